@@ -1,0 +1,264 @@
+/*
+ * pa.h — C ABI of the paged-KV-cache decode library (libpa.so), sm_100a.
+ *
+ * The library implements the data-parallel hot path of PagedAttention: the
+ * KV cache is cut into fixed-size blocks of BLOCK_SIZE tokens, a per-sequence
+ * block table maps logical blocks to non-contiguous physical blocks, blocks
+ * are handed out on demand, and parallel samples share prompt blocks through
+ * reference counts with copy-on-write (vLLM launch blog, "PagedAttention"
+ * section, summarised on the CSDN discovery note, item 2; agientry.com
+ * overview, opening section; gitcode repo walkthrough, section 2.1).
+ *
+ * Conventions for every call:
+ *  - Device memory and streams belong to the caller.  No call allocates or
+ *    frees device memory; scratch space is passed in through pa_opts.
+ *  - Device calls are asynchronous on opts->stream (NULL opts or NULL stream
+ *    means the legacy default stream) on the current CUDA device; pointers
+ *    must belong to that device.
+ *  - Argument errors are reported before anything is launched, with no side
+ *    effects.  Errors that only the device can see (a block id outside the
+ *    pool, a slot outside the cache, a context longer than its block-table
+ *    row, a bounded wait that gave up) set bits in a per-device status word
+ *    and the offending element is skipped (see pa_get_device_status).
+ *  - Tensors are described by pa_tensor: a data pointer, a dtype, a rank and
+ *    per-dimension sizes and strides (in elements).  Only the layouts listed
+ *    at each call are accepted.
+ *
+ * Physical KV layout (part of this ABI): k_cache and v_cache are each
+ *   [num_blocks, num_kv_heads, block_size, head_size], contiguous, row-major,
+ * so that the page of one (block, kv head) — block_size x head_size elements,
+ * 4 KiB for bf16 / head_size 128 or fp32 / head_size 64 — is one contiguous
+ * run that a single bulk copy moves.  The historical layout printed on the
+ * pages (K split as head_size/x by x, V transposed; gitcode walkthrough,
+ * section 2.1) served per-thread-group 16-byte loads on older GPUs and is not
+ * used.
+ *
+ * Supported: block_size 16; (bf16, head_size 128), (bf16, head_size 64),
+ * (fp32, head_size 64), (fp32, head_size 128); num_heads / num_kv_heads in
+ * {1, 2, 4, 8}.  Anything else returns PA_ERR_UNSUPPORTED.
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARG = 1,    /* bad pointer, shape, stride, dtype or id */
+  PA_ERR_UNSUPPORTED = 2,    /* valid but not implemented (dtype/head size/group) */
+  PA_ERR_OUT_OF_BLOCKS = 3,  /* allocator: free blocks exhausted, state unchanged */
+  PA_ERR_CUDA = 4,           /* a CUDA runtime call failed */
+  PA_ERR_DEVICE_TIMEOUT = 5, /* a device-side bounded wait gave up */
+  PA_ERR_DEVICE_BOUNDS = 6   /* a device-side index check failed; element skipped */
+} pa_status;
+
+typedef enum { PA_F32 = 0, PA_BF16 = 1, PA_I32 = 2, PA_I64 = 3 } pa_dtype;
+
+/* A strided view of caller-owned memory.  Strides are in elements. */
+typedef struct {
+  void* data;
+  int32_t dtype; /* pa_dtype */
+  int32_t ndim;  /* 1..5 */
+  int64_t shape[5];
+  int64_t stride[5];
+} pa_tensor;
+
+typedef struct {
+  void* stream;             /* cudaStream_t, NULL = legacy default stream */
+  void* workspace;          /* device scratch for split decode, 256-byte aligned, may be NULL */
+  size_t workspace_bytes;   /* size of workspace */
+  int32_t partition_tokens; /* pa_decode context split:
+                                 0  = auto: balanced split over all SMs when the
+                                      workspace is large enough, else no split;
+                                 >0 = fixed partitions of this many tokens (a
+                                      multiple of block_size), one partial result
+                                      per partition, then a log-sum-exp merge;
+                                 -1 = no split: each (sequence, kv head) is
+                                      reduced by one warp, no workspace needed */
+  int32_t timeout_ms;       /* bound on every device-side wait; 0 = 1000 ms */
+} pa_opts;
+
+/* Device status bits (pa_get_device_status). */
+#define PA_DEV_TIMEOUT 0x1u     /* a bounded wait gave up */
+#define PA_DEV_BAD_BLOCK 0x2u   /* block-table entry or copy pair outside [0, num_blocks) */
+#define PA_DEV_BAD_CONTEXT 0x4u /* context_len < 0 or > block-table row capacity */
+#define PA_DEV_BAD_SLOT 0x8u    /* slot_mapping entry < -1 or >= num_blocks*block_size */
+
+/* ---------------------------------------------------------------------------
+ * Cache write (the step that stores each new token's K/V at its slot).
+ * The pages imply it — tokens land in the block the table names, at their
+ * offset (launch blog "PagedAttention" section; CSDN note item 2) — without
+ * naming it.
+ *
+ *   for t, h:  s = slot_mapping[t];  if s == -1: skip
+ *              k_cache[s / block_size, h, s % block_size, :] = key[t, h, :]
+ *              v_cache[s / block_size, h, s % block_size, :] = value[t, h, :]
+ *
+ * key, value:   [T, num_kv_heads, head_size], dtype of the cache, last dim
+ *               contiguous, token/head strides multiples of 16 bytes, data
+ *               16-byte aligned.  T may be 0 (nothing is launched).
+ * k_cache, v_cache: [num_blocks, num_kv_heads, block_size, head_size],
+ *               contiguous, 16-byte aligned.
+ * slot_mapping: [T] int64, contiguous.  Entries outside [-1, num_blocks*bs)
+ *               set PA_DEV_BAD_SLOT and are skipped.
+ * Bit copy: the cache receives the exact input bits.  Two tokens with the same
+ * slot in one call race (undefined which one lands).
+ * ------------------------------------------------------------------------- */
+pa_status pa_reshape_and_cache(const pa_tensor* key, const pa_tensor* value, pa_tensor* k_cache,
+                               pa_tensor* v_cache, const pa_tensor* slot_mapping, const pa_opts* opts);
+
+/* ---------------------------------------------------------------------------
+ * Copy-on-write block copy (launch blog "PagedAttention" section; CSDN note
+ * item 2: a write into a block shared by several samples first copies it).
+ *
+ *   for each pair (src, dst):  k_cache[dst] = k_cache[src];  v_cache[dst] = v_cache[src]
+ *   (whole block: every head, every offset)
+ *
+ * pairs: [n, 2] int64 in DEVICE memory, contiguous (the allocator's
+ *        copy-on-write output, uploaded by the caller on the same stream).
+ *        n may be 0.  A pair with an id outside [0, num_blocks) sets
+ *        PA_DEV_BAD_BLOCK and is skipped.  Destinations must be distinct and
+ *        no destination may be another pair's source (the allocator never
+ *        emits such pairs).
+ * ------------------------------------------------------------------------- */
+pa_status pa_copy_blocks(pa_tensor* k_cache, pa_tensor* v_cache, const pa_tensor* pairs, const pa_opts* opts);
+
+/* ---------------------------------------------------------------------------
+ * Paged decode attention (gitcode walkthrough, section 2.1: the query-key dot
+ * product, softmax normalisation and weighted sum of V over K/V gathered
+ * block by block; launch blog "PagedAttention" section).
+ *
+ *   for sequence i < B, query head h < H, with g = h / (H / num_kv_heads):
+ *     s_t = scale * <query[i,h,:], K_i[t, g, :]>,  t < context_lens[i]
+ *     out[i,h,:] = sum_t softmax(s)_t V_i[t, g, :]
+ *   where K_i[t] = k_cache[block_tables[i][t / bs], g, t % bs, :] (same for V).
+ *   context_lens[i] == 0 gives a zero row.
+ *
+ * out:          [B, H, head_size], cache dtype, last dim contiguous, strides
+ *               multiples of 16 bytes, 16-byte aligned.  Written, never read.
+ * query:        [B, H, head_size], cache dtype, same layout rules.
+ * k_cache, v_cache: see the physical layout above.
+ * block_tables: [B, max_blocks_per_seq] int32, last dim contiguous.  Only the
+ *               first ceil(context_lens[i] / bs) entries of row i are read;
+ *               each must be in [0, num_blocks) (else PA_DEV_BAD_BLOCK and the
+ *               page is replaced by block 0).
+ * context_lens: [B] int32.  Values above max_blocks_per_seq * bs, or below 0,
+ *               set PA_DEV_BAD_CONTEXT and are clamped.
+ * scale:        softmax scale (usually 1/sqrt(head_size)).
+ * num_kv_heads: must equal k_cache's second dimension and divide H.
+ * Accumulation is fp32; the output is rounded to the cache dtype (bf16:
+ * round-to-nearest-even).  Split modes (opts->partition_tokens) change only
+ * fp32 rounding order.  Fixed-partition mode leaves its per-partition
+ * results in the workspace: float o[B][H][P][head_size] (normalised) followed
+ * by float lse[B][H][P] (natural log of the partition's softmax denominator
+ * plus its max logit), P = ceil(max_blocks_per_seq*bs / partition_tokens);
+ * entries of partitions past a sequence's end are left unwritten.
+ * B may be 0.  B must be < 2^20.
+ * ------------------------------------------------------------------------- */
+pa_status pa_decode(pa_tensor* out, const pa_tensor* query, const pa_tensor* k_cache, const pa_tensor* v_cache,
+                    const pa_tensor* block_tables, const pa_tensor* context_lens, float scale,
+                    int32_t num_kv_heads, const pa_opts* opts);
+
+/* Launch shape of pa_decode on the current process (a tuning knob; 0 keeps
+ * the default): warps per CTA (each warp is one worker with its own page
+ * ring; default 8, at most 8), ring stages per warp (default 3; lowered
+ * automatically to fit shared memory), CTAs per SM (default 1).  Changes
+ * the workspace size of the auto mode.  Not thread-safe. */
+pa_status pa_set_decode_tuning(int32_t warps_per_cta, int32_t stages, int32_t ctas_per_sm);
+
+/* Workspace bytes pa_decode needs on the current device for these sizes and
+ * this partition_tokens setting (0 = auto/balanced, >0 = fixed, -1 = none).
+ * Needs a CUDA device for the auto mode (it depends on the SM count). */
+pa_status pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
+                                    int32_t head_size, int32_t max_blocks_per_seq, int32_t partition_tokens,
+                                    size_t* bytes_out);
+
+/* ---------------------------------------------------------------------------
+ * Host block allocator (launch blog "PagedAttention" section; CSDN note item
+ * 2; agientry.com overview).  Pure host code, not thread-safe (the caller
+ * serialises), no CUDA needed.
+ *
+ * Rules (the pages give the mechanism; the orders are this library's):
+ *  - free blocks form a LIFO stack seeded from free_order (free_order[0] is
+ *    handed out first; NULL = 0, 1, 2, ...); a freed block goes on top;
+ *  - appending token at position p: if p % bs == 0 a fresh block is taken;
+ *    otherwise, if the last block's reference count is above 1, a fresh block
+ *    is taken, the pair (old, new) is reported for pa_copy_blocks, the old
+ *    block loses one reference and the table points at the new block
+ *    (copy-on-write; at most one pair per append call); the token's slot is
+ *    table[p / bs] * bs + p % bs;
+ *  - an append is all-or-nothing: PA_ERR_OUT_OF_BLOCKS leaves every state
+ *    unchanged;
+ *  - fork: the child gets a copy of the parent's table and length; each block
+ *    gains one reference;
+ *  - free: blocks lose one reference in table order; a block reaching 0 is
+ *    pushed on the free stack.
+ * Sequence ids are arbitrary int64 values.
+ * ------------------------------------------------------------------------- */
+typedef struct pa_allocator pa_allocator;
+
+typedef struct {
+  int32_t num_blocks;
+  int32_t num_free;
+  int32_t num_seqs;
+  int32_t block_size;
+  int64_t num_tokens;  /* sum of sequence lengths (shared tokens counted per sequence) */
+  int64_t waste_slots; /* unused slots of blocks in use (bs minus the most any holder filled) */
+} pa_alloc_stats;
+
+pa_status pa_alloc_create(int32_t num_blocks, int32_t block_size, const int32_t* free_order, pa_allocator** out);
+void pa_alloc_destroy(pa_allocator* a);
+pa_status pa_seq_add(pa_allocator* a, int64_t seq_id);
+/* slots_out: [n_tokens]; cow_pair_out: [2], written (src, dst) when *n_cow_out == 1. */
+pa_status pa_seq_append(pa_allocator* a, int64_t seq_id, int32_t n_tokens, int64_t* slots_out,
+                        int64_t* cow_pair_out, int32_t* n_cow_out);
+/* Appends n_tokens[k] tokens to seq_ids[k] for k = 0..n-1 in order.  Each
+ * sequence's append is all-or-nothing; the call stops at the first failure and
+ * *n_done_out says how many sequences were served.  slots_out holds the slots
+ * of the served sequences back to back; cow_pairs_out [n, 2] holds the
+ * *n_cow_out copy pairs in order. */
+pa_status pa_seq_append_batch(pa_allocator* a, const int64_t* seq_ids, const int32_t* n_tokens, int32_t n,
+                              int64_t* slots_out, int64_t* cow_pairs_out, int32_t* n_cow_out, int32_t* n_done_out);
+pa_status pa_seq_fork(pa_allocator* a, int64_t parent, int64_t child);
+pa_status pa_seq_free(pa_allocator* a, int64_t seq_id);
+pa_status pa_seq_len(const pa_allocator* a, int64_t seq_id, int32_t* len_out);
+pa_status pa_seq_block_table(const pa_allocator* a, int64_t seq_id, int32_t* out, int32_t cap, int32_t* n_out);
+/* Fills out [n, max_blocks] (row-major) with the tables of seq_ids, padding
+ * with -1, and context_lens_out [n] (nullable) with their lengths.  A table
+ * longer than max_blocks is PA_ERR_INVALID_ARG (nothing written). */
+pa_status pa_alloc_block_tables(const pa_allocator* a, const int64_t* seq_ids, int32_t n, int32_t* out,
+                                int32_t max_blocks, int32_t* context_lens_out);
+int32_t pa_alloc_num_free(const pa_allocator* a);
+int32_t pa_block_refcount(const pa_allocator* a, int32_t block); /* -1 if out of range */
+pa_status pa_alloc_get_stats(const pa_allocator* a, pa_alloc_stats* out);
+
+/* ---------------------------------------------------------------------------
+ * Device status and diagnostics
+ * ------------------------------------------------------------------------- */
+/* Synchronises opts->stream, then reads and clears the current device's
+ * status word into *bits_out (nullable).  Returns PA_ERR_DEVICE_TIMEOUT if the
+ * timeout bit was set, else PA_ERR_DEVICE_BOUNDS if any bounds bit was set,
+ * else PA_OK. */
+pa_status pa_get_device_status(const pa_opts* opts, uint32_t* bits_out);
+
+/* Launches one warp that waits, with the same bounded wait the decode
+ * pipeline uses, on a barrier nothing completes.  It must give up after
+ * opts->timeout_ms and set PA_DEV_TIMEOUT; the context stays usable.  No copy
+ * is in flight during the wait. */
+pa_status pa_debug_wait_selftest(const pa_opts* opts);
+
+const char* pa_status_string(pa_status s);
+
+/* Library version, for the Python loader's sanity check. */
+int32_t pa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H_ */

@@ -1,0 +1,255 @@
+"""Python binding of libpa.so — paged KV cache decode for B200 (sm_100a).
+
+Thin wrappers with the C ABI's names (include/pa.h).  They only turn torch
+tensors and numpy arrays into the ABI's plain pointers, shapes and strides;
+all device work runs in the library's CUDA kernels.  PyTorch is used by
+callers for device memory and streams.  A non-OK status raises
+``PagedAttentionError``.  When no stream is given, the current torch CUDA
+stream is used.
+"""
+
+from __future__ import annotations
+
+import ctypes
+from typing import Optional, Sequence, Tuple
+
+import numpy as np
+
+from . import _lib
+from ._lib import (PA_DEV_BAD_BLOCK, PA_DEV_BAD_CONTEXT, PA_DEV_BAD_SLOT,  # noqa: F401
+                   PA_DEV_TIMEOUT, PaAllocStats, PaOpts, PaTensor)
+
+__all__ = [
+    "PagedAttentionError", "OutOfBlocksError", "pa_reshape_and_cache", "pa_copy_blocks", "pa_decode",
+    "pa_decode_workspace_bytes", "pa_set_decode_tuning", "pa_get_device_status", "pa_debug_wait_selftest",
+    "Allocator", "library",
+]
+
+_lib_handle = _lib.load()
+
+
+def library():
+    """The loaded ctypes library (for tests of the raw ABI)."""
+    return _lib_handle
+
+
+class PagedAttentionError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = _lib_handle.pa_status_string(status)
+        super().__init__(f"{where}: {_lib.STATUS_NAMES.get(status, status)} ({msg.decode() if msg else ''})")
+
+
+class OutOfBlocksError(PagedAttentionError):
+    pass
+
+
+def _check(st: int, where: str) -> None:
+    if st != 0:
+        if st == 3:
+            raise OutOfBlocksError(st, where)
+        raise PagedAttentionError(st, where)
+
+
+def _dtype_code(t) -> int:
+    import torch
+
+    codes = {torch.float32: _lib.PA_F32, torch.bfloat16: _lib.PA_BF16, torch.int32: _lib.PA_I32,
+             torch.int64: _lib.PA_I64}
+    if t.dtype not in codes:
+        raise TypeError(f"unsupported dtype {t.dtype}")
+    return codes[t.dtype]
+
+
+def _tensor(t) -> PaTensor:
+    """torch.Tensor -> pa_tensor (pointer, dtype, shape, strides in elements)."""
+    pt = PaTensor()
+    pt.data = t.data_ptr() if t.numel() > 0 else (t.data_ptr() or None)
+    pt.dtype = _dtype_code(t)
+    if t.dim() > 5:
+        raise ValueError("at most 5 dimensions")
+    pt.ndim = t.dim()
+    for k in range(t.dim()):
+        pt.shape[k] = t.shape[k]
+        pt.stride[k] = t.stride(k)
+    return pt
+
+
+def _stream_ptr(stream) -> Optional[int]:
+    import torch
+
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, int):
+        return stream or None
+    return stream.cuda_stream or None
+
+
+def _opts(stream=None, workspace=None, partition_tokens: int = 0, timeout_ms: int = 0) -> PaOpts:
+    o = PaOpts()
+    o.stream = _stream_ptr(stream)
+    if workspace is not None:
+        o.workspace = workspace.data_ptr()
+        o.workspace_bytes = workspace.numel() * workspace.element_size()
+    else:
+        o.workspace = None
+        o.workspace_bytes = 0
+    o.partition_tokens = partition_tokens
+    o.timeout_ms = timeout_ms
+    return o
+
+
+# ---------------------------------------------------------------------------
+# device entry points
+# ---------------------------------------------------------------------------
+
+def pa_reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, stream=None) -> None:
+    """Write each token's K/V [T, H_kv, D] into its slot of the paged cache."""
+    tk, tv, kc, vc, sm = (_tensor(x) for x in (key, value, k_cache, v_cache, slot_mapping))
+    o = _opts(stream)
+    _check(_lib_handle.pa_reshape_and_cache(ctypes.byref(tk), ctypes.byref(tv), ctypes.byref(kc), ctypes.byref(vc),
+                                            ctypes.byref(sm), ctypes.byref(o)), "pa_reshape_and_cache")
+
+
+def pa_copy_blocks(k_cache, v_cache, pairs, stream=None) -> None:
+    """Copy whole blocks (K and V) for each (src, dst) row of the int64 [n, 2] device tensor."""
+    kc, vc, pr = (_tensor(x) for x in (k_cache, v_cache, pairs))
+    o = _opts(stream)
+    _check(_lib_handle.pa_copy_blocks(ctypes.byref(kc), ctypes.byref(vc), ctypes.byref(pr), ctypes.byref(o)),
+           "pa_copy_blocks")
+
+
+def pa_decode(out, query, k_cache, v_cache, block_tables, context_lens, scale: float, num_kv_heads: int,
+              workspace=None, partition_tokens: int = 0, stream=None, timeout_ms: int = 0) -> None:
+    """Paged decode attention; writes out [B, H, D].  ``partition_tokens``:
+    0 = auto (balanced split when ``workspace`` is large enough), >0 = fixed
+    partitions, -1 = no split."""
+    to, tq, kc, vc, bt, cl = (_tensor(x) for x in (out, query, k_cache, v_cache, block_tables, context_lens))
+    o = _opts(stream, workspace, partition_tokens, timeout_ms)
+    _check(_lib_handle.pa_decode(ctypes.byref(to), ctypes.byref(tq), ctypes.byref(kc), ctypes.byref(vc),
+                                 ctypes.byref(bt), ctypes.byref(cl), ctypes.c_float(scale), int(num_kv_heads),
+                                 ctypes.byref(o)), "pa_decode")
+
+
+def pa_decode_workspace_bytes(num_seqs: int, num_heads: int, num_kv_heads: int, head_size: int,
+                              max_blocks_per_seq: int, partition_tokens: int = 0) -> int:
+    n = ctypes.c_size_t(0)
+    _check(_lib_handle.pa_decode_workspace_bytes(num_seqs, num_heads, num_kv_heads, head_size, max_blocks_per_seq,
+                                                 partition_tokens, ctypes.byref(n)), "pa_decode_workspace_bytes")
+    return int(n.value)
+
+
+def pa_set_decode_tuning(warps_per_cta: int = 0, stages: int = 0, ctas_per_sm: int = 0) -> None:
+    _check(_lib_handle.pa_set_decode_tuning(warps_per_cta, stages, ctas_per_sm), "pa_set_decode_tuning")
+
+
+def pa_get_device_status(stream=None) -> Tuple[int, int]:
+    """Synchronise the stream; return (status, bits) and clear the device status word."""
+    bits = ctypes.c_uint32(0)
+    o = _opts(stream)
+    st = _lib_handle.pa_get_device_status(ctypes.byref(o), ctypes.byref(bits))
+    return int(st), int(bits.value)
+
+
+def pa_debug_wait_selftest(timeout_ms: int, stream=None) -> None:
+    o = _opts(stream, timeout_ms=timeout_ms)
+    _check(_lib_handle.pa_debug_wait_selftest(ctypes.byref(o)), "pa_debug_wait_selftest")
+
+
+# ---------------------------------------------------------------------------
+# host allocator
+# ---------------------------------------------------------------------------
+
+def _i64p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int64))
+
+
+def _i32p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+
+
+class Allocator:
+    """Host block allocator of libpa (pa_alloc_* / pa_seq_*)."""
+
+    def __init__(self, num_blocks: int, block_size: int, free_order: Optional[Sequence[int]] = None):
+        h = ctypes.c_void_p()
+        if free_order is not None:
+            self._order = np.ascontiguousarray(np.asarray(free_order, dtype=np.int32))
+            if self._order.shape != (num_blocks,):
+                raise ValueError("free_order must list every block once")
+            ptr = _i32p(self._order)
+        else:
+            ptr = None
+        _check(_lib_handle.pa_alloc_create(num_blocks, block_size, ptr, ctypes.byref(h)), "pa_alloc_create")
+        self._h = h
+        self.num_blocks = num_blocks
+        self.block_size = block_size
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h is not None and h.value:
+            _lib_handle.pa_alloc_destroy(h)
+            self._h = None
+
+    def add(self, seq: int) -> None:
+        _check(_lib_handle.pa_seq_add(self._h, seq), "pa_seq_add")
+
+    def append(self, seq: int, n: int):
+        """Returns (slots int64 [n], copy-on-write pairs as a list of (src, dst))."""
+        slots = np.zeros(max(n, 1), np.int64)
+        pair = np.zeros(2, np.int64)
+        ncow = ctypes.c_int32(0)
+        _check(_lib_handle.pa_seq_append(self._h, seq, n, _i64p(slots), _i64p(pair), ctypes.byref(ncow)),
+               "pa_seq_append")
+        return slots[:n], ([(int(pair[0]), int(pair[1]))] if ncow.value else [])
+
+    def append_batch(self, seqs: Sequence[int], counts: Sequence[int]):
+        """Returns (slots of all tokens back to back, pairs int64 [n_cow, 2])."""
+        ids = np.ascontiguousarray(np.asarray(seqs, np.int64))
+        cnt = np.ascontiguousarray(np.asarray(counts, np.int32))
+        slots = np.zeros(max(1, int(cnt.sum())), np.int64)
+        pairs = np.zeros((max(1, len(ids)), 2), np.int64)
+        ncow = ctypes.c_int32(0)
+        ndone = ctypes.c_int32(0)
+        st = _lib_handle.pa_seq_append_batch(self._h, _i64p(ids), _i32p(cnt), len(ids), _i64p(slots),
+                                             _i64p(pairs), ctypes.byref(ncow), ctypes.byref(ndone))
+        _check(st, f"pa_seq_append_batch (served {ndone.value} of {len(ids)})")
+        return slots[: int(cnt.sum())], pairs[: ncow.value]
+
+    def fork(self, parent: int, child: int) -> None:
+        _check(_lib_handle.pa_seq_fork(self._h, parent, child), "pa_seq_fork")
+
+    def free(self, seq: int) -> None:
+        _check(_lib_handle.pa_seq_free(self._h, seq), "pa_seq_free")
+
+    def length(self, seq: int) -> int:
+        n = ctypes.c_int32(0)
+        _check(_lib_handle.pa_seq_len(self._h, seq, ctypes.byref(n)), "pa_seq_len")
+        return int(n.value)
+
+    def block_table(self, seq: int):
+        cap = self.length(seq) // self.block_size + 1
+        out = np.zeros(cap, np.int32)
+        n = ctypes.c_int32(0)
+        _check(_lib_handle.pa_seq_block_table(self._h, seq, _i32p(out), cap, ctypes.byref(n)), "pa_seq_block_table")
+        return out[: n.value].tolist()
+
+    def block_tables(self, seqs: Sequence[int], max_blocks: int):
+        """(tables int32 [n, max_blocks] padded with -1, context lengths int32 [n])."""
+        ids = np.ascontiguousarray(np.asarray(seqs, np.int64))
+        out = np.zeros((len(ids), max(max_blocks, 1)), np.int32)
+        lens = np.zeros(max(len(ids), 1), np.int32)
+        _check(_lib_handle.pa_alloc_block_tables(self._h, _i64p(ids), len(ids), _i32p(out), max_blocks,
+                                                 _i32p(lens)), "pa_alloc_block_tables")
+        return out[:, :max_blocks], lens[: len(ids)]
+
+    def num_free(self) -> int:
+        return int(_lib_handle.pa_alloc_num_free(self._h))
+
+    def refcount(self, block: int) -> int:
+        return int(_lib_handle.pa_block_refcount(self._h, block))
+
+    def stats(self) -> dict:
+        s = PaAllocStats()
+        _check(_lib_handle.pa_alloc_get_stats(self._h, ctypes.byref(s)), "pa_alloc_get_stats")
+        return {f: getattr(s, f) for f, _ in PaAllocStats._fields_}

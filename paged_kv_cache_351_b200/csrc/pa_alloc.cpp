@@ -1,0 +1,251 @@
+// Host block allocator of the paged KV cache: fixed-size blocks, per-sequence
+// block tables, blocks handed out on demand, reference counts and
+// copy-on-write for shared prompt blocks (vLLM launch blog, "PagedAttention"
+// section, as summarised on the CSDN discovery note, item 2; agientry.com
+// overview, opening section).  The exact orders (LIFO free stack seeded from
+// the caller's order, copy-on-write trigger, free in table order) are stated
+// in include/pa.h.
+//
+// Plain host code: O(1) per token, no CUDA.  Every request checks its
+// arguments and its block needs before changing anything, so a failed call
+// leaves the state untouched.
+
+#include <cstdint>
+#include <cstring>
+#include <new>
+#include <unordered_map>
+#include <vector>
+
+#include "../../include/pa.h"
+
+namespace {
+
+struct Seq {
+  std::vector<int32_t> table;
+  int32_t len = 0;
+};
+
+}  // namespace
+
+struct pa_allocator {
+  int32_t num_blocks = 0;
+  int32_t block_size = 0;
+  std::vector<int32_t> free_stack;  // top = back()
+  std::vector<int32_t> ref;
+  std::unordered_map<int64_t, Seq> seqs;
+
+  // Blocks an append of n tokens to s needs (copy-on-write + fresh blocks).
+  int64_t blocks_needed(const Seq& s, int64_t n) const {
+    const int64_t bs = block_size;
+    const int64_t pos = s.len;
+    int64_t need = 0;
+    if (n > 0 && pos % bs != 0 && ref[s.table.back()] > 1) need += 1;
+    const int64_t first = (pos + bs - 1) / bs * bs;  // first position >= pos opening a block
+    if (first < pos + n) need += (pos + n - 1 - first) / bs + 1;
+    return need;
+  }
+
+  pa_status append(int64_t seq_id, int32_t n, int64_t* slots, int64_t* cow_pair, int32_t* n_cow) {
+    auto it = seqs.find(seq_id);
+    if (it == seqs.end() || n < 0) return PA_ERR_INVALID_ARG;
+    if (n > 0 && slots == nullptr) return PA_ERR_INVALID_ARG;
+    Seq& s = it->second;
+    if (static_cast<int64_t>(s.len) + n > INT32_MAX) return PA_ERR_INVALID_ARG;
+    if (blocks_needed(s, n) > static_cast<int64_t>(free_stack.size())) return PA_ERR_OUT_OF_BLOCKS;
+    const int32_t bs = block_size;
+    int32_t cows = 0;
+    for (int32_t k = 0; k < n; ++k) {
+      const int32_t pos = s.len;
+      if (pos % bs == 0) {
+        const int32_t b = free_stack.back();
+        free_stack.pop_back();
+        ref[b] = 1;
+        s.table.push_back(b);
+      } else {
+        const int32_t last = s.table.back();
+        if (ref[last] > 1) {
+          const int32_t b = free_stack.back();
+          free_stack.pop_back();
+          ref[b] = 1;
+          ref[last] -= 1;
+          s.table.back() = b;
+          if (cow_pair != nullptr) {
+            cow_pair[0] = last;
+            cow_pair[1] = b;
+          }
+          ++cows;
+        }
+      }
+      slots[k] = static_cast<int64_t>(s.table[pos / bs]) * bs + pos % bs;
+      s.len = pos + 1;
+    }
+    if (n_cow != nullptr) *n_cow = cows;
+    return PA_OK;
+  }
+};
+
+extern "C" {
+
+pa_status pa_alloc_create(int32_t num_blocks, int32_t block_size, const int32_t* free_order, pa_allocator** out) {
+  if (out == nullptr || num_blocks <= 0 || block_size <= 0) return PA_ERR_INVALID_ARG;
+  *out = nullptr;
+  pa_allocator* a = new (std::nothrow) pa_allocator();
+  if (a == nullptr) return PA_ERR_INVALID_ARG;
+  a->num_blocks = num_blocks;
+  a->block_size = block_size;
+  a->ref.assign(num_blocks, 0);
+  a->free_stack.resize(num_blocks);
+  if (free_order != nullptr) {
+    std::vector<uint8_t> seen(num_blocks, 0);
+    for (int32_t k = 0; k < num_blocks; ++k) {
+      const int32_t b = free_order[k];
+      if (b < 0 || b >= num_blocks || seen[b]) {
+        delete a;
+        return PA_ERR_INVALID_ARG;
+      }
+      seen[b] = 1;
+      a->free_stack[num_blocks - 1 - k] = b;
+    }
+  } else {
+    for (int32_t k = 0; k < num_blocks; ++k) a->free_stack[num_blocks - 1 - k] = k;
+  }
+  *out = a;
+  return PA_OK;
+}
+
+void pa_alloc_destroy(pa_allocator* a) { delete a; }
+
+pa_status pa_seq_add(pa_allocator* a, int64_t seq_id) {
+  if (a == nullptr) return PA_ERR_INVALID_ARG;
+  if (a->seqs.count(seq_id)) return PA_ERR_INVALID_ARG;
+  a->seqs.emplace(seq_id, Seq());
+  return PA_OK;
+}
+
+pa_status pa_seq_append(pa_allocator* a, int64_t seq_id, int32_t n_tokens, int64_t* slots_out,
+                        int64_t* cow_pair_out, int32_t* n_cow_out) {
+  if (a == nullptr) return PA_ERR_INVALID_ARG;
+  return a->append(seq_id, n_tokens, slots_out, cow_pair_out, n_cow_out);
+}
+
+pa_status pa_seq_append_batch(pa_allocator* a, const int64_t* seq_ids, const int32_t* n_tokens, int32_t n,
+                              int64_t* slots_out, int64_t* cow_pairs_out, int32_t* n_cow_out, int32_t* n_done_out) {
+  if (a == nullptr || n < 0 || (n > 0 && (seq_ids == nullptr || n_tokens == nullptr))) return PA_ERR_INVALID_ARG;
+  int64_t off = 0;
+  int32_t cows = 0;
+  pa_status st = PA_OK;
+  int32_t k = 0;
+  for (; k < n; ++k) {
+    int32_t c = 0;
+    int64_t pair[2] = {-1, -1};
+    st = a->append(seq_ids[k], n_tokens[k], slots_out == nullptr ? nullptr : slots_out + off, pair, &c);
+    if (st != PA_OK) break;
+    off += n_tokens[k];
+    if (c) {
+      if (cow_pairs_out != nullptr) {
+        cow_pairs_out[2 * cows] = pair[0];
+        cow_pairs_out[2 * cows + 1] = pair[1];
+      }
+      ++cows;
+    }
+  }
+  if (n_cow_out != nullptr) *n_cow_out = cows;
+  if (n_done_out != nullptr) *n_done_out = k;
+  return st;
+}
+
+pa_status pa_seq_fork(pa_allocator* a, int64_t parent, int64_t child) {
+  if (a == nullptr) return PA_ERR_INVALID_ARG;
+  auto it = a->seqs.find(parent);
+  if (it == a->seqs.end() || a->seqs.count(child)) return PA_ERR_INVALID_ARG;
+  Seq c = it->second;  // copy before emplace may rehash
+  for (int32_t b : c.table) a->ref[b] += 1;
+  a->seqs.emplace(child, std::move(c));
+  return PA_OK;
+}
+
+pa_status pa_seq_free(pa_allocator* a, int64_t seq_id) {
+  if (a == nullptr) return PA_ERR_INVALID_ARG;
+  auto it = a->seqs.find(seq_id);
+  if (it == a->seqs.end()) return PA_ERR_INVALID_ARG;
+  for (int32_t b : it->second.table) {
+    a->ref[b] -= 1;
+    if (a->ref[b] == 0) a->free_stack.push_back(b);
+  }
+  a->seqs.erase(it);
+  return PA_OK;
+}
+
+pa_status pa_seq_len(const pa_allocator* a, int64_t seq_id, int32_t* len_out) {
+  if (a == nullptr || len_out == nullptr) return PA_ERR_INVALID_ARG;
+  auto it = a->seqs.find(seq_id);
+  if (it == a->seqs.end()) return PA_ERR_INVALID_ARG;
+  *len_out = it->second.len;
+  return PA_OK;
+}
+
+pa_status pa_seq_block_table(const pa_allocator* a, int64_t seq_id, int32_t* out, int32_t cap, int32_t* n_out) {
+  if (a == nullptr || n_out == nullptr) return PA_ERR_INVALID_ARG;
+  auto it = a->seqs.find(seq_id);
+  if (it == a->seqs.end()) return PA_ERR_INVALID_ARG;
+  const auto& t = it->second.table;
+  *n_out = static_cast<int32_t>(t.size());
+  if (static_cast<int64_t>(t.size()) > cap || (!t.empty() && out == nullptr)) return PA_ERR_INVALID_ARG;
+  if (!t.empty()) std::memcpy(out, t.data(), t.size() * sizeof(int32_t));
+  return PA_OK;
+}
+
+pa_status pa_alloc_block_tables(const pa_allocator* a, const int64_t* seq_ids, int32_t n, int32_t* out,
+                                int32_t max_blocks, int32_t* context_lens_out) {
+  if (a == nullptr || n < 0 || max_blocks < 0) return PA_ERR_INVALID_ARG;
+  if (n > 0 && (seq_ids == nullptr || (out == nullptr && max_blocks > 0))) return PA_ERR_INVALID_ARG;
+  for (int32_t r = 0; r < n; ++r) {
+    auto it = a->seqs.find(seq_ids[r]);
+    if (it == a->seqs.end() || static_cast<int64_t>(it->second.table.size()) > max_blocks) return PA_ERR_INVALID_ARG;
+  }
+  for (int32_t r = 0; r < n; ++r) {
+    const Seq& s = a->seqs.find(seq_ids[r])->second;
+    int32_t* row = out + static_cast<int64_t>(r) * max_blocks;
+    const int32_t nt = static_cast<int32_t>(s.table.size());
+    for (int32_t k = 0; k < max_blocks; ++k) row[k] = k < nt ? s.table[k] : -1;
+    if (context_lens_out != nullptr) context_lens_out[r] = s.len;
+  }
+  return PA_OK;
+}
+
+int32_t pa_alloc_num_free(const pa_allocator* a) {
+  return a == nullptr ? -1 : static_cast<int32_t>(a->free_stack.size());
+}
+
+int32_t pa_block_refcount(const pa_allocator* a, int32_t block) {
+  if (a == nullptr || block < 0 || block >= a->num_blocks) return -1;
+  return a->ref[block];
+}
+
+pa_status pa_alloc_get_stats(const pa_allocator* a, pa_alloc_stats* out) {
+  if (a == nullptr || out == nullptr) return PA_ERR_INVALID_ARG;
+  const int32_t bs = a->block_size;
+  std::vector<int32_t> filled(a->num_blocks, 0);
+  int64_t tokens = 0;
+  for (const auto& kv : a->seqs) {
+    const Seq& s = kv.second;
+    tokens += s.len;
+    for (size_t k = 0; k < s.table.size(); ++k) {
+      const int64_t f = std::min<int64_t>(bs, s.len - static_cast<int64_t>(k) * bs);
+      int32_t& slot = filled[s.table[k]];
+      if (f > slot) slot = static_cast<int32_t>(f);
+    }
+  }
+  int64_t waste = 0;
+  for (int32_t b = 0; b < a->num_blocks; ++b)
+    if (a->ref[b] > 0) waste += bs - filled[b];
+  out->num_blocks = a->num_blocks;
+  out->num_free = static_cast<int32_t>(a->free_stack.size());
+  out->num_seqs = static_cast<int32_t>(a->seqs.size());
+  out->block_size = bs;
+  out->num_tokens = tokens;
+  out->waste_slots = waste;
+  return PA_OK;
+}
+
+}  // extern "C"

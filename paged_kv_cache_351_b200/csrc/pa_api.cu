@@ -1,0 +1,511 @@
+// C ABI of libpa.so: argument validation, launch configuration and the
+// device-status word.  All kernels live in this one translation unit (the
+// status word is a plain __device__ variable, no relocatable device code).
+// The host allocator is in pa_alloc.cpp.
+
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/pa.h"
+#include "pa_cache.cuh"
+#include "pa_common.cuh"
+#include "pa_decode.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kMaxBatch = 8192;  // decode: one int per sequence of shared memory per CTA
+
+struct DeviceInfo {
+  bool ready = false;
+  int sms = 0;
+  int smem_optin = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+struct Tuning {
+  int warps = 8;
+  int stages = 3;
+  int ctas_per_sm = 1;
+};
+Tuning g_tuning;
+
+pa_status device_info(DeviceInfo* out, int* dev_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return PA_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+      return PA_ERR_CUDA;
+    d.ready = true;
+  }
+  *out = d;
+  if (dev_out) *dev_out = dev;
+  return PA_OK;
+}
+
+inline cudaStream_t stream_of(const pa_opts* o) {
+  return o ? reinterpret_cast<cudaStream_t>(o->stream) : nullptr;
+}
+
+inline uint64_t timeout_of(const pa_opts* o) {
+  const int ms = (o && o->timeout_ms > 0) ? o->timeout_ms : 1000;
+  return uint64_t(ms) * 1000000ull;
+}
+
+inline int esize(int32_t dt) { return dt == PA_F32 ? 4 : dt == PA_BF16 ? 2 : dt == PA_I32 ? 4 : dt == PA_I64 ? 8 : 0; }
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// The cache: [NB, Hkv, 16, D] contiguous, 16-byte aligned.
+pa_status check_cache(const pa_tensor* t) {
+  if (t == nullptr || t->ndim != 4 || (t->dtype != PA_F32 && t->dtype != PA_BF16)) return PA_ERR_INVALID_ARG;
+  const int64_t* s = t->shape;
+  if (s[0] <= 0 || s[1] <= 0 || s[2] <= 0 || s[3] <= 0) return PA_ERR_INVALID_ARG;
+  if (t->stride[3] != 1 || t->stride[2] != s[3] || t->stride[1] != s[2] * s[3] || t->stride[0] != s[1] * s[2] * s[3])
+    return PA_ERR_INVALID_ARG;
+  if (t->data == nullptr || !aligned16(t->data)) return PA_ERR_INVALID_ARG;
+  if (s[2] != 16) return PA_ERR_UNSUPPORTED;
+  if (s[3] != 64 && s[3] != 128) return PA_ERR_UNSUPPORTED;
+  if (s[0] > INT32_MAX || s[1] > 1024) return PA_ERR_UNSUPPORTED;
+  return PA_OK;
+}
+
+pa_status check_pair(const pa_tensor* k, const pa_tensor* v) {
+  pa_status st = check_cache(k);
+  if (st != PA_OK) return st;
+  st = check_cache(v);
+  if (st != PA_OK) return st;
+  if (k->dtype != v->dtype) return PA_ERR_INVALID_ARG;
+  for (int d = 0; d < 4; ++d)
+    if (k->shape[d] != v->shape[d]) return PA_ERR_INVALID_ARG;
+  return PA_OK;
+}
+
+// [n0, n1, D] rows: last dim contiguous, other strides multiples of 16 bytes.
+pa_status check_rows3(const pa_tensor* t, int32_t dtype, int64_t n0, int64_t n1, int64_t D) {
+  if (t == nullptr || t->ndim != 3 || t->dtype != dtype) return PA_ERR_INVALID_ARG;
+  if (t->shape[0] != n0 || t->shape[1] != n1 || t->shape[2] != D || t->stride[2] != 1) return PA_ERR_INVALID_ARG;
+  const int e = esize(dtype);
+  if (t->stride[0] < 0 || t->stride[1] < 0 || (t->stride[0] * e) % 16 || (t->stride[1] * e) % 16)
+    return PA_ERR_INVALID_ARG;
+  if (n0 > 0 && (t->data == nullptr || !aligned16(t->data))) return PA_ERR_INVALID_ARG;
+  return PA_OK;
+}
+
+pa_status launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+template <typename Kern, typename... Args>
+cudaError_t launch_pdl(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+// ---------------------------------------------------------------------------
+// decode launch plumbing
+// ---------------------------------------------------------------------------
+struct DecodePlan {
+  int mode;
+  int grid;
+  int warps;
+  int stages;
+  size_t smem;
+  int part_pages;
+  int P_max;
+  size_t ws_need;
+};
+
+template <typename T, int D, int G>
+size_t stage_fit(int B, int warps, int want, int optin, int* stages_out) {
+  using C = pa::DecodeCfg<T, D, G>;
+  for (int st = want; st >= 1; --st) {
+    const size_t bytes = pa::decode_prefix_bytes(B) + size_t(warps) * C::warp_bytes(st);
+    if (bytes <= size_t(optin)) {
+      *stages_out = st;
+      return bytes;
+    }
+  }
+  return 0;
+}
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+size_t fixed_ws_bytes(int64_t B, int64_t H, int64_t D, int64_t P) {
+  return align_up(size_t(B * H * P * D) * 4, 256) + align_up(size_t(B * H * P) * 4, 256);
+}
+
+size_t balanced_ws_bytes(int64_t workers, int64_t G, int64_t D) {
+  return align_up(size_t(workers * 2 * G * D) * 4, 256) + align_up(size_t(workers * 2 * G) * 4, 256) +
+         align_up(size_t(workers) * 16, 256);
+}
+
+template <typename T, int D, int G>
+pa_status run_decode(const pa::DecodeArgs& base, const DecodePlan& p, cudaStream_t st, int dev) {
+  static bool attr_set[kMaxDevices] = {};
+  static size_t attr_bytes[kMaxDevices] = {};
+  auto kern = pa::decode_kernel<T, D, G>;
+  if (!attr_set[dev] || attr_bytes[dev] < p.smem) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(p.smem)) != cudaSuccess)
+      return PA_ERR_CUDA;
+    attr_set[dev] = true;
+    attr_bytes[dev] = p.smem;
+  }
+  pa::DecodeArgs a = base;
+  a.stages = p.stages;
+  a.mode = p.mode;
+  a.part_pages = p.part_pages;
+  a.P_max = p.P_max;
+  if (launch_pdl(kern, dim3(p.grid), dim3(p.warps * 32), p.smem, st, true, a) != cudaSuccess) return launch_status();
+  const int64_t nworkers = int64_t(p.grid) * p.warps;
+  if (p.mode == pa::kFixed) {
+    const int64_t tasks = int64_t(a.B) * a.H;
+    const int blocks = int((tasks + 7) / 8);
+    if (launch_pdl(pa::merge_fixed_kernel<T, D>, dim3(blocks), dim3(256), 0, st, true, a,
+                   p.part_pages * pa::kBS) != cudaSuccess)
+      return launch_status();
+  } else if (p.mode == pa::kBalanced) {
+    const int64_t tasks = nworkers * G;
+    const int blocks = int((tasks + 7) / 8);
+    if (launch_pdl(pa::merge_balanced_kernel<T, D, G>, dim3(blocks), dim3(256), 0, st, true, a, nworkers) !=
+        cudaSuccess)
+      return launch_status();
+  }
+  return launch_status();
+}
+
+template <typename T, int D>
+pa_status dispatch_group(int G, const pa::DecodeArgs& a, const DecodePlan& p, cudaStream_t st, int dev) {
+  switch (G) {
+    case 1:
+      return run_decode<T, D, 1>(a, p, st, dev);
+    case 2:
+      return run_decode<T, D, 2>(a, p, st, dev);
+    case 4:
+      return run_decode<T, D, 4>(a, p, st, dev);
+    case 8:
+      return run_decode<T, D, 8>(a, p, st, dev);
+    default:
+      return PA_ERR_UNSUPPORTED;
+  }
+}
+
+template <typename T, int D>
+size_t fit_for_group(int G, int B, int warps, int want, int optin, int* stages) {
+  switch (G) {
+    case 1:
+      return stage_fit<T, D, 1>(B, warps, want, optin, stages);
+    case 2:
+      return stage_fit<T, D, 2>(B, warps, want, optin, stages);
+    case 4:
+      return stage_fit<T, D, 4>(B, warps, want, optin, stages);
+    case 8:
+      return stage_fit<T, D, 8>(B, warps, want, optin, stages);
+    default:
+      return 0;
+  }
+}
+
+size_t fit_stages(int32_t dtype, int D, int G, int B, int warps, int want, int optin, int* stages) {
+  if (dtype == PA_BF16 && D == 128) return fit_for_group<__nv_bfloat16, 128>(G, B, warps, want, optin, stages);
+  if (dtype == PA_BF16 && D == 64) return fit_for_group<__nv_bfloat16, 64>(G, B, warps, want, optin, stages);
+  if (dtype == PA_F32 && D == 64) return fit_for_group<float, 64>(G, B, warps, want, optin, stages);
+  if (dtype == PA_F32 && D == 128) return fit_for_group<float, 128>(G, B, warps, want, optin, stages);
+  return 0;
+}
+
+// Mode, grid, smem and workspace of one decode call.
+pa_status plan_decode(int32_t dtype, int64_t B, int64_t H, int64_t Hkv, int64_t D, int64_t max_nb, int32_t part_tokens,
+                      size_t ws_bytes, bool ws_given, DecodePlan* p) {
+  DeviceInfo di;
+  int dev = 0;
+  pa_status s = device_info(&di, &dev);
+  if (s != PA_OK) return s;
+  const int G = int(H / Hkv);
+  p->warps = g_tuning.warps;
+  p->grid = di.sms * g_tuning.ctas_per_sm;
+  p->smem = fit_stages(dtype, int(D), G, int(B), p->warps, g_tuning.stages, di.smem_optin, &p->stages);
+  if (p->smem == 0) return PA_ERR_UNSUPPORTED;
+  p->part_pages = 0;
+  p->P_max = 0;
+  p->ws_need = 0;
+  const int64_t nworkers = int64_t(p->grid) * p->warps;
+  if (part_tokens > 0) {
+    if (part_tokens % pa::kBS) return PA_ERR_INVALID_ARG;
+    p->mode = pa::kFixed;
+    p->part_pages = part_tokens / pa::kBS;
+    p->P_max = int((max_nb + p->part_pages - 1) / p->part_pages);
+    if (p->P_max < 1) p->P_max = 1;
+    p->ws_need = fixed_ws_bytes(B, H, D, p->P_max);
+  } else if (part_tokens == 0) {
+    const size_t need = balanced_ws_bytes(nworkers, G, D);
+    if (ws_given && ws_bytes >= need) {
+      p->mode = pa::kBalanced;
+      p->ws_need = need;
+    } else {
+      p->mode = pa::kNoSplit;
+    }
+  } else if (part_tokens == -1) {
+    p->mode = pa::kNoSplit;
+  } else {
+    return PA_ERR_INVALID_ARG;
+  }
+  return PA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t pa_version(void) { return 1; }
+
+const char* pa_status_string(pa_status s) {
+  switch (s) {
+    case PA_OK:
+      return "ok";
+    case PA_ERR_INVALID_ARG:
+      return "invalid argument";
+    case PA_ERR_UNSUPPORTED:
+      return "unsupported shape or dtype";
+    case PA_ERR_OUT_OF_BLOCKS:
+      return "out of free blocks";
+    case PA_ERR_CUDA:
+      return "CUDA runtime error";
+    case PA_ERR_DEVICE_TIMEOUT:
+      return "device wait timed out";
+    case PA_ERR_DEVICE_BOUNDS:
+      return "device index check failed";
+  }
+  return "unknown status";
+}
+
+pa_status pa_set_decode_tuning(int32_t warps_per_cta, int32_t stages, int32_t ctas_per_sm) {
+  if (warps_per_cta < 0 || warps_per_cta > 8 || stages < 0 || stages > 16 || ctas_per_sm < 0 || ctas_per_sm > 8)
+    return PA_ERR_INVALID_ARG;
+  g_tuning.warps = warps_per_cta ? warps_per_cta : 8;
+  g_tuning.stages = stages ? stages : 3;
+  g_tuning.ctas_per_sm = ctas_per_sm ? ctas_per_sm : 1;
+  return PA_OK;
+}
+
+pa_status pa_reshape_and_cache(const pa_tensor* key, const pa_tensor* value, pa_tensor* k_cache, pa_tensor* v_cache,
+                               const pa_tensor* slot_mapping, const pa_opts* opts) {
+  pa_status st = check_pair(k_cache, v_cache);
+  if (st != PA_OK) return st;
+  const int64_t NB = k_cache->shape[0], Hkv = k_cache->shape[1], D = k_cache->shape[3];
+  if (slot_mapping == nullptr || slot_mapping->ndim != 1 || slot_mapping->dtype != PA_I64) return PA_ERR_INVALID_ARG;
+  const int64_t T = slot_mapping->shape[0];
+  if (T < 0 || (T > 0 && (slot_mapping->stride[0] != 1 || slot_mapping->data == nullptr))) return PA_ERR_INVALID_ARG;
+  st = check_rows3(key, k_cache->dtype, T, Hkv, D);
+  if (st != PA_OK) return st;
+  st = check_rows3(value, k_cache->dtype, T, Hkv, D);
+  if (st != PA_OK) return st;
+  if (T == 0) return PA_OK;
+  const int e = esize(k_cache->dtype);
+  const int vpr = int(D * e / 16);
+  const int64_t vec = 16 / e;  // elements per 16-byte vector
+  const int64_t total = T * Hkv * vpr;
+  DeviceInfo di;
+  st = device_info(&di, nullptr);
+  if (st != PA_OK) return st;
+  const int64_t want = (total + 255) / 256;
+  const int blocks = int(want < int64_t(di.sms) * 16 ? want : int64_t(di.sms) * 16);
+  cudaStream_t s = stream_of(opts);
+  const uint4* kp = static_cast<const uint4*>(key->data);
+  const uint4* vp = static_cast<const uint4*>(value->data);
+  uint4* kc = static_cast<uint4*>(k_cache->data);
+  uint4* vc = static_cast<uint4*>(v_cache->data);
+  const int64_t* sl = static_cast<const int64_t*>(slot_mapping->data);
+  const int64_t ks0 = key->stride[0] / vec, ks1 = key->stride[1] / vec;
+  const int64_t vs0 = value->stride[0] / vec, vs1 = value->stride[1] / vec;
+  const int64_t nslots = NB * 16;
+  cudaError_t err;
+  switch (vpr) {
+    case 8:
+      err = launch_pdl(pa::reshape_and_cache_kernel<8>, dim3(blocks), dim3(256), 0, s, false, kp, vp, kc, vc, sl, T,
+                       int(Hkv), ks0, ks1, vs0, vs1, nslots);
+      break;
+    case 16:
+      err = launch_pdl(pa::reshape_and_cache_kernel<16>, dim3(blocks), dim3(256), 0, s, false, kp, vp, kc, vc, sl, T,
+                       int(Hkv), ks0, ks1, vs0, vs1, nslots);
+      break;
+    case 32:
+      err = launch_pdl(pa::reshape_and_cache_kernel<32>, dim3(blocks), dim3(256), 0, s, false, kp, vp, kc, vc, sl, T,
+                       int(Hkv), ks0, ks1, vs0, vs1, nslots);
+      break;
+    default:
+      return PA_ERR_UNSUPPORTED;
+  }
+  return err == cudaSuccess ? PA_OK : launch_status();
+}
+
+pa_status pa_copy_blocks(pa_tensor* k_cache, pa_tensor* v_cache, const pa_tensor* pairs, const pa_opts* opts) {
+  pa_status st = check_pair(k_cache, v_cache);
+  if (st != PA_OK) return st;
+  if (pairs == nullptr || pairs->ndim != 2 || pairs->dtype != PA_I64 || pairs->shape[1] != 2) return PA_ERR_INVALID_ARG;
+  const int64_t n = pairs->shape[0];
+  if (n < 0) return PA_ERR_INVALID_ARG;
+  if (n == 0) return PA_OK;
+  if (pairs->stride[1] != 1 || pairs->stride[0] != 2 || pairs->data == nullptr) return PA_ERR_INVALID_ARG;
+  const int64_t NB = k_cache->shape[0];
+  const int e = esize(k_cache->dtype);
+  const int64_t block_vecs = k_cache->shape[1] * 16 * k_cache->shape[3] * e / 16;
+  const int gx = int((block_vecs + 1023) / 1024);
+  const int gy = int(n < 65535 ? n : 65535);
+  const cudaError_t err = launch_pdl(pa::copy_blocks_kernel, dim3(gx, gy), dim3(256), 0, stream_of(opts), false,
+                                     static_cast<uint4*>(k_cache->data), static_cast<uint4*>(v_cache->data),
+                                     static_cast<const int64_t*>(pairs->data), n, block_vecs, NB);
+  return err == cudaSuccess ? PA_OK : launch_status();
+}
+
+pa_status pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads, int32_t head_size,
+                                    int32_t max_blocks_per_seq, int32_t partition_tokens, size_t* bytes_out) {
+  if (bytes_out == nullptr || num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_size <= 0 ||
+      max_blocks_per_seq < 0 || num_heads % num_kv_heads)
+    return PA_ERR_INVALID_ARG;
+  *bytes_out = 0;
+  if (partition_tokens == -1) return PA_OK;
+  if (partition_tokens > 0) {
+    if (partition_tokens % pa::kBS) return PA_ERR_INVALID_ARG;
+    const int64_t pp = partition_tokens / pa::kBS;
+    int64_t P = (max_blocks_per_seq + pp - 1) / pp;
+    if (P < 1) P = 1;
+    *bytes_out = fixed_ws_bytes(num_seqs, num_heads, head_size, P);
+    return PA_OK;
+  }
+  if (partition_tokens != 0) return PA_ERR_INVALID_ARG;
+  DeviceInfo di;
+  pa_status st = device_info(&di, nullptr);
+  if (st != PA_OK) return st;
+  const int64_t workers = int64_t(di.sms) * g_tuning.ctas_per_sm * g_tuning.warps;
+  *bytes_out = balanced_ws_bytes(workers, num_heads / num_kv_heads, head_size);
+  return PA_OK;
+}
+
+pa_status pa_decode(pa_tensor* out, const pa_tensor* query, const pa_tensor* k_cache, const pa_tensor* v_cache,
+                    const pa_tensor* block_tables, const pa_tensor* context_lens, float scale, int32_t num_kv_heads,
+                    const pa_opts* opts) {
+  pa_status st = check_pair(k_cache, v_cache);
+  if (st != PA_OK) return st;
+  const int64_t NB = k_cache->shape[0], Hkv = k_cache->shape[1], D = k_cache->shape[3];
+  const int32_t dt = k_cache->dtype;
+  if (num_kv_heads != Hkv) return PA_ERR_INVALID_ARG;
+  if (query == nullptr || query->ndim != 3) return PA_ERR_INVALID_ARG;
+  const int64_t B = query->shape[0], H = query->shape[1];
+  if (B < 0 || H <= 0 || H % Hkv) return PA_ERR_INVALID_ARG;
+  st = check_rows3(query, dt, B, H, D);
+  if (st != PA_OK) return st;
+  st = check_rows3(out, dt, B, H, D);
+  if (st != PA_OK) return st;
+  if (block_tables == nullptr || block_tables->ndim != 2 || block_tables->dtype != PA_I32 ||
+      block_tables->shape[0] != B || block_tables->shape[1] < 0)
+    return PA_ERR_INVALID_ARG;
+  const int64_t max_nb = block_tables->shape[1];
+  if (B > 0 && max_nb > 0 && (block_tables->stride[1] != 1 || block_tables->stride[0] < max_nb ||
+                              block_tables->data == nullptr))
+    return PA_ERR_INVALID_ARG;
+  if (context_lens == nullptr || context_lens->ndim != 1 || context_lens->dtype != PA_I32 ||
+      context_lens->shape[0] != B || (B > 0 && (context_lens->stride[0] != 1 || context_lens->data == nullptr)))
+    return PA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
+  const int64_t G = H / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return PA_ERR_UNSUPPORTED;
+  if (B >= (int64_t(1) << 20) || B > kMaxBatch) return PA_ERR_UNSUPPORTED;
+  if (B * Hkv * max_nb >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
+  if (max_nb * 16 > INT32_MAX) return PA_ERR_UNSUPPORTED;
+  if (B == 0) return PA_OK;
+
+  const int32_t part = opts ? opts->partition_tokens : 0;
+  if (part < -1 || (part > 0 && part % pa::kBS)) return PA_ERR_INVALID_ARG;
+  const bool ws_given = opts && opts->workspace != nullptr;
+  const size_t ws_bytes = ws_given ? opts->workspace_bytes : 0;
+  if (ws_given && (reinterpret_cast<uintptr_t>(opts->workspace) & 255u)) return PA_ERR_INVALID_ARG;
+  DecodePlan plan;
+  st = plan_decode(dt, B, H, Hkv, D, max_nb, part, ws_bytes, ws_given, &plan);
+  if (st != PA_OK) return st;
+  if (plan.mode != pa::kNoSplit && (!ws_given || ws_bytes < plan.ws_need)) return PA_ERR_INVALID_ARG;
+
+  pa::DecodeArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.out = out->data;
+  a.q = query->data;
+  a.kc = k_cache->data;
+  a.vc = v_cache->data;
+  a.bt = static_cast<const int32_t*>(block_tables->data);
+  a.ctx = static_cast<const int32_t*>(context_lens->data);
+  a.q_sb = query->stride[0];
+  a.q_sh = query->stride[1];
+  a.o_sb = out->stride[0];
+  a.o_sh = out->stride[1];
+  a.bt_stride = block_tables->stride[0];
+  a.B = int32_t(B);
+  a.H = int32_t(H);
+  a.Hkv = int32_t(Hkv);
+  a.max_nb = int32_t(max_nb);
+  a.num_blocks = int32_t(NB);
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.timeout_ns = timeout_of(opts);
+  if (plan.mode == pa::kFixed) {
+    char* w = static_cast<char*>(opts->workspace);
+    a.ws_o = reinterpret_cast<float*>(w);
+    a.ws_lse = reinterpret_cast<float*>(w + align_up(size_t(B * H * plan.P_max * D) * 4, 256));
+  } else if (plan.mode == pa::kBalanced) {
+    const int64_t workers = int64_t(plan.grid) * plan.warps;
+    char* w = static_cast<char*>(opts->workspace);
+    const size_t o_bytes = align_up(size_t(workers * 2 * G * D) * 4, 256);
+    const size_t l_bytes = align_up(size_t(workers * 2 * G) * 4, 256);
+    a.ws_o = reinterpret_cast<float*>(w);
+    a.ws_lse = reinterpret_cast<float*>(w + o_bytes);
+    a.ws_task = reinterpret_cast<int4*>(w + o_bytes + l_bytes);
+  }
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
+  cudaStream_t s = stream_of(opts);
+  if (dt == PA_BF16 && D == 128) return dispatch_group<__nv_bfloat16, 128>(int(G), a, plan, s, dev);
+  if (dt == PA_BF16 && D == 64) return dispatch_group<__nv_bfloat16, 64>(int(G), a, plan, s, dev);
+  if (dt == PA_F32 && D == 64) return dispatch_group<float, 64>(int(G), a, plan, s, dev);
+  if (dt == PA_F32 && D == 128) return dispatch_group<float, 128>(int(G), a, plan, s, dev);
+  return PA_ERR_UNSUPPORTED;
+}
+
+pa_status pa_get_device_status(const pa_opts* opts, uint32_t* bits_out) {
+  cudaStream_t s = stream_of(opts);
+  unsigned int bits = 0;
+  const unsigned int zero = 0;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return PA_ERR_CUDA;
+  if (cudaMemcpyFromSymbolAsync(&bits, pa::g_status, sizeof(bits), 0, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return PA_ERR_CUDA;
+  if (cudaMemcpyToSymbolAsync(pa::g_status, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return PA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return PA_ERR_CUDA;
+  if (bits_out) *bits_out = bits;
+  if (bits & PA_DEV_TIMEOUT) return PA_ERR_DEVICE_TIMEOUT;
+  if (bits) return PA_ERR_DEVICE_BOUNDS;
+  return PA_OK;
+}
+
+pa_status pa_debug_wait_selftest(const pa_opts* opts) {
+  const uint64_t t = timeout_of(opts);
+  pa::wait_selftest_kernel<<<1, 32, 0, stream_of(opts)>>>(t);
+  return launch_status();
+}
+
+}  // extern "C"

@@ -1,0 +1,87 @@
+// Byte-moving kernels of the paged KV cache (sm_100a): the per-token cache
+// write by slot and the whole-block copy of copy-on-write.
+//
+// Both are pure HBM traffic.  Every (token, kv head) row of K or V is
+// head_size * elem bytes (256 B for bf16/128 and fp32/64) and contiguous on
+// both sides in the layout [num_blocks, num_kv_heads, 16, head_size], so a
+// thread moves one 16-byte vector and 16 consecutive lanes move one row
+// with fully coalesced loads and stores.
+#pragma once
+
+#include "pa_common.cuh"
+
+namespace pa {
+
+// Cache write: for token t, head h, vector c of the row:
+//   k_cache[slot / 16, h, slot % 16, c] = key[t, h, c]   (same for V)
+// slot == -1 skips the token; any other slot outside [0, num_slots) sets
+// PA_DEV_BAD_SLOT and skips it.  Strides are in 16-byte vectors.
+template <int VPR>  // 16-byte vectors per row
+__global__ void __launch_bounds__(256) reshape_and_cache_kernel(const uint4* __restrict__ key,
+                                                                const uint4* __restrict__ value, uint4* kc,
+                                                                uint4* vc, const int64_t* __restrict__ slots,
+                                                                int64_t T, int Hkv, int64_t k_st, int64_t k_sh,
+                                                                int64_t v_st, int64_t v_sh, int64_t num_slots) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int64_t per_tok = int64_t(Hkv) * VPR;
+  const int64_t total = T * per_tok;
+  const int64_t step = int64_t(gridDim.x) * blockDim.x;
+  for (int64_t idx = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; idx < total; idx += step) {
+    const int64_t t = idx / per_tok;
+    const int r = int(idx - t * per_tok);
+    const int h = r / VPR, c = r % VPR;
+    const int64_t s = slots[t];
+    if (s == -1) continue;
+    if (s < -1 || s >= num_slots) {
+      if (h == 0 && c == 0) flag(PA_DEV_BAD_SLOT);
+      continue;
+    }
+    const int64_t dst = (((s >> 4) * Hkv + h) * 16 + (s & 15)) * VPR + c;
+    const uint4 kv = ld_nc_v4(key + t * k_st + h * k_sh + c);
+    const uint4 vv = ld_nc_v4(value + t * v_st + h * v_sh + c);
+    kc[dst] = kv;
+    vc[dst] = vv;
+  }
+}
+
+// Copy-on-write: for each pair (src, dst) copy the whole block, K and V.
+// block_vecs = num_kv_heads * 16 * head_size * elem / 16.  grid.y strides
+// over pairs, grid.x over the block's vectors.
+__global__ void __launch_bounds__(256) copy_blocks_kernel(uint4* kc, uint4* vc, const int64_t* __restrict__ pairs,
+                                                          int64_t n, int64_t block_vecs, int64_t num_blocks) {
+  pdl_wait();
+  pdl_launch_dependents();
+  for (int64_t p = blockIdx.y; p < n; p += gridDim.y) {
+    const int64_t src = pairs[2 * p], dst = pairs[2 * p + 1];
+    if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+      if (blockIdx.x == 0 && threadIdx.x == 0) flag(PA_DEV_BAD_BLOCK);
+      continue;
+    }
+    const uint4* ks = kc + src * block_vecs;
+    const uint4* vs = vc + src * block_vecs;
+    uint4* kd = kc + dst * block_vecs;
+    uint4* vd = vc + dst * block_vecs;
+    for (int64_t v = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; v < block_vecs;
+         v += int64_t(gridDim.x) * blockDim.x) {
+      const uint4 a = ks[v];
+      const uint4 b = vs[v];
+      kd[v] = a;
+      vd[v] = b;
+    }
+  }
+}
+
+// One warp waits on a barrier that nothing completes; the bounded wait must
+// give up and set PA_DEV_TIMEOUT.  No copy is in flight.
+__global__ void wait_selftest_kernel(uint64_t timeout_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
+  mbar_wait_bounded(smem_u32(&bar), 0, timeout_ns);
+}
+
+}  // namespace pa

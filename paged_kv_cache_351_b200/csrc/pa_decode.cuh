@@ -1,0 +1,683 @@
+// Paged decode attention for sm_100a.
+//
+// What it computes (gitcode repo walkthrough, section 2.1 "PagedAttention":
+// the query-key dot product, the softmax normalisation and the weighted sum
+// of V, over K/V that the block table gathers block by block):
+//   out[i, h] = sum_t softmax_t(scale * <q[i,h], K_i[t, g]>) V_i[t, g],
+//   g = h / G, K_i[t] = k_cache[block_tables[i][t / 16], g, t % 16, :].
+//
+// Design (a B200 re-design; the pages' thread-group/warp/block kernel and its
+// x-split K layout are prior art only):
+//  * The work is the list of "rows" (sequence i, kv head g) — each row is
+//    ceil(ctx_i / 16) pages of 16 tokens.  One warp is one worker; all
+//    workers of a persistent grid (one CTA per SM) take equal, contiguous
+//    ranges of the flattened page list, so every SM streams the same number
+//    of bytes whatever the length mix.  A row cut by a range boundary yields
+//    per-worker partial results (max, denominator, normalised output) that a
+//    small log-sum-exp merge kernel combines.  Fixed-size partitions (each
+//    partition its own partial, then the merge) and an unsplit mode are the
+//    same loop with boundaries snapped to partitions or rows.
+//  * Each page of a row — 16 tokens x head_size for one kv head, 4 KiB for
+//    bf16/128 — is one contiguous run in the cache layout
+//    [num_blocks, num_kv_heads, 16, head_size], so a worker moves it with a
+//    single 1-D bulk copy (TMA engine, no tensor map, no multicast) into its
+//    own shared-memory ring, completing on an mbarrier.  The worker's lane 0
+//    issues the copies; the ring keeps several pages per warp in flight.
+//  * The G = H / H_kv query heads that share a kv head are handled by the
+//    same worker, so every K/V page is read from HBM once per group.
+//  * Online softmax in fp32 with base-2 exponentials: q is pre-scaled by
+//    scale * log2(e); running max, denominator and output per head are
+//    rescaled when the max grows.
+//  * Lane layout inside a page: a token row is LPT 16-byte vectors; lane
+//    (tg, c) = (lane / LPT, lane % LPT) handles vector c of tokens
+//    tg + TPI*k, k < NT.  Partial dot products are summed across the LPT
+//    lanes of a token by a halving butterfly that leaves each lane one token
+//    (and half the heads), then the page max is a warp reduction and the
+//    probabilities go through a small shared buffer to the lanes that
+//    multiply them into V.
+#pragma once
+
+#include "pa_common.cuh"
+
+namespace pa {
+
+constexpr int kBS = 16;  // tokens per block (block_size)
+
+enum DecodeMode : int32_t { kBalanced = 0, kFixed = 1, kNoSplit = 2 };
+
+struct DecodeArgs {
+  void* out;
+  const void* q;
+  const void* kc;
+  const void* vc;
+  const int32_t* bt;
+  const int32_t* ctx;
+  int64_t q_sb, q_sh;  // query strides (elements)
+  int64_t o_sb, o_sh;  // out strides (elements)
+  int64_t bt_stride;   // block-table row stride (elements)
+  int32_t B, H, Hkv, max_nb, num_blocks;
+  float scale_log2;  // scale * log2(e)
+  int32_t mode;
+  int32_t part_pages;  // fixed mode: pages per partition
+  int32_t P_max;       // fixed mode: partition capacity per (seq, head)
+  int32_t stages;      // ring depth per warp
+  float* ws_o;         // partial outputs
+  float* ws_lse;       // partial log-sum-exp (natural log)
+  int4* ws_task;       // balanced mode: one merge task per worker
+  uint64_t timeout_ns;
+};
+
+template <typename T, int D, int G>
+struct DecodeCfg {
+  static constexpr int ROWB = D * int(sizeof(T));  // bytes of one token's K (or V) for one head
+  static constexpr int LPT = ROWB / 16;            // lanes per token row
+  static constexpr int TPI = 32 / LPT;             // token rows per warp-wide 16-byte load
+  static constexpr int NT = kBS / TPI;             // tokens per lane per page
+  static constexpr int EPV = 16 / int(sizeof(T));  // elements per 16-byte vector
+  static constexpr int PAGE = kBS * ROWB;          // bytes of one page
+  static constexpr int QBYTES = G * ROWB;          // the group's query rows
+  static constexpr int STAGE = 2 * PAGE + QBYTES;  // K page, V page, query rows
+  static constexpr int GH = G >= 2 ? G / 2 : 1;    // heads a lane holds after the butterfly
+  static constexpr int PBUF = G * kBS * 4;         // probabilities of one page
+  static constexpr int LOG2_NT = NT == 16 ? 4 : NT == 8 ? 3 : NT == 4 ? 2 : NT == 2 ? 1 : 0;
+  static_assert(LPT >= 8 && LPT <= 32 && (LPT & (LPT - 1)) == 0, "row of 128, 256 or 512 bytes");
+  static_assert(2 * NT == LPT, "lane layout");
+  static_assert(G == 1 || G == 2 || G == 4 || G == 8, "group size");
+  // per-warp region: [ring: stages * STAGE][probabilities: PBUF][mbarriers: stages * 8], 128-byte multiple
+  static constexpr size_t warp_bytes(int stages) {
+    return (size_t(stages) * STAGE + PBUF + size_t(stages) * 8 + 127) / 128 * 128;
+  }
+};
+
+// smem carve-up: [scan scratch: 32 int32][S: (B+1) int32], padded to 128 bytes,
+// then one region per warp (DecodeCfg::warp_bytes).
+__host__ __device__ inline size_t decode_prefix_bytes(int B) { return (size_t(B + 1 + 32) * 4 + 127) / 128 * 128; }
+
+// Block-wide exclusive scan of one int per thread; returns the prefix and
+// writes the total to *total.  scratch: >= 32 ints of shared memory.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* scratch, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) scratch[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int t = lane < nw ? scratch[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += y;
+    }
+    scratch[lane] = t;  // inclusive prefix of warp totals
+  }
+  __syncthreads();
+  const int warp_prefix = warp ? scratch[warp - 1] : 0;
+  *total = scratch[nw - 1];
+  __syncthreads();
+  return warp_prefix + x - v;
+}
+
+__device__ __forceinline__ int clamp_ctx(int c, int cap) { return c < 0 ? 0 : (c > cap ? cap : c); }
+
+// Position of flat page index x in the row list: seq i, kv head g, page p.
+struct RowPos {
+  int i, g, p, np;
+};
+
+__device__ __forceinline__ RowPos locate(const int* S, int B, int Hkv, int64_t x) {
+  // largest i in [0, B) with S[i] <= x (S nondecreasing, S[B] > x)
+  int lo = 0, hi = B - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (S[mid] <= x)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  RowPos r;
+  r.i = lo;
+  r.np = (S[lo + 1] - S[lo]) / Hkv;
+  const int off = int(x - S[lo]);
+  r.g = off / r.np;
+  r.p = off - r.g * r.np;
+  return r;
+}
+
+// Snap a range boundary down to the start of its partition (fixed mode) or
+// row (unsplit mode); balanced mode keeps page granularity.
+__device__ __forceinline__ int64_t snap_boundary(const int* S, int B, int Hkv, int64_t b, int64_t W, int mode,
+                                                 int part_pages) {
+  if (b >= W || mode == kBalanced) return b < W ? b : W;
+  const RowPos r = locate(S, B, Hkv, b);
+  const int p0 = mode == kNoSplit ? 0 : (r.p / part_pages) * part_pages;
+  return int64_t(S[r.i]) + int64_t(r.g) * r.np + p0;
+}
+
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(256, 1) decode_kernel(const DecodeArgs a) {
+  using C = DecodeCfg<T, D, G>;
+  constexpr int LPT = C::LPT, TPI = C::TPI, NT = C::NT, EPV = C::EPV, GH = C::GH;
+  extern __shared__ __align__(128) unsigned char smem[];
+
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int nwarps = blockDim.x >> 5;
+  const int tg = lane / LPT, c = lane % LPT;
+  const int B = a.B, Hkv = a.Hkv, H = a.H;
+  const int ctx_cap = a.max_nb * kBS;
+
+  int* scan_scratch = reinterpret_cast<int*>(smem);
+  int* S = scan_scratch + 32;
+  unsigned char* wbase = smem + decode_prefix_bytes(B) + size_t(warp) * C::warp_bytes(a.stages);
+  unsigned char* ring = wbase;
+  float* pbuf = reinterpret_cast<float*>(wbase + size_t(a.stages) * C::STAGE);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(wbase + size_t(a.stages) * C::STAGE + C::PBUF);
+
+  if (lane == 0) {
+    for (int s = 0; s < a.stages; ++s) mbar_init(smem_u32(&bars[s]), 1);
+    fence_barrier_init();
+  }
+
+  // Inputs may come from the kernel just before this one in the stream.
+  pdl_wait();
+  pdl_launch_dependents();
+
+  // ---- prologue: page prefix over sequences (every CTA computes it) ------
+  {
+    const int nt = blockDim.x;
+    const int per = (B + nt - 1) / nt;
+    const int i0 = threadIdx.x * per;
+    const int i1 = min(B, i0 + per);
+    int local = 0;
+    for (int i = i0; i < i1; ++i) {
+      const int raw = a.ctx[i];
+      if ((raw < 0 || raw > ctx_cap) && blockIdx.x == 0) flag(PA_DEV_BAD_CONTEXT);
+      local += (clamp_ctx(raw, ctx_cap) + kBS - 1) / kBS * Hkv;
+    }
+    int total;
+    int run = block_exclusive_scan(local, scan_scratch, &total);
+    for (int i = i0; i < i1; ++i) {
+      S[i] = run;
+      run += (clamp_ctx(a.ctx[i], ctx_cap) + kBS - 1) / kBS * Hkv;
+    }
+    if (threadIdx.x == 0) S[B] = total;
+    __syncthreads();
+  }
+  __syncwarp();
+
+  const int64_t W = S[B];
+  const int64_t nworkers = int64_t(gridDim.x) * nwarps;
+  const int64_t wid = int64_t(blockIdx.x) * nwarps + warp;
+  int64_t lo = (wid * W + nworkers - 1) / nworkers;
+  int64_t hi = ((wid + 1) * W + nworkers - 1) / nworkers;
+  lo = snap_boundary(S, B, Hkv, lo, W, a.mode, a.part_pages);
+  hi = snap_boundary(S, B, Hkv, hi, W, a.mode, a.part_pages);
+  if (a.mode == kBalanced) {
+    if (lane == 0) a.ws_task[wid] = make_int4(-1, -1, -1, -1);
+    if (lo >= hi) {
+      // an empty worker contributes nothing to a merge that spans it
+      float* po = a.ws_o + wid * 2 * G * D;
+      for (int k = lane; k < G * D; k += 32) po[k] = 0.f;
+      if (lane < G) a.ws_lse[wid * 2 * G + lane] = -INFINITY;
+    }
+  }
+
+  const uint64_t pol = policy_evict_first();
+  const T* qg = reinterpret_cast<const T*>(a.q);
+  const unsigned char* kcb = reinterpret_cast<const unsigned char*>(a.kc);
+  const unsigned char* vcb = reinterpret_cast<const unsigned char*>(a.vc);
+
+  if (lo < hi) {
+    // ---- producer cursor (warp-uniform) ----
+    RowPos pc = locate(S, B, Hkv, lo);
+    int64_t px = lo;
+    int win_seq = -1, win_base = 0, win_blk = 0;  // lane-held window of 32 block ids
+    int p_seg_first = 1;                          // next issued page opens a segment
+
+    auto issue = [&](int s) {
+      // block id of page pc.p of sequence pc.i (warp-collective)
+      if (pc.i != win_seq || pc.p < win_base || pc.p >= win_base + 32) {
+        win_seq = pc.i;
+        win_base = pc.p & ~31;
+        const int pp = win_base + lane;
+        win_blk = pp < pc.np ? a.bt[int64_t(pc.i) * a.bt_stride + pp] : 0;
+      }
+      int blk = __shfl_sync(0xffffffffu, win_blk, pc.p - win_base);
+      if (unsigned(blk) >= unsigned(a.num_blocks)) {
+        if (lane == 0) flag(PA_DEV_BAD_BLOCK);
+        blk = 0;
+      }
+      if (lane == 0) {
+        const uint32_t bar = smem_u32(&bars[s]);
+        unsigned char* st = ring + size_t(s) * C::STAGE;
+        const int64_t page_off = (int64_t(blk) * Hkv + pc.g) * C::PAGE;
+        // order this warp's earlier shared-memory reads of the stage before the async-proxy refill
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_arrive_expect_tx(bar, 2 * C::PAGE + (p_seg_first ? C::QBYTES : 0));
+        bulk_g2s(smem_u32(st), kcb + page_off, C::PAGE, bar, pol);
+        bulk_g2s(smem_u32(st + C::PAGE), vcb + page_off, C::PAGE, bar, pol);
+        if (p_seg_first) {
+#pragma unroll
+          for (int j = 0; j < G; ++j)
+            bulk_g2s(smem_u32(st + 2 * C::PAGE + j * C::ROWB),
+                     qg + int64_t(pc.i) * a.q_sb + int64_t(pc.g * G + j) * a.q_sh, C::ROWB, bar, pol);
+        }
+      }
+      // advance the producer cursor
+      ++px;
+      ++pc.p;
+      p_seg_first = 0;
+      if (pc.p == pc.np) {
+        pc.p = 0;
+        p_seg_first = 1;
+        if (++pc.g == Hkv) {
+          pc.g = 0;
+          do {
+            ++pc.i;
+          } while (pc.i < B && S[pc.i + 1] == S[pc.i]);
+          if (pc.i < B) pc.np = (S[pc.i + 1] - S[pc.i]) / Hkv;
+        }
+      } else if (a.mode == kFixed && pc.p % a.part_pages == 0) {
+        p_seg_first = 1;
+      }
+    };
+
+    const int npre = int(hi - lo < int64_t(a.stages) ? hi - lo : int64_t(a.stages));
+    for (int s = 0; s < npre; ++s) issue(s);
+
+    // ---- consumer state ----
+    RowPos cc = locate(S, B, Hkv, lo);
+    int64_t cx = lo;
+    int seg_p0 = cc.p;
+    bool seg_first = true;
+    float q[G][EPV];
+    float o[G][EPV];
+    float m[G], lpart[GH];
+    int ctx_i = 0;
+    uint32_t phase = 0;  // bit s = parity of the next wait on stage s
+    int s = 0;
+
+    while (cx < hi) {
+      unsigned char* st = ring + size_t(s) * C::STAGE;
+      const uint32_t bar = smem_u32(&bars[s]);
+      if (!mbar_wait_bounded(bar, (phase >> s) & 1u, a.timeout_ns)) {
+        // give up: wait (bounded) for every other copy still in flight, then stop
+        // (at most `stages` pages are in flight, each in its own stage)
+        for (int64_t y = cx + 1; y < px; ++y) {
+          const int s2 = int((s + (y - cx)) % a.stages);
+          mbar_wait_bounded(smem_u32(&bars[s2]), (phase >> s2) & 1u, a.timeout_ns);
+        }
+        return;
+      }
+      phase ^= 1u << s;
+
+      if (seg_first) {
+        const uint4* qs = reinterpret_cast<const uint4*>(st + 2 * C::PAGE);
+#pragma unroll
+        for (int j = 0; j < G; ++j) {
+          float f[EPV];
+          Elem<T>::unpack(qs[j * LPT + c], f);
+#pragma unroll
+          for (int e = 0; e < EPV; ++e) {
+            q[j][e] = f[e] * a.scale_log2;
+            o[j][e] = 0.f;
+          }
+          m[j] = -INFINITY;
+        }
+#pragma unroll
+        for (int jj = 0; jj < GH; ++jj) lpart[jj] = 0.f;
+        ctx_i = clamp_ctx(a.ctx[cc.i], ctx_cap);  // consumed at the row's last page
+        seg_p0 = cc.p;
+      }
+      const bool last_of_row = (cc.p == cc.np - 1);
+      const int valid = last_of_row ? ctx_i - cc.p * kBS : kBS;
+
+      const uint4* Ks = reinterpret_cast<const uint4*>(st);
+      const uint4* Vs = reinterpret_cast<const uint4*>(st + C::PAGE);
+
+      // ---- scores: partial dot products, then the halving butterfly ----
+      float acc[G][NT];
+#pragma unroll
+      for (int k = 0; k < NT; ++k) {
+        float kf[EPV];
+        Elem<T>::unpack(Ks[(tg + TPI * k) * LPT + c], kf);
+#pragma unroll
+        for (int j = 0; j < G; ++j) {
+          float sum = 0.f;
+#pragma unroll
+          for (int e = 0; e < EPV; ++e) sum = fmaf(q[j][e], kf[e], sum);
+          acc[j][k] = sum;
+        }
+      }
+#pragma unroll
+      for (int step = 0; step < C::LOG2_NT; ++step) {
+        const int half = (NT >> step) / 2;
+        const int mask = LPT >> (step + 1);
+        const bool upper = (c & mask) != 0;
+#pragma unroll
+        for (int j = 0; j < G; ++j) {
+#pragma unroll
+          for (int k = 0; k < half; ++k) {
+            const float send = upper ? acc[j][k] : acc[j][k + half];
+            const float keep = upper ? acc[j][k + half] : acc[j][k];
+            acc[j][k] = keep + __shfl_xor_sync(0xffffffffu, send, mask);
+          }
+        }
+      }
+      const bool hi_half = (c & 1) != 0;
+      float sc[GH];
+      if constexpr (G >= 2) {
+#pragma unroll
+        for (int jj = 0; jj < GH; ++jj) {
+          const float send = hi_half ? acc[jj][0] : acc[jj + GH][0];
+          const float keep = hi_half ? acc[jj + GH][0] : acc[jj][0];
+          sc[jj] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+        }
+      } else {
+        sc[0] = acc[0][0] + __shfl_xor_sync(0xffffffffu, acc[0][0], 1);
+      }
+      const int t_own = tg + TPI * (c >> 1);
+      if (t_own >= valid) {
+#pragma unroll
+        for (int jj = 0; jj < GH; ++jj) sc[jj] = -INFINITY;
+      }
+
+      // ---- page max, new running max, rescale factors ----
+      float pm[GH];
+#pragma unroll
+      for (int jj = 0; jj < GH; ++jj) {
+        float x = sc[jj];
+#pragma unroll
+        for (int msk = 2; msk < 32; msk <<= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, msk));
+        pm[jj] = x;
+      }
+      float pmall[G];
+      if constexpr (G >= 2) {
+#pragma unroll
+        for (int jj = 0; jj < GH; ++jj) {
+          const float other = __shfl_xor_sync(0xffffffffu, pm[jj], 1);
+          pmall[jj] = hi_half ? other : pm[jj];
+          pmall[jj + GH] = hi_half ? pm[jj] : other;
+        }
+      } else {
+        pmall[0] = pm[0];
+      }
+      float alpha[G];
+      bool grew = false;
+#pragma unroll
+      for (int j = 0; j < G; ++j) {
+        const float mn = fmaxf(m[j], pmall[j]);
+        alpha[j] = ex2(m[j] - mn);
+        grew |= (mn != m[j]);
+        m[j] = mn;
+      }
+
+      // ---- probabilities of this lane's (token, heads); denominators ----
+#pragma unroll
+      for (int jj = 0; jj < GH; ++jj) {
+        const float mj = (G >= 2 && hi_half) ? m[(jj + GH) % G] : m[jj];
+        const float aj = (G >= 2 && hi_half) ? alpha[(jj + GH) % G] : alpha[jj];
+        const float p = ex2(sc[jj] - mj);
+        const bool own = (G >= 2) || !hi_half;
+        lpart[jj] = lpart[jj] * aj + (own ? p : 0.f);
+        if (own) {
+          const int j = (G >= 2 && hi_half) ? jj + GH : jj;
+          pbuf[(j * TPI + tg) * NT + (c >> 1)] = p;
+        }
+      }
+      __syncwarp();
+      float pk[G][NT];
+#pragma unroll
+      for (int j = 0; j < G; ++j) {
+        const float4* src = reinterpret_cast<const float4*>(pbuf + (j * TPI + tg) * NT);
+#pragma unroll
+        for (int k4 = 0; k4 < NT / 4; ++k4) {
+          const float4 v4 = src[k4];
+          pk[j][4 * k4 + 0] = v4.x;
+          pk[j][4 * k4 + 1] = v4.y;
+          pk[j][4 * k4 + 2] = v4.z;
+          pk[j][4 * k4 + 3] = v4.w;
+        }
+      }
+      __syncwarp();
+      if (grew) {
+#pragma unroll
+        for (int j = 0; j < G; ++j)
+#pragma unroll
+          for (int e = 0; e < EPV; ++e) o[j][e] *= alpha[j];
+      }
+
+      // ---- weighted sum of V ----
+#pragma unroll
+      for (int k = 0; k < NT; ++k) {
+        float vf[EPV];
+        Elem<T>::unpack(Vs[(tg + TPI * k) * LPT + c], vf);
+        if (tg + TPI * k >= valid) {
+#pragma unroll
+          for (int e = 0; e < EPV; ++e) vf[e] = 0.f;  // unused slots may hold any bits
+        }
+#pragma unroll
+        for (int j = 0; j < G; ++j)
+#pragma unroll
+          for (int e = 0; e < EPV; ++e) o[j][e] = fmaf(pk[j][k], vf[e], o[j][e]);
+      }
+      __syncwarp();  // every lane is done with stage s
+
+      // ---- refill stage s with the next page of this worker's range ----
+      if (px < hi) issue(s);
+
+      // ---- segment end: combine lanes and write ----
+      const bool seg_last = (cx == hi - 1) || last_of_row || (a.mode == kFixed && (cc.p + 1) % a.part_pages == 0);
+      if (seg_last) {
+#pragma unroll
+        for (int msk = LPT; msk < 32; msk <<= 1)
+#pragma unroll
+          for (int j = 0; j < G; ++j)
+#pragma unroll
+            for (int e = 0; e < EPV; ++e) o[j][e] += __shfl_xor_sync(0xffffffffu, o[j][e], msk);
+        float lall[G];
+#pragma unroll
+        for (int jj = 0; jj < GH; ++jj) {
+          float x = lpart[jj];
+#pragma unroll
+          for (int msk = 2; msk < 32; msk <<= 1) x += __shfl_xor_sync(0xffffffffu, x, msk);
+          if constexpr (G >= 2) {
+            const float other = __shfl_xor_sync(0xffffffffu, x, 1);
+            lall[jj] = hi_half ? other : x;
+            lall[jj + GH] = hi_half ? x : other;
+          } else {
+            lall[0] = x + __shfl_xor_sync(0xffffffffu, x, 1);
+          }
+        }
+        const bool whole_row = (seg_p0 == 0) && last_of_row;
+        if (whole_row) {
+          if (tg == 0) {
+            T* ob = reinterpret_cast<T*>(a.out) + int64_t(cc.i) * a.o_sb;
+#pragma unroll
+            for (int j = 0; j < G; ++j) {
+              const float inv = 1.f / lall[j];
+              float f[EPV];
+#pragma unroll
+              for (int e = 0; e < EPV; ++e) f[e] = o[j][e] * inv;
+              *reinterpret_cast<uint4*>(ob + int64_t(cc.g * G + j) * a.o_sh + c * EPV) = Elem<T>::pack(f);
+            }
+          }
+        } else {
+          int64_t base;  // index of the (head 0) partial slot
+          bool task = false;
+          if (a.mode == kFixed) {
+            base = (int64_t(cc.i) * H + int64_t(cc.g) * G) * a.P_max + cc.p / a.part_pages;
+          } else {
+            const int slot = seg_p0 == 0 ? 1 : 0;
+            base = (wid * 2 + slot) * G;
+            task = (slot == 1);
+          }
+          const int64_t hstride = a.mode == kFixed ? a.P_max : 1;
+          if (tg == 0) {
+#pragma unroll
+            for (int j = 0; j < G; ++j) {
+              const float inv = 1.f / lall[j];
+              float4* dst = reinterpret_cast<float4*>(a.ws_o + (base + j * hstride) * D + c * EPV);
+#pragma unroll
+              for (int e4 = 0; e4 < EPV / 4; ++e4)
+                dst[e4] = make_float4(o[j][4 * e4] * inv, o[j][4 * e4 + 1] * inv, o[j][4 * e4 + 2] * inv,
+                                      o[j][4 * e4 + 3] * inv);
+            }
+          }
+          if (lane < G) {
+            float mj = m[0], lj = lall[0];
+#pragma unroll
+            for (int j = 1; j < G; ++j)
+              if (lane == j) {
+                mj = m[j];
+                lj = lall[j];
+              }
+            a.ws_lse[base + lane * hstride] = (mj + log2f(lj)) * 0.69314718055994530942f;
+          }
+          if (task && lane == 0) {
+            const int64_t row_last = int64_t(S[cc.i]) + int64_t(cc.g) * cc.np + cc.np - 1;
+            const int wb = int(row_last * nworkers / W);
+            a.ws_task[wid] = make_int4(cc.i, cc.g, int(wid), wb);
+          }
+        }
+      }
+
+      // ---- advance the consumer cursor ----
+      ++cx;
+      seg_first = seg_last;
+      if (++cc.p == cc.np) {
+        cc.p = 0;
+        if (++cc.g == Hkv) {
+          cc.g = 0;
+          do {
+            ++cc.i;
+          } while (cc.i < B && S[cc.i + 1] == S[cc.i]);
+          if (cc.i < B) cc.np = (S[cc.i + 1] - S[cc.i]) / Hkv;
+        }
+      }
+      if (++s == a.stages) s = 0;
+    }
+  }
+
+  // ---- sequences with no context: zero output rows ----
+  for (int64_t i = wid; i < B; i += nworkers) {
+    if (S[i + 1] != S[i]) continue;
+    T* ob = reinterpret_cast<T*>(a.out) + i * a.o_sb;
+    for (int idx = lane; idx < H * LPT; idx += 32) {
+      const int h = idx / LPT, cc2 = idx % LPT;
+      *reinterpret_cast<uint4*>(ob + int64_t(h) * a.o_sh + cc2 * EPV) = make_uint4(0, 0, 0, 0);
+    }
+  }
+}
+
+// ---- log-sum-exp merge of partial results ----------------------------------
+// out = sum_p exp(lse_p - LSE) o_p, LSE = log sum_p exp(lse_p), with o_p the
+// normalised partial outputs.  One warp merges one (sequence, query head).
+// Fixed partitions: one warp per (sequence, query head) with > 1 partition.
+// Each lane walks the partitions with a running max (one pass).
+template <typename T, int D>
+__global__ void __launch_bounds__(256) merge_fixed_kernel(const DecodeArgs a, int part_tokens) {
+  pdl_wait();
+  constexpr int PER = D / 32;
+  const int lane = threadIdx.x & 31;
+  const int64_t task = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (task >= int64_t(a.B) * a.H) return;
+  const int i = int(task / a.H), h = int(task % a.H);
+  const int ctx = clamp_ctx(a.ctx[i], a.max_nb * kBS);
+  const int np = (ctx + part_tokens - 1) / part_tokens;
+  if (np <= 1) return;
+  const int64_t row = int64_t(i) * a.H + h;
+  const float* lse = a.ws_lse + row * a.P_max;
+  const float* ob = a.ws_o + row * a.P_max * D;
+  float mx = -INFINITY, wsum = 0.f;
+  float acc[PER];
+#pragma unroll
+  for (int e = 0; e < PER; ++e) acc[e] = 0.f;
+  for (int p = 0; p < np; ++p) {
+    const float l = lse[p];
+    const float mn = fmaxf(mx, l);
+    const float sc = ex2((mx - mn) * 1.4426950408889634f);
+    const float w = ex2((l - mn) * 1.4426950408889634f);
+    mx = mn;
+    wsum = wsum * sc + w;
+    const float* src = ob + int64_t(p) * D + lane * PER;
+    float v[PER];
+    if constexpr (PER == 4) {
+      const float4 v4 = *reinterpret_cast<const float4*>(src);
+      v[0] = v4.x, v[1] = v4.y, v[2] = v4.z, v[3] = v4.w;
+    } else {
+      const float2 v2 = *reinterpret_cast<const float2*>(src);
+      v[0] = v2.x, v[1] = v2.y;
+    }
+#pragma unroll
+    for (int e = 0; e < PER; ++e) acc[e] = fmaf(w, v[e], acc[e] * sc);
+  }
+  const float inv = 1.f / wsum;
+  T* dst = reinterpret_cast<T*>(a.out) + int64_t(i) * a.o_sb + int64_t(h) * a.o_sh + lane * PER;
+  float f[PER];
+#pragma unroll
+  for (int e = 0; e < PER; ++e) f[e] = acc[e] * inv;
+  if constexpr (sizeof(T) == 4) {
+#pragma unroll
+    for (int e = 0; e < PER; ++e) reinterpret_cast<float*>(dst)[e] = f[e];
+  } else {
+#pragma unroll
+    for (int e = 0; e < PER; e += 2) {
+      __nv_bfloat162 hh = __floats2bfloat162_rn(f[e], f[e + 1]);
+      *reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(dst) + e) = hh;
+    }
+  }
+}
+
+// Balanced mode: one warp per (worker, query head of the group); the worker's
+// task names the row it started and the last worker the row reaches.
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(256) merge_balanced_kernel(const DecodeArgs a, int64_t nworkers) {
+  pdl_wait();
+  constexpr int PER = D / 32;
+  const int lane = threadIdx.x & 31;
+  const int64_t t = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= nworkers * G) return;
+  const int64_t w = t / G;
+  const int j = int(t % G);
+  const int4 task = a.ws_task[w];
+  if (task.x < 0) return;
+  const int i = task.x, g = task.y, wa = task.z, wb = task.w;
+  float mx = -INFINITY, wsum = 0.f;
+  float acc[PER];
+#pragma unroll
+  for (int e = 0; e < PER; ++e) acc[e] = 0.f;
+  for (int wk = wa; wk <= wb; ++wk) {
+    const int64_t slot = (int64_t(wk) * 2 + (wk == wa ? 1 : 0)) * G + j;
+    const float l = a.ws_lse[slot];
+    const float mn = fmaxf(mx, l);
+    const float sc = ex2((mx - mn) * 1.4426950408889634f);
+    const float wgt = ex2((l - mn) * 1.4426950408889634f);
+    mx = mn;
+    wsum = wsum * sc + wgt;
+    const float* src = a.ws_o + slot * D + lane * PER;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) acc[e] = fmaf(wgt, src[e], acc[e] * sc);
+  }
+  const float inv = 1.f / wsum;
+  T* dst = reinterpret_cast<T*>(a.out) + int64_t(i) * a.o_sb + int64_t(g * G + j) * a.o_sh + lane * PER;
+  float f[PER];
+#pragma unroll
+  for (int e = 0; e < PER; ++e) f[e] = acc[e] * inv;
+  if constexpr (sizeof(T) == 4) {
+#pragma unroll
+    for (int e = 0; e < PER; ++e) reinterpret_cast<float*>(dst)[e] = f[e];
+  } else {
+#pragma unroll
+    for (int e = 0; e < PER; e += 2) {
+      __nv_bfloat162 hh = __floats2bfloat162_rn(f[e], f[e + 1]);
+      *reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(dst) + e) = hh;
+    }
+  }
+}
+
+}  // namespace pa

@@ -1,0 +1,79 @@
+"""A paged KV cache on one GPU: the host allocator plus the device pools,
+driven through the library's entry points.
+
+This is bookkeeping around libpa: the allocator decides slots and
+copy-on-write pairs on the host; the pairs are copied with pa_copy_blocks
+and the tokens written with pa_reshape_and_cache (in that order, on one
+stream); decode reads through int32 block tables.  Device memory comes from
+torch; every byte is moved by the library's kernels.
+"""
+
+from __future__ import annotations
+
+from typing import Optional, Sequence, Tuple
+
+import numpy as np
+import torch
+
+from . import Allocator, pa_copy_blocks, pa_decode, pa_decode_workspace_bytes, pa_reshape_and_cache
+
+_DT = {"f32": torch.float32, "bf16": torch.bfloat16}
+
+
+class PagedKVCacheGPU:
+    """K/V pools [num_blocks, num_kv_heads, block_size, head_size] on one device."""
+
+    def __init__(self, num_blocks: int, num_kv_heads: int, head_size: int, dtype: str = "bf16",
+                 block_size: int = 16, free_order: Optional[Sequence[int]] = None, device="cuda"):
+        self.num_blocks, self.num_kv_heads, self.head_size = num_blocks, num_kv_heads, head_size
+        self.block_size, self.dtype, self.device = block_size, dtype, torch.device(device)
+        shape = (num_blocks, num_kv_heads, block_size, head_size)
+        self.k_cache = torch.empty(shape, dtype=_DT[dtype], device=self.device)
+        self.v_cache = torch.empty(shape, dtype=_DT[dtype], device=self.device)
+        self.alloc = Allocator(num_blocks, block_size, free_order)
+        self._ws = None
+
+    # -- host bookkeeping ------------------------------------------------------
+    def add(self, seq: int) -> None:
+        self.alloc.add(seq)
+
+    def fork(self, parent: int, child: int) -> None:
+        self.alloc.fork(parent, child)
+
+    def free(self, seq: int) -> None:
+        self.alloc.free(seq)
+
+    def append(self, seqs: Sequence[int], counts: Sequence[int]) -> Tuple[np.ndarray, np.ndarray]:
+        """Reserve slots for counts[k] new tokens of seqs[k]; returns (slots
+        int64 [sum(counts)], copy-on-write pairs int64 [n, 2])."""
+        return self.alloc.append_batch(seqs, counts)
+
+    def block_tables(self, seqs: Sequence[int], max_blocks: int) -> Tuple[np.ndarray, np.ndarray]:
+        return self.alloc.block_tables(seqs, max_blocks)
+
+    # -- device steps -------------------------------------------------------------
+    def write(self, slots: torch.Tensor, key: torch.Tensor, value: torch.Tensor,
+              pairs: Optional[torch.Tensor] = None, stream=None) -> None:
+        """Copy-on-write copies first (they must precede writes into the
+        copied blocks), then the tokens' K/V at their slots."""
+        if pairs is not None and pairs.shape[0]:
+            pa_copy_blocks(self.k_cache, self.v_cache, pairs, stream=stream)
+        pa_reshape_and_cache(key, value, self.k_cache, self.v_cache, slots, stream=stream)
+
+    def workspace(self, num_seqs: int, num_heads: int, max_blocks: int, partition_tokens: int = 0):
+        n = pa_decode_workspace_bytes(num_seqs, num_heads, self.num_kv_heads, self.head_size, max_blocks,
+                                      partition_tokens)
+        if n == 0:
+            return None
+        if self._ws is None or self._ws.numel() < n:
+            self._ws = torch.empty(n, dtype=torch.uint8, device=self.device)
+        return self._ws
+
+    def decode(self, out: torch.Tensor, query: torch.Tensor, block_tables: torch.Tensor,
+               context_lens: torch.Tensor, scale: float, partition_tokens: int = 0, stream=None,
+               workspace=None) -> torch.Tensor:
+        if workspace is None:
+            workspace = self.workspace(query.shape[0], query.shape[1], block_tables.shape[1], partition_tokens)
+        pa_decode(out, query, self.k_cache, self.v_cache, block_tables, context_lens, scale, self.num_kv_heads,
+                  workspace=workspace, partition_tokens=partition_tokens, stream=stream)
+        return out

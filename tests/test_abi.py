@@ -1,0 +1,258 @@
+"""CPU-only checks of libpa.so: it loads, exports every function that
+include/pa.h declares, rejects bad arguments before touching the GPU, and
+its host allocator reproduces the oracle block manager bit for bit (slots,
+copy-on-write pairs, tables, reference counts, free counts, waste) — on the
+hand-worked example, on random request sequences and on the replays of
+every seeded workload."""
+
+import os
+import random
+import re
+
+import numpy as np
+import pytest
+import torch
+
+import paged_kv_cache_351_b200 as pa
+from oracle.allocator import BlockAllocator, OutOfBlocks
+from workloads import WORKLOADS, AddOp, AppendOp, ForkOp, make_plan
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    with open(os.path.join(ROOT, "include", "pa.h")) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pa_\w+)\s*\(", text)))
+
+
+def test_exports_every_declared_function():
+    names = _declared_functions()
+    assert len(names) >= 20
+    lib = pa.library()
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+    assert lib.pa_version() == 1
+
+
+def test_status_strings():
+    lib = pa.library()
+    for s in range(7):
+        assert lib.pa_status_string(s)
+
+
+# ---------------------------------------------------------------------------
+# argument validation (returns before any CUDA call)
+# ---------------------------------------------------------------------------
+
+def _cache(nb=8, hk=2, d=128, dtype=torch.bfloat16):
+    return torch.empty(nb, hk, 16, d, dtype=dtype)
+
+
+def _expect(status, fn, *args, **kw):
+    with pytest.raises(pa.PagedAttentionError) as e:
+        fn(*args, **kw)
+    assert e.value.status == status, str(e.value)
+
+
+INVALID, UNSUPPORTED = 1, 2
+
+
+def test_reshape_and_cache_validation():
+    kc, vc = _cache(), _cache()
+    key = torch.empty(4, 2, 128, dtype=torch.bfloat16)
+    slots = torch.zeros(4, dtype=torch.int64)
+    _expect(INVALID, pa.pa_reshape_and_cache, key, key, kc, vc, slots.to(torch.int32), stream=0)
+    _expect(INVALID, pa.pa_reshape_and_cache, key[:3], key, kc, vc, slots, stream=0)
+    _expect(INVALID, pa.pa_reshape_and_cache, key.float(), key.float(), kc, vc, slots, stream=0)
+    _expect(INVALID, pa.pa_reshape_and_cache, key, key, kc, vc.float(), slots, stream=0)
+    _expect(INVALID, pa.pa_reshape_and_cache, key, key, kc.transpose(0, 1), vc, slots, stream=0)
+    _expect(UNSUPPORTED, pa.pa_reshape_and_cache, key[..., :96].contiguous(), key[..., :96].contiguous(),
+            _cache(d=96), _cache(d=96), slots, stream=0)
+    _expect(UNSUPPORTED, pa.pa_reshape_and_cache, key, key, torch.empty(8, 2, 32, 128, dtype=torch.bfloat16),
+            torch.empty(8, 2, 32, 128, dtype=torch.bfloat16), slots, stream=0)
+    # a token stride that is not a multiple of 16 bytes
+    wide = torch.empty(4, 2, 132, dtype=torch.bfloat16)[..., :128]
+    assert wide.stride(1) * 2 % 16 != 0
+    _expect(INVALID, pa.pa_reshape_and_cache, wide, wide, kc, vc, slots, stream=0)
+
+
+def test_copy_blocks_validation():
+    kc, vc = _cache(), _cache()
+    _expect(INVALID, pa.pa_copy_blocks, kc, vc, torch.zeros(3, 3, dtype=torch.int64), stream=0)
+    _expect(INVALID, pa.pa_copy_blocks, kc, vc, torch.zeros(3, 2, dtype=torch.int32), stream=0)
+    _expect(INVALID, pa.pa_copy_blocks, kc, vc, torch.zeros(2, 3, dtype=torch.int64).t(), stream=0)
+    pa.pa_copy_blocks(kc, vc, torch.zeros(0, 2, dtype=torch.int64), stream=0)  # n == 0: nothing launched
+
+
+def test_decode_validation():
+    kc, vc = _cache(hk=2), _cache(hk=2)
+    B, H = 3, 8
+    q = torch.empty(B, H, 128, dtype=torch.bfloat16)
+    out = torch.empty_like(q)
+    bt = torch.zeros(B, 4, dtype=torch.int32)
+    cl = torch.zeros(B, dtype=torch.int32)
+    _expect(INVALID, pa.pa_decode, out, q, kc, vc, bt, cl, 0.1, 4, stream=0)  # num_kv_heads mismatch
+    _expect(INVALID, pa.pa_decode, out, q, kc, vc, bt.long(), cl, 0.1, 2, stream=0)
+    _expect(INVALID, pa.pa_decode, out, q, kc, vc, bt[:2], cl, 0.1, 2, stream=0)
+    _expect(INVALID, pa.pa_decode, out, q, kc, vc, bt, cl[:2], 0.1, 2, stream=0)
+    _expect(INVALID, pa.pa_decode, out.float(), q, kc, vc, bt, cl, 0.1, 2, stream=0)
+    _expect(INVALID, pa.pa_decode, out, q, kc, vc, bt, cl, float("nan"), 2, stream=0)
+    _expect(INVALID, pa.pa_decode, out, q, kc, vc, bt.t().contiguous().t(), cl, 0.1, 2, stream=0)
+    q6 = torch.empty(B, 6, 128, dtype=torch.bfloat16)
+    _expect(UNSUPPORTED, pa.pa_decode, torch.empty_like(q6), q6, _cache(hk=2), _cache(hk=2), bt, cl, 0.1, 2,
+            stream=0)  # group of 3
+    q3 = torch.empty(B, 3, 128, dtype=torch.bfloat16)
+    _expect(INVALID, pa.pa_decode, torch.empty_like(q3), q3, kc, vc, bt, cl, 0.1, 2, stream=0)  # H % H_kv
+    # partition size not a multiple of the block size
+    _expect(INVALID, pa.pa_decode, out, q, kc, vc, bt, cl, 0.1, 2, partition_tokens=100, stream=0)
+    # B == 0: valid, nothing launched
+    z = torch.empty(0, H, 128, dtype=torch.bfloat16)
+    pa.pa_decode(z, z, kc, vc, torch.zeros(0, 4, dtype=torch.int32), torch.zeros(0, dtype=torch.int32), 0.1, 2,
+                 stream=0)
+
+
+def test_fixed_workspace_size():
+    n = pa.pa_decode_workspace_bytes(8, 32, 8, 128, 8192, 512)
+    P = 8192 * 16 // 512
+    assert n == 8 * 32 * P * 128 * 4 + 8 * 32 * P * 4
+    assert pa.pa_decode_workspace_bytes(8, 32, 8, 128, 8192, -1) == 0
+
+
+# ---------------------------------------------------------------------------
+# host allocator vs oracle
+# ---------------------------------------------------------------------------
+
+def _compare_state(c: pa.Allocator, o: BlockAllocator):
+    assert c.num_free() == o.num_free()
+    assert [c.refcount(b) for b in range(o.num_blocks)] == [o.refcount(b) for b in range(o.num_blocks)]
+    for s in o.sequences():
+        assert c.block_table(s) == o.block_table(s)
+        assert c.length(s) == o.length(s)
+    st = c.stats()
+    assert st["num_free"] == o.num_free() and st["num_seqs"] == len(o.sequences())
+    assert st["waste_slots"] == o.waste_slots()
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_allocator_matches_oracle_random(seed):
+    rnd = random.Random(100 + seed)
+    nb, bs = 40, 4
+    order = list(range(nb))
+    rnd.shuffle(order)
+    c = pa.Allocator(nb, bs, order)
+    o = BlockAllocator(nb, bs, order)
+    live, nxt = [], 0
+    for _ in range(400):
+        r = rnd.random()
+        if r < 0.12 or not live:
+            c.add(nxt)
+            o.add(nxt)
+            live.append(nxt)
+            nxt += 1
+        elif r < 0.27:
+            p = rnd.choice(live)
+            c.fork(p, nxt)
+            o.fork(p, nxt)
+            live.append(nxt)
+            nxt += 1
+        elif r < 0.38:
+            s = live.pop(rnd.randrange(len(live)))
+            c.free(s)
+            o.free(s)
+        else:
+            s = rnd.choice(live)
+            n = rnd.choice([0, 1, 1, 2, 3, 4, 5, 9])
+            try:
+                oslots, ocow = o.append(s, n)
+            except OutOfBlocks:
+                with pytest.raises(pa.OutOfBlocksError):
+                    c.append(s, n)
+            else:
+                cslots, ccow = c.append(s, n)
+                assert cslots.tolist() == oslots and ccow == ocow
+        _compare_state(c, o)
+
+
+def test_allocator_golden_example():
+    import json
+
+    with open(os.path.join(ROOT, "tests", "golden", "fork_cow_example.json")) as f:
+        g = json.load(f)
+    c = pa.Allocator(g["num_blocks"], g["block_size"], g["free_order"])
+    for stp in g["steps"]:
+        if stp["op"] == "add":
+            c.add(stp["seq"])
+        elif stp["op"] == "fork":
+            c.fork(stp["parent"], stp["child"])
+        elif stp["op"] == "free":
+            c.free(stp["seq"])
+        elif stp.get("error"):
+            with pytest.raises(pa.OutOfBlocksError):
+                c.append(stp["seq"], stp["n"])
+        else:
+            slots, cow = c.append(stp["seq"], stp["n"])
+            assert slots.tolist() == stp["slots"] and [list(p) for p in cow] == stp["cow"]
+    fin = g["final"]
+    assert [c.refcount(b) for b in range(g["num_blocks"])] == fin["refcounts"]
+    assert c.stats()["waste_slots"] == fin["waste_slots"]
+    for s, t in fin["tables"].items():
+        assert c.block_table(int(s)) == t
+
+
+def test_allocator_bad_requests():
+    c = pa.Allocator(4, 4)
+    c.add(1)
+    for fn, args in ((c.add, (1,)), (c.append, (9, 1)), (c.fork, (9, 10)), (c.fork, (1, 1)), (c.free, (9,))):
+        with pytest.raises(pa.PagedAttentionError):
+            fn(*args)
+    with pytest.raises(pa.PagedAttentionError):
+        pa.Allocator(3, 4, [0, 1, 1])
+    assert c.refcount(99) == -1
+
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_workload_replay_matches_oracle(name):
+    """Every seeded workload's request stream gives identical slots,
+    copy-on-write pairs and block tables in C++ and in the oracle."""
+    from oracle.replay import block_table_array, replay
+
+    plan = make_plan(name)
+    alloc_o, _, log = replay(plan, write_values=False)
+    c = pa.Allocator(plan.num_blocks, plan.workload.block_size, plan.free_order)
+    k = 0
+    for op in plan.setup_ops + plan.step_ops:
+        if isinstance(op, AddOp):
+            c.add(op.seq)
+        elif isinstance(op, ForkOp):
+            c.fork(op.parent, op.child)
+        elif isinstance(op, AppendOp):
+            slots, cow = c.append(op.seq, op.n)
+            seq, oslots, ocow = log.appends[k]
+            k += 1
+            assert seq == op.seq and np.array_equal(slots, np.asarray(oslots, np.int64)) and cow == ocow
+    tables, lens = c.block_tables(plan.batch, plan.max_blocks_per_seq)
+    assert np.array_equal(tables, block_table_array(alloc_o, plan.batch, plan.max_blocks_per_seq))
+    assert np.array_equal(lens, plan.context_lens)
+    assert c.stats()["waste_slots"] == alloc_o.waste_slots()
+
+
+def test_append_batch_matches_single_appends():
+    order = list(range(64))
+    random.Random(3).shuffle(order)
+    c1, c2 = pa.Allocator(64, 16, order), pa.Allocator(64, 16, order)
+    for c in (c1, c2):
+        for s in range(4):
+            c.add(s)
+            c.append(s, 10 + s)
+        c.fork(0, 10)
+        c.fork(1, 11)
+    seqs, counts = [0, 10, 1, 11, 2, 3], [1, 1, 3, 1, 0, 20]
+    slots_b, pairs_b = c1.append_batch(seqs, counts)
+    slots_s, pairs_s = [], []
+    for s, n in zip(seqs, counts):
+        sl, cw = c2.append(s, n)
+        slots_s += sl.tolist()
+        pairs_s += cw
+    assert slots_b.tolist() == slots_s and [tuple(p) for p in pairs_b.tolist()] == pairs_s
