@@ -122,6 +122,25 @@ def ncu_traffic(workload, launch_bytes_scale=1.0):
         return None
 
 
+def max_over_ranks(values, device, world):
+    """Each rank's device-timed values -> their maximum over all ranks (the
+    job is as slow as its slowest replica)."""
+    if world <= 1:
+        return [float(v) for v in values]
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def aggregate_value(bytes_per_step, ms_per_step, world):
+    """Whole-job GB/s: every replica moves bytes_per_step per step; the step
+    time is the max over ranks."""
+    return bytes_per_step * world / (ms_per_step * 1e-3) / 1e9
+
+
 # ---------------------------------------------------------------------------
 # device setup through the library
 # ---------------------------------------------------------------------------
@@ -388,12 +407,9 @@ def run_ours(args):
     st, bits = pa.pa_get_device_status(stream)
     if st != 0:
         raise RuntimeError(f"device status {st} bits {bits:#x} after the timed region")
-    if world > 1:
-        t = torch.tensor([elapsed, dec_ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed, dec_ms = float(t[0]), float(t[1])
+    elapsed, dec_ms = max_over_ranks([elapsed, dec_ms], device, world)
     ms_step = elapsed / K
-    value = nbytes["step"] * world / (ms_step * 1e-3) / 1e9
+    value = aggregate_value(nbytes["step"], ms_step, world)
     tok_s = plan.B * world / (ms_step * 1e-3)
     peak, peak_kind = measured_peaks()
 
@@ -434,13 +450,9 @@ def run_ours(args):
                 e2e_step()
             f1.record(stream)
         torch.cuda.synchronize()
-        e_ms = f0.elapsed_time(f1)
-        if world > 1:
-            t = torch.tensor([e_ms], device=device)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t[0])
+        e_ms = max_over_ranks([f0.elapsed_time(f1)], device, world)[0]
         e_step = e_ms / K
-        e2e = {"value": round(nbytes["step"] * world / (e_step * 1e-3) / 1e9, 3), "unit": "GB/s",
+        e2e = {"value": round(aggregate_value(nbytes["step"], e_step, world), 3), "unit": "GB/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": round(e_step, 5), "tok_per_s": round(plan.B * world / (e_step * 1e-3), 1)}
 
