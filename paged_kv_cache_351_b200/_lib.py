@@ -97,11 +97,15 @@ def load():
         return _lib
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"{LIB_PATH} is missing; build it with `python -m paged_kv_cache_351_b200.build` "
+            f"{LIB_PATH} is missing; build it with `python paged_kv_cache_351_b200/build.py` "
             "(the CUDA library is the only implementation)")
     lib = ctypes.CDLL(LIB_PATH)
     for name, (res, args) in SIGNATURES.items():
-        fn = getattr(lib, name)
+        try:
+            fn = getattr(lib, name)
+        except AttributeError as e:
+            raise ImportError(f"{LIB_PATH} lacks {name}: rebuild it with "
+                              "`python paged_kv_cache_351_b200/build.py`") from e
         fn.restype = res
         fn.argtypes = args
     if lib.pa_version() != 1:

@@ -1,6 +1,9 @@
 """Build libpa.so (sm_100a kernels + C ABI + host allocator) in-tree.
 
-    python -m paged_kv_cache_351_b200.build [--force] [--verbose]
+    python paged_kv_cache_351_b200/build.py [--force] [--verbose] [--ptxas-info]
+
+(run it by path: it does not import the package, whose import loads the
+library it is about to rebuild)
 
 nvcc compiles the single CUDA translation unit for sm_100a only
 (``-gencode arch=compute_100a,code=sm_100a``); g++ compiles the host
