@@ -54,7 +54,8 @@ typedef enum {
   PA_ERR_OUT_OF_BLOCKS = 3,  /* allocator: free blocks exhausted, state unchanged */
   PA_ERR_CUDA = 4,           /* a CUDA runtime call failed */
   PA_ERR_DEVICE_TIMEOUT = 5, /* a device-side bounded wait gave up */
-  PA_ERR_DEVICE_BOUNDS = 6   /* a device-side index check failed; element skipped */
+  PA_ERR_DEVICE_BOUNDS = 6,  /* a device-side index check failed; element skipped */
+  PA_ERR_SCRATCH_LIMIT = 7   /* pa_decode_no_alloc: the call needs more scratch than the library's fixed buffer */
 } pa_status;
 
 typedef enum { PA_F32 = 0, PA_BF16 = 1, PA_I32 = 2, PA_I64 = 3 } pa_dtype;
@@ -170,6 +171,35 @@ pa_status pa_decode(pa_tensor* out, const pa_tensor* query, const pa_tensor* k_c
  * automatically to fit shared memory), CTAs per SM (default 1).  Changes
  * the workspace size of the auto mode.  Not thread-safe. */
 pa_status pa_set_decode_tuning(int32_t warps_per_cta, int32_t stages, int32_t ctas_per_sm);
+
+/* ---------------------------------------------------------------------------
+ * pa_decode without a caller workspace.  The pages have no counterpart to
+ * this call; it exists for callers that cannot provide device scratch: for
+ * instance code running inside a host framework that owns every device
+ * allocation and passes plugins no scratch buffer, or a serving loop that
+ * must not call cudaMalloc (which can synchronise the device and stall other
+ * streams).  It computes exactly what pa_decode computes, with the same
+ * arguments and split modes (opts->partition_tokens, stream, timeout_ms;
+ * opts->workspace and workspace_bytes are ignored), but its split-context
+ * scratch is a fixed array of PA_NO_ALLOC_SCRATCH_BYTES inside the library,
+ * which every GPU that loads the library holds until the process exits.
+ *  - It allocates nothing: no cudaMalloc, no cudaFree, no allocating library
+ *    routine.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - A call whose split needs more scratch than PA_NO_ALLOC_SCRATCH_BYTES
+ *    returns PA_ERR_SCRATCH_LIMIT before launching anything (use
+ *    partition_tokens -1, no split, which needs none).
+ *  - All calls share the array and it keeps the last call's contents.  No
+ *    byte of it has to start at zero: every byte a call reads was written
+ *    earlier in that same call.  Calls whose kernels overlap on the GPU (two
+ *    streams, or two host threads) race on it: issue them on one stream.
+ * ------------------------------------------------------------------------- */
+#define PA_NO_ALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+pa_status pa_decode_no_alloc(pa_tensor* out, const pa_tensor* query, const pa_tensor* k_cache,
+                             const pa_tensor* v_cache, const pa_tensor* block_tables,
+                             const pa_tensor* context_lens, float scale, int32_t num_kv_heads, const pa_opts* opts);
 
 /* Workspace bytes pa_decode needs on the current device for these sizes and
  * this partition_tokens setting (0 = auto/balanced, >0 = fixed, -1 = none).

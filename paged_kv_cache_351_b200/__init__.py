@@ -21,7 +21,7 @@ from ._lib import (PA_DEV_BAD_BLOCK, PA_DEV_BAD_CONTEXT, PA_DEV_BAD_SLOT,  # noq
 
 __all__ = [
     "PagedAttentionError", "OutOfBlocksError", "pa_reshape_and_cache", "pa_copy_blocks", "pa_decode",
-    "pa_decode_workspace_bytes", "pa_set_decode_tuning", "pa_get_device_status", "pa_debug_wait_selftest",
+    "pa_decode_workspace_bytes", "pa_decode_no_alloc", "pa_set_decode_tuning", "pa_get_device_status", "pa_debug_wait_selftest",
     "Allocator", "library",
 ]
 
@@ -129,6 +129,25 @@ def pa_decode(out, query, k_cache, v_cache, block_tables, context_lens, scale: f
     _check(_lib_handle.pa_decode(ctypes.byref(to), ctypes.byref(tq), ctypes.byref(kc), ctypes.byref(vc),
                                  ctypes.byref(bt), ctypes.byref(cl), ctypes.c_float(scale), int(num_kv_heads),
                                  ctypes.byref(o)), "pa_decode")
+
+
+NO_ALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
+
+
+def pa_decode_no_alloc(out, query, k_cache, v_cache, block_tables, context_lens, scale: float, num_kv_heads: int,
+                       partition_tokens: int = 0, stream=None, timeout_ms: int = 0) -> None:
+    """pa_decode for callers that cannot provide device scratch (a host
+    framework that owns all device memory and gives plugins no scratch
+    buffer, or a loop that must not call cudaMalloc, which can synchronise
+    the device).  The split scratch is a fixed 16 MiB array inside the
+    library; a call needing more raises PA_ERR_SCRATCH_LIMIT.  The first call
+    on a device looks up that array's address, so make it before any stream
+    capture.  Calls share the array: issue them on one stream."""
+    to, tq, kc, vc, bt, cl = (_tensor(x) for x in (out, query, k_cache, v_cache, block_tables, context_lens))
+    o = _opts(stream, None, partition_tokens, timeout_ms)
+    _check(_lib_handle.pa_decode_no_alloc(ctypes.byref(to), ctypes.byref(tq), ctypes.byref(kc), ctypes.byref(vc),
+                                          ctypes.byref(bt), ctypes.byref(cl), ctypes.c_float(scale),
+                                          int(num_kv_heads), ctypes.byref(o)), "pa_decode_no_alloc")
 
 
 def pa_decode_workspace_bytes(num_seqs: int, num_heads: int, num_kv_heads: int, head_size: int,

@@ -293,6 +293,8 @@ const char* pa_status_string(pa_status s) {
       return "device wait timed out";
     case PA_ERR_DEVICE_BOUNDS:
       return "device index check failed";
+    case PA_ERR_SCRATCH_LIMIT:
+      return "needs more split scratch than the library's fixed no-alloc buffer holds";
   }
   return "unknown status";
 }
@@ -500,6 +502,74 @@ pa_status pa_get_device_status(const pa_opts* opts, uint32_t* bits_out) {
   if (bits & PA_DEV_TIMEOUT) return PA_ERR_DEVICE_TIMEOUT;
   if (bits) return PA_ERR_DEVICE_BOUNDS;
   return PA_OK;
+}
+
+// ---------------------------------------------------------------------------
+// pa_decode_no_alloc: pa_decode with its split scratch in a fixed device
+// array of this library instead of a caller workspace.
+// ---------------------------------------------------------------------------
+}  // extern "C"
+
+namespace {
+
+static __device__ __align__(256) unsigned char g_no_alloc_scratch[PA_NO_ALLOC_SCRATCH_BYTES];
+
+// In host code g_no_alloc_scratch names a host-side stand-in, not device
+// memory; the kernels must be given the address cudaGetSymbolAddress returns,
+// looked up once per device with that device current.
+void* g_no_alloc_ptr[kMaxDevices] = {};
+std::mutex g_no_alloc_mu;
+
+pa_status no_alloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_no_alloc_mu);
+  if (g_no_alloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_no_alloc_scratch) != cudaSuccess || p == nullptr) return PA_ERR_CUDA;
+    g_no_alloc_ptr[dev] = p;
+  }
+  *out = g_no_alloc_ptr[dev];
+  return PA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+pa_status pa_decode_no_alloc(pa_tensor* out, const pa_tensor* query, const pa_tensor* k_cache,
+                             const pa_tensor* v_cache, const pa_tensor* block_tables, const pa_tensor* context_lens,
+                             float scale, int32_t num_kv_heads, const pa_opts* opts) {
+  if (query == nullptr || query->ndim != 3 || k_cache == nullptr || k_cache->ndim != 4 || block_tables == nullptr ||
+      block_tables->ndim != 2)
+    return PA_ERR_INVALID_ARG;
+  const int32_t part = opts ? opts->partition_tokens : 0;
+  if (part < -1 || (part > 0 && part % pa::kBS)) return PA_ERR_INVALID_ARG;
+  const int64_t B = query->shape[0], H = query->shape[1], D = query->shape[2];
+  const int64_t max_nb = block_tables->shape[1];
+  if (B < 0 || H <= 0 || num_kv_heads <= 0 || H % num_kv_heads || B > INT32_MAX || max_nb < 0 || max_nb > INT32_MAX ||
+      D <= 0 || D > INT32_MAX || H > INT32_MAX)
+    return PA_ERR_INVALID_ARG;
+  size_t need = 0;
+  if (part != -1 && B > 0) {
+    const pa_status st = pa_decode_workspace_bytes(int32_t(B), int32_t(H), num_kv_heads, int32_t(D),
+                                                   int32_t(max_nb), part, &need);
+    if (st != PA_OK) return st;
+    if (need > PA_NO_ALLOC_SCRATCH_BYTES) return PA_ERR_SCRATCH_LIMIT;
+  }
+  pa_opts o;
+  std::memset(&o, 0, sizeof(o));
+  if (opts) o = *opts;
+  o.workspace = nullptr;
+  o.workspace_bytes = 0;
+  if (part != -1 && B > 0) {
+    void* p = nullptr;
+    const pa_status st = no_alloc_scratch(&p);
+    if (st != PA_OK) return st;
+    o.workspace = p;
+    o.workspace_bytes = PA_NO_ALLOC_SCRATCH_BYTES;
+  }
+  return pa_decode(out, query, k_cache, v_cache, block_tables, context_lens, scale, num_kv_heads, &o);
 }
 
 pa_status pa_debug_wait_selftest(const pa_opts* opts) {
