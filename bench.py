@@ -176,8 +176,7 @@ def setup_device(plan, device):
 
     for op in plan.setup_ops:
         if isinstance(op, AddOp):
-            flush()
-            kv.add(op.seq)
+            kv.add(op.seq)  # a new sequence touches no pending block
         elif isinstance(op, ForkOp):
             flush()
             kv.fork(op.parent, op.child)

@@ -201,13 +201,15 @@ class Allocator:
             ptr = None
         _check(_lib_handle.pa_alloc_create(num_blocks, block_size, ptr, ctypes.byref(h)), "pa_alloc_create")
         self._h = h
+        self._destroy = _lib_handle.pa_alloc_destroy  # kept: module globals may be gone at exit
         self.num_blocks = num_blocks
         self.block_size = block_size
 
     def __del__(self):
         h = getattr(self, "_h", None)
-        if h is not None and h.value:
-            _lib_handle.pa_alloc_destroy(h)
+        destroy = getattr(self, "_destroy", None)
+        if h is not None and h.value and destroy is not None:
+            destroy(h)
             self._h = None
 
     def add(self, seq: int) -> None:

@@ -76,6 +76,35 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
   }
 }
 
+// ---- flags between CTAs of one grid ---------------------------------------
+__device__ __forceinline__ void st_release_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Wait until *p == want, giving up after timeout_ns (sets PA_DEV_TIMEOUT).
+__device__ __forceinline__ bool wait_flag_bounded(const unsigned long long* p, unsigned long long want,
+                                                  uint64_t timeout_ns) {
+  if (ld_acquire_u64(p) == want) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int k = 0; k < 32; ++k) {
+      __nanosleep(64);
+      if (ld_acquire_u64(p) == want) return true;
+    }
+    if (globaltimer_ns() - t0 > timeout_ns) {
+      flag(PA_DEV_TIMEOUT);
+      return false;
+    }
+  }
+}
+
 // ---- bulk copy (TMA engine, 1-D, no tensor map, no multicast) --------------
 // dst and src 16-byte aligned, bytes a multiple of 16.
 __device__ __forceinline__ void bulk_g2s(uint32_t dst_smem, const void* src, uint32_t bytes, uint32_t bar,
@@ -108,6 +137,18 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// d = a * b + d on two fp32 lanes at once (packed FMA, sm_100).
+__device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %5};\n\t"
+      "mov.b64 rd, {%0, %1};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rd;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "+f"(d0), "+f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
 // Storage-type traits: a 16-byte vector holds EPV elements.

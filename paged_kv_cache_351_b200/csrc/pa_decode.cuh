@@ -13,10 +13,14 @@
 //    workers of a persistent grid (one CTA per SM) take equal, contiguous
 //    ranges of the flattened page list, so every SM streams the same number
 //    of bytes whatever the length mix.  A row cut by a range boundary yields
-//    per-worker partial results (max, denominator, normalised output) that a
-//    small log-sum-exp merge kernel combines.  Fixed-size partitions (each
-//    partition its own partial, then the merge) and an unsplit mode are the
-//    same loop with boundaries snapped to partitions or rows.
+//    per-worker partial results (normalised output and log-sum-exp).  The
+//    worker holding the row's first page merges them at the end of its own
+//    range: the later workers publish their share with a per-call tag, and
+//    the merging warp waits (bounded) for the tags, so no separate merge
+//    kernel and no zeroed workspace are needed.  Fixed-size partitions (each
+//    partition its own partial, merged by a small log-sum-exp kernel) and an
+//    unsplit mode are the same loop with boundaries snapped to partitions or
+//    rows.
 //  * Each page of a row — 16 tokens x head_size for one kv head, 4 KiB for
 //    bf16/128 — is one contiguous run in the cache layout
 //    [num_blocks, num_kv_heads, 16, head_size], so a worker moves it with a
@@ -41,7 +45,11 @@
 
 namespace pa {
 
-constexpr int kBS = 16;  // tokens per block (block_size)
+constexpr int kBS = 16;        // tokens per block (block_size)
+constexpr int kMaxWarps = 12;  // workers per CTA (registers allow 12 at G <= 4)
+
+// Warps per CTA the register budget allows without spills (8 at G = 8).
+__host__ __device__ constexpr int max_warps_for_group(int G) { return G >= 8 ? 8 : kMaxWarps; }
 
 enum DecodeMode : int32_t { kBalanced = 0, kFixed = 1, kNoSplit = 2 };
 
@@ -61,9 +69,10 @@ struct DecodeArgs {
   int32_t part_pages;  // fixed mode: pages per partition
   int32_t P_max;       // fixed mode: partition capacity per (seq, head)
   int32_t stages;      // ring depth per warp
-  float* ws_o;         // partial outputs
+  float* ws_o;         // partial outputs (normalised)
   float* ws_lse;       // partial log-sum-exp (natural log)
-  int4* ws_task;       // balanced mode: one merge task per worker
+  unsigned long long* ws_flag;  // balanced mode: per worker, the call tag once its partial is published
+  unsigned long long call_tag;  // distinct per call, so no flag has to start at zero
   uint64_t timeout_ns;
 };
 
@@ -158,7 +167,7 @@ __device__ __forceinline__ int64_t snap_boundary(const int* S, int B, int Hkv, i
 }
 
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(256, 1) decode_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(max_warps_for_group(G) * 32, 1) decode_kernel(const DecodeArgs a) {
   using C = DecodeCfg<T, D, G>;
   constexpr int LPT = C::LPT, TPI = C::TPI, NT = C::NT, EPV = C::EPV, GH = C::GH;
   extern __shared__ __align__(128) unsigned char smem[];
@@ -216,16 +225,6 @@ __global__ void __launch_bounds__(256, 1) decode_kernel(const DecodeArgs a) {
   int64_t hi = ((wid + 1) * W + nworkers - 1) / nworkers;
   lo = snap_boundary(S, B, Hkv, lo, W, a.mode, a.part_pages);
   hi = snap_boundary(S, B, Hkv, hi, W, a.mode, a.part_pages);
-  if (a.mode == kBalanced) {
-    if (lane == 0) a.ws_task[wid] = make_int4(-1, -1, -1, -1);
-    if (lo >= hi) {
-      // an empty worker contributes nothing to a merge that spans it
-      float* po = a.ws_o + wid * 2 * G * D;
-      for (int k = lane; k < G * D; k += 32) po[k] = 0.f;
-      if (lane < G) a.ws_lse[wid * 2 * G + lane] = -INFINITY;
-    }
-  }
-
   const uint64_t pol = policy_evict_first();
   const T* qg = reinterpret_cast<const T*>(a.q);
   const unsigned char* kcb = reinterpret_cast<const unsigned char*>(a.kc);
@@ -347,10 +346,11 @@ __global__ void __launch_bounds__(256, 1) decode_kernel(const DecodeArgs a) {
         Elem<T>::unpack(Ks[(tg + TPI * k) * LPT + c], kf);
 #pragma unroll
         for (int j = 0; j < G; ++j) {
-          float sum = 0.f;
+          // two interleaved partial sums on the packed-FMA pipe
+          float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-          for (int e = 0; e < EPV; ++e) sum = fmaf(q[j][e], kf[e], sum);
-          acc[j][k] = sum;
+          for (int e = 0; e < EPV; e += 2) ffma2(s0, s1, q[j][e], q[j][e + 1], kf[e], kf[e + 1]);
+          acc[j][k] = s0 + s1;
         }
       }
 #pragma unroll
@@ -426,21 +426,7 @@ __global__ void __launch_bounds__(256, 1) decode_kernel(const DecodeArgs a) {
         lpart[jj] = lpart[jj] * aj + (own ? p : 0.f);
         if (own) {
           const int j = (G >= 2 && hi_half) ? jj + GH : jj;
-          pbuf[(j * TPI + tg) * NT + (c >> 1)] = p;
-        }
-      }
-      __syncwarp();
-      float pk[G][NT];
-#pragma unroll
-      for (int j = 0; j < G; ++j) {
-        const float4* src = reinterpret_cast<const float4*>(pbuf + (j * TPI + tg) * NT);
-#pragma unroll
-        for (int k4 = 0; k4 < NT / 4; ++k4) {
-          const float4 v4 = src[k4];
-          pk[j][4 * k4 + 0] = v4.x;
-          pk[j][4 * k4 + 1] = v4.y;
-          pk[j][4 * k4 + 2] = v4.z;
-          pk[j][4 * k4 + 3] = v4.w;
+          pbuf[(tg * NT + (c >> 1)) * G + j] = p;
         }
       }
       __syncwarp();
@@ -451,9 +437,25 @@ __global__ void __launch_bounds__(256, 1) decode_kernel(const DecodeArgs a) {
           for (int e = 0; e < EPV; ++e) o[j][e] *= alpha[j];
       }
 
-      // ---- weighted sum of V ----
+      // ---- weighted sum of V (probabilities read per token, heads contiguous) ----
 #pragma unroll
       for (int k = 0; k < NT; ++k) {
+        float pk[G];
+        {
+          const float* src = pbuf + (tg * NT + k) * G;
+          if constexpr (G % 4 == 0) {
+#pragma unroll
+            for (int j4 = 0; j4 < G; j4 += 4) {
+              const float4 v4 = *reinterpret_cast<const float4*>(src + j4);
+              pk[j4] = v4.x, pk[j4 + 1] = v4.y, pk[j4 + 2] = v4.z, pk[j4 + 3] = v4.w;
+            }
+          } else if constexpr (G == 2) {
+            const float2 v2 = *reinterpret_cast<const float2*>(src);
+            pk[0] = v2.x, pk[1] = v2.y;
+          } else {
+            pk[0] = src[0];
+          }
+        }
         float vf[EPV];
         Elem<T>::unpack(Vs[(tg + TPI * k) * LPT + c], vf);
         if (tg + TPI * k >= valid) {
@@ -461,11 +463,12 @@ __global__ void __launch_bounds__(256, 1) decode_kernel(const DecodeArgs a) {
           for (int e = 0; e < EPV; ++e) vf[e] = 0.f;  // unused slots may hold any bits
         }
 #pragma unroll
-        for (int j = 0; j < G; ++j)
+        for (int j = 0; j < G; ++j) {
 #pragma unroll
-          for (int e = 0; e < EPV; ++e) o[j][e] = fmaf(pk[j][k], vf[e], o[j][e]);
+          for (int e = 0; e < EPV; e += 2) ffma2(o[j][e], o[j][e + 1], pk[j], pk[j], vf[e], vf[e + 1]);
+        }
       }
-      __syncwarp();  // every lane is done with stage s
+      __syncwarp();  // every lane is done with stage s and with pbuf
 
       // ---- refill stage s with the next page of this worker's range ----
       if (px < hi) issue(s);
@@ -506,22 +509,14 @@ __global__ void __launch_bounds__(256, 1) decode_kernel(const DecodeArgs a) {
               *reinterpret_cast<uint4*>(ob + int64_t(cc.g * G + j) * a.o_sh + c * EPV) = Elem<T>::pack(f);
             }
           }
-        } else {
-          int64_t base;  // index of the (head 0) partial slot
-          bool task = false;
-          if (a.mode == kFixed) {
-            base = (int64_t(cc.i) * H + int64_t(cc.g) * G) * a.P_max + cc.p / a.part_pages;
-          } else {
-            const int slot = seg_p0 == 0 ? 1 : 0;
-            base = (wid * 2 + slot) * G;
-            task = (slot == 1);
-          }
-          const int64_t hstride = a.mode == kFixed ? a.P_max : 1;
+        } else if (a.mode == kFixed) {
+          // one partial per partition; a separate kernel merges them
+          const int64_t base = (int64_t(cc.i) * H + int64_t(cc.g) * G) * a.P_max + cc.p / a.part_pages;
           if (tg == 0) {
 #pragma unroll
             for (int j = 0; j < G; ++j) {
               const float inv = 1.f / lall[j];
-              float4* dst = reinterpret_cast<float4*>(a.ws_o + (base + j * hstride) * D + c * EPV);
+              float4* dst = reinterpret_cast<float4*>(a.ws_o + (base + j * a.P_max) * D + c * EPV);
 #pragma unroll
               for (int e4 = 0; e4 < EPV / 4; ++e4)
                 dst[e4] = make_float4(o[j][4 * e4] * inv, o[j][4 * e4 + 1] * inv, o[j][4 * e4 + 2] * inv,
@@ -536,12 +531,91 @@ __global__ void __launch_bounds__(256, 1) decode_kernel(const DecodeArgs a) {
                 mj = m[j];
                 lj = lall[j];
               }
-            a.ws_lse[base + lane * hstride] = (mj + log2f(lj)) * 0.69314718055994530942f;
+            a.ws_lse[base + lane * a.P_max] = (mj + log2f(lj)) * 0.69314718055994530942f;
           }
-          if (task && lane == 0) {
-            const int64_t row_last = int64_t(S[cc.i]) + int64_t(cc.g) * cc.np + cc.np - 1;
-            const int wb = int(row_last * nworkers / W);
-            a.ws_task[wid] = make_int4(cc.i, cc.g, int(wid), wb);
+        } else if (seg_p0 != 0) {
+          // Balanced mode, a row that began in an earlier worker: publish this
+          // share (normalised output + log-sum-exp), then the call tag.
+          if (tg == 0) {
+#pragma unroll
+            for (int j = 0; j < G; ++j) {
+              const float inv = 1.f / lall[j];
+              float4* dst = reinterpret_cast<float4*>(a.ws_o + (wid * G + j) * D + c * EPV);
+#pragma unroll
+              for (int e4 = 0; e4 < EPV / 4; ++e4)
+                dst[e4] = make_float4(o[j][4 * e4] * inv, o[j][4 * e4 + 1] * inv, o[j][4 * e4 + 2] * inv,
+                                      o[j][4 * e4 + 3] * inv);
+            }
+          }
+          if (lane < G) {
+            float mj = m[0], lj = lall[0];
+#pragma unroll
+            for (int j = 1; j < G; ++j)
+              if (lane == j) {
+                mj = m[j];
+                lj = lall[j];
+              }
+            a.ws_lse[wid * G + lane] = (mj + log2f(lj)) * 0.69314718055994530942f;
+          }
+          __syncwarp();
+          if (lane == 0) {
+            __threadfence();
+            st_release_u64(a.ws_flag + wid, a.call_tag);
+          }
+        } else {
+          // Balanced mode, a row that began here and continues in later
+          // workers.  This is the last segment of this worker's range; the
+          // later workers published their shares at the start (or, for a
+          // range inside the row, the end) of theirs.  Merge them into this
+          // share by log-sum-exp and write the row.
+          const int64_t row_last = int64_t(S[cc.i]) + int64_t(cc.g) * cc.np + cc.np - 1;
+          const int64_t wb = row_last * nworkers / W;
+          float mx[G], wsum[G], acc[G][EPV];
+#pragma unroll
+          for (int j = 0; j < G; ++j) {
+            mx[j] = (m[j] + log2f(lall[j])) * 0.69314718055994530942f;
+            wsum[j] = 1.f;
+            const float inv = 1.f / lall[j];
+#pragma unroll
+            for (int e = 0; e < EPV; ++e) acc[j][e] = o[j][e] * inv;
+          }
+          for (int64_t k = wid + 1; k <= wb; ++k) {
+            const int64_t klo = (k * W + nworkers - 1) / nworkers;
+            const int64_t khi = ((k + 1) * W + nworkers - 1) / nworkers;
+            if (klo == khi) continue;  // an empty worker holds no share
+            if (lane == 0) wait_flag_bounded(a.ws_flag + k, a.call_tag, a.timeout_ns);
+            __syncwarp();
+#pragma unroll
+            for (int j = 0; j < G; ++j) {
+              const float lk = __ldcg(a.ws_lse + k * G + j);
+              const float mn = fmaxf(mx[j], lk);
+              const float sc = ex2((mx[j] - mn) * 1.4426950408889634f);
+              const float wk = ex2((lk - mn) * 1.4426950408889634f);
+              mx[j] = mn;
+              wsum[j] = wsum[j] * sc + wk;
+              if (tg == 0) {
+                const float4* src = reinterpret_cast<const float4*>(a.ws_o + (k * G + j) * D + c * EPV);
+#pragma unroll
+                for (int e4 = 0; e4 < EPV / 4; ++e4) {
+                  const float4 v = __ldcg(src + e4);
+                  acc[j][4 * e4 + 0] = fmaf(wk, v.x, acc[j][4 * e4 + 0] * sc);
+                  acc[j][4 * e4 + 1] = fmaf(wk, v.y, acc[j][4 * e4 + 1] * sc);
+                  acc[j][4 * e4 + 2] = fmaf(wk, v.z, acc[j][4 * e4 + 2] * sc);
+                  acc[j][4 * e4 + 3] = fmaf(wk, v.w, acc[j][4 * e4 + 3] * sc);
+                }
+              }
+            }
+          }
+          if (tg == 0) {
+            T* ob = reinterpret_cast<T*>(a.out) + int64_t(cc.i) * a.o_sb;
+#pragma unroll
+            for (int j = 0; j < G; ++j) {
+              const float inv = 1.f / wsum[j];
+              float f[EPV];
+#pragma unroll
+              for (int e = 0; e < EPV; ++e) f[e] = acc[j][e] * inv;
+              *reinterpret_cast<uint4*>(ob + int64_t(cc.g * G + j) * a.o_sh + c * EPV) = Elem<T>::pack(f);
+            }
           }
         }
       }
@@ -618,53 +692,6 @@ __global__ void __launch_bounds__(256) merge_fixed_kernel(const DecodeArgs a, in
   }
   const float inv = 1.f / wsum;
   T* dst = reinterpret_cast<T*>(a.out) + int64_t(i) * a.o_sb + int64_t(h) * a.o_sh + lane * PER;
-  float f[PER];
-#pragma unroll
-  for (int e = 0; e < PER; ++e) f[e] = acc[e] * inv;
-  if constexpr (sizeof(T) == 4) {
-#pragma unroll
-    for (int e = 0; e < PER; ++e) reinterpret_cast<float*>(dst)[e] = f[e];
-  } else {
-#pragma unroll
-    for (int e = 0; e < PER; e += 2) {
-      __nv_bfloat162 hh = __floats2bfloat162_rn(f[e], f[e + 1]);
-      *reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(dst) + e) = hh;
-    }
-  }
-}
-
-// Balanced mode: one warp per (worker, query head of the group); the worker's
-// task names the row it started and the last worker the row reaches.
-template <typename T, int D, int G>
-__global__ void __launch_bounds__(256) merge_balanced_kernel(const DecodeArgs a, int64_t nworkers) {
-  pdl_wait();
-  constexpr int PER = D / 32;
-  const int lane = threadIdx.x & 31;
-  const int64_t t = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (t >= nworkers * G) return;
-  const int64_t w = t / G;
-  const int j = int(t % G);
-  const int4 task = a.ws_task[w];
-  if (task.x < 0) return;
-  const int i = task.x, g = task.y, wa = task.z, wb = task.w;
-  float mx = -INFINITY, wsum = 0.f;
-  float acc[PER];
-#pragma unroll
-  for (int e = 0; e < PER; ++e) acc[e] = 0.f;
-  for (int wk = wa; wk <= wb; ++wk) {
-    const int64_t slot = (int64_t(wk) * 2 + (wk == wa ? 1 : 0)) * G + j;
-    const float l = a.ws_lse[slot];
-    const float mn = fmaxf(mx, l);
-    const float sc = ex2((mx - mn) * 1.4426950408889634f);
-    const float wgt = ex2((l - mn) * 1.4426950408889634f);
-    mx = mn;
-    wsum = wsum * sc + wgt;
-    const float* src = a.ws_o + slot * D + lane * PER;
-#pragma unroll
-    for (int e = 0; e < PER; ++e) acc[e] = fmaf(wgt, src[e], acc[e] * sc);
-  }
-  const float inv = 1.f / wsum;
-  T* dst = reinterpret_cast<T*>(a.out) + int64_t(i) * a.o_sb + int64_t(g * G + j) * a.o_sh + lane * PER;
   float f[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) f[e] = acc[e] * inv;

@@ -88,8 +88,7 @@ def build_device_state(plan: Plan, device="cuda", include_step=True, write_step=
     step_slots = []
     for idx, op in enumerate(ops):
         if isinstance(op, AddOp):
-            flush()
-            alloc.add(op.seq)
+            alloc.add(op.seq)  # a new sequence touches no pending block
         elif isinstance(op, ForkOp):
             flush()
             alloc.fork(op.parent, op.child)
