@@ -108,16 +108,21 @@ def kernel_source_hash():
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(workload, launch_bytes_scale=1.0):
-    """DRAM bytes per launch of the decode kernel from the committed ncu
-    summary, if it was taken on the current kernel source."""
-    p = os.path.join(ROOT, "profiles", "decode_traffic.json")
+def ncu_traffic(workload):
+    """DRAM bytes (read + write) per launch of the decode kernel from the
+    committed ncu summary of this workload, if it was taken on the current
+    kernel source; else None."""
+    p = os.path.join(ROOT, "profiles", f"decode_kernel_{workload}.md")
     try:
+        vals = {}
         with open(p) as f:
-            d = json.load(f)
-        if d.get("kernel_sha") != kernel_source_hash() or d.get("workload") != workload:
+            for line in f:
+                k, _, v = line.strip().partition(":")
+                if k in ("workload", "kernel_source_sha", "dram_bytes_per_launch"):
+                    vals[k] = v.strip()
+        if vals.get("kernel_source_sha") != kernel_source_hash() or vals.get("workload") != workload:
             return None
-        return float(d["dram_bytes_per_launch"]) * launch_bytes_scale
+        return float(vals["dram_bytes_per_launch"])
     except Exception:
         return None
 
@@ -357,7 +362,8 @@ def run_ours(args):
     scale = 1.0 / math.sqrt(w.head_size)
     ws = kv.workspace(plan.B, w.num_heads, bt.shape[1], args.partition)
     stream = torch.cuda.Stream(device)
-    launches_per_step = 2 + (1 if (args.partition > 0 or (args.partition == 0 and ws is not None)) else 0)
+    # cache write + decode; fixed partitions add the log-sum-exp merge kernel
+    launches_per_step = 2 + (1 if args.partition > 0 else 0)
 
     def step():
         pa.pa_reshape_and_cache(key, value, kv.k_cache, kv.v_cache, slots, stream=stream)
@@ -477,7 +483,7 @@ def run_ours(args):
         "frac_of_hbm_peak": round(value / world / peak, 4),
         "frac_of_8tbs_spec": round(value / world / 8000.0, 4),
         "bytes_per_step": nbytes,
-        "roofline": {"bound": "hbm", "kernel": "pa_decode (decode_kernel + lse merge)",
+        "roofline": {"bound": "hbm", "kernel": "pa_decode (decode_kernel, log-sum-exp merge fused)",
                      "achieved": round(achieved, 2), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
                      "algorithmic_bytes_per_launch": nbytes["decode"], "avg_launch_ms": round(dec_ms, 5)},
