@@ -11,6 +11,9 @@ definitions:
   discovery note, item 2; agientry.com overview, opening section).
 * ``cache``      — physical K/V storage and the two byte-moving steps: the
   per-token cache write by slot and the whole-block copy of copy-on-write.
+* ``quant``      — FP8 (e4m3) codes of a quantized KV cache with per-head
+  scales (the pages only say the KV cache can be quantized; gitcode repo
+  walkthrough, section 三 "量化").
 * ``attention``  — single-query attention softmax(q K^T * scale) V over the
   tokens a block table names, walked logically, in fp64; and the
   log-sum-exp merge of per-partition partial results.
@@ -28,6 +31,7 @@ routine; none is "parity unpinned".
 
 from .allocator import BlockAllocator, OutOfBlocks, AllocatorError  # noqa: F401
 from .cache import PagedKVCache  # noqa: F401
+from .quant import e4m3_decode, e4m3_encode, quantize_kv  # noqa: F401
 from .attention import (  # noqa: F401
     widen,
     paged_decode,

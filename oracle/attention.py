@@ -39,10 +39,15 @@ import numpy as np
 
 
 def widen(raw: np.ndarray, dtype: str) -> np.ndarray:
-    """Exact widening of stored values (float32, or bf16 bits) to fp64."""
+    """Exact widening of stored values (float32, bf16 bits, or e4m3 codes
+    without their scale) to fp64."""
     raw = np.asarray(raw)
     if dtype == "f32":
         return raw.astype(np.float64)
+    if dtype == "fp8":
+        from .quant import e4m3_decode
+
+        return e4m3_decode(raw)
     if dtype == "bf16":
         bits = raw.astype(np.uint16).astype(np.uint32) << np.uint32(16)
         return bits.view(np.float32).astype(np.float64)
@@ -63,6 +68,9 @@ def gather_sequence(cache, block_table: Sequence[int], ctx: int) -> Tuple[np.nda
             raise IndexError(f"block {b} read at offsets that were never written")
         k[t0:t0 + n] = widen(cache.k_page(b)[:, :n, :], cache.dtype).transpose(1, 0, 2)
         v[t0:t0 + n] = widen(cache.v_page(b)[:, :n, :], cache.dtype).transpose(1, 0, 2)
+    if cache.dtype == "fp8":  # dequantize: code value times the head's scale
+        k *= cache.k_scale.astype(np.float64)[None, :, None]
+        v *= cache.v_scale.astype(np.float64)[None, :, None]
     return k, v
 
 
@@ -86,13 +94,15 @@ def attend_contiguous(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float)
 
 
 def paged_decode_rows(query, cache, block_tables, context_lens, scale: float,
-                      seqs: Iterable[int]) -> Dict[int, np.ndarray]:
-    """Outputs [H, D] (fp64) of the chosen batch rows only."""
+                      seqs: Iterable[int], query_dtype: str = "") -> Dict[int, np.ndarray]:
+    """Outputs [H, D] (fp64) of the chosen batch rows only.  The query is in
+    the cache's storage type, or bf16 for an fp8 cache (unless given)."""
+    qd = query_dtype or ("bf16" if cache.dtype == "fp8" else cache.dtype)
     res: Dict[int, np.ndarray] = {}
     for i in seqs:
         i = int(i)
         ctx = int(context_lens[i])
-        q = widen(query[i], cache.dtype)
+        q = widen(query[i], qd)
         k, v = gather_sequence(cache, block_tables[i], ctx)
         res[i] = attend_contiguous(q, k, v, scale)
     return res

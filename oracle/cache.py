@@ -4,8 +4,9 @@ A block holds the K (and, separately, the V) of ``block_size`` consecutive
 tokens for every KV head: the pages state that one block stores BLOCK_SIZE
 tokens of one head, e.g. 2048 elements per block per head at block size 16
 and head size 128 (gitcode repo walkthrough, section 2.1 "PagedAttention").
-Values are kept as their raw storage bits (float32, or bfloat16 bit patterns
-in uint16) so that byte-moving steps can be compared bit for bit.
+Values are kept as their raw storage bits (float32, bfloat16 bit patterns in
+uint16, or FP8 e4m3 codes in uint8 with per-kv-head scales) so that
+byte-moving steps can be compared bit for bit.
 
 * ``write``: the cache write — token t's K/V for head h go to slot
   ``slots[t]``, i.e. block ``slot // bs``, offset ``slot % bs``; slot -1 means
@@ -26,15 +27,21 @@ import numpy as np
 
 
 class PagedKVCache:
-    def __init__(self, num_blocks: int, num_kv_heads: int, head_size: int, block_size: int, dtype: str):
-        if dtype not in ("f32", "bf16"):
-            raise ValueError("dtype must be 'f32' or 'bf16'")
+    def __init__(self, num_blocks: int, num_kv_heads: int, head_size: int, block_size: int, dtype: str,
+                 k_scale=None, v_scale=None):
+        if dtype not in ("f32", "bf16", "fp8"):
+            raise ValueError("dtype must be 'f32', 'bf16' or 'fp8'")
+        if dtype == "fp8" and (k_scale is None or v_scale is None):
+            raise ValueError("an fp8 cache needs per-head k_scale and v_scale")
         self.num_blocks = num_blocks
         self.num_kv_heads = num_kv_heads
         self.head_size = head_size
         self.block_size = block_size
         self.dtype = dtype
-        self.raw_dtype = np.float32 if dtype == "f32" else np.uint16
+        self.raw_dtype = {"f32": np.float32, "bf16": np.uint16, "fp8": np.uint8}[dtype]
+        # fp8: stored codes are value / scale[h] (see oracle.quant)
+        self.k_scale = None if k_scale is None else np.asarray(k_scale, np.float32)
+        self.v_scale = None if v_scale is None else np.asarray(v_scale, np.float32)
         self._k: Dict[int, np.ndarray] = {}
         self._v: Dict[int, np.ndarray] = {}
         self._written: Dict[int, np.ndarray] = {}

@@ -14,10 +14,12 @@ from typing import List, Optional, Tuple
 
 import numpy as np
 
-from workloads import AddOp, ForkOp, AppendOp, Plan, stream_kv
+from workloads import AddOp, ForkOp, AppendOp, Plan, kv_scales, stream_kv
 
 from .allocator import BlockAllocator
+from .attention import widen
 from .cache import PagedKVCache
+from .quant import quantize_kv
 
 
 @dataclass
@@ -34,7 +36,11 @@ def replay(plan: Plan, stop_after: Optional[int] = None, include_step: bool = Tr
     allocator-only checks of large workloads)."""
     w = plan.workload
     alloc = BlockAllocator(plan.num_blocks, w.block_size, plan.free_order)
-    cache = PagedKVCache(plan.num_blocks, w.num_kv_heads, w.head_size, w.block_size, w.dtype)
+    if w.cache_dtype == "fp8":
+        ks, vs = kv_scales(plan)
+        cache = PagedKVCache(plan.num_blocks, w.num_kv_heads, w.head_size, w.block_size, "fp8", ks, vs)
+    else:
+        cache = PagedKVCache(plan.num_blocks, w.num_kv_heads, w.head_size, w.block_size, w.dtype)
     log = ReplayLog()
     ops = list(plan.setup_ops) + (list(plan.step_ops) if include_step else [])
     if stop_after is not None:
@@ -50,6 +56,9 @@ def replay(plan: Plan, stop_after: Optional[int] = None, include_step: bool = Tr
             if write_values:
                 cache.copy_blocks(cow)
                 k, v = stream_kv(plan, op.stream, op.start, op.n)
+                if w.cache_dtype == "fp8":  # the write quantizes the bf16 inputs
+                    k = quantize_kv(widen(k, w.dtype).astype(np.float32), cache.k_scale)
+                    v = quantize_kv(widen(v, w.dtype).astype(np.float32), cache.v_scale)
                 cache.write(slots, k, v)
         else:
             raise TypeError(op)

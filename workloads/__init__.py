@@ -18,6 +18,7 @@ from .synth import (  # noqa: F401
     stream_kv,
     seq_token_sources,
     query_values,
+    kv_scales,
     to_bf16_bits,
     bf16_bits_to_f32,
     workload_by_name,

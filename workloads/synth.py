@@ -50,6 +50,7 @@ class Workload:
     head_size: int
     block_size: int = BLOCK_SIZE
     description: str = ""
+    kv_dtype: str = ""  # cache storage type when it differs from dtype ("fp8": e4m3 codes + per-head scales)
 
     @property
     def seed(self) -> int:
@@ -62,6 +63,14 @@ class Workload:
     @property
     def elem_bytes(self) -> int:
         return 4 if self.dtype == "f32" else 2
+
+    @property
+    def cache_dtype(self) -> str:
+        return self.kv_dtype or self.dtype
+
+    @property
+    def cache_elem_bytes(self) -> int:
+        return {"f32": 4, "bf16": 2, "fp8": 1}[self.cache_dtype]
 
 
 WORKLOADS: Dict[str, Workload] = {
@@ -81,6 +90,12 @@ WORKLOADS: Dict[str, Workload] = {
         Workload("long_ctx_splitk", 4, "bf16", 32, 8, 128,
                  description="B=8, ctx {32,48,64,80,96,112,128,128}k, H=32 on H_kv=8, D=128, bf16, "
                              "512-token partitions + LSE reduce"),
+        # FP8 KV-cache variants: same seeds, lengths and bf16 token values; the
+        # cache stores e4m3 codes with per-kv-head scales (kv_scales).
+        Workload("llama7b_bs64_fp8", 1, "bf16", 32, 32, 128, kv_dtype="fp8",
+                 description="llama7b_bs64 with an e4m3 KV cache (per-head scales), bf16 query/output"),
+        Workload("gqa_bs256_fp8", 2, "bf16", 32, 8, 128, kv_dtype="fp8",
+                 description="gqa_bs256 with an e4m3 KV cache (per-head scales), bf16 query/output"),
     )
 }
 
@@ -199,6 +214,14 @@ def make_plan(w: Union[Workload, str]) -> Plan:
     """Build the seeded instance of a named workload."""
     if isinstance(w, str):
         w = WORKLOADS[w]
+    if w.kv_dtype == "fp8":
+        base = make_plan(w.name[: -len("_fp8")])
+        base.workload = w
+        if w.name.startswith("llama7b"):
+            # the same 40 GB of pool, now of 1-byte elements
+            base.num_blocks = int(40_000_000_000 // (2 * w.num_kv_heads * w.block_size * w.head_size))
+            base.free_order = _rng(w, _TAG_PERM).permutation(base.num_blocks).astype(np.int32)
+        return base
     bs = w.block_size
     if w.name == "tiny_fp32":
         ctx = np.array([1, 17, 33, 100], np.int32)
@@ -327,6 +350,20 @@ def seq_token_sources(plan: Plan) -> Dict[int, List[Tuple[int, int, int]]]:
             else:
                 r.append((op.stream, op.start, op.n))
     return runs
+
+
+def kv_scales(plan: Plan) -> Tuple[np.ndarray, np.ndarray]:
+    """Per-kv-head FP8 scales (k_scale, v_scale), float32 [H_kv]: about the
+    largest |value| of a head over 448, so the N(0,1) values use the e4m3
+    range; heads holding an x8 outlier channel get an 8x larger K scale."""
+    w = plan.workload
+    h = np.arange(w.num_kv_heads)
+    k = (6.0 / 448.0) * (1.0 + 0.25 * (h % 3))
+    if plan.outlier_channels.shape[0]:
+        hot = np.isin(h, plan.outlier_channels[:, 0])
+        k = np.where(hot, 8.0 * k, k)
+    v = (5.0 / 448.0) * (1.0 + 0.25 * ((h + 1) % 3))
+    return k.astype(np.float32), v.astype(np.float32)
 
 
 def query_values(plan: Plan, step: int = 0) -> np.ndarray:
