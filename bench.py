@@ -69,7 +69,7 @@ def workload_plan(name, pool_gb=None):
         import numpy as np
 
         w = plan.workload
-        nb = int(pool_gb * 1e9) // (2 * w.num_kv_heads * w.block_size * w.head_size * w.elem_bytes)
+        nb = int(pool_gb * 1e9) // (2 * w.num_kv_heads * w.block_size * w.head_size * w.cache_elem_bytes)
         need = sum(-(-int(c) // w.block_size) for c in plan.context_lens)
         nb = max(nb, need)
         plan.num_blocks = nb
@@ -78,16 +78,20 @@ def workload_plan(name, pool_gb=None):
 
 
 def step_bytes(plan):
+    """Algorithmic bytes: the decode reads every context token's K and V (in
+    the cache's element size), the query and writes the output (in the
+    query's), plus block tables and lengths; the write reads the new tokens'
+    K/V and writes them into the cache."""
     w = plan.workload
-    e, bs = w.elem_bytes, w.block_size
+    e, ec, bs = w.elem_bytes, w.cache_elem_bytes, w.block_size
     ctx = [int(c) for c in plan.context_lens]
-    kv = sum(ctx) * 2 * w.num_kv_heads * w.head_size * e
+    kv = sum(ctx) * 2 * w.num_kv_heads * w.head_size * ec
     qo = 2 * plan.B * w.num_heads * w.head_size * e
     tables = sum(4 * (-(-c // bs)) for c in ctx)
     lens = 4 * plan.B
     decode = kv + qo + tables + lens
     n_new = len(plan.step_ops)
-    write = n_new * w.num_kv_heads * w.head_size * e * 2 * 2 + 8 * n_new
+    write = n_new * w.num_kv_heads * w.head_size * 2 * (e + ec) + 8 * n_new
     return {"kv": kv, "decode": decode, "write": write, "step": decode + write}
 
 
@@ -158,18 +162,19 @@ def setup_device(plan, device):
     import torch
 
     from paged_kv_cache_351_b200.runtime import PagedKVCacheGPU
-    from workloads import AddOp, AppendOp, ForkOp, query_values, stream_kv
+    from workloads import AddOp, AppendOp, ForkOp, kv_scales, query_values, stream_kv
 
     w = plan.workload
-    tdt = torch.float32 if w.dtype == "f32" else torch.bfloat16
+    tdt = torch.float32 if w.dtype == "f32" else torch.bfloat16  # query/output and new-token type
 
     def dev(raw):
         if w.dtype == "f32":
             return torch.from_numpy(np.ascontiguousarray(raw)).to(device)
         return torch.from_numpy(np.ascontiguousarray(raw).view(np.int16)).to(device).view(torch.bfloat16)
 
-    kv = PagedKVCacheGPU(plan.num_blocks, w.num_kv_heads, w.head_size, w.dtype, w.block_size, plan.free_order,
-                         device=device)
+    scales = kv_scales(plan) if w.cache_dtype == "fp8" else (None, None)
+    kv = PagedKVCacheGPU(plan.num_blocks, w.num_kv_heads, w.head_size, w.cache_dtype, w.block_size,
+                         plan.free_order, device=device, k_scale=scales[0], v_scale=scales[1])
     pend = {"seqs": set(), "slots": [], "k": [], "v": [], "pairs": []}
 
     def flush():
@@ -275,7 +280,7 @@ def oracle_timing(plan, seconds, max_rows=None):
     q = query_values(plan)
     scale = 1.0 / math.sqrt(plan.workload.head_size)
     w = plan.workload
-    per_tok = 2 * w.num_kv_heads * w.head_size * w.elem_bytes
+    per_tok = 2 * w.num_kv_heads * w.head_size * w.cache_elem_bytes
     done_bytes, rows_done, i = 0, 0, 0
     t0 = time.perf_counter()
     while True:
@@ -366,7 +371,7 @@ def run_ours(args):
     launches_per_step = 2 + (1 if args.partition > 0 else 0)
 
     def step():
-        pa.pa_reshape_and_cache(key, value, kv.k_cache, kv.v_cache, slots, stream=stream)
+        kv.write(slots, key, value, None, stream=stream)
         kv.decode(out, q, bt, cl, scale, partition_tokens=args.partition, stream=stream, workspace=ws)
 
     with torch.cuda.stream(stream):
@@ -379,8 +384,6 @@ def run_ours(args):
 
     K = args.steps
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    ea = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    eb = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     uuid = str(torch.cuda.get_device_properties(device).uuid)
     uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
     sampler = ClockSampler(uuid)
@@ -388,18 +391,28 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    # Timed region: K whole steps, events only at its ends (an event between
+    # the write and the decode would block the decode's early launch).
     with torch.cuda.stream(stream):
         ev0.record(stream)
-        for k in range(K):
-            pa.pa_reshape_and_cache(key, value, kv.k_cache, kv.v_cache, slots, stream=stream)
-            ea[k].record(stream)
-            kv.decode(out, q, bt, cl, scale, partition_tokens=args.partition, stream=stream, workspace=ws)
-            eb[k].record(stream)
+        for _ in range(K):
+            step()
         ev1.record(stream)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     elapsed = ev0.elapsed_time(ev1)  # ms
+    # Roofline of the dominant kernel: K decode launches on the same stream,
+    # each bracketed by events, right after the timed region.
+    ea = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    eb = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    with torch.cuda.stream(stream):
+        for k in range(K):
+            ea[k].record(stream)
+            kv.decode(out, q, bt, cl, scale, partition_tokens=args.partition, stream=stream, workspace=ws)
+            eb[k].record(stream)
+    torch.cuda.synchronize()
+    dec_ms = statistics.mean(ea[k].elapsed_time(eb[k]) for k in range(K))
     # keep the same load a little longer if the timed region was too short for clock samples
     t_soak = time.perf_counter()
     with torch.cuda.stream(stream):
@@ -408,7 +421,6 @@ def run_ours(args):
                 step()
             torch.cuda.synchronize()
     clocks = sampler.stop()
-    dec_ms = statistics.mean(ea[k].elapsed_time(eb[k]) for k in range(K))
     st, bits = pa.pa_get_device_status(stream)
     if st != 0:
         raise RuntimeError(f"device status {st} bits {bits:#x} after the timed region")
@@ -418,48 +430,86 @@ def run_ours(args):
     tok_s = plan.B * world / (ms_step * 1e-3)
     peak, peak_kind = measured_peaks()
 
-    # end to end through the public API: host (pinned) inputs in, output out
+    # End to end through the public API: every step copies its inputs from
+    # pinned host memory and reads its output back.  Two buffer sets let the
+    # copies of steps k+1 (in) and k-1 (out) run on copy streams while step k
+    # computes, as a serving loop would.
     e2e = None
     if not args.no_e2e:
         pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()  # noqa: E731
         raw = (lambda r: r if w.dtype == "f32" else r.view(np.int16))
-        h_q, h_k, h_v = pin(raw(inp["query"])), pin(raw(inp["key"])), pin(raw(inp["value"]))
-        h_s, h_bt, h_cl = pin(inp["slots"]), pin(inp["tables"]), pin(inp["lens"])
-        h_out = torch.empty(out.shape, dtype=torch.int16 if w.dtype == "bf16" else torch.float32).pin_memory()
-        d_q = torch.empty(h_q.shape, dtype=h_q.dtype, device=device)
-        d_k = torch.empty(h_k.shape, dtype=h_k.dtype, device=device)
-        d_v = torch.empty(h_v.shape, dtype=h_v.dtype, device=device)
-        d_s, d_bt, d_cl = (torch.empty_like(x, device=device) for x in (h_s, h_bt, h_cl))
         view = (lambda t: t if w.dtype == "f32" else t.view(torch.bfloat16))
-        h2d = sum(x.numel() * x.element_size() for x in (h_q, h_k, h_v, h_s, h_bt, h_cl))
-        d2h = h_out.numel() * h_out.element_size()
+        hosts = [(pin(raw(inp["query"])), pin(raw(inp["key"])), pin(raw(inp["value"])), pin(inp["slots"]),
+                  pin(inp["tables"]), pin(inp["lens"])) for _ in range(2)]
+        h_out = [torch.empty(out.shape, dtype=torch.int16 if w.dtype == "bf16" else torch.float32).pin_memory()
+                 for _ in range(2)]
+        devs = [tuple(torch.empty(x.shape, dtype=x.dtype, device=device) for x in hosts[b]) for b in range(2)]
+        d_out = [torch.empty_like(out) for _ in range(2)]
+        h2d = sum(x.numel() * x.element_size() for x in hosts[0])
+        d2h = h_out[0].numel() * h_out[0].element_size()
+        s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_done = [torch.cuda.Event() for _ in range(2)]
+        ev_read = [torch.cuda.Event() for _ in range(2)]
 
-        def e2e_step():
-            for d, h in ((d_q, h_q), (d_k, h_k), (d_v, h_v), (d_s, h_s), (d_bt, h_bt), (d_cl, h_cl)):
-                d.copy_(h, non_blocking=True)
+        def copy_in(k):
+            b = k % 2
+            with torch.cuda.stream(s_in):
+                if k >= 2:
+                    s_in.wait_event(ev_done[b])  # step k-2 no longer reads buffer set b
+                for d, h in zip(devs[b], hosts[b]):
+                    d.copy_(h, non_blocking=True)
+                ev_in[b].record(s_in)
+
+        def compute(k):
+            b = k % 2
+            d_q, d_k, d_v, d_s, d_bt, d_cl = devs[b]
+            stream.wait_event(ev_in[b])
+            if k >= 2:
+                stream.wait_event(ev_read[b])  # step k-2's output has been read back
             kv.write(d_s, view(d_k), view(d_v), None, stream=stream)
-            kv.decode(out, view(d_q), d_bt, d_cl, scale, partition_tokens=args.partition, stream=stream,
+            kv.decode(d_out[b], view(d_q), d_bt, d_cl, scale, partition_tokens=args.partition, stream=stream,
                       workspace=ws)
-            h_out.copy_(out.view(h_out.dtype), non_blocking=True)
+            ev_done[b].record(stream)
 
-        with torch.cuda.stream(stream):
-            for _ in range(max(3, args.warmup)):
-                e2e_step()
+        def copy_out(k):
+            b = k % 2
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_done[b])
+                h_out[b].copy_(d_out[b].view(h_out[b].dtype), non_blocking=True)
+                ev_read[b].record(s_out)
+
+        def run_e2e(n):
+            copy_in(0)
+            for k in range(n):
+                if k + 1 < n:
+                    copy_in(k + 1)
+                compute(k)
+                copy_out(k)
+
+        run_e2e(max(3, args.warmup))
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
         f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            f0.record(stream)
-            for _ in range(K):
-                e2e_step()
-            f1.record(stream)
+        f0.record(s_in)
+        stream.wait_event(f0)
+        s_out.wait_event(f0)
+        run_e2e(K)
+        s_out.wait_stream(stream)
+        s_out.wait_stream(s_in)
+        f1.record(s_out)
         torch.cuda.synchronize()
         e_ms = max_over_ranks([f0.elapsed_time(f1)], device, world)[0]
         e_step = e_ms / K
+        got = h_out[(K - 1) % 2].view(torch.bfloat16 if w.dtype == "bf16" else torch.float32)
+        if not torch.equal(got.view(torch.int16 if w.dtype == "bf16" else torch.int32),
+                           out.view(torch.int16 if w.dtype == "bf16" else torch.int32).cpu()):
+            raise RuntimeError("end-to-end output differs from the device-resident step's output")
         e2e = {"value": round(aggregate_value(nbytes["step"], e_step, world), 3), "unit": "GB/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "ms_per_step": round(e_step, 5), "tok_per_s": round(plan.B * world / (e_step * 1e-3), 1)}
+               "ms_per_step": round(e_step, 5), "tok_per_s": round(plan.B * world / (e_step * 1e-3), 1),
+               "overlap": "double-buffered: copies of steps k+1 (in) and k-1 (out) overlap step k"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -486,7 +536,8 @@ def run_ours(args):
         "roofline": {"bound": "hbm", "kernel": "pa_decode (decode_kernel, log-sum-exp merge fused)",
                      "achieved": round(achieved, 2), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
-                     "algorithmic_bytes_per_launch": nbytes["decode"], "avg_launch_ms": round(dec_ms, 5)},
+                     "algorithmic_bytes_per_launch": nbytes["decode"], "avg_launch_ms": round(dec_ms, 5),
+                     "timing": f"{K} decode launches, each bracketed by CUDA events, after the timed region"},
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": launches_per_step * K,

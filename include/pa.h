@@ -34,8 +34,10 @@
  * used.
  *
  * Supported: block_size 16; (bf16, head_size 128), (bf16, head_size 64),
- * (fp32, head_size 64), (fp32, head_size 128); num_heads / num_kv_heads in
- * {1, 2, 4, 8}.  Anything else returns PA_ERR_UNSUPPORTED.
+ * (fp32, head_size 64), (fp32, head_size 128), and an FP8 e4m3 cache with
+ * head_size 128 and bf16 query/output (pa_reshape_and_cache_fp8,
+ * pa_decode_fp8); num_heads / num_kv_heads in {1, 2, 4, 8}.  Anything else
+ * returns PA_ERR_UNSUPPORTED.
  */
 #ifndef PA_H_
 #define PA_H_
@@ -58,7 +60,7 @@ typedef enum {
   PA_ERR_SCRATCH_LIMIT = 7   /* pa_decode_no_alloc: the call needs more scratch than the library's fixed buffer */
 } pa_status;
 
-typedef enum { PA_F32 = 0, PA_BF16 = 1, PA_I32 = 2, PA_I64 = 3 } pa_dtype;
+typedef enum { PA_F32 = 0, PA_BF16 = 1, PA_I32 = 2, PA_I64 = 3, PA_FP8_E4M3 = 4 } pa_dtype;
 
 /* A strided view of caller-owned memory.  Strides are in elements. */
 typedef struct {
@@ -201,6 +203,30 @@ pa_status pa_set_decode_tuning(int32_t warps_per_cta, int32_t stages, int32_t ct
 pa_status pa_decode_no_alloc(pa_tensor* out, const pa_tensor* query, const pa_tensor* k_cache,
                              const pa_tensor* v_cache, const pa_tensor* block_tables,
                              const pa_tensor* context_lens, float scale, int32_t num_kv_heads, const pa_opts* opts);
+
+/* ---------------------------------------------------------------------------
+ * FP8 (e4m3) KV cache.  The pages say only that the KV cache itself can be
+ * quantized to save memory (gitcode walkthrough, section 三 "量化", the
+ * quantized_kvcache item); this library's form: every K (V) element is stored
+ * as one OCP e4m3 code of value / k_scale[h] (v_scale[h]), h the kv head,
+ * so a page is 2 KiB at head_size 128 and the decode reads half the bytes.
+ *
+ * pa_reshape_and_cache_fp8: as pa_reshape_and_cache, with key/value bf16 or
+ *   fp32 and k_cache/v_cache of dtype PA_FP8_E4M3 [num_blocks, H_kv, 16, 128];
+ *   code = e4m3(float(x) / scale[h]) with IEEE fp32 division, rounding to
+ *   nearest even and saturation to +-448 (NaN stays NaN).
+ * pa_decode_fp8: as pa_decode over an FP8 cache with bf16 query and output;
+ *   K[t] = e4m3_value(code) * k_scale[g], V likewise; fp32 accumulation.
+ * k_scale, v_scale: [H_kv] fp32 on the device, contiguous, positive.
+ * pa_reshape_and_cache and pa_decode reject FP8 caches (they have no scales).
+ * ------------------------------------------------------------------------- */
+pa_status pa_reshape_and_cache_fp8(const pa_tensor* key, const pa_tensor* value, pa_tensor* k_cache,
+                                   pa_tensor* v_cache, const pa_tensor* slot_mapping, const pa_tensor* k_scale,
+                                   const pa_tensor* v_scale, const pa_opts* opts);
+pa_status pa_decode_fp8(pa_tensor* out, const pa_tensor* query, const pa_tensor* k_cache, const pa_tensor* v_cache,
+                        const pa_tensor* block_tables, const pa_tensor* context_lens, float scale,
+                        int32_t num_kv_heads, const pa_tensor* k_scale, const pa_tensor* v_scale,
+                        const pa_opts* opts);
 
 /* Workspace bytes pa_decode needs on the current device for these sizes and
  * this partition_tokens setting (0 = auto/balanced, >0 = fixed, -1 = none).

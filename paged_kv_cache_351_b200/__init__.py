@@ -21,7 +21,7 @@ from ._lib import (PA_DEV_BAD_BLOCK, PA_DEV_BAD_CONTEXT, PA_DEV_BAD_SLOT,  # noq
 
 __all__ = [
     "PagedAttentionError", "OutOfBlocksError", "pa_reshape_and_cache", "pa_copy_blocks", "pa_decode",
-    "pa_decode_workspace_bytes", "pa_decode_no_alloc", "pa_set_decode_tuning", "pa_get_device_status", "pa_debug_wait_selftest",
+    "pa_decode_workspace_bytes", "pa_decode_no_alloc", "pa_reshape_and_cache_fp8", "pa_decode_fp8", "pa_set_decode_tuning", "pa_get_device_status", "pa_debug_wait_selftest",
     "Allocator", "library",
 ]
 
@@ -55,7 +55,7 @@ def _dtype_code(t) -> int:
     import torch
 
     codes = {torch.float32: _lib.PA_F32, torch.bfloat16: _lib.PA_BF16, torch.int32: _lib.PA_I32,
-             torch.int64: _lib.PA_I64}
+             torch.int64: _lib.PA_I64, torch.float8_e4m3fn: _lib.PA_FP8_E4M3}
     if t.dtype not in codes:
         raise TypeError(f"unsupported dtype {t.dtype}")
     return codes[t.dtype]
@@ -129,6 +129,25 @@ def pa_decode(out, query, k_cache, v_cache, block_tables, context_lens, scale: f
     _check(_lib_handle.pa_decode(ctypes.byref(to), ctypes.byref(tq), ctypes.byref(kc), ctypes.byref(vc),
                                  ctypes.byref(bt), ctypes.byref(cl), ctypes.c_float(scale), int(num_kv_heads),
                                  ctypes.byref(o)), "pa_decode")
+
+
+def pa_reshape_and_cache_fp8(key, value, k_cache, v_cache, slot_mapping, k_scale, v_scale, stream=None) -> None:
+    """Quantizing cache write into an FP8 (torch.float8_e4m3fn) cache: each
+    value is stored as the e4m3 code of value / scale[kv head]."""
+    ts = [_tensor(x) for x in (key, value, k_cache, v_cache, slot_mapping, k_scale, v_scale)]
+    o = _opts(stream)
+    _check(_lib_handle.pa_reshape_and_cache_fp8(*[ctypes.byref(t) for t in ts], ctypes.byref(o)),
+           "pa_reshape_and_cache_fp8")
+
+
+def pa_decode_fp8(out, query, k_cache, v_cache, block_tables, context_lens, scale: float, num_kv_heads: int,
+                  k_scale, v_scale, workspace=None, partition_tokens: int = 0, stream=None, timeout_ms: int = 0) -> None:
+    """Paged decode over an FP8 cache with per-kv-head scales; bf16 query and output."""
+    ts = [_tensor(x) for x in (out, query, k_cache, v_cache, block_tables, context_lens)]
+    ks, vs = _tensor(k_scale), _tensor(v_scale)
+    o = _opts(stream, workspace, partition_tokens, timeout_ms)
+    _check(_lib_handle.pa_decode_fp8(*[ctypes.byref(t) for t in ts], ctypes.c_float(scale), int(num_kv_heads),
+                                     ctypes.byref(ks), ctypes.byref(vs), ctypes.byref(o)), "pa_decode_fp8")
 
 
 NO_ALLOC_SCRATCH_BYTES = 16 * 1024 * 1024

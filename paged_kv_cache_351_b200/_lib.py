@@ -54,7 +54,7 @@ STATUS_NAMES = {
     6: "PA_ERR_DEVICE_BOUNDS",
     7: "PA_ERR_SCRATCH_LIMIT",
 }
-PA_F32, PA_BF16, PA_I32, PA_I64 = 0, 1, 2, 3
+PA_F32, PA_BF16, PA_I32, PA_I64, PA_FP8_E4M3 = 0, 1, 2, 3, 4
 PA_DEV_TIMEOUT, PA_DEV_BAD_BLOCK, PA_DEV_BAD_CONTEXT, PA_DEV_BAD_SLOT = 0x1, 0x2, 0x4, 0x8
 
 _T = POINTER(PaTensor)
@@ -68,6 +68,8 @@ SIGNATURES = {
     "pa_copy_blocks": (c_int32, [_T, _T, _T, _O]),
     "pa_decode": (c_int32, [_T, _T, _T, _T, _T, _T, c_float, c_int32, _O]),
     "pa_decode_no_alloc": (c_int32, [_T, _T, _T, _T, _T, _T, c_float, c_int32, _O]),
+    "pa_reshape_and_cache_fp8": (c_int32, [_T, _T, _T, _T, _T, _T, _T, _O]),
+    "pa_decode_fp8": (c_int32, [_T, _T, _T, _T, _T, _T, c_float, c_int32, _T, _T, _O]),
     "pa_decode_workspace_bytes": (c_int32, [c_int32, c_int32, c_int32, c_int32, c_int32, c_int32, POINTER(c_size_t)]),
     "pa_set_decode_tuning": (c_int32, [c_int32, c_int32, c_int32]),
     "pa_alloc_create": (c_int32, [c_int32, c_int32, _I32P, POINTER(_A)]),

@@ -45,11 +45,17 @@ Tuning g_tuning;
 // pages in flight; grouped heads (G = 2, 4) do more math per page and need
 // 12 warps to hide it (+15% on the GQA workload); G = 8 is capped at 8 by
 // registers.
-int default_warps(int G) { return (G == 2 || G == 4) ? 12 : 8; }
+// An FP8 cache doubles the dequantization and math per byte, so it wants 12
+// warps even at G = 1 (+20% on the LLaMA-7B shape).
+int default_warps(int G, bool fp8 = false) { return (G == 2 || G == 4 || fp8) ? 12 : 8; }
 
-int warps_for(int G) {
-  const int w = g_tuning.warps ? g_tuning.warps : default_warps(G);
-  return w < pa::max_warps_for_group(G) ? w : pa::max_warps_for_group(G);
+// Cache elements per 16-byte vector (dims per lane) of a cache dtype.
+int epv_of(int32_t kv_dtype) { return kv_dtype == PA_F32 ? 4 : kv_dtype == PA_FP8_E4M3 ? 16 : 8; }
+
+int warps_for(int G, int32_t kv_dtype) {
+  const int w = g_tuning.warps ? g_tuning.warps : default_warps(G, kv_dtype == PA_FP8_E4M3);
+  const int cap = pa::max_warps_for(G, epv_of(kv_dtype));
+  return w < cap ? w : cap;
 }
 
 pa_status device_info(DeviceInfo* out, int* dev_out) {
@@ -77,13 +83,16 @@ inline uint64_t timeout_of(const pa_opts* o) {
   return uint64_t(ms) * 1000000ull;
 }
 
-inline int esize(int32_t dt) { return dt == PA_F32 ? 4 : dt == PA_BF16 ? 2 : dt == PA_I32 ? 4 : dt == PA_I64 ? 8 : 0; }
+inline int esize(int32_t dt) {
+  return dt == PA_F32 ? 4 : dt == PA_BF16 ? 2 : dt == PA_I32 ? 4 : dt == PA_I64 ? 8 : dt == PA_FP8_E4M3 ? 1 : 0;
+}
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // The cache: [NB, Hkv, 16, D] contiguous, 16-byte aligned.
 pa_status check_cache(const pa_tensor* t) {
-  if (t == nullptr || t->ndim != 4 || (t->dtype != PA_F32 && t->dtype != PA_BF16)) return PA_ERR_INVALID_ARG;
+  if (t == nullptr || t->ndim != 4 || (t->dtype != PA_F32 && t->dtype != PA_BF16 && t->dtype != PA_FP8_E4M3))
+    return PA_ERR_INVALID_ARG;
   const int64_t* s = t->shape;
   if (s[0] <= 0 || s[1] <= 0 || s[2] <= 0 || s[3] <= 0) return PA_ERR_INVALID_ARG;
   if (t->stride[3] != 1 || t->stride[2] != s[3] || t->stride[1] != s[2] * s[3] || t->stride[0] != s[1] * s[2] * s[3])
@@ -91,6 +100,7 @@ pa_status check_cache(const pa_tensor* t) {
   if (t->data == nullptr || !aligned16(t->data)) return PA_ERR_INVALID_ARG;
   if (s[2] != 16) return PA_ERR_UNSUPPORTED;
   if (s[3] != 64 && s[3] != 128) return PA_ERR_UNSUPPORTED;
+  if (t->dtype == PA_FP8_E4M3 && s[3] != 128) return PA_ERR_UNSUPPORTED;
   if (s[0] > INT32_MAX || s[1] > 1024) return PA_ERR_UNSUPPORTED;
   return PA_OK;
 }
@@ -114,6 +124,16 @@ pa_status check_rows3(const pa_tensor* t, int32_t dtype, int64_t n0, int64_t n1,
   if (t->stride[0] < 0 || t->stride[1] < 0 || (t->stride[0] * e) % 16 || (t->stride[1] * e) % 16)
     return PA_ERR_INVALID_ARG;
   if (n0 > 0 && (t->data == nullptr || !aligned16(t->data))) return PA_ERR_INVALID_ARG;
+  return PA_OK;
+}
+
+// Per-kv-head FP8 scales: [Hkv] fp32, contiguous, every value finite and > 0
+// (the values are not checked on the host: they live on the device).
+pa_status check_scale(const pa_tensor* t, int64_t Hkv) {
+  if (t == nullptr || t->ndim != 1 || t->dtype != PA_F32 || t->shape[0] != Hkv || t->data == nullptr)
+    return PA_ERR_INVALID_ARG;
+  if (Hkv > 1 && t->stride[0] != 1) return PA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(t->data) & 3u) return PA_ERR_INVALID_ARG;
   return PA_OK;
 }
 
@@ -151,9 +171,9 @@ struct DecodePlan {
   size_t ws_need;
 };
 
-template <typename T, int D, int G>
+template <typename Tkv, typename Tq, int D, int G>
 size_t stage_fit(int B, int warps, int want, int optin, int* stages_out) {
-  using C = pa::DecodeCfg<T, D, G>;
+  using C = pa::DecodeCfg<Tkv, Tq, D, G>;
   for (int st = want; st >= 1; --st) {
     const size_t bytes = pa::decode_prefix_bytes(B) + size_t(warps) * C::warp_bytes(st);
     if (bytes <= size_t(optin)) {
@@ -197,11 +217,11 @@ unsigned long long next_call_tag() {
   return g_call_tag.fetch_add(2ull);
 }
 
-template <typename T, int D, int G>
+template <typename Tkv, typename Tq, int D, int G>
 pa_status run_decode(const pa::DecodeArgs& base, const DecodePlan& p, cudaStream_t st, int dev) {
   static bool attr_set[kMaxDevices] = {};
   static size_t attr_bytes[kMaxDevices] = {};
-  auto kern = pa::decode_kernel<T, D, G>;
+  auto kern = pa::decode_kernel<Tkv, Tq, D, G>;
   if (!attr_set[dev] || attr_bytes[dev] < p.smem) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(p.smem)) != cudaSuccess)
       return PA_ERR_CUDA;
@@ -218,7 +238,7 @@ pa_status run_decode(const pa::DecodeArgs& base, const DecodePlan& p, cudaStream
   if (p.mode == pa::kFixed) {
     const int64_t tasks = int64_t(a.B) * a.H;
     const int blocks = int((tasks + 7) / 8);
-    if (launch_pdl(pa::merge_fixed_kernel<T, D>, dim3(blocks), dim3(256), 0, st, true, a,
+    if (launch_pdl(pa::merge_fixed_kernel<Tq, D>, dim3(blocks), dim3(256), 0, st, true, a,
                    p.part_pages * pa::kBS) != cudaSuccess)
       return launch_status();
   }
@@ -226,43 +246,48 @@ pa_status run_decode(const pa::DecodeArgs& base, const DecodePlan& p, cudaStream
   return launch_status();
 }
 
-template <typename T, int D>
+template <typename Tkv, typename Tq, int D>
 pa_status dispatch_group(int G, const pa::DecodeArgs& a, const DecodePlan& p, cudaStream_t st, int dev) {
   switch (G) {
     case 1:
-      return run_decode<T, D, 1>(a, p, st, dev);
+      return run_decode<Tkv, Tq, D, 1>(a, p, st, dev);
     case 2:
-      return run_decode<T, D, 2>(a, p, st, dev);
+      return run_decode<Tkv, Tq, D, 2>(a, p, st, dev);
     case 4:
-      return run_decode<T, D, 4>(a, p, st, dev);
+      return run_decode<Tkv, Tq, D, 4>(a, p, st, dev);
     case 8:
-      return run_decode<T, D, 8>(a, p, st, dev);
+      return run_decode<Tkv, Tq, D, 8>(a, p, st, dev);
     default:
       return PA_ERR_UNSUPPORTED;
   }
 }
 
-template <typename T, int D>
+template <typename Tkv, typename Tq, int D>
 size_t fit_for_group(int G, int B, int warps, int want, int optin, int* stages) {
   switch (G) {
     case 1:
-      return stage_fit<T, D, 1>(B, warps, want, optin, stages);
+      return stage_fit<Tkv, Tq, D, 1>(B, warps, want, optin, stages);
     case 2:
-      return stage_fit<T, D, 2>(B, warps, want, optin, stages);
+      return stage_fit<Tkv, Tq, D, 2>(B, warps, want, optin, stages);
     case 4:
-      return stage_fit<T, D, 4>(B, warps, want, optin, stages);
+      return stage_fit<Tkv, Tq, D, 4>(B, warps, want, optin, stages);
     case 8:
-      return stage_fit<T, D, 8>(B, warps, want, optin, stages);
+      return stage_fit<Tkv, Tq, D, 8>(B, warps, want, optin, stages);
     default:
       return 0;
   }
 }
 
-size_t fit_stages(int32_t dtype, int D, int G, int B, int warps, int want, int optin, int* stages) {
-  if (dtype == PA_BF16 && D == 128) return fit_for_group<__nv_bfloat16, 128>(G, B, warps, want, optin, stages);
-  if (dtype == PA_BF16 && D == 64) return fit_for_group<__nv_bfloat16, 64>(G, B, warps, want, optin, stages);
-  if (dtype == PA_F32 && D == 64) return fit_for_group<float, 64>(G, B, warps, want, optin, stages);
-  if (dtype == PA_F32 && D == 128) return fit_for_group<float, 128>(G, B, warps, want, optin, stages);
+// The (cache type, query/output type, head size) combinations built.
+size_t fit_stages(int32_t kv_dtype, int D, int G, int B, int warps, int want, int optin, int* stages) {
+  if (kv_dtype == PA_BF16 && D == 128)
+    return fit_for_group<__nv_bfloat16, __nv_bfloat16, 128>(G, B, warps, want, optin, stages);
+  if (kv_dtype == PA_BF16 && D == 64)
+    return fit_for_group<__nv_bfloat16, __nv_bfloat16, 64>(G, B, warps, want, optin, stages);
+  if (kv_dtype == PA_F32 && D == 64) return fit_for_group<float, float, 64>(G, B, warps, want, optin, stages);
+  if (kv_dtype == PA_F32 && D == 128) return fit_for_group<float, float, 128>(G, B, warps, want, optin, stages);
+  if (kv_dtype == PA_FP8_E4M3 && D == 128)
+    return fit_for_group<__nv_fp8_e4m3, __nv_bfloat16, 128>(G, B, warps, want, optin, stages);
   return 0;
 }
 
@@ -274,7 +299,7 @@ pa_status plan_decode(int32_t dtype, int64_t B, int64_t H, int64_t Hkv, int64_t 
   pa_status s = device_info(&di, &dev);
   if (s != PA_OK) return s;
   const int G = int(H / Hkv);
-  p->warps = warps_for(G);
+  p->warps = warps_for(G, dtype);
   p->grid = di.sms * g_tuning.ctas_per_sm;
   p->smem = fit_stages(dtype, int(D), G, int(B), p->warps, g_tuning.stages, di.smem_optin, &p->stages);
   if (p->smem == 0) return PA_ERR_UNSUPPORTED;
@@ -393,6 +418,54 @@ pa_status pa_reshape_and_cache(const pa_tensor* key, const pa_tensor* value, pa_
   return err == cudaSuccess ? PA_OK : launch_status();
 }
 
+pa_status pa_reshape_and_cache_fp8(const pa_tensor* key, const pa_tensor* value, pa_tensor* k_cache,
+                                   pa_tensor* v_cache, const pa_tensor* slot_mapping, const pa_tensor* k_scale,
+                                   const pa_tensor* v_scale, const pa_opts* opts) {
+  pa_status st = check_pair(k_cache, v_cache);
+  if (st != PA_OK) return st;
+  if (k_cache->dtype != PA_FP8_E4M3) return PA_ERR_INVALID_ARG;
+  const int64_t NB = k_cache->shape[0], Hkv = k_cache->shape[1], D = k_cache->shape[3];
+  if (slot_mapping == nullptr || slot_mapping->ndim != 1 || slot_mapping->dtype != PA_I64) return PA_ERR_INVALID_ARG;
+  const int64_t T = slot_mapping->shape[0];
+  if (T < 0 || (T > 0 && (slot_mapping->stride[0] != 1 || slot_mapping->data == nullptr))) return PA_ERR_INVALID_ARG;
+  if (key == nullptr || (key->dtype != PA_BF16 && key->dtype != PA_F32)) return PA_ERR_INVALID_ARG;
+  const int32_t in_dt = key->dtype;
+  st = check_rows3(key, in_dt, T, Hkv, D);
+  if (st != PA_OK) return st;
+  st = check_rows3(value, in_dt, T, Hkv, D);
+  if (st != PA_OK) return st;
+  st = check_scale(k_scale, Hkv);
+  if (st != PA_OK) return st;
+  st = check_scale(v_scale, Hkv);
+  if (st != PA_OK) return st;
+  if (T == 0) return PA_OK;
+  constexpr int OPR = 128 / 16;  // e4m3 codes of one 128-element row: 8 vectors
+  const int64_t total = T * Hkv * OPR;
+  DeviceInfo di;
+  st = device_info(&di, nullptr);
+  if (st != PA_OK) return st;
+  const int64_t want = (total + 255) / 256;
+  const int blocks = int(want < int64_t(di.sms) * 16 ? want : int64_t(di.sms) * 16);
+  cudaStream_t s = stream_of(opts);
+  uint4* kc = static_cast<uint4*>(k_cache->data);
+  uint4* vc = static_cast<uint4*>(v_cache->data);
+  const int64_t* sl = static_cast<const int64_t*>(slot_mapping->data);
+  const float* ks = static_cast<const float*>(k_scale->data);
+  const float* vs = static_cast<const float*>(v_scale->data);
+  cudaError_t err;
+  if (in_dt == PA_BF16) {
+    err = launch_pdl(pa::reshape_and_cache_fp8_kernel<__nv_bfloat16, OPR>, dim3(blocks), dim3(256), 0, s, false,
+                     static_cast<const __nv_bfloat16*>(key->data), static_cast<const __nv_bfloat16*>(value->data),
+                     kc, vc, sl, T, int(Hkv), key->stride[0], key->stride[1], value->stride[0], value->stride[1],
+                     NB * 16, ks, vs);
+  } else {
+    err = launch_pdl(pa::reshape_and_cache_fp8_kernel<float, OPR>, dim3(blocks), dim3(256), 0, s, false,
+                     static_cast<const float*>(key->data), static_cast<const float*>(value->data), kc, vc, sl, T,
+                     int(Hkv), key->stride[0], key->stride[1], value->stride[0], value->stride[1], NB * 16, ks, vs);
+  }
+  return err == cudaSuccess ? PA_OK : launch_status();
+}
+
 pa_status pa_copy_blocks(pa_tensor* k_cache, pa_tensor* v_cache, const pa_tensor* pairs, const pa_opts* opts) {
   pa_status st = check_pair(k_cache, v_cache);
   if (st != PA_OK) return st;
@@ -432,26 +505,36 @@ pa_status pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_heads, int32_t
   pa_status st = device_info(&di, nullptr);
   if (st != PA_OK) return st;
   const int G = num_heads / num_kv_heads;
-  const int64_t workers = int64_t(di.sms) * g_tuning.ctas_per_sm * warps_for(G);
+  // an upper bound over cache types (FP8 may cap the warps lower)
+  const int64_t workers = int64_t(di.sms) * g_tuning.ctas_per_sm * (g_tuning.warps ? g_tuning.warps : default_warps(G, true));
   *bytes_out = balanced_ws_bytes(workers, G, head_size);
   return PA_OK;
 }
 
-pa_status pa_decode(pa_tensor* out, const pa_tensor* query, const pa_tensor* k_cache, const pa_tensor* v_cache,
-                    const pa_tensor* block_tables, const pa_tensor* context_lens, float scale, int32_t num_kv_heads,
-                    const pa_opts* opts) {
+// Both decode entry points: k_scale/v_scale are null unless the cache is FP8.
+static pa_status decode_impl(pa_tensor* out, const pa_tensor* query, const pa_tensor* k_cache,
+                             const pa_tensor* v_cache, const pa_tensor* block_tables, const pa_tensor* context_lens,
+                             float scale, int32_t num_kv_heads, const pa_tensor* k_scale, const pa_tensor* v_scale,
+                             const pa_opts* opts) {
   pa_status st = check_pair(k_cache, v_cache);
   if (st != PA_OK) return st;
   const int64_t NB = k_cache->shape[0], Hkv = k_cache->shape[1], D = k_cache->shape[3];
   const int32_t dt = k_cache->dtype;
+  const int32_t qdt = dt == PA_FP8_E4M3 ? PA_BF16 : dt;  // query/output type
   if (num_kv_heads != Hkv) return PA_ERR_INVALID_ARG;
   if (query == nullptr || query->ndim != 3) return PA_ERR_INVALID_ARG;
   const int64_t B = query->shape[0], H = query->shape[1];
   if (B < 0 || H <= 0 || H % Hkv) return PA_ERR_INVALID_ARG;
-  st = check_rows3(query, dt, B, H, D);
+  st = check_rows3(query, qdt, B, H, D);
   if (st != PA_OK) return st;
-  st = check_rows3(out, dt, B, H, D);
+  st = check_rows3(out, qdt, B, H, D);
   if (st != PA_OK) return st;
+  if (dt == PA_FP8_E4M3) {
+    st = check_scale(k_scale, Hkv);
+    if (st != PA_OK) return st;
+    st = check_scale(v_scale, Hkv);
+    if (st != PA_OK) return st;
+  }
   if (block_tables == nullptr || block_tables->ndim != 2 || block_tables->dtype != PA_I32 ||
       block_tables->shape[0] != B || block_tables->shape[1] < 0)
     return PA_ERR_INVALID_ARG;
@@ -500,6 +583,10 @@ pa_status pa_decode(pa_tensor* out, const pa_tensor* query, const pa_tensor* k_c
   a.num_blocks = int32_t(NB);
   a.scale_log2 = scale * 1.4426950408889634f;
   a.timeout_ns = timeout_of(opts);
+  if (dt == PA_FP8_E4M3) {
+    a.k_scale = static_cast<const float*>(k_scale->data);
+    a.v_scale = static_cast<const float*>(v_scale->data);
+  }
   if (plan.mode == pa::kFixed) {
     char* w = static_cast<char*>(opts->workspace);
     a.ws_o = reinterpret_cast<float*>(w);
@@ -517,11 +604,30 @@ pa_status pa_decode(pa_tensor* out, const pa_tensor* query, const pa_tensor* k_c
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
   cudaStream_t s = stream_of(opts);
-  if (dt == PA_BF16 && D == 128) return dispatch_group<__nv_bfloat16, 128>(int(G), a, plan, s, dev);
-  if (dt == PA_BF16 && D == 64) return dispatch_group<__nv_bfloat16, 64>(int(G), a, plan, s, dev);
-  if (dt == PA_F32 && D == 64) return dispatch_group<float, 64>(int(G), a, plan, s, dev);
-  if (dt == PA_F32 && D == 128) return dispatch_group<float, 128>(int(G), a, plan, s, dev);
+  if (dt == PA_BF16 && D == 128) return dispatch_group<__nv_bfloat16, __nv_bfloat16, 128>(int(G), a, plan, s, dev);
+  if (dt == PA_BF16 && D == 64) return dispatch_group<__nv_bfloat16, __nv_bfloat16, 64>(int(G), a, plan, s, dev);
+  if (dt == PA_F32 && D == 64) return dispatch_group<float, float, 64>(int(G), a, plan, s, dev);
+  if (dt == PA_F32 && D == 128) return dispatch_group<float, float, 128>(int(G), a, plan, s, dev);
+  if (dt == PA_FP8_E4M3 && D == 128)
+    return dispatch_group<__nv_fp8_e4m3, __nv_bfloat16, 128>(int(G), a, plan, s, dev);
   return PA_ERR_UNSUPPORTED;
+}
+
+pa_status pa_decode(pa_tensor* out, const pa_tensor* query, const pa_tensor* k_cache, const pa_tensor* v_cache,
+                    const pa_tensor* block_tables, const pa_tensor* context_lens, float scale, int32_t num_kv_heads,
+                    const pa_opts* opts) {
+  if (k_cache != nullptr && k_cache->dtype == PA_FP8_E4M3) return PA_ERR_INVALID_ARG;  // needs scales
+  return decode_impl(out, query, k_cache, v_cache, block_tables, context_lens, scale, num_kv_heads, nullptr, nullptr,
+                     opts);
+}
+
+pa_status pa_decode_fp8(pa_tensor* out, const pa_tensor* query, const pa_tensor* k_cache, const pa_tensor* v_cache,
+                        const pa_tensor* block_tables, const pa_tensor* context_lens, float scale,
+                        int32_t num_kv_heads, const pa_tensor* k_scale, const pa_tensor* v_scale,
+                        const pa_opts* opts) {
+  if (k_cache == nullptr || k_cache->dtype != PA_FP8_E4M3) return PA_ERR_INVALID_ARG;
+  return decode_impl(out, query, k_cache, v_cache, block_tables, context_lens, scale, num_kv_heads, k_scale, v_scale,
+                     opts);
 }
 
 pa_status pa_get_device_status(const pa_opts* opts, uint32_t* bits_out) {

@@ -1,5 +1,6 @@
 // Byte-moving kernels of the paged KV cache (sm_100a): the per-token cache
-// write by slot and the whole-block copy of copy-on-write.
+// write by slot (plain, or quantizing into an FP8 cache) and the whole-block
+// copy of copy-on-write.
 //
 // Both are pure HBM traffic.  Every (token, kv head) row of K or V is
 // head_size * elem bytes (256 B for bf16/128 and fp32/64) and contiguous on
@@ -42,6 +43,54 @@ __global__ void __launch_bounds__(256) reshape_and_cache_kernel(const uint4* __r
     const uint4 vv = ld_nc_v4(value + t * v_st + h * v_sh + c);
     kc[dst] = kv;
     vc[dst] = vv;
+  }
+}
+
+// Cache write into an FP8 (e4m3) cache: the same scatter, but each value is
+// stored as the e4m3 code of float(x) / scale[h] (IEEE fp32 division, round
+// to nearest even, saturating).  A thread produces one 16-byte vector of 16
+// codes from 16 input elements.  Strides are in input elements.
+template <typename Tin, int OPR>  // OPR: 16-byte code vectors per row (head_size / 16)
+__global__ void __launch_bounds__(256) reshape_and_cache_fp8_kernel(
+    const Tin* __restrict__ key, const Tin* __restrict__ value, uint4* kc, uint4* vc,
+    const int64_t* __restrict__ slots, int64_t T, int Hkv, int64_t k_st, int64_t k_sh, int64_t v_st,
+    int64_t v_sh, int64_t num_slots, const float* __restrict__ k_scale, const float* __restrict__ v_scale) {
+  pdl_wait();
+  pdl_launch_dependents();
+  constexpr int EPQ = 16 / int(sizeof(Tin));
+  const int64_t per_tok = int64_t(Hkv) * OPR;
+  const int64_t total = T * per_tok;
+  const int64_t step = int64_t(gridDim.x) * blockDim.x;
+  for (int64_t idx = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; idx < total; idx += step) {
+    const int64_t t = idx / per_tok;
+    const int r = int(idx - t * per_tok);
+    const int h = r / OPR, c = r % OPR;
+    const int64_t s = slots[t];
+    if (s == -1) continue;
+    if (s < -1 || s >= num_slots) {
+      if (h == 0 && c == 0) flag(PA_DEV_BAD_SLOT);
+      continue;
+    }
+    float kf[16], vf[16];
+    const uint4* kp = reinterpret_cast<const uint4*>(key + t * k_st + h * k_sh + c * 16);
+    const uint4* vp = reinterpret_cast<const uint4*>(value + t * v_st + h * v_sh + c * 16);
+#pragma unroll
+    for (int v = 0; v < 16 / EPQ; ++v) {
+      Elem<Tin>::unpack(ld_nc_v4(kp + v), kf + v * EPQ);
+      Elem<Tin>::unpack(ld_nc_v4(vp + v), vf + v * EPQ);
+    }
+    const float ks = k_scale[h], vs = v_scale[h];
+    uint32_t kw[4], vw[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      kw[i] = quantize_e4m3x2(__fdiv_rn(kf[4 * i], ks), __fdiv_rn(kf[4 * i + 1], ks)) |
+              (quantize_e4m3x2(__fdiv_rn(kf[4 * i + 2], ks), __fdiv_rn(kf[4 * i + 3], ks)) << 16);
+      vw[i] = quantize_e4m3x2(__fdiv_rn(vf[4 * i], vs), __fdiv_rn(vf[4 * i + 1], vs)) |
+              (quantize_e4m3x2(__fdiv_rn(vf[4 * i + 2], vs), __fdiv_rn(vf[4 * i + 3], vs)) << 16);
+    }
+    const int64_t dst = (((s >> 4) * Hkv + h) * 16 + (s & 15)) * OPR + c;
+    kc[dst] = make_uint4(kw[0], kw[1], kw[2], kw[3]);
+    vc[dst] = make_uint4(vw[0], vw[1], vw[2], vw[3]);
   }
 }
 

@@ -8,6 +8,8 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -191,6 +193,35 @@ struct Elem<__nv_bfloat16> {
     return make_uint4(w[0], w[1], w[2], w[3]);
   }
 };
+
+// FP8 e4m3 codes (a quantized KV cache): a 16-byte vector holds 16 codes.
+// Decoding goes e4m3x2 -> f16x2 -> 2 x f32, all exact; the per-head scale is
+// applied by the caller.  Only decoding exists here: codes are produced by the
+// cache write (quantize_e4m3x2).
+template <>
+struct Elem<__nv_fp8_e4m3> {
+  static constexpr int EPV = 16;
+  __device__ __forceinline__ static void unpack(const uint4& v, float* f) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[k] & 0xFFFFu), __NV_E4M3);
+      const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[k] >> 16), __NV_E4M3);
+      const float2 a = __half22float2(__half2(lo));
+      const float2 b = __half22float2(__half2(hi));
+      f[4 * k + 0] = a.x;
+      f[4 * k + 1] = a.y;
+      f[4 * k + 2] = b.x;
+      f[4 * k + 3] = b.y;
+    }
+  }
+};
+
+// Two floats -> two e4m3 codes (round to nearest even, saturating to +-448;
+// NaN stays NaN), first value in the low byte.
+__device__ __forceinline__ uint32_t quantize_e4m3x2(float a, float b) {
+  return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3));
+}
 
 __device__ __forceinline__ uint4 ld_nc_v4(const uint4* p) {
   uint4 r;

@@ -48,8 +48,10 @@ namespace pa {
 constexpr int kBS = 16;        // tokens per block (block_size)
 constexpr int kMaxWarps = 12;  // workers per CTA (registers allow 12 at G <= 4)
 
-// Warps per CTA the register budget allows without spills (8 at G = 8).
-__host__ __device__ constexpr int max_warps_for_group(int G) { return G >= 8 ? 8 : kMaxWarps; }
+// Warps per CTA the register budget allows without spills: a lane keeps the
+// query and output of G heads x EPV dims in registers (2 G EPV floats); at
+// 128 or more (bf16 G = 8, FP8 G = 4) only 8 warps fit.
+__host__ __device__ constexpr int max_warps_for(int G, int EPV) { return 2 * G * EPV >= 128 ? 8 : kMaxWarps; }
 
 enum DecodeMode : int32_t { kBalanced = 0, kFixed = 1, kNoSplit = 2 };
 
@@ -74,17 +76,23 @@ struct DecodeArgs {
   unsigned long long* ws_flag;  // balanced mode: per worker, the call tag once its partial is published
   unsigned long long call_tag;  // distinct per call, so no flag has to start at zero
   uint64_t timeout_ns;
+  const float* k_scale;  // FP8 cache: per-kv-head dequantization scales (else null)
+  const float* v_scale;
 };
 
-template <typename T, int D, int G>
+// Tkv: cache element type (fp32, bf16 or e4m3 codes); Tq: query/output type.
+template <typename Tkv, typename Tq, int D, int G>
 struct DecodeCfg {
-  static constexpr int ROWB = D * int(sizeof(T));  // bytes of one token's K (or V) for one head
-  static constexpr int LPT = ROWB / 16;            // lanes per token row
-  static constexpr int TPI = 32 / LPT;             // token rows per warp-wide 16-byte load
-  static constexpr int NT = kBS / TPI;             // tokens per lane per page
-  static constexpr int EPV = 16 / int(sizeof(T));  // elements per 16-byte vector
-  static constexpr int PAGE = kBS * ROWB;          // bytes of one page
-  static constexpr int QBYTES = G * ROWB;          // the group's query rows
+  static constexpr int ROWB = D * int(sizeof(Tkv));  // bytes of one token's K (or V) for one head
+  static constexpr int LPT = ROWB / 16;              // lanes per token row
+  static constexpr int TPI = 32 / LPT;               // token rows per warp-wide 16-byte load
+  static constexpr int NT = kBS / TPI;               // tokens per lane per page
+  static constexpr int EPV = 16 / int(sizeof(Tkv));  // cache elements per 16-byte vector (dims per lane)
+  static constexpr int QROWB = D * int(sizeof(Tq));  // bytes of one query (or output) row
+  static constexpr int EPQ = 16 / int(sizeof(Tq));   // query elements per 16-byte vector
+  static constexpr int QV = EPV / EPQ;               // query vectors per lane per head
+  static constexpr int PAGE = kBS * ROWB;            // bytes of one page
+  static constexpr int QBYTES = G * QROWB;           // the group's query rows
   static constexpr int STAGE = 2 * PAGE + QBYTES;  // K page, V page, query rows
   static constexpr int GH = G >= 2 ? G / 2 : 1;    // heads a lane holds after the butterfly
   static constexpr int PBUF = G * kBS * 4;         // probabilities of one page
@@ -92,6 +100,7 @@ struct DecodeCfg {
   static_assert(LPT >= 8 && LPT <= 32 && (LPT & (LPT - 1)) == 0, "row of 128, 256 or 512 bytes");
   static_assert(2 * NT == LPT, "lane layout");
   static_assert(G == 1 || G == 2 || G == 4 || G == 8, "group size");
+  static_assert(QV >= 1 && QV * EPQ == EPV, "query row split");
   // per-warp region: [ring: stages * STAGE][probabilities: PBUF][mbarriers: stages * 8], 128-byte multiple
   static constexpr size_t warp_bytes(int stages) {
     return (size_t(stages) * STAGE + PBUF + size_t(stages) * 8 + 127) / 128 * 128;
@@ -166,10 +175,19 @@ __device__ __forceinline__ int64_t snap_boundary(const int* S, int B, int Hkv, i
   return int64_t(S[r.i]) + int64_t(r.g) * r.np + p0;
 }
 
-template <typename T, int D, int G>
-__global__ void __launch_bounds__(max_warps_for_group(G) * 32, 1) decode_kernel(const DecodeArgs a) {
-  using C = DecodeCfg<T, D, G>;
-  constexpr int LPT = C::LPT, TPI = C::TPI, NT = C::NT, EPV = C::EPV, GH = C::GH;
+// Writes one lane's EPV output values of a row (QV 16-byte vectors of Tq).
+template <typename Tq, int EPV>
+__device__ __forceinline__ void store_out(Tq* dst, const float* f) {
+  constexpr int EPQ = 16 / int(sizeof(Tq));
+#pragma unroll
+  for (int v = 0; v < EPV / EPQ; ++v) *reinterpret_cast<uint4*>(dst + v * EPQ) = Elem<Tq>::pack(f + v * EPQ);
+}
+
+template <typename Tkv, typename Tq, int D, int G>
+__global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 1) decode_kernel(const DecodeArgs a) {
+  using C = DecodeCfg<Tkv, Tq, D, G>;
+  using T = Tkv;
+  constexpr int LPT = C::LPT, TPI = C::TPI, NT = C::NT, EPV = C::EPV, GH = C::GH, QV = C::QV, EPQ = C::EPQ;
   extern __shared__ __align__(128) unsigned char smem[];
 
   const int lane = threadIdx.x & 31;
@@ -226,7 +244,7 @@ __global__ void __launch_bounds__(max_warps_for_group(G) * 32, 1) decode_kernel(
   lo = snap_boundary(S, B, Hkv, lo, W, a.mode, a.part_pages);
   hi = snap_boundary(S, B, Hkv, hi, W, a.mode, a.part_pages);
   const uint64_t pol = policy_evict_first();
-  const T* qg = reinterpret_cast<const T*>(a.q);
+  const Tq* qg = reinterpret_cast<const Tq*>(a.q);
   const unsigned char* kcb = reinterpret_cast<const unsigned char*>(a.kc);
   const unsigned char* vcb = reinterpret_cast<const unsigned char*>(a.vc);
 
@@ -262,8 +280,8 @@ __global__ void __launch_bounds__(max_warps_for_group(G) * 32, 1) decode_kernel(
         if (p_seg_first) {
 #pragma unroll
           for (int j = 0; j < G; ++j)
-            bulk_g2s(smem_u32(st + 2 * C::PAGE + j * C::ROWB),
-                     qg + int64_t(pc.i) * a.q_sb + int64_t(pc.g * G + j) * a.q_sh, C::ROWB, bar, pol);
+            bulk_g2s(smem_u32(st + 2 * C::PAGE + j * C::QROWB),
+                     qg + int64_t(pc.i) * a.q_sb + int64_t(pc.g * G + j) * a.q_sh, C::QROWB, bar, pol);
         }
       }
       // advance the producer cursor
@@ -296,6 +314,7 @@ __global__ void __launch_bounds__(max_warps_for_group(G) * 32, 1) decode_kernel(
     float q[G][EPV];
     float o[G][EPV];
     float m[G], lpart[GH];
+    float vscale = 1.f;
     int ctx_i = 0;
     uint32_t phase = 0;  // bit s = parity of the next wait on stage s
     int s = 0;
@@ -316,13 +335,17 @@ __global__ void __launch_bounds__(max_warps_for_group(G) * 32, 1) decode_kernel(
 
       if (seg_first) {
         const uint4* qs = reinterpret_cast<const uint4*>(st + 2 * C::PAGE);
+        // FP8 cache: fold the K dequantization scale into the query
+        const float qscale = a.scale_log2 * (a.k_scale ? __ldg(a.k_scale + cc.g) : 1.f);
+        vscale = a.v_scale ? __ldg(a.v_scale + cc.g) : 1.f;
 #pragma unroll
         for (int j = 0; j < G; ++j) {
           float f[EPV];
-          Elem<T>::unpack(qs[j * LPT + c], f);
+#pragma unroll
+          for (int v = 0; v < QV; ++v) Elem<Tq>::unpack(qs[j * (C::QROWB / 16) + c * QV + v], f + v * EPQ);
 #pragma unroll
           for (int e = 0; e < EPV; ++e) {
-            q[j][e] = f[e] * a.scale_log2;
+            q[j][e] = f[e] * qscale;
             o[j][e] = 0.f;
           }
           m[j] = -INFINITY;
@@ -499,14 +522,14 @@ __global__ void __launch_bounds__(max_warps_for_group(G) * 32, 1) decode_kernel(
         const bool whole_row = (seg_p0 == 0) && last_of_row;
         if (whole_row) {
           if (tg == 0) {
-            T* ob = reinterpret_cast<T*>(a.out) + int64_t(cc.i) * a.o_sb;
+            Tq* ob = reinterpret_cast<Tq*>(a.out) + int64_t(cc.i) * a.o_sb;
 #pragma unroll
             for (int j = 0; j < G; ++j) {
-              const float inv = 1.f / lall[j];
+              const float inv = vscale / lall[j];
               float f[EPV];
 #pragma unroll
               for (int e = 0; e < EPV; ++e) f[e] = o[j][e] * inv;
-              *reinterpret_cast<uint4*>(ob + int64_t(cc.g * G + j) * a.o_sh + c * EPV) = Elem<T>::pack(f);
+              store_out<Tq, EPV>(ob + int64_t(cc.g * G + j) * a.o_sh + c * EPV, f);
             }
           }
         } else if (a.mode == kFixed) {
@@ -515,7 +538,7 @@ __global__ void __launch_bounds__(max_warps_for_group(G) * 32, 1) decode_kernel(
           if (tg == 0) {
 #pragma unroll
             for (int j = 0; j < G; ++j) {
-              const float inv = 1.f / lall[j];
+              const float inv = vscale / lall[j];
               float4* dst = reinterpret_cast<float4*>(a.ws_o + (base + j * a.P_max) * D + c * EPV);
 #pragma unroll
               for (int e4 = 0; e4 < EPV / 4; ++e4)
@@ -539,7 +562,7 @@ __global__ void __launch_bounds__(max_warps_for_group(G) * 32, 1) decode_kernel(
           if (tg == 0) {
 #pragma unroll
             for (int j = 0; j < G; ++j) {
-              const float inv = 1.f / lall[j];
+              const float inv = vscale / lall[j];
               float4* dst = reinterpret_cast<float4*>(a.ws_o + (wid * G + j) * D + c * EPV);
 #pragma unroll
               for (int e4 = 0; e4 < EPV / 4; ++e4)
@@ -575,7 +598,7 @@ __global__ void __launch_bounds__(max_warps_for_group(G) * 32, 1) decode_kernel(
           for (int j = 0; j < G; ++j) {
             mx[j] = (m[j] + log2f(lall[j])) * 0.69314718055994530942f;
             wsum[j] = 1.f;
-            const float inv = 1.f / lall[j];
+            const float inv = vscale / lall[j];
 #pragma unroll
             for (int e = 0; e < EPV; ++e) acc[j][e] = o[j][e] * inv;
           }
@@ -607,14 +630,14 @@ __global__ void __launch_bounds__(max_warps_for_group(G) * 32, 1) decode_kernel(
             }
           }
           if (tg == 0) {
-            T* ob = reinterpret_cast<T*>(a.out) + int64_t(cc.i) * a.o_sb;
+            Tq* ob = reinterpret_cast<Tq*>(a.out) + int64_t(cc.i) * a.o_sb;
 #pragma unroll
             for (int j = 0; j < G; ++j) {
               const float inv = 1.f / wsum[j];
               float f[EPV];
 #pragma unroll
               for (int e = 0; e < EPV; ++e) f[e] = acc[j][e] * inv;
-              *reinterpret_cast<uint4*>(ob + int64_t(cc.g * G + j) * a.o_sh + c * EPV) = Elem<T>::pack(f);
+              store_out<Tq, EPV>(ob + int64_t(cc.g * G + j) * a.o_sh + c * EPV, f);
             }
           }
         }
@@ -640,10 +663,11 @@ __global__ void __launch_bounds__(max_warps_for_group(G) * 32, 1) decode_kernel(
   // ---- sequences with no context: zero output rows ----
   for (int64_t i = wid; i < B; i += nworkers) {
     if (S[i + 1] != S[i]) continue;
-    T* ob = reinterpret_cast<T*>(a.out) + i * a.o_sb;
-    for (int idx = lane; idx < H * LPT; idx += 32) {
-      const int h = idx / LPT, cc2 = idx % LPT;
-      *reinterpret_cast<uint4*>(ob + int64_t(h) * a.o_sh + cc2 * EPV) = make_uint4(0, 0, 0, 0);
+    Tq* ob = reinterpret_cast<Tq*>(a.out) + i * a.o_sb;
+    constexpr int OVR = C::QROWB / 16;  // 16-byte vectors per output row
+    for (int idx = lane; idx < H * OVR; idx += 32) {
+      const int h = idx / OVR, cc2 = idx % OVR;
+      *reinterpret_cast<uint4*>(ob + int64_t(h) * a.o_sh + cc2 * EPQ) = make_uint4(0, 0, 0, 0);
     }
   }
 }

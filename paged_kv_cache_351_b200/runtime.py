@@ -15,16 +15,20 @@ from typing import Optional, Sequence, Tuple
 import numpy as np
 import torch
 
-from . import Allocator, pa_copy_blocks, pa_decode, pa_decode_workspace_bytes, pa_reshape_and_cache
+from . import (Allocator, pa_copy_blocks, pa_decode, pa_decode_fp8, pa_decode_workspace_bytes,
+               pa_reshape_and_cache, pa_reshape_and_cache_fp8)
 
-_DT = {"f32": torch.float32, "bf16": torch.bfloat16}
+_DT = {"f32": torch.float32, "bf16": torch.bfloat16, "fp8": torch.float8_e4m3fn}
 
 
 class PagedKVCacheGPU:
     """K/V pools [num_blocks, num_kv_heads, block_size, head_size] on one device."""
 
     def __init__(self, num_blocks: int, num_kv_heads: int, head_size: int, dtype: str = "bf16",
-                 block_size: int = 16, free_order: Optional[Sequence[int]] = None, device="cuda"):
+                 block_size: int = 16, free_order: Optional[Sequence[int]] = None, device="cuda",
+                 k_scale=None, v_scale=None):
+        """dtype "fp8" stores e4m3 codes and needs per-kv-head k_scale/v_scale
+        (float32 [num_kv_heads])."""
         self.num_blocks, self.num_kv_heads, self.head_size = num_blocks, num_kv_heads, head_size
         self.block_size, self.dtype, self.device = block_size, dtype, torch.device(device)
         shape = (num_blocks, num_kv_heads, block_size, head_size)
@@ -32,6 +36,12 @@ class PagedKVCacheGPU:
         self.v_cache = torch.empty(shape, dtype=_DT[dtype], device=self.device)
         self.alloc = Allocator(num_blocks, block_size, free_order)
         self._ws = None
+        self.k_scale = self.v_scale = None
+        if dtype == "fp8":
+            if k_scale is None or v_scale is None:
+                raise ValueError("an fp8 cache needs k_scale and v_scale")
+            self.k_scale = torch.as_tensor(k_scale, dtype=torch.float32).to(self.device).contiguous()
+            self.v_scale = torch.as_tensor(v_scale, dtype=torch.float32).to(self.device).contiguous()
 
     # -- host bookkeeping ------------------------------------------------------
     def add(self, seq: int) -> None:
@@ -58,7 +68,11 @@ class PagedKVCacheGPU:
         copied blocks), then the tokens' K/V at their slots."""
         if pairs is not None and pairs.shape[0]:
             pa_copy_blocks(self.k_cache, self.v_cache, pairs, stream=stream)
-        pa_reshape_and_cache(key, value, self.k_cache, self.v_cache, slots, stream=stream)
+        if self.dtype == "fp8":
+            pa_reshape_and_cache_fp8(key, value, self.k_cache, self.v_cache, slots, self.k_scale, self.v_scale,
+                                     stream=stream)
+        else:
+            pa_reshape_and_cache(key, value, self.k_cache, self.v_cache, slots, stream=stream)
 
     def workspace(self, num_seqs: int, num_heads: int, max_blocks: int, partition_tokens: int = 0):
         n = pa_decode_workspace_bytes(num_seqs, num_heads, self.num_kv_heads, self.head_size, max_blocks,
@@ -74,6 +88,11 @@ class PagedKVCacheGPU:
                workspace=None) -> torch.Tensor:
         if workspace is None:
             workspace = self.workspace(query.shape[0], query.shape[1], block_tables.shape[1], partition_tokens)
-        pa_decode(out, query, self.k_cache, self.v_cache, block_tables, context_lens, scale, self.num_kv_heads,
-                  workspace=workspace, partition_tokens=partition_tokens, stream=stream)
+        if self.dtype == "fp8":
+            pa_decode_fp8(out, query, self.k_cache, self.v_cache, block_tables, context_lens, scale,
+                          self.num_kv_heads, self.k_scale, self.v_scale, workspace=workspace,
+                          partition_tokens=partition_tokens, stream=stream)
+        else:
+            pa_decode(out, query, self.k_cache, self.v_cache, block_tables, context_lens, scale, self.num_kv_heads,
+                      workspace=workspace, partition_tokens=partition_tokens, stream=stream)
         return out

@@ -17,9 +17,9 @@ import torch
 
 import paged_kv_cache_351_b200 as pa
 from oracle.attention import widen
-from workloads import AddOp, AppendOp, ForkOp, Plan, query_values, stream_kv
+from workloads import AddOp, AppendOp, ForkOp, Plan, kv_scales, query_values, stream_kv
 
-TORCH_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16}
+TORCH_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16, "fp8": torch.float8_e4m3fn}
 TOL = {"f32": 1e-5, "bf16": 1e-2}
 
 
@@ -35,6 +35,8 @@ def to_host_raw(t: torch.Tensor, dtype: str) -> np.ndarray:
     t = t.detach().cpu().contiguous()
     if dtype == "f32":
         return t.numpy()
+    if dtype == "fp8":
+        return t.view(torch.uint8).numpy()
     return t.view(torch.int16).numpy().view(np.uint16)
 
 
@@ -52,15 +54,27 @@ class DeviceState:
     step_slots: Optional[torch.Tensor] = None  # int64 [B] device: slots of the step's new tokens
     step_key: Optional[torch.Tensor] = None
     step_value: Optional[torch.Tensor] = None
+    k_scale: Optional[torch.Tensor] = None  # FP8 cache only
+    v_scale: Optional[torch.Tensor] = None
+
+    def write(self, key, value, slots):
+        if self.k_scale is not None:
+            pa.pa_reshape_and_cache_fp8(key, value, self.k_cache, self.v_cache, slots, self.k_scale, self.v_scale)
+        else:
+            pa.pa_reshape_and_cache(key, value, self.k_cache, self.v_cache, slots)
 
 
 def build_device_state(plan: Plan, device="cuda", include_step=True, write_step=True,
                        stop_after: Optional[int] = None) -> DeviceState:
     w = plan.workload
-    dt = TORCH_DTYPE[w.dtype]
+    dt = TORCH_DTYPE[w.cache_dtype]
     shape = (plan.num_blocks, w.num_kv_heads, w.block_size, w.head_size)
     k_cache = torch.empty(shape, dtype=dt, device=device)
     v_cache = torch.empty(shape, dtype=dt, device=device)
+    ks = vs = None
+    if w.cache_dtype == "fp8":
+        ks_np, vs_np = kv_scales(plan)
+        ks, vs = torch.from_numpy(ks_np).to(device), torch.from_numpy(vs_np).to(device)
     alloc = pa.Allocator(plan.num_blocks, w.block_size, plan.free_order)
     cow_all: List[tuple] = []
 
@@ -78,7 +92,10 @@ def build_device_state(plan: Plan, device="cuda", include_step=True, write_step=
             slots = torch.from_numpy(np.concatenate(pend_slots)).to(device)
             key = to_device_values(np.concatenate(pend_k), w.dtype, device)
             value = to_device_values(np.concatenate(pend_v), w.dtype, device)
-            pa.pa_reshape_and_cache(key, value, k_cache, v_cache, slots)
+            if ks is not None:
+                pa.pa_reshape_and_cache_fp8(key, value, k_cache, v_cache, slots, ks, vs)
+            else:
+                pa.pa_reshape_and_cache(key, value, k_cache, v_cache, slots)
         pend_slots.clear(), pend_k.clear(), pend_v.clear(), pend_pairs.clear(), pend_seqs.clear()
 
     ops = list(plan.setup_ops) + (list(plan.step_ops) if include_step else [])
@@ -113,7 +130,7 @@ def build_device_state(plan: Plan, device="cuda", include_step=True, write_step=
     max_nb = plan.max_blocks_per_seq
     tables, lens = alloc.block_tables(plan.batch, max_nb)
     st = DeviceState(plan, alloc, k_cache, v_cache, torch.from_numpy(tables).to(device),
-                     torch.from_numpy(lens).to(device), tables, lens, cow_all)
+                     torch.from_numpy(lens).to(device), tables, lens, cow_all, k_scale=ks, v_scale=vs)
     if include_step and plan.step_ops:
         st.step_slots = torch.from_numpy(np.concatenate(step_slots)).to(device)
         ks, vs = [], []
@@ -135,8 +152,13 @@ def decode_on_device(st: DeviceState, query: torch.Tensor, partition_tokens: int
     n = pa.pa_decode_workspace_bytes(st.plan.B, w.num_heads, w.num_kv_heads, w.head_size,
                                      st.block_tables.shape[1], partition_tokens)
     ws = torch.empty(max(n, 256), dtype=torch.uint8, device=query.device) if n else None
-    pa.pa_decode(out, query, st.k_cache, st.v_cache, st.block_tables, st.context_lens,
-                 1.0 / np.sqrt(w.head_size), w.num_kv_heads, workspace=ws, partition_tokens=partition_tokens)
+    if st.k_scale is not None:
+        pa.pa_decode_fp8(out, query, st.k_cache, st.v_cache, st.block_tables, st.context_lens,
+                         1.0 / np.sqrt(w.head_size), w.num_kv_heads, st.k_scale, st.v_scale, workspace=ws,
+                         partition_tokens=partition_tokens)
+    else:
+        pa.pa_decode(out, query, st.k_cache, st.v_cache, st.block_tables, st.context_lens,
+                     1.0 / np.sqrt(w.head_size), w.num_kv_heads, workspace=ws, partition_tokens=partition_tokens)
     return out
 
 

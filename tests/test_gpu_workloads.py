@@ -29,9 +29,11 @@ pytestmark = pytest.mark.gpu
 def _check_cache(st, cache_o, blocks):
     w = st.plan.workload
     idx = torch.tensor(sorted(blocks), dtype=torch.int64, device="cuda")
-    kh = to_host_raw(st.k_cache.index_select(0, idx), w.dtype)
-    vh = to_host_raw(st.v_cache.index_select(0, idx), w.dtype)
-    view = np.uint32 if w.dtype == "f32" else np.uint16
+    kc = st.k_cache.view(torch.uint8) if w.cache_dtype == "fp8" else st.k_cache
+    vc = st.v_cache.view(torch.uint8) if w.cache_dtype == "fp8" else st.v_cache
+    kh = to_host_raw(kc.index_select(0, idx), "fp8" if w.cache_dtype == "fp8" else w.dtype)
+    vh = to_host_raw(vc.index_select(0, idx), "fp8" if w.cache_dtype == "fp8" else w.dtype)
+    view = {"f32": np.uint32, "bf16": np.uint16, "fp8": np.uint8}[w.cache_dtype]
     for r, b in enumerate(sorted(blocks)):
         wr = cache_o.written(b)
         assert np.array_equal(kh[r][:, wr].view(view), cache_o.k_page(b)[:, wr].view(view)), b
@@ -43,7 +45,7 @@ def _run_workload(name, sample_rows=None, modes=(0, 512), check_all_blocks=True)
     st = build_device_state(plan, write_step=False)
     # the step: write the new tokens, then decode
     if st.step_slots is not None:
-        pa.pa_reshape_and_cache(st.step_key, st.step_value, st.k_cache, st.v_cache, st.step_slots)
+        st.write(st.step_key, st.step_value, st.step_slots)
     alloc_o, cache_o, log = replay(plan)
     assert np.array_equal(st.tables_host, block_table_array(alloc_o, plan.batch, plan.max_blocks_per_seq))
     assert np.array_equal(st.lens_host, plan.context_lens)
@@ -87,6 +89,17 @@ def test_parallel_sampling_13b():
     # 3 copies per prompt whose length is not a multiple of the block size
     plen = [op.n for op in st.plan.setup_ops if hasattr(op, "n") and op.n > 64]
     assert len(st.cow_pairs) == 3 * sum(1 for n in plen if n % 16)
+
+
+def test_llama7b_bs64_fp8():
+    _run_workload("llama7b_bs64_fp8", modes=(0, -1, 512))
+
+
+def test_gqa_bs256_fp8():
+    plan = make_plan("gqa_bs256_fp8")
+    order = np.argsort(-plan.context_lens)
+    rows = sorted(set(order[:6].tolist() + order[-4:].tolist() + list(range(0, 256, 16))))
+    _run_workload("gqa_bs256_fp8", sample_rows=rows, modes=(0, 512), check_all_blocks=False)
 
 
 def test_long_ctx_splitk():
