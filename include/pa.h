@@ -261,11 +261,13 @@ typedef struct pa_allocator pa_allocator;
 
 typedef struct {
   int32_t num_blocks;
-  int32_t num_free;
+  int32_t num_free;      /* blocks available to allocation: free + evictable */
   int32_t num_seqs;
   int32_t block_size;
-  int64_t num_tokens;  /* sum of sequence lengths (shared tokens counted per sequence) */
-  int64_t waste_slots; /* unused slots of blocks in use (bs minus the most any holder filled) */
+  int64_t num_tokens;    /* sum of sequence lengths (shared tokens counted per sequence) */
+  int64_t waste_slots;   /* unused slots of blocks in use (bs minus the most any holder filled) */
+  int32_t num_cached;    /* registered prefix-cache blocks (held or evictable) */
+  int32_t num_evictable; /* registered blocks nobody holds */
 } pa_alloc_stats;
 
 pa_status pa_alloc_create(int32_t num_blocks, int32_t block_size, const int32_t* free_order, pa_allocator** out);
@@ -282,6 +284,35 @@ pa_status pa_seq_append(pa_allocator* a, int64_t seq_id, int32_t n_tokens, int64
 pa_status pa_seq_append_batch(pa_allocator* a, const int64_t* seq_ids, const int32_t* n_tokens, int32_t n,
                               int64_t* slots_out, int64_t* cow_pairs_out, int32_t* n_cow_out, int32_t* n_done_out);
 pa_status pa_seq_fork(pa_allocator* a, int64_t parent, int64_t child);
+
+/* Prefix caching.  The pages give the effect — requests reuse the computed
+ * KV of an identical prefix such as a system prompt (gitcode walkthrough,
+ * section 2.2, "Prefix caching (APC)"); blocks can be shared across requests
+ * (agientry.com overview, opening section) — and this is the mechanism:
+ *  - a sequence whose token ids are all known (created by pa_seq_add or
+ *    pa_seq_add_prefix and extended only by pa_seq_append_tokens) registers
+ *    each block when it becomes full, under the key (previous block of the
+ *    sequence or -1, the block's token ids), if that previous block is
+ *    registered (or it is the first block) and the key is not taken; so a key
+ *    match means the whole prefix matches, exactly (no hashing shortcut);
+ *  - pa_seq_add_prefix(seq, tokens, n) creates the sequence on the longest
+ *    chain of registered keys along tokens, at most (n - 1) / bs blocks so
+ *    one token is left to compute; *n_cached_out = tokens reused (a multiple
+ *    of bs).  The caller then appends tokens[*n_cached_out:] with
+ *    pa_seq_append_tokens and writes only their K/V;
+ *  - a registered block whose count drops to 0 becomes evictable (kept in
+ *    least-recently-freed order) instead of free; allocation takes the free
+ *    stack first, then evicts the least recently freed evictable block;
+ *    unregistering a block (eviction) unregisters its registered children in
+ *    increasing block order, depth first, and frees those nobody holds;
+ *  - pa_seq_append (token ids unknown) turns a sequence's registration off.
+ * Without these calls the allocator behaves exactly as described above. */
+pa_status pa_seq_add_prefix(pa_allocator* a, int64_t seq_id, const int64_t* tokens, int32_t n_tokens,
+                            int32_t* n_cached_out);
+pa_status pa_seq_append_tokens(pa_allocator* a, int64_t seq_id, const int64_t* tokens, int32_t n_tokens,
+                               int64_t* slots_out, int64_t* cow_pair_out, int32_t* n_cow_out);
+/* Evictable blocks, least recently freed first. */
+pa_status pa_alloc_evictable(const pa_allocator* a, int32_t* out, int32_t cap, int32_t* n_out);
 pa_status pa_seq_free(pa_allocator* a, int64_t seq_id);
 pa_status pa_seq_len(const pa_allocator* a, int64_t seq_id, int32_t* len_out);
 pa_status pa_seq_block_table(const pa_allocator* a, int64_t seq_id, int32_t* out, int32_t cap, int32_t* n_out);

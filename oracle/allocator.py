@@ -25,11 +25,33 @@ What the pages leave open, and the reading taken here:
 * ``append`` is all-or-nothing: if the free stack cannot cover every block the
   call needs, it raises ``OutOfBlocks`` and changes nothing.
 * slot of logical position t of a sequence: ``table[t // bs] * bs + t % bs``.
+
+Prefix caching (gitcode repo walkthrough, section 2.2: requests reuse the
+already computed KV of an identical prefix such as a system prompt;
+agientry.com overview, opening section: blocks can be shared across requests)
+— the pages give the effect, not the mechanism; the reading taken here:
+
+* sequences created with ``add_prefix`` and extended with ``append_tokens``
+  carry their token ids; when such a block becomes full it is registered
+  under the key (parent block, its token ids), the parent being the
+  sequence's previous block (-1 for the first).  A block is registered only
+  if its parent is registered (or it is a first block) and no block holds the
+  key yet, so a key match implies the whole prefix matches, exactly.
+* ``add_prefix`` follows the longest chain of registered keys along the
+  prompt, over at most (n - 1) // bs full blocks so that one token is left to
+  compute, and starts the sequence on those blocks (one more reference each).
+* a registered block whose count drops to 0 is not freed but becomes
+  evictable, kept in least-recently-freed order; blocks are taken from the
+  free stack first, then by evicting the least recently freed evictable
+  block.  Evicting (or otherwise unregistering) a block unregisters its
+  registered children in increasing block order, depth first; an evictable
+  child that loses its key goes onto the free stack.
 """
 
 from __future__ import annotations
 
-from typing import Dict, List, Optional, Sequence, Tuple
+from collections import OrderedDict
+from typing import Dict, List, Optional, Sequence, Set, Tuple
 
 
 class AllocatorError(ValueError):
@@ -56,10 +78,26 @@ class BlockAllocator:
         self._ref: List[int] = [0] * num_blocks
         self._table: Dict[int, List[int]] = {}
         self._len: Dict[int, int] = {}
+        # prefix caching
+        self._tokens: Dict[int, Optional[List[int]]] = {}  # None: token ids unknown
+        self._cache: Dict[Tuple[int, Tuple[int, ...]], int] = {}
+        self._key_of: Dict[int, Tuple[int, Tuple[int, ...]]] = {}
+        self._children: Dict[int, Set[int]] = {}
+        self._evictable: "OrderedDict[int, None]" = OrderedDict()
 
     # -- queries ---------------------------------------------------------
     def num_free(self) -> int:
-        return len(self._free)
+        """Blocks available to allocation: free plus evictable."""
+        return len(self._free) + len(self._evictable)
+
+    def num_cached(self) -> int:
+        return len(self._cache)
+
+    def num_evictable(self) -> int:
+        return len(self._evictable)
+
+    def is_cached(self, block: int) -> bool:
+        return block in self._key_of
 
     def refcount(self, block: int) -> int:
         return self._ref[block]
@@ -83,6 +121,74 @@ class BlockAllocator:
             raise AllocatorError(f"sequence {seq} exists")
         self._table[seq] = []
         self._len[seq] = 0
+        self._tokens[seq] = []
+
+    # -- prefix-cache primitives ------------------------------------------
+    def _take_block(self) -> int:
+        if self._free:
+            return self._free.pop()
+        b, _ = self._evictable.popitem(last=False)
+        self._unregister(b)
+        return b
+
+    def _unregister(self, b: int) -> None:
+        key = self._key_of.pop(b)
+        del self._cache[key]
+        parent = key[0]
+        if parent >= 0 and parent in self._children:
+            self._children[parent].discard(b)
+        for c in sorted(self._children.pop(b, set())):
+            self._unregister_subtree(c)
+
+    def _unregister_subtree(self, c: int) -> None:
+        self._unregister(c)
+        if c in self._evictable:
+            del self._evictable[c]
+            self._free.append(c)
+
+    def _register(self, b: int, parent: int, toks: Tuple[int, ...]) -> None:
+        if parent >= 0 and parent not in self._key_of:
+            return
+        key = (parent, toks)
+        if key in self._cache or b in self._key_of:
+            return
+        self._cache[key] = b
+        self._key_of[b] = key
+        if parent >= 0:
+            self._children.setdefault(parent, set()).add(b)
+
+    def _release(self, b: int) -> None:
+        self._ref[b] -= 1
+        if self._ref[b] == 0:
+            if b in self._key_of:
+                self._evictable[b] = None
+            else:
+                self._free.append(b)
+
+    def add_prefix(self, seq: int, tokens: Sequence[int]) -> int:
+        """Add a sequence whose prompt is ``tokens``; reuse the longest chain
+        of registered full blocks (leaving at least one token).  Returns the
+        number of prompt tokens already in the cache (a multiple of bs)."""
+        if seq in self._table:
+            raise AllocatorError(f"sequence {seq} exists")
+        bs = self.block_size
+        tokens = [int(t) for t in tokens]
+        hits: List[int] = []
+        parent = -1
+        for k in range(max(0, (len(tokens) - 1) // bs)):
+            b = self._cache.get((parent, tuple(tokens[k * bs:(k + 1) * bs])))
+            if b is None:
+                break
+            hits.append(b)
+            parent = b
+        for b in hits:
+            if self._ref[b] == 0:
+                del self._evictable[b]
+            self._ref[b] += 1
+        self._table[seq] = list(hits)
+        self._len[seq] = len(hits) * bs
+        self._tokens[seq] = tokens[:len(hits) * bs]
+        return len(hits) * bs
 
     def _blocks_needed(self, seq: int, n: int) -> int:
         bs = self.block_size
@@ -102,28 +208,48 @@ class BlockAllocator:
             raise AllocatorError(f"unknown sequence {seq}")
         if n < 0:
             raise AllocatorError("negative token count")
-        if self._blocks_needed(seq, n) > len(self._free):
-            raise OutOfBlocks(f"sequence {seq}: {n} tokens need more than {len(self._free)} free blocks")
+        return self._append(seq, n, None)
+
+    def append_tokens(self, seq: int, tokens: Sequence[int]) -> Tuple[List[int], List[Tuple[int, int]]]:
+        """Append tokens with known ids (the sequence's ids so far must be
+        known); blocks that become full are registered for prefix reuse."""
+        if seq not in self._table:
+            raise AllocatorError(f"unknown sequence {seq}")
+        if self._tokens.get(seq) is None:
+            raise AllocatorError(f"sequence {seq} has tokens of unknown id")
+        return self._append(seq, len(tokens), [int(t) for t in tokens])
+
+    def _append(self, seq: int, n: int, ids: Optional[List[int]]):
+        if self._blocks_needed(seq, n) > self.num_free():
+            raise OutOfBlocks(f"sequence {seq}: {n} tokens need more than {self.num_free()} free blocks")
         bs = self.block_size
         table = self._table[seq]
+        if ids is None:
+            self._tokens[seq] = None
+        toks = self._tokens[seq]
         slots: List[int] = []
         cow: List[Tuple[int, int]] = []
-        for _ in range(n):
+        for k in range(n):
             pos = self._len[seq]
             if pos % bs == 0:
-                b = self._free.pop()
+                b = self._take_block()
                 self._ref[b] = 1
                 table.append(b)
             else:
                 last = table[-1]
                 if self._ref[last] > 1:
-                    b = self._free.pop()
+                    b = self._take_block()
                     self._ref[b] = 1
                     self._ref[last] -= 1
                     table[-1] = b
                     cow.append((last, b))
             slots.append(table[pos // bs] * bs + pos % bs)
             self._len[seq] = pos + 1
+            if toks is not None:
+                toks.append(ids[k])
+                if (pos + 1) % bs == 0:
+                    j = pos // bs
+                    self._register(table[j], table[j - 1] if j else -1, tuple(toks[j * bs:(j + 1) * bs]))
         return slots, cow
 
     def fork(self, parent: int, child: int) -> None:
@@ -135,6 +261,8 @@ class BlockAllocator:
             raise AllocatorError(f"sequence {child} exists")
         self._table[child] = list(self._table[parent])
         self._len[child] = self._len[parent]
+        t = self._tokens.get(parent)
+        self._tokens[child] = None if t is None else list(t)
         for b in self._table[child]:
             self._ref[b] += 1
 
@@ -142,10 +270,9 @@ class BlockAllocator:
         if seq not in self._table:
             raise AllocatorError(f"unknown sequence {seq}")
         for b in self._table.pop(seq):
-            self._ref[b] -= 1
-            if self._ref[b] == 0:
-                self._free.append(b)
+            self._release(b)
         del self._len[seq]
+        del self._tokens[seq]
 
     # -- statistics and invariants ----------------------------------------
     def waste_slots(self) -> int:
@@ -173,6 +300,14 @@ class BlockAllocator:
         free = set(self._free)
         if len(free) != len(self._free):
             raise AssertionError("a block is on the free stack twice")
+        evict = set(self._evictable)
         used = {b for b in range(self.num_blocks) if self._ref[b] > 0}
-        if free & used or (free | used) != set(range(self.num_blocks)):
-            raise AssertionError("free and used blocks do not partition the pool")
+        if (free & used) or (free & evict) or (evict & used) or (free | used | evict) != set(range(self.num_blocks)):
+            raise AssertionError("free, evictable and used blocks do not partition the pool")
+        for key, b in self._cache.items():
+            if self._key_of.get(b) != key:
+                raise AssertionError("cache key and block disagree")
+            if key[0] >= 0 and key[0] not in self._key_of:
+                raise AssertionError("a registered block's parent is not registered")
+        if not evict <= set(self._key_of):
+            raise AssertionError("an evictable block is not registered")

@@ -259,6 +259,33 @@ class Allocator:
     def fork(self, parent: int, child: int) -> None:
         _check(_lib_handle.pa_seq_fork(self._h, parent, child), "pa_seq_fork")
 
+    def add_prefix(self, seq: int, tokens: Sequence[int]) -> int:
+        """Prefix caching: add a sequence on the longest registered chain of
+        its prompt's full blocks; returns the number of tokens reused."""
+        ids = np.ascontiguousarray(np.asarray(tokens, np.int64))
+        n = ctypes.c_int32(0)
+        _check(_lib_handle.pa_seq_add_prefix(self._h, seq, _i64p(ids) if ids.size else None, int(ids.size),
+                                             ctypes.byref(n)), "pa_seq_add_prefix")
+        return int(n.value)
+
+    def append_tokens(self, seq: int, tokens: Sequence[int]):
+        """Append tokens with known ids (blocks register when full)."""
+        ids = np.ascontiguousarray(np.asarray(tokens, np.int64))
+        n = int(ids.size)
+        slots = np.zeros(max(n, 1), np.int64)
+        pair = np.zeros(2, np.int64)
+        ncow = ctypes.c_int32(0)
+        _check(_lib_handle.pa_seq_append_tokens(self._h, seq, _i64p(ids) if n else _i64p(slots), n, _i64p(slots),
+                                                _i64p(pair), ctypes.byref(ncow)), "pa_seq_append_tokens")
+        return slots[:n], ([(int(pair[0]), int(pair[1]))] if ncow.value else [])
+
+    def evictable(self):
+        out = np.zeros(max(1, self.num_blocks), np.int32)
+        n = ctypes.c_int32(0)
+        _check(_lib_handle.pa_alloc_evictable(self._h, _i32p(out), self.num_blocks, ctypes.byref(n)),
+               "pa_alloc_evictable")
+        return out[: n.value].tolist()
+
     def free(self, seq: int) -> None:
         _check(_lib_handle.pa_seq_free(self._h, seq), "pa_seq_free")
 

@@ -40,6 +40,8 @@ class PaAllocStats(ctypes.Structure):
         ("block_size", c_int32),
         ("num_tokens", c_int64),
         ("waste_slots", c_int64),
+        ("num_cached", c_int32),
+        ("num_evictable", c_int32),
     ]
 
 
@@ -78,6 +80,9 @@ SIGNATURES = {
     "pa_seq_append": (c_int32, [_A, c_int64, c_int32, _I64P, _I64P, _I32P]),
     "pa_seq_append_batch": (c_int32, [_A, _I64P, _I32P, c_int32, _I64P, _I64P, _I32P, _I32P]),
     "pa_seq_fork": (c_int32, [_A, c_int64, c_int64]),
+    "pa_seq_add_prefix": (c_int32, [_A, c_int64, _I64P, c_int32, _I32P]),
+    "pa_seq_append_tokens": (c_int32, [_A, c_int64, _I64P, c_int32, _I64P, _I64P, _I32P]),
+    "pa_alloc_evictable": (c_int32, [_A, _I32P, c_int32, _I32P]),
     "pa_seq_free": (c_int32, [_A, c_int64]),
     "pa_seq_len": (c_int32, [_A, c_int64, _I32P]),
     "pa_seq_block_table": (c_int32, [_A, c_int64, _I32P, c_int32, _I32P]),

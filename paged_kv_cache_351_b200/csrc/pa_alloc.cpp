@@ -10,9 +10,12 @@
 // arguments and its block needs before changing anything, so a failed call
 // leaves the state untouched.
 
+#include <algorithm>
 #include <cstdint>
 #include <cstring>
+#include <list>
 #include <new>
+#include <set>
 #include <unordered_map>
 #include <vector>
 
@@ -23,6 +26,27 @@ namespace {
 struct Seq {
   std::vector<int32_t> table;
   int32_t len = 0;
+  bool tracked = true;          // token ids of every position are known
+  std::vector<int64_t> tokens;  // (prefix caching) ids of positions 0..len-1
+};
+
+// Prefix-cache key of a full block: its parent block (-1 for a sequence's
+// first block) and its token ids.  Exact comparison: a match never relies on
+// a hash alone.
+struct Key {
+  int32_t parent;
+  std::vector<int64_t> toks;
+  bool operator==(const Key& o) const { return parent == o.parent && toks == o.toks; }
+};
+
+struct KeyHash {
+  size_t operator()(const Key& k) const {
+    uint64_t h = 0x9E3779B97F4A7C15ull ^ static_cast<uint64_t>(static_cast<uint32_t>(k.parent));
+    for (int64_t t : k.toks) {
+      h ^= static_cast<uint64_t>(t) + 0x9E3779B97F4A7C15ull + (h << 6) + (h >> 2);
+    }
+    return static_cast<size_t>(h);
+  }
 };
 
 }  // namespace
@@ -33,6 +57,79 @@ struct pa_allocator {
   std::vector<int32_t> free_stack;  // top = back()
   std::vector<int32_t> ref;
   std::unordered_map<int64_t, Seq> seqs;
+
+  // Prefix caching: registered full blocks, their children, and the
+  // registered blocks nobody holds (evictable, least recently freed first).
+  std::unordered_map<Key, int32_t, KeyHash> cache;
+  std::vector<uint8_t> reg;
+  std::vector<Key> key_of;
+  std::vector<std::set<int32_t>> children;
+  std::list<int32_t> lru;
+  std::vector<std::list<int32_t>::iterator> lru_pos;
+  std::vector<uint8_t> in_lru;
+
+  void init_cache_state() {
+    reg.assign(num_blocks, 0);
+    key_of.assign(num_blocks, Key{-1, {}});
+    children.assign(num_blocks, {});
+    lru_pos.assign(num_blocks, lru.end());
+    in_lru.assign(num_blocks, 0);
+  }
+
+  int64_t available() const { return static_cast<int64_t>(free_stack.size()) + static_cast<int64_t>(lru.size()); }
+
+  void unregister(int32_t b) {
+    cache.erase(key_of[b]);
+    reg[b] = 0;
+    const int32_t parent = key_of[b].parent;
+    if (parent >= 0) children[parent].erase(b);
+    std::set<int32_t> kids;
+    kids.swap(children[b]);
+    for (int32_t c : kids) {  // increasing block order, depth first
+      unregister(c);
+      if (in_lru[c]) {
+        lru.erase(lru_pos[c]);
+        in_lru[c] = 0;
+        free_stack.push_back(c);
+      }
+    }
+  }
+
+  int32_t take_block() {
+    if (!free_stack.empty()) {
+      const int32_t b = free_stack.back();
+      free_stack.pop_back();
+      return b;
+    }
+    const int32_t b = lru.front();
+    lru.pop_front();
+    in_lru[b] = 0;
+    unregister(b);
+    return b;
+  }
+
+  void register_block(int32_t b, int32_t parent, const int64_t* toks) {
+    if (parent >= 0 && !reg[parent]) return;
+    Key k{parent, std::vector<int64_t>(toks, toks + block_size)};
+    if (reg[b] || cache.count(k)) return;
+    key_of[b] = k;
+    cache.emplace(std::move(k), b);
+    reg[b] = 1;
+    if (parent >= 0) children[parent].insert(b);
+  }
+
+  void release(int32_t b) {
+    ref[b] -= 1;
+    if (ref[b] == 0) {
+      if (reg[b]) {
+        lru.push_back(b);
+        lru_pos[b] = std::prev(lru.end());
+        in_lru[b] = 1;
+      } else {
+        free_stack.push_back(b);
+      }
+    }
+  }
 
   // Blocks an append of n tokens to s needs (copy-on-write + fresh blocks).
   int64_t blocks_needed(const Seq& s, int64_t n) const {
@@ -45,27 +142,33 @@ struct pa_allocator {
     return need;
   }
 
-  pa_status append(int64_t seq_id, int32_t n, int64_t* slots, int64_t* cow_pair, int32_t* n_cow) {
+  // ids: token ids of the n tokens (prefix caching), or null (unknown ids).
+  pa_status append(int64_t seq_id, int32_t n, const int64_t* ids, int64_t* slots, int64_t* cow_pair,
+                   int32_t* n_cow) {
     auto it = seqs.find(seq_id);
     if (it == seqs.end() || n < 0) return PA_ERR_INVALID_ARG;
     if (n > 0 && slots == nullptr) return PA_ERR_INVALID_ARG;
     Seq& s = it->second;
+    if (ids != nullptr && !s.tracked) return PA_ERR_INVALID_ARG;
     if (static_cast<int64_t>(s.len) + n > INT32_MAX) return PA_ERR_INVALID_ARG;
-    if (blocks_needed(s, n) > static_cast<int64_t>(free_stack.size())) return PA_ERR_OUT_OF_BLOCKS;
+    if (blocks_needed(s, n) > available()) return PA_ERR_OUT_OF_BLOCKS;
+    if (ids == nullptr) {
+      s.tracked = false;
+      s.tokens.clear();
+      s.tokens.shrink_to_fit();
+    }
     const int32_t bs = block_size;
     int32_t cows = 0;
     for (int32_t k = 0; k < n; ++k) {
       const int32_t pos = s.len;
       if (pos % bs == 0) {
-        const int32_t b = free_stack.back();
-        free_stack.pop_back();
+        const int32_t b = take_block();
         ref[b] = 1;
         s.table.push_back(b);
       } else {
         const int32_t last = s.table.back();
         if (ref[last] > 1) {
-          const int32_t b = free_stack.back();
-          free_stack.pop_back();
+          const int32_t b = take_block();
           ref[b] = 1;
           ref[last] -= 1;
           s.table.back() = b;
@@ -78,6 +181,13 @@ struct pa_allocator {
       }
       slots[k] = static_cast<int64_t>(s.table[pos / bs]) * bs + pos % bs;
       s.len = pos + 1;
+      if (s.tracked) {
+        s.tokens.push_back(ids[k]);
+        if ((pos + 1) % bs == 0) {
+          const int32_t j = pos / bs;
+          register_block(s.table[j], j ? s.table[j - 1] : -1, s.tokens.data() + static_cast<int64_t>(j) * bs);
+        }
+      }
     }
     if (n_cow != nullptr) *n_cow = cows;
     return PA_OK;
@@ -94,6 +204,7 @@ pa_status pa_alloc_create(int32_t num_blocks, int32_t block_size, const int32_t*
   a->num_blocks = num_blocks;
   a->block_size = block_size;
   a->ref.assign(num_blocks, 0);
+  a->init_cache_state();
   a->free_stack.resize(num_blocks);
   if (free_order != nullptr) {
     std::vector<uint8_t> seen(num_blocks, 0);
@@ -125,7 +236,55 @@ pa_status pa_seq_add(pa_allocator* a, int64_t seq_id) {
 pa_status pa_seq_append(pa_allocator* a, int64_t seq_id, int32_t n_tokens, int64_t* slots_out,
                         int64_t* cow_pair_out, int32_t* n_cow_out) {
   if (a == nullptr) return PA_ERR_INVALID_ARG;
-  return a->append(seq_id, n_tokens, slots_out, cow_pair_out, n_cow_out);
+  return a->append(seq_id, n_tokens, nullptr, slots_out, cow_pair_out, n_cow_out);
+}
+
+pa_status pa_seq_add_prefix(pa_allocator* a, int64_t seq_id, const int64_t* tokens, int32_t n_tokens,
+                            int32_t* n_cached_out) {
+  if (a == nullptr || n_tokens < 0 || (n_tokens > 0 && tokens == nullptr)) return PA_ERR_INVALID_ARG;
+  if (a->seqs.count(seq_id)) return PA_ERR_INVALID_ARG;
+  const int32_t bs = a->block_size;
+  std::vector<int32_t> hits;
+  int32_t parent = -1;
+  Key k{-1, std::vector<int64_t>(bs)};
+  for (int32_t j = 0; j < (n_tokens > 0 ? (n_tokens - 1) / bs : 0); ++j) {
+    k.parent = parent;
+    std::copy(tokens + static_cast<int64_t>(j) * bs, tokens + static_cast<int64_t>(j + 1) * bs, k.toks.begin());
+    auto it = a->cache.find(k);
+    if (it == a->cache.end()) break;
+    hits.push_back(it->second);
+    parent = it->second;
+  }
+  for (int32_t b : hits) {
+    if (a->ref[b] == 0 && a->in_lru[b]) {
+      a->lru.erase(a->lru_pos[b]);
+      a->in_lru[b] = 0;
+    }
+    a->ref[b] += 1;
+  }
+  Seq s;
+  s.table = hits;
+  s.len = static_cast<int32_t>(hits.size()) * bs;
+  s.tokens.assign(tokens, tokens + s.len);
+  a->seqs.emplace(seq_id, std::move(s));
+  if (n_cached_out != nullptr) *n_cached_out = static_cast<int32_t>(hits.size()) * bs;
+  return PA_OK;
+}
+
+pa_status pa_seq_append_tokens(pa_allocator* a, int64_t seq_id, const int64_t* tokens, int32_t n_tokens,
+                               int64_t* slots_out, int64_t* cow_pair_out, int32_t* n_cow_out) {
+  if (a == nullptr || (n_tokens > 0 && tokens == nullptr)) return PA_ERR_INVALID_ARG;
+  static const int64_t kNone = 0;
+  return a->append(seq_id, n_tokens, n_tokens > 0 ? tokens : &kNone, slots_out, cow_pair_out, n_cow_out);
+}
+
+pa_status pa_alloc_evictable(const pa_allocator* a, int32_t* out, int32_t cap, int32_t* n_out) {
+  if (a == nullptr || n_out == nullptr) return PA_ERR_INVALID_ARG;
+  *n_out = static_cast<int32_t>(a->lru.size());
+  if (static_cast<int64_t>(a->lru.size()) > cap || (!a->lru.empty() && out == nullptr)) return PA_ERR_INVALID_ARG;
+  int32_t k = 0;
+  for (int32_t b : a->lru) out[k++] = b;
+  return PA_OK;
 }
 
 pa_status pa_seq_append_batch(pa_allocator* a, const int64_t* seq_ids, const int32_t* n_tokens, int32_t n,
@@ -138,7 +297,7 @@ pa_status pa_seq_append_batch(pa_allocator* a, const int64_t* seq_ids, const int
   for (; k < n; ++k) {
     int32_t c = 0;
     int64_t pair[2] = {-1, -1};
-    st = a->append(seq_ids[k], n_tokens[k], slots_out == nullptr ? nullptr : slots_out + off, pair, &c);
+    st = a->append(seq_ids[k], n_tokens[k], nullptr, slots_out == nullptr ? nullptr : slots_out + off, pair, &c);
     if (st != PA_OK) break;
     off += n_tokens[k];
     if (c) {
@@ -168,10 +327,7 @@ pa_status pa_seq_free(pa_allocator* a, int64_t seq_id) {
   if (a == nullptr) return PA_ERR_INVALID_ARG;
   auto it = a->seqs.find(seq_id);
   if (it == a->seqs.end()) return PA_ERR_INVALID_ARG;
-  for (int32_t b : it->second.table) {
-    a->ref[b] -= 1;
-    if (a->ref[b] == 0) a->free_stack.push_back(b);
-  }
+  for (int32_t b : it->second.table) a->release(b);
   a->seqs.erase(it);
   return PA_OK;
 }
@@ -213,9 +369,7 @@ pa_status pa_alloc_block_tables(const pa_allocator* a, const int64_t* seq_ids, i
   return PA_OK;
 }
 
-int32_t pa_alloc_num_free(const pa_allocator* a) {
-  return a == nullptr ? -1 : static_cast<int32_t>(a->free_stack.size());
-}
+int32_t pa_alloc_num_free(const pa_allocator* a) { return a == nullptr ? -1 : static_cast<int32_t>(a->available()); }
 
 int32_t pa_block_refcount(const pa_allocator* a, int32_t block) {
   if (a == nullptr || block < 0 || block >= a->num_blocks) return -1;
@@ -240,7 +394,9 @@ pa_status pa_alloc_get_stats(const pa_allocator* a, pa_alloc_stats* out) {
   for (int32_t b = 0; b < a->num_blocks; ++b)
     if (a->ref[b] > 0) waste += bs - filled[b];
   out->num_blocks = a->num_blocks;
-  out->num_free = static_cast<int32_t>(a->free_stack.size());
+  out->num_free = static_cast<int32_t>(a->available());
+  out->num_cached = static_cast<int32_t>(a->cache.size());
+  out->num_evictable = static_cast<int32_t>(a->lru.size());
   out->num_seqs = static_cast<int32_t>(a->seqs.size());
   out->block_size = bs;
   out->num_tokens = tokens;

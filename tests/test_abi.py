@@ -256,3 +256,81 @@ def test_append_batch_matches_single_appends():
         slots_s += sl.tolist()
         pairs_s += cw
     assert slots_b.tolist() == slots_s and [tuple(p) for p in pairs_b.tolist()] == pairs_s
+
+
+# ---------------------------------------------------------------------------
+# prefix caching: C++ vs oracle
+# ---------------------------------------------------------------------------
+
+def test_prefix_cache_golden_example_cpp():
+    from test_oracle_allocator import run_prefix_example
+
+    a = run_prefix_example(pa.Allocator, lambda a, s, n: a.append(s, n), lambda a, s, t: a.append_tokens(s, t),
+                           lambda a, s, t: a.add_prefix(s, t), lambda a: a.evictable(),
+                           lambda a: a.stats()["num_cached"])
+    assert a.num_free() == 0
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_prefix_cache_matches_oracle_random(seed):
+    rnd = random.Random(300 + seed)
+    nb, bs = 36, 4
+    order = list(range(nb))
+    rnd.shuffle(order)
+    c = pa.Allocator(nb, bs, order)
+    o = BlockAllocator(nb, bs, order)
+    systems = [[rnd.randrange(3) for _ in range(rnd.choice([4, 8, 9, 12]))] for _ in range(3)]
+    live, nxt, tracked = [], 0, set()
+    for _ in range(500):
+        r = rnd.random()
+        if r < 0.25 or not live:
+            prompt = rnd.choice(systems) + [rnd.randrange(3) for _ in range(rnd.randrange(0, 7))]
+            hit_o = o.add_prefix(nxt, prompt)
+            assert c.add_prefix(nxt, prompt) == hit_o
+            live.append(nxt)
+            tracked.add(nxt)
+            toks = prompt[hit_o:]
+            seq = nxt
+            nxt += 1
+            try:
+                so, co = o.append_tokens(seq, toks)
+            except OutOfBlocks:
+                with pytest.raises(pa.OutOfBlocksError):
+                    c.append_tokens(seq, toks)
+            else:
+                sc, cc = c.append_tokens(seq, toks)
+                assert sc.tolist() == so and cc == co
+        elif r < 0.35:
+            p = rnd.choice(live)
+            o.fork(p, nxt)
+            c.fork(p, nxt)
+            if p in tracked:
+                tracked.add(nxt)
+            live.append(nxt)
+            nxt += 1
+        elif r < 0.55:
+            s = live.pop(rnd.randrange(len(live)))
+            o.free(s)
+            c.free(s)
+            tracked.discard(s)
+        else:
+            s = rnd.choice(live)
+            use_tokens = s in tracked and rnd.random() < 0.8
+            if use_tokens:
+                toks = [rnd.randrange(3) for _ in range(rnd.choice([1, 2, 3, 5]))]
+                fo, fc = (lambda: o.append_tokens(s, toks)), (lambda: c.append_tokens(s, toks))
+            else:
+                tracked.discard(s)
+                n = rnd.choice([1, 2, 5])
+                fo, fc = (lambda: o.append(s, n)), (lambda: c.append(s, n))
+            try:
+                so, co = fo()
+            except OutOfBlocks:
+                with pytest.raises(pa.OutOfBlocksError):
+                    fc()
+            else:
+                sc, cc = fc()
+                assert sc.tolist() == so and cc == co
+        _compare_state(c, o)
+        assert c.evictable() == list(o._evictable)
+        assert c.stats()["num_cached"] == o.num_cached()

@@ -268,3 +268,178 @@ def test_pins_catch_planted_mistakes(mutant):
     except AssertionError:
         failed = True
     assert failed
+
+
+# ---------------------------------------------------------------------------
+# prefix caching
+# ---------------------------------------------------------------------------
+
+def run_prefix_example(alloc_factory, appendf, append_tokensf, add_prefixf, evictable_of, cached_of):
+    g = _load("prefix_cache_example.json")
+    a = alloc_factory(g["num_blocks"], g["block_size"], g["free_order"])
+    for st in g["steps"]:
+        op = st["op"]
+        if op == "add":
+            a.add(st["seq"])
+        elif op == "free":
+            a.free(st["seq"])
+        elif op == "add_prefix":
+            assert add_prefixf(a, st["seq"], st["tokens"]) == st["hit"], st
+        elif op == "append_tokens":
+            slots, cow = append_tokensf(a, st["seq"], st["tokens"])
+            assert list(slots) == st["slots"] and [list(p) for p in cow] == st["cow"], st
+        elif op == "append":
+            slots, cow = appendf(a, st["seq"], st["n"])
+            assert list(slots) == st["slots"] and [list(p) for p in cow] == st["cow"], st
+        elif op == "check":
+            assert a.num_free() == st["num_free"], st
+            assert evictable_of(a) == st["evictable"], st
+            assert cached_of(a) == st["cached"], st
+    assert [a.refcount(b) for b in range(g["num_blocks"])] == g["final_refcounts"]
+    return a
+
+
+def test_prefix_cache_hand_worked_example():
+    a = run_prefix_example(BlockAllocator, lambda a, s, n: a.append(s, n), lambda a, s, t: a.append_tokens(s, t),
+                           lambda a, s, t: a.add_prefix(s, t), lambda a: list(a._evictable), lambda a: a.num_cached())
+    a.check_invariants()
+
+
+class PrefixIsolationModel(IsolationModel):
+    """Context model with prefix reuse.  A token's K/V depends on every token
+    before it, so the content of a slot is the whole token prefix of the
+    sequence that wrote it, up to that token.  A sequence must read back its
+    own prefixes at every position; a reused block must therefore have been
+    written under exactly the same prefix, and a false prefix hit is caught."""
+
+    def add_prefix(self, s, toks):
+        hit = self.a.add_prefix(s, toks)
+        self.logical[s] = list(toks[:hit])
+        return hit
+
+    def _write(self, s, slots, cow, ids):
+        bs = self.a.block_size
+        for src, dst in cow:
+            self.phys[dst * bs:(dst + 1) * bs] = self.phys[src * bs:(src + 1) * bs]
+        for sl, t in zip(slots, ids):
+            self.logical[s].append(t)
+            self.phys[sl] = tuple(self.logical[s])
+
+    def append_tokens(self, s, toks):
+        slots, cow = self.a.append_tokens(s, toks)
+        self._write(s, slots, cow, list(toks))
+        return slots, cow
+
+    def append(self, s, n):
+        slots, cow = self.a.append(s, n)
+        ids = [-1 - self.next_id - k for k in range(n)]  # unknown tokens: ids no prompt uses
+        self.next_id += n
+        self._write(s, slots, cow, ids)
+        return slots, cow
+
+    def check(self):
+        self.a.check_invariants()
+        for s, toks in self.logical.items():
+            got = [self.phys[self.a.slot(s, t)] for t in range(self.a.length(s))]
+            assert got == [tuple(toks[:t + 1]) for t in range(len(toks))], f"sequence {s} reads a foreign prefix"
+
+
+def _prefix_session(seed, num_blocks=30, bs=4, steps=400):
+    rnd = random.Random(seed)
+    order = list(range(num_blocks))
+    rnd.shuffle(order)
+    m = PrefixIsolationModel(BlockAllocator(num_blocks, bs, order))
+    systems = [[rnd.randrange(3) for _ in range(rnd.choice([4, 8, 9, 12]))] for _ in range(3)]
+    nxt = 0
+    hits = 0
+    for _ in range(steps):
+        live = list(m.logical)
+        r = rnd.random()
+        try:
+            if r < 0.25 or not live:
+                prompt = rnd.choice(systems) + [rnd.randrange(3) for _ in range(rnd.randrange(0, 7))]
+                if not prompt:
+                    prompt = [0]
+                hit = m.add_prefix(nxt, prompt)
+                hits += hit > 0
+                nxt += 1
+                m.append_tokens(nxt - 1, prompt[hit:])
+            elif r < 0.35:
+                m.fork(rnd.choice(live), nxt)
+                nxt += 1
+            elif r < 0.55:
+                m.free(rnd.choice(live))
+            elif r < 0.85:
+                s = rnd.choice(live)
+                if m.a._tokens.get(s) is not None:
+                    m.append_tokens(s, [rnd.randrange(3) for _ in range(rnd.choice([1, 2, 3, 5]))])
+                else:
+                    m.append(s, rnd.choice([1, 2, 5]))
+            else:
+                m.append(rnd.choice(live), rnd.choice([1, 3]))
+        except OutOfBlocks:
+            pass
+        m.check()
+    return hits
+
+
+@pytest.mark.parametrize("seed", range(10))
+def test_prefix_sessions_keep_invariants_and_isolation(seed):
+    assert _prefix_session(seed) > 0
+
+
+class _MutantPrefixIgnoresParent(BlockAllocator):
+    """Planted mistake: matches a block by its own tokens only."""
+
+    def add_prefix(self, seq, tokens):
+        bs = self.block_size
+        saved = dict(self._cache)
+        self._cache = {(-1, k[1]): b for k, b in saved.items()} | saved
+        try:
+            hits = []
+            for k in range(max(0, (len(tokens) - 1) // bs)):
+                b = self._cache.get((-1, tuple(tokens[k * bs:(k + 1) * bs])))
+                if b is None:
+                    break
+                hits.append(b)
+        finally:
+            self._cache = saved
+        if seq in self._table:
+            raise AllocatorError("exists")
+        for b in hits:
+            if self._ref[b] == 0:
+                del self._evictable[b]
+            self._ref[b] += 1
+        self._table[seq] = hits
+        self._len[seq] = len(hits) * bs
+        self._tokens[seq] = list(tokens[:len(hits) * bs])
+        return len(hits) * bs
+
+
+def test_prefix_pins_catch_planted_mistake():
+    m = PrefixIsolationModel(_MutantPrefixIgnoresParent(20, 4, list(range(20))))
+    m.add_prefix(0, [1, 1, 1, 1, 2, 2, 2, 2, 3])
+    m.append_tokens(0, [1, 1, 1, 1, 2, 2, 2, 2, 3])
+    m.check()
+    # the same four tokens as seq 0's second block, but at the start of a prompt
+    hit = m.add_prefix(1, [2, 2, 2, 2, 9])
+    assert hit == 4  # the mutant reuses a block written under another prefix
+    with pytest.raises(AssertionError):
+        m.check()
+
+
+def test_forks_of_forks_share_and_copy():
+    """Beam-search style: forks of forks share every full block and copy the
+    shared partial one on their first write."""
+    m = IsolationModel(BlockAllocator(40, 4, list(range(40))))
+    m.add(0)
+    m.append(0, 6)
+    m.fork(0, 1)
+    m.fork(1, 2)
+    m.fork(2, 3)
+    assert m.a.refcount(m.a.block_table(0)[1]) == 4
+    for s in (3, 2, 1, 0):
+        m.append(s, 1)
+        m.check()
+    assert len({m.a.block_table(s)[1] for s in range(4)}) == 4
+    assert len({m.a.block_table(s)[0] for s in range(4)}) == 1
