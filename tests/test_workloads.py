@@ -26,7 +26,9 @@ def test_plans_are_reproducible_and_shaped():
         assert sorted(p1.free_order.tolist()) == list(range(p1.num_blocks))
         assert p1.context_lens.shape[0] == p1.B
         q = query_values(p1)
-        assert q.shape == (p1.B, w.num_heads, w.head_size)
+        rows = p1.B if np.all(p1.query_lens == 1) else p1.num_query_rows
+        assert q.shape == (rows, w.num_heads, w.head_size)
+        assert p1.query_start[-1] == p1.num_query_rows and np.all(p1.query_lens <= p1.context_lens)
 
 
 def test_documented_sizes():
@@ -43,6 +45,25 @@ def test_documented_sizes():
     assert int(p.context_lens.sum()) == 704512
     p = make_plan("parallel_sampling_13b")
     assert p.B == 256 and p.context_lens.max() <= 1024 + 64
+    p = make_plan("prefill_chunks_llama7b")
+    assert p.B == 16 and p.num_query_rows == 16 * 512 and p.context_lens.max() <= 3584 + 512
+    p = make_plan("prefill_mixed_gqa")
+    assert p.B == 64 and p.num_query_rows == 4 * 512 + 60
+    assert p.query_lens.tolist() == [512] * 4 + [1] * 60
+    p = make_plan("prefill_tiny")
+    assert (0 in p.query_lens.tolist()) and (0 in p.context_lens.tolist())
+
+
+def test_prefill_step_appends_new_tokens_after_prior_context():
+    for name in ("prefill_tiny", "prefill_mixed_gqa"):
+        p = make_plan(name)
+        step = {op.seq: op for op in p.step_ops}
+        for i in range(p.B):
+            q, c = int(p.query_lens[i]), int(p.context_lens[i])
+            if q == 0:
+                assert i not in step
+            else:
+                assert step[i].n == q and step[i].start == c - q and step[i].stream == i
 
 
 def test_stream_slices_agree_across_chunks():

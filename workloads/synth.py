@@ -96,6 +96,17 @@ WORKLOADS: Dict[str, Workload] = {
                  description="llama7b_bs64 with an e4m3 KV cache (per-head scales), bf16 query/output"),
         Workload("gqa_bs256_fp8", 2, "bf16", 32, 8, 128, kv_dtype="fp8",
                  description="gqa_bs256 with an e4m3 KV cache (per-head scales), bf16 query/output"),
+        # Multi-token (chunked-prefill) steps: each sequence appends q_len
+        # tokens at once and every new token is a query row (causal).
+        Workload("prefill_tiny", 7, "bf16", 4, 2, 128,
+                 description="11 seqs of (prior context, new tokens) edge cases incl. empty and decode rows, "
+                             "H=4 on H_kv=2, D=128, bf16"),
+        Workload("prefill_chunks_llama7b", 8, "bf16", 32, 32, 128,
+                 description="16 prefill chunks of 512 tokens over prior contexts U{0..3584}, H=H_kv=32, "
+                             "D=128, bf16"),
+        Workload("prefill_mixed_gqa", 9, "bf16", 32, 8, 128,
+                 description="4 prefill chunks of 512 tokens (prior U{0..7680}) mixed with 60 decode rows "
+                             "(ctx lognormal median 1024), H=32 on H_kv=8, D=128, bf16"),
     )
 }
 
@@ -174,6 +185,22 @@ class Plan:
     outlier_channels: np.ndarray = field(default_factory=lambda: np.zeros((0, 2), np.int64))
     # parallel sampling only: ops after the first append round (for a mid-replay check)
     first_round_end: int = -1
+    # new tokens of each batch sequence in the step (1 for a decode step); the
+    # step's query rows are these tokens, sequence by sequence
+    query_lens: np.ndarray = None
+
+    def __post_init__(self):
+        if self.query_lens is None:
+            self.query_lens = np.ones(len(self.context_lens), np.int32)
+
+    @property
+    def num_query_rows(self) -> int:
+        return int(np.sum(self.query_lens))
+
+    @property
+    def query_start(self) -> np.ndarray:
+        """int32 [B + 1]: row offset of each sequence's queries."""
+        return np.concatenate([[0], np.cumsum(self.query_lens)]).astype(np.int32)
 
     @property
     def B(self) -> int:
@@ -204,6 +231,25 @@ def _single_plan(w: Workload, ctx: np.ndarray, num_blocks: int) -> Plan:
             step.append(AppendOp(i, 1, i, c - 1))
     order = _rng(w, _TAG_PERM).permutation(num_blocks).astype(np.int32)
     return Plan(w, num_blocks, order, setup, step, np.arange(len(ctx), dtype=np.int64), ctx.astype(np.int32))
+
+
+def _prefill_plan(w: Workload, prior: np.ndarray, qlen: np.ndarray, spare: float = 1.25) -> Plan:
+    """Sequence i holds prior[i] tokens before the step (stream i, positions
+    [0, prior)) and appends qlen[i] tokens in it (positions [prior, prior+qlen))."""
+    setup: List[Op] = []
+    step: List[Op] = []
+    for i, (c, q) in enumerate(zip(prior.tolist(), qlen.tolist())):
+        setup.append(AddOp(i))
+        if c > 0:
+            setup.append(AppendOp(i, c, i, 0))
+    for i, (c, q) in enumerate(zip(prior.tolist(), qlen.tolist())):
+        if q > 0:
+            step.append(AppendOp(i, q, i, c))
+    ctx = (prior + qlen).astype(np.int32)
+    nb = max(1, int(math.ceil(spare * _blocks_needed(ctx, w.block_size))))
+    order = _rng(w, _TAG_PERM).permutation(nb).astype(np.int32)
+    return Plan(w, nb, order, setup, step, np.arange(len(ctx), dtype=np.int64), ctx,
+                query_lens=qlen.astype(np.int32))
 
 
 def _blocks_needed(ctx: np.ndarray, bs: int) -> int:
@@ -245,6 +291,22 @@ def make_plan(w: Union[Workload, str]) -> Plan:
         return _single_plan(w, ctx, int(math.ceil(1.25 * _blocks_needed(ctx, bs))))
     if w.name == "parallel_sampling_13b":
         return _parallel_sampling_plan(w)
+    if w.name == "prefill_tiny":
+        pairs = [(0, 1), (0, 17), (23, 7), (0, 300), (16, 16), (100, 129), (511, 1), (257, 256), (40, 0), (0, 0),
+                 (5, 33)]
+        prior = np.array([a for a, _ in pairs], np.int32)
+        qlen = np.array([b for _, b in pairs], np.int32)
+        return _prefill_plan(w, prior, qlen, spare=1.5)
+    if w.name == "prefill_chunks_llama7b":
+        prior = _rng(w, _TAG_CTX).integers(0, 3584, size=16, endpoint=True).astype(np.int32)
+        return _prefill_plan(w, prior, np.full(16, 512, np.int32))
+    if w.name == "prefill_mixed_gqa":
+        r = _rng(w, _TAG_CTX)
+        prior_chunks = r.integers(0, 7680, size=4, endpoint=True).astype(np.int32)
+        dec = np.clip(np.rint(np.exp(r.normal(math.log(1024.0), 0.75, size=60))), 32, 8192).astype(np.int32)
+        prior = np.concatenate([prior_chunks, dec - 1]).astype(np.int32)
+        qlen = np.concatenate([np.full(4, 512, np.int32), np.ones(60, np.int32)])
+        return _prefill_plan(w, prior, qlen)
     raise KeyError(w.name)
 
 
@@ -367,8 +429,11 @@ def kv_scales(plan: Plan) -> Tuple[np.ndarray, np.ndarray]:
 
 
 def query_values(plan: Plan, step: int = 0) -> np.ndarray:
-    """Query of the decode step, [B, H, D] in storage form."""
+    """Query of the decode step, [B, H, D] in storage form; for a multi-token
+    step, [num_query_rows, H, D] (the rows of sequence i start at
+    ``plan.query_start[i]``)."""
     w = plan.workload
     r = _rng(w, _TAG_Q, step)
-    q = r.standard_normal(size=(plan.B, w.num_heads, w.head_size), dtype=np.float32)
+    n = plan.B if np.all(plan.query_lens == 1) else plan.num_query_rows
+    q = r.standard_normal(size=(n, w.num_heads, w.head_size), dtype=np.float32)
     return _store(w, q)
