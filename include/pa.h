@@ -132,6 +132,20 @@ pa_status pa_reshape_and_cache(const pa_tensor* key, const pa_tensor* value, pa_
 pa_status pa_copy_blocks(pa_tensor* k_cache, pa_tensor* v_cache, const pa_tensor* pairs, const pa_opts* opts);
 
 /* ---------------------------------------------------------------------------
+ * Swap copy between a device pool and a pinned host pool (either direction):
+ *   for each pair (src, dst): dst_k[dst] = src_k[src]; dst_v[dst] = src_v[src]
+ * src_k/src_v and dst_k/dst_v: caches of the same dtype and [*, H_kv, 16, D]
+ * shape (block counts may differ), each in device memory of the current
+ * device or in page-locked host memory the device can address (e.g.
+ * cudaHostAlloc, torch pin_memory); anything else is PA_ERR_INVALID_ARG.
+ * pairs: [n, 2] int64 in device or pinned memory (the allocator's swap pairs).
+ * Ids outside their pool set PA_DEV_BAD_BLOCK and are skipped.  One kernel
+ * moves every pair; the host side of the copy crosses the host link.
+ * ------------------------------------------------------------------------- */
+pa_status pa_swap_blocks(const pa_tensor* src_k, const pa_tensor* src_v, pa_tensor* dst_k, pa_tensor* dst_v,
+                         const pa_tensor* pairs, const pa_opts* opts);
+
+/* ---------------------------------------------------------------------------
  * Paged decode attention (gitcode walkthrough, section 2.1: the query-key dot
  * product, softmax normalisation and weighted sum of V over K/V gathered
  * block by block; launch blog "PagedAttention" section).
@@ -313,6 +327,28 @@ pa_status pa_seq_append_tokens(pa_allocator* a, int64_t seq_id, const int64_t* t
                                int64_t* slots_out, int64_t* cow_pair_out, int32_t* n_cow_out);
 /* Evictable blocks, least recently freed first. */
 pa_status pa_alloc_evictable(const pa_allocator* a, int32_t* out, int32_t cap, int32_t* n_out);
+
+/* Swapping.  The pages say blocks can be swapped out (agientry.com overview,
+ * opening section); this library's form:
+ *  - pa_alloc_set_host_pool gives the allocator num_host_blocks host blocks
+ *    (LIFO, host_free_order[0] first; NULL = 0, 1, ...); not while any
+ *    sequence is swapped out;
+ *  - pa_seq_swap_out gives each block of the sequence, in table order, a host
+ *    block (all or nothing: PA_ERR_OUT_OF_BLOCKS), writes (device, host) pairs
+ *    to pairs_out [n, 2] (cap pairs of room), then releases the device blocks
+ *    as pa_seq_free would; shared blocks are copied and keep their holders;
+ *  - pa_seq_swap_in takes device blocks for the host blocks in order (all or
+ *    nothing), writes (host, device) pairs, returns the host blocks, and
+ *    re-registers the full blocks for prefix reuse when the token ids are
+ *    known;
+ *  - a swapped-out sequence accepts only pa_seq_swap_in and pa_seq_free;
+ *  - the caller moves the bytes with pa_swap_blocks (out: before any device
+ *    block it released is written again; in: before the sequence is read). */
+pa_status pa_alloc_set_host_pool(pa_allocator* a, int32_t num_host_blocks, const int32_t* host_free_order);
+pa_status pa_seq_swap_out(pa_allocator* a, int64_t seq_id, int64_t* pairs_out, int32_t cap, int32_t* n_out);
+pa_status pa_seq_swap_in(pa_allocator* a, int64_t seq_id, int64_t* pairs_out, int32_t cap, int32_t* n_out);
+int32_t pa_alloc_num_host_free(const pa_allocator* a);
+pa_status pa_seq_host_table(const pa_allocator* a, int64_t seq_id, int32_t* out, int32_t cap, int32_t* n_out);
 pa_status pa_seq_free(pa_allocator* a, int64_t seq_id);
 pa_status pa_seq_len(const pa_allocator* a, int64_t seq_id, int32_t* len_out);
 pa_status pa_seq_block_table(const pa_allocator* a, int64_t seq_id, int32_t* out, int32_t cap, int32_t* n_out);

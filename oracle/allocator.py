@@ -46,6 +46,17 @@ agientry.com overview, opening section: blocks can be shared across requests)
   block.  Evicting (or otherwise unregistering) a block unregisters its
   registered children in increasing block order, depth first; an evictable
   child that loses its key goes onto the free stack.
+
+Swapping (agientry.com overview, opening section: blocks can be swapped out)
+— the reading taken here: a second pool of host blocks with its own LIFO free
+stack.  ``swap_out`` gives each of a sequence's blocks, in table order, a
+host block (all or nothing), reports (device, host) pairs for the copy, then
+releases the device blocks as ``free`` would (a shared block is copied and
+keeps its other holders).  ``swap_in`` takes device blocks for the host blocks
+in order (all or nothing), reports (host, device) pairs, returns the host
+blocks to their free stack in order, and re-registers the sequence's full
+blocks for prefix reuse when its token ids are known.  A swapped-out sequence
+can only be swapped in or freed.
 """
 
 from __future__ import annotations
@@ -84,6 +95,10 @@ class BlockAllocator:
         self._key_of: Dict[int, Tuple[int, Tuple[int, ...]]] = {}
         self._children: Dict[int, Set[int]] = {}
         self._evictable: "OrderedDict[int, None]" = OrderedDict()
+        # swapping
+        self.num_host_blocks = 0
+        self._host_free: List[int] = []
+        self._swapped: Dict[int, List[int]] = {}
 
     # -- queries ---------------------------------------------------------
     def num_free(self) -> int:
@@ -115,7 +130,72 @@ class BlockAllocator:
         bs = self.block_size
         return self._table[seq][pos // bs] * bs + pos % bs
 
+    def num_host_free(self) -> int:
+        return len(self._host_free)
+
+    def is_swapped(self, seq: int) -> bool:
+        return seq in self._swapped
+
+    def host_table(self, seq: int) -> List[int]:
+        return list(self._swapped[seq])
+
     # -- requests --------------------------------------------------------
+    def set_host_pool(self, num_host_blocks: int, host_free_order: Optional[Sequence[int]] = None) -> None:
+        if self._swapped:
+            raise AllocatorError("sequences are swapped out")
+        order = list(range(num_host_blocks)) if host_free_order is None else [int(b) for b in host_free_order]
+        if sorted(order) != list(range(num_host_blocks)):
+            raise AllocatorError("host_free_order must be a permutation")
+        self.num_host_blocks = num_host_blocks
+        self._host_free = list(reversed(order))
+
+    def _check_resident(self, seq: int) -> None:
+        if seq not in self._table:
+            raise AllocatorError(f"unknown sequence {seq}")
+        if seq in self._swapped:
+            raise AllocatorError(f"sequence {seq} is swapped out")
+
+    def swap_out(self, seq: int) -> List[Tuple[int, int]]:
+        self._check_resident(seq)
+        table = self._table[seq]
+        if len(table) > len(self._host_free):
+            raise OutOfBlocks(f"sequence {seq}: {len(table)} blocks, {len(self._host_free)} host blocks free")
+        pairs = []
+        host = []
+        for b in table:
+            h = self._host_free.pop()
+            pairs.append((b, h))
+            host.append(h)
+        for b in table:
+            self._release(b)
+        self._table[seq] = []
+        self._swapped[seq] = host
+        return pairs
+
+    def swap_in(self, seq: int) -> List[Tuple[int, int]]:
+        if seq not in self._swapped:
+            raise AllocatorError(f"sequence {seq} is not swapped out")
+        host = self._swapped[seq]
+        if len(host) > self.num_free():
+            raise OutOfBlocks(f"sequence {seq}: {len(host)} blocks, {self.num_free()} free")
+        pairs = []
+        table = []
+        for h in host:
+            b = self._take_block()
+            self._ref[b] = 1
+            table.append(b)
+            pairs.append((h, b))
+        for h in host:
+            self._host_free.append(h)
+        del self._swapped[seq]
+        self._table[seq] = table
+        toks = self._tokens.get(seq)
+        if toks is not None:
+            bs = self.block_size
+            for j in range(self._len[seq] // bs):
+                self._register(table[j], table[j - 1] if j else -1, tuple(toks[j * bs:(j + 1) * bs]))
+        return pairs
+
     def add(self, seq: int) -> None:
         if seq in self._table:
             raise AllocatorError(f"sequence {seq} exists")
@@ -204,8 +284,7 @@ class BlockAllocator:
 
     def append(self, seq: int, n: int) -> Tuple[List[int], List[Tuple[int, int]]]:
         """Append n tokens; return (slots of the new tokens, copy-on-write pairs)."""
-        if seq not in self._table:
-            raise AllocatorError(f"unknown sequence {seq}")
+        self._check_resident(seq)
         if n < 0:
             raise AllocatorError("negative token count")
         return self._append(seq, n, None)
@@ -213,8 +292,7 @@ class BlockAllocator:
     def append_tokens(self, seq: int, tokens: Sequence[int]) -> Tuple[List[int], List[Tuple[int, int]]]:
         """Append tokens with known ids (the sequence's ids so far must be
         known); blocks that become full are registered for prefix reuse."""
-        if seq not in self._table:
-            raise AllocatorError(f"unknown sequence {seq}")
+        self._check_resident(seq)
         if self._tokens.get(seq) is None:
             raise AllocatorError(f"sequence {seq} has tokens of unknown id")
         return self._append(seq, len(tokens), [int(t) for t in tokens])
@@ -255,8 +333,7 @@ class BlockAllocator:
     def fork(self, parent: int, child: int) -> None:
         """The child starts as a copy of the parent's table; every block it
         names gains one reference."""
-        if parent not in self._table:
-            raise AllocatorError(f"unknown sequence {parent}")
+        self._check_resident(parent)
         if child in self._table:
             raise AllocatorError(f"sequence {child} exists")
         self._table[child] = list(self._table[parent])
@@ -271,6 +348,8 @@ class BlockAllocator:
             raise AllocatorError(f"unknown sequence {seq}")
         for b in self._table.pop(seq):
             self._release(b)
+        for h in self._swapped.pop(seq, []):
+            self._host_free.append(h)
         del self._len[seq]
         del self._tokens[seq]
 
@@ -291,6 +370,10 @@ class BlockAllocator:
         bs = self.block_size
         count = [0] * self.num_blocks
         for seq, table in self._table.items():
+            if seq in self._swapped:
+                if table or len(self._swapped[seq]) != -(-self._len[seq] // bs):
+                    raise AssertionError(f"swapped sequence {seq}: table and host blocks disagree")
+                continue
             if len(table) != -(-self._len[seq] // bs):
                 raise AssertionError(f"sequence {seq}: table length does not match its token count")
             for b in table:
@@ -311,3 +394,7 @@ class BlockAllocator:
                 raise AssertionError("a registered block's parent is not registered")
         if not evict <= set(self._key_of):
             raise AssertionError("an evictable block is not registered")
+        host_used = [h for hs in self._swapped.values() for h in hs]
+        if len(set(host_used)) != len(host_used) or set(host_used) & set(self._host_free) or \
+                len(host_used) + len(self._host_free) != self.num_host_blocks:
+            raise AssertionError("host blocks are not partitioned")

@@ -84,6 +84,16 @@ class PagedKVCache:
             vd[...] = vs
             wd[...] = ws
 
+    def copy_blocks_to(self, dst: "PagedKVCache", pairs: Iterable[Tuple[int, int]]) -> None:
+        """Whole-block copies into another pool (swap out / swap in): for each
+        (src, dst) pair, dst's block becomes a copy of this cache's block."""
+        for s_, d_ in pairs:
+            ks, vs, ws = self._page(int(s_))
+            kd, vd, wd = dst._page(int(d_))
+            kd[...] = ks
+            vd[...] = vs
+            wd[...] = ws
+
     def blocks(self):
         return sorted(self._k.keys())
 

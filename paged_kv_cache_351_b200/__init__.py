@@ -21,7 +21,7 @@ from ._lib import (PA_DEV_BAD_BLOCK, PA_DEV_BAD_CONTEXT, PA_DEV_BAD_SLOT,  # noq
 
 __all__ = [
     "PagedAttentionError", "OutOfBlocksError", "pa_reshape_and_cache", "pa_copy_blocks", "pa_decode",
-    "pa_decode_workspace_bytes", "pa_decode_no_alloc", "pa_reshape_and_cache_fp8", "pa_decode_fp8", "pa_set_decode_tuning", "pa_get_device_status", "pa_debug_wait_selftest",
+    "pa_decode_workspace_bytes", "pa_decode_no_alloc", "pa_reshape_and_cache_fp8", "pa_decode_fp8", "pa_swap_blocks", "pa_set_decode_tuning", "pa_get_device_status", "pa_debug_wait_selftest",
     "Allocator", "library",
 ]
 
@@ -148,6 +148,14 @@ def pa_decode_fp8(out, query, k_cache, v_cache, block_tables, context_lens, scal
     o = _opts(stream, workspace, partition_tokens, timeout_ms)
     _check(_lib_handle.pa_decode_fp8(*[ctypes.byref(t) for t in ts], ctypes.c_float(scale), int(num_kv_heads),
                                      ctypes.byref(ks), ctypes.byref(vs), ctypes.byref(o)), "pa_decode_fp8")
+
+
+def pa_swap_blocks(src_k, src_v, dst_k, dst_v, pairs, stream=None) -> None:
+    """Copy whole blocks between a device pool and a pinned host pool (either
+    direction) for each (src, dst) row of ``pairs``."""
+    ts = [_tensor(x) for x in (src_k, src_v, dst_k, dst_v, pairs)]
+    o = _opts(stream)
+    _check(_lib_handle.pa_swap_blocks(*[ctypes.byref(t) for t in ts], ctypes.byref(o)), "pa_swap_blocks")
 
 
 NO_ALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
@@ -278,6 +286,39 @@ class Allocator:
         _check(_lib_handle.pa_seq_append_tokens(self._h, seq, _i64p(ids) if n else _i64p(slots), n, _i64p(slots),
                                                 _i64p(pair), ctypes.byref(ncow)), "pa_seq_append_tokens")
         return slots[:n], ([(int(pair[0]), int(pair[1]))] if ncow.value else [])
+
+    def set_host_pool(self, num_host_blocks: int, host_free_order: Optional[Sequence[int]] = None) -> None:
+        self._host_order = (np.ascontiguousarray(np.asarray(host_free_order, np.int32))
+                            if host_free_order is not None else None)
+        _check(_lib_handle.pa_alloc_set_host_pool(self._h, num_host_blocks,
+                                                  _i32p(self._host_order) if self._host_order is not None else None),
+               "pa_alloc_set_host_pool")
+        self.num_host_blocks = num_host_blocks
+
+    def _swap(self, fn, seq, where):
+        cap = self.length(seq) // self.block_size + 2
+        out = np.zeros((cap, 2), np.int64)
+        n = ctypes.c_int32(0)
+        _check(fn(self._h, seq, _i64p(out), cap, ctypes.byref(n)), where)
+        return out[: n.value]
+
+    def swap_out(self, seq: int):
+        """(device, host) block pairs int64 [n, 2]; the device blocks are released."""
+        return self._swap(_lib_handle.pa_seq_swap_out, seq, "pa_seq_swap_out")
+
+    def swap_in(self, seq: int):
+        """(host, device) block pairs int64 [n, 2]."""
+        return self._swap(_lib_handle.pa_seq_swap_in, seq, "pa_seq_swap_in")
+
+    def num_host_free(self) -> int:
+        return int(_lib_handle.pa_alloc_num_host_free(self._h))
+
+    def host_table(self, seq: int):
+        cap = self.length(seq) // self.block_size + 1
+        out = np.zeros(cap, np.int32)
+        n = ctypes.c_int32(0)
+        _check(_lib_handle.pa_seq_host_table(self._h, seq, _i32p(out), cap, ctypes.byref(n)), "pa_seq_host_table")
+        return out[: n.value].tolist()
 
     def evictable(self):
         out = np.zeros(max(1, self.num_blocks), np.int32)

@@ -83,6 +83,12 @@ SIGNATURES = {
     "pa_seq_add_prefix": (c_int32, [_A, c_int64, _I64P, c_int32, _I32P]),
     "pa_seq_append_tokens": (c_int32, [_A, c_int64, _I64P, c_int32, _I64P, _I64P, _I32P]),
     "pa_alloc_evictable": (c_int32, [_A, _I32P, c_int32, _I32P]),
+    "pa_alloc_set_host_pool": (c_int32, [_A, c_int32, _I32P]),
+    "pa_seq_swap_out": (c_int32, [_A, c_int64, _I64P, c_int32, _I32P]),
+    "pa_seq_swap_in": (c_int32, [_A, c_int64, _I64P, c_int32, _I32P]),
+    "pa_alloc_num_host_free": (c_int32, [_A]),
+    "pa_seq_host_table": (c_int32, [_A, c_int64, _I32P, c_int32, _I32P]),
+    "pa_swap_blocks": (c_int32, [_T, _T, _T, _T, _T, _O]),
     "pa_seq_free": (c_int32, [_A, c_int64]),
     "pa_seq_len": (c_int32, [_A, c_int64, _I32P]),
     "pa_seq_block_table": (c_int32, [_A, c_int64, _I32P, c_int32, _I32P]),

@@ -28,6 +28,8 @@ struct Seq {
   int32_t len = 0;
   bool tracked = true;          // token ids of every position are known
   std::vector<int64_t> tokens;  // (prefix caching) ids of positions 0..len-1
+  bool swapped = false;         // swapped out: table is empty, host holds the blocks
+  std::vector<int32_t> host;    // host blocks of a swapped-out sequence, in table order
 };
 
 // Prefix-cache key of a full block: its parent block (-1 for a sequence's
@@ -67,6 +69,10 @@ struct pa_allocator {
   std::list<int32_t> lru;
   std::vector<std::list<int32_t>::iterator> lru_pos;
   std::vector<uint8_t> in_lru;
+
+  // Swapping: a pool of host blocks with its own LIFO free stack.
+  int32_t num_host_blocks = 0;
+  std::vector<int32_t> host_free;
 
   void init_cache_state() {
     reg.assign(num_blocks, 0);
@@ -146,7 +152,7 @@ struct pa_allocator {
   pa_status append(int64_t seq_id, int32_t n, const int64_t* ids, int64_t* slots, int64_t* cow_pair,
                    int32_t* n_cow) {
     auto it = seqs.find(seq_id);
-    if (it == seqs.end() || n < 0) return PA_ERR_INVALID_ARG;
+    if (it == seqs.end() || n < 0 || it->second.swapped) return PA_ERR_INVALID_ARG;
     if (n > 0 && slots == nullptr) return PA_ERR_INVALID_ARG;
     Seq& s = it->second;
     if (ids != nullptr && !s.tracked) return PA_ERR_INVALID_ARG;
@@ -278,6 +284,89 @@ pa_status pa_seq_append_tokens(pa_allocator* a, int64_t seq_id, const int64_t* t
   return a->append(seq_id, n_tokens, n_tokens > 0 ? tokens : &kNone, slots_out, cow_pair_out, n_cow_out);
 }
 
+pa_status pa_alloc_set_host_pool(pa_allocator* a, int32_t num_host_blocks, const int32_t* host_free_order) {
+  if (a == nullptr || num_host_blocks < 0) return PA_ERR_INVALID_ARG;
+  for (const auto& kv : a->seqs)
+    if (kv.second.swapped) return PA_ERR_INVALID_ARG;
+  std::vector<int32_t> st(num_host_blocks);
+  std::vector<uint8_t> seen(num_host_blocks, 0);
+  for (int32_t k = 0; k < num_host_blocks; ++k) {
+    const int32_t h = host_free_order ? host_free_order[k] : k;
+    if (h < 0 || h >= num_host_blocks || seen[h]) return PA_ERR_INVALID_ARG;
+    seen[h] = 1;
+    st[num_host_blocks - 1 - k] = h;
+  }
+  a->num_host_blocks = num_host_blocks;
+  a->host_free.swap(st);
+  return PA_OK;
+}
+
+pa_status pa_seq_swap_out(pa_allocator* a, int64_t seq_id, int64_t* pairs_out, int32_t cap, int32_t* n_out) {
+  if (a == nullptr || n_out == nullptr) return PA_ERR_INVALID_ARG;
+  auto it = a->seqs.find(seq_id);
+  if (it == a->seqs.end() || it->second.swapped) return PA_ERR_INVALID_ARG;
+  Seq& s = it->second;
+  const int32_t n = static_cast<int32_t>(s.table.size());
+  *n_out = n;
+  if (n > cap || (n > 0 && pairs_out == nullptr)) return PA_ERR_INVALID_ARG;
+  if (n > static_cast<int32_t>(a->host_free.size())) return PA_ERR_OUT_OF_BLOCKS;
+  s.host.resize(n);
+  for (int32_t k = 0; k < n; ++k) {
+    const int32_t h = a->host_free.back();
+    a->host_free.pop_back();
+    s.host[k] = h;
+    pairs_out[2 * k] = s.table[k];
+    pairs_out[2 * k + 1] = h;
+  }
+  for (int32_t b : s.table) a->release(b);
+  s.table.clear();
+  s.swapped = true;
+  return PA_OK;
+}
+
+pa_status pa_seq_swap_in(pa_allocator* a, int64_t seq_id, int64_t* pairs_out, int32_t cap, int32_t* n_out) {
+  if (a == nullptr || n_out == nullptr) return PA_ERR_INVALID_ARG;
+  auto it = a->seqs.find(seq_id);
+  if (it == a->seqs.end() || !it->second.swapped) return PA_ERR_INVALID_ARG;
+  Seq& s = it->second;
+  const int32_t n = static_cast<int32_t>(s.host.size());
+  *n_out = n;
+  if (n > cap || (n > 0 && pairs_out == nullptr)) return PA_ERR_INVALID_ARG;
+  if (n > a->available()) return PA_ERR_OUT_OF_BLOCKS;
+  s.table.resize(n);
+  for (int32_t k = 0; k < n; ++k) {
+    const int32_t b = a->take_block();
+    a->ref[b] = 1;
+    s.table[k] = b;
+    pairs_out[2 * k] = s.host[k];
+    pairs_out[2 * k + 1] = b;
+  }
+  for (int32_t h : s.host) a->host_free.push_back(h);
+  s.host.clear();
+  s.swapped = false;
+  if (s.tracked) {
+    const int32_t bs = a->block_size;
+    for (int32_t j = 0; j < s.len / bs; ++j)
+      a->register_block(s.table[j], j ? s.table[j - 1] : -1, s.tokens.data() + static_cast<int64_t>(j) * bs);
+  }
+  return PA_OK;
+}
+
+int32_t pa_alloc_num_host_free(const pa_allocator* a) {
+  return a == nullptr ? -1 : static_cast<int32_t>(a->host_free.size());
+}
+
+pa_status pa_seq_host_table(const pa_allocator* a, int64_t seq_id, int32_t* out, int32_t cap, int32_t* n_out) {
+  if (a == nullptr || n_out == nullptr) return PA_ERR_INVALID_ARG;
+  auto it = a->seqs.find(seq_id);
+  if (it == a->seqs.end() || !it->second.swapped) return PA_ERR_INVALID_ARG;
+  const auto& h = it->second.host;
+  *n_out = static_cast<int32_t>(h.size());
+  if (static_cast<int64_t>(h.size()) > cap || (!h.empty() && out == nullptr)) return PA_ERR_INVALID_ARG;
+  if (!h.empty()) std::memcpy(out, h.data(), h.size() * sizeof(int32_t));
+  return PA_OK;
+}
+
 pa_status pa_alloc_evictable(const pa_allocator* a, int32_t* out, int32_t cap, int32_t* n_out) {
   if (a == nullptr || n_out == nullptr) return PA_ERR_INVALID_ARG;
   *n_out = static_cast<int32_t>(a->lru.size());
@@ -316,7 +405,7 @@ pa_status pa_seq_append_batch(pa_allocator* a, const int64_t* seq_ids, const int
 pa_status pa_seq_fork(pa_allocator* a, int64_t parent, int64_t child) {
   if (a == nullptr) return PA_ERR_INVALID_ARG;
   auto it = a->seqs.find(parent);
-  if (it == a->seqs.end() || a->seqs.count(child)) return PA_ERR_INVALID_ARG;
+  if (it == a->seqs.end() || it->second.swapped || a->seqs.count(child)) return PA_ERR_INVALID_ARG;
   Seq c = it->second;  // copy before emplace may rehash
   for (int32_t b : c.table) a->ref[b] += 1;
   a->seqs.emplace(child, std::move(c));
@@ -328,6 +417,7 @@ pa_status pa_seq_free(pa_allocator* a, int64_t seq_id) {
   auto it = a->seqs.find(seq_id);
   if (it == a->seqs.end()) return PA_ERR_INVALID_ARG;
   for (int32_t b : it->second.table) a->release(b);
+  for (int32_t h : it->second.host) a->host_free.push_back(h);
   a->seqs.erase(it);
   return PA_OK;
 }

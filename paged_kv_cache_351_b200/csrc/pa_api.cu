@@ -485,6 +485,59 @@ pa_status pa_copy_blocks(pa_tensor* k_cache, pa_tensor* v_cache, const pa_tensor
   return err == cudaSuccess ? PA_OK : launch_status();
 }
 
+// Device address of one pool of a swap: device memory of the current device,
+// or page-locked host memory the device can reach (else the kernel would
+// fault on it).
+static pa_status swap_pool_ptr(const pa_tensor* t, void** dptr) {
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, t->data) != cudaSuccess) {
+    cudaGetLastError();
+    return PA_ERR_INVALID_ARG;
+  }
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
+  if (at.type == cudaMemoryTypeDevice && at.device == dev) {
+    *dptr = t->data;
+    return PA_OK;
+  }
+  if (at.type == cudaMemoryTypeHost && at.devicePointer != nullptr) {
+    *dptr = at.devicePointer;
+    return PA_OK;
+  }
+  return PA_ERR_INVALID_ARG;  // pageable host memory, managed memory or another device's memory
+}
+
+pa_status pa_swap_blocks(const pa_tensor* src_k, const pa_tensor* src_v, pa_tensor* dst_k, pa_tensor* dst_v,
+                         const pa_tensor* pairs, const pa_opts* opts) {
+  pa_status st = check_pair(src_k, src_v);
+  if (st != PA_OK) return st;
+  st = check_pair(dst_k, dst_v);
+  if (st != PA_OK) return st;
+  if (src_k->dtype != dst_k->dtype) return PA_ERR_INVALID_ARG;
+  for (int d = 1; d < 4; ++d)
+    if (src_k->shape[d] != dst_k->shape[d]) return PA_ERR_INVALID_ARG;
+  if (pairs == nullptr || pairs->ndim != 2 || pairs->dtype != PA_I64 || pairs->shape[1] != 2) return PA_ERR_INVALID_ARG;
+  const int64_t n = pairs->shape[0];
+  if (n < 0) return PA_ERR_INVALID_ARG;
+  if (n == 0) return PA_OK;
+  if (pairs->stride[1] != 1 || pairs->stride[0] != 2 || pairs->data == nullptr) return PA_ERR_INVALID_ARG;
+  void *sk, *sv, *dk, *dv, *pp;
+  if ((st = swap_pool_ptr(src_k, &sk)) != PA_OK || (st = swap_pool_ptr(src_v, &sv)) != PA_OK ||
+      (st = swap_pool_ptr(dst_k, &dk)) != PA_OK || (st = swap_pool_ptr(dst_v, &dv)) != PA_OK ||
+      (st = swap_pool_ptr(pairs, &pp)) != PA_OK)
+    return st;
+  const int e = esize(src_k->dtype);
+  const int64_t block_vecs = src_k->shape[1] * 16 * src_k->shape[3] * e / 16;
+  const int gx = int((block_vecs + 1023) / 1024);
+  const int gy = int(n < 65535 ? n : 65535);
+  const cudaError_t err = launch_pdl(pa::swap_blocks_kernel, dim3(gx, gy), dim3(256), 0, stream_of(opts), false,
+                                     static_cast<const uint4*>(sk), static_cast<const uint4*>(sv),
+                                     static_cast<uint4*>(dk), static_cast<uint4*>(dv),
+                                     static_cast<const int64_t*>(pp), n, block_vecs, src_k->shape[0],
+                                     dst_k->shape[0]);
+  return err == cudaSuccess ? PA_OK : launch_status();
+}
+
 pa_status pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads, int32_t head_size,
                                     int32_t max_blocks_per_seq, int32_t partition_tokens, size_t* bytes_out) {
   if (bytes_out == nullptr || num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_size <= 0 ||

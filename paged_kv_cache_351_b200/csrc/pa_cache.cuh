@@ -121,6 +121,35 @@ __global__ void __launch_bounds__(256) copy_blocks_kernel(uint4* kc, uint4* vc, 
   }
 }
 
+// Swap copy: whole blocks from one pool to another (device <-> pinned host,
+// reached through unified addressing).  For each pair (src, dst):
+// dst_k[dst] = src_k[src], dst_v[dst] = src_v[src]; ids outside their pool
+// set PA_DEV_BAD_BLOCK and are skipped.
+__global__ void __launch_bounds__(256) swap_blocks_kernel(const uint4* sk, const uint4* sv, uint4* dk, uint4* dv,
+                                                          const int64_t* __restrict__ pairs, int64_t n,
+                                                          int64_t block_vecs, int64_t n_src, int64_t n_dst) {
+  pdl_wait();
+  pdl_launch_dependents();
+  for (int64_t p = blockIdx.y; p < n; p += gridDim.y) {
+    const int64_t src = pairs[2 * p], dst = pairs[2 * p + 1];
+    if (src < 0 || src >= n_src || dst < 0 || dst >= n_dst) {
+      if (blockIdx.x == 0 && threadIdx.x == 0) flag(PA_DEV_BAD_BLOCK);
+      continue;
+    }
+    const uint4* ks = sk + src * block_vecs;
+    const uint4* vs = sv + src * block_vecs;
+    uint4* kd = dk + dst * block_vecs;
+    uint4* vd = dv + dst * block_vecs;
+    for (int64_t v = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; v < block_vecs;
+         v += int64_t(gridDim.x) * blockDim.x) {
+      const uint4 a = ks[v];
+      const uint4 b = vs[v];
+      kd[v] = a;
+      vd[v] = b;
+    }
+  }
+}
+
 // One warp waits on a barrier that nothing completes; the bounded wait must
 // give up and set PA_DEV_TIMEOUT.  No copy is in flight.
 __global__ void wait_selftest_kernel(uint64_t timeout_ns) {

@@ -334,3 +334,76 @@ def test_prefix_cache_matches_oracle_random(seed):
         _compare_state(c, o)
         assert c.evictable() == list(o._evictable)
         assert c.stats()["num_cached"] == o.num_cached()
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_swap_matches_oracle_random(seed):
+    """Swap-out/in requests (with prefix caching and forks) give identical
+    pairs, tables, host tables and free counts in C++ and in the oracle."""
+    rnd = random.Random(500 + seed)
+    nb, nh, bs = 24, 18, 4
+    order = list(range(nb))
+    rnd.shuffle(order)
+    horder = list(range(nh))
+    rnd.shuffle(horder)
+    c, o = pa.Allocator(nb, bs, order), BlockAllocator(nb, bs, order)
+    c.set_host_pool(nh, horder)
+    o.set_host_pool(nh, horder)
+    live, nxt = [], 0
+
+    def both(fo, fc):
+        try:
+            ro = fo()
+        except OutOfBlocks:
+            with pytest.raises(pa.OutOfBlocksError):
+                fc()
+            return None
+        rc = fc()
+        return ro, rc
+
+    for _ in range(500):
+        resident = [s for s in live if not o.is_swapped(s)]
+        swapped = [s for s in live if o.is_swapped(s)]
+        r = rnd.random()
+        if r < 0.2 or not live:
+            prompt = [rnd.randrange(2) for _ in range(rnd.randrange(1, 14))]
+            assert c.add_prefix(nxt, prompt) == o.add_prefix(nxt, prompt)
+            hit = o.length(nxt)
+            live.append(nxt)
+            res = both(lambda: o.append_tokens(nxt, prompt[hit:]), lambda: c.append_tokens(nxt, prompt[hit:]))
+            if res:
+                assert res[1][0].tolist() == res[0][0] and res[1][1] == res[0][1]
+            nxt += 1
+        elif r < 0.3 and resident:
+            p = rnd.choice(resident)
+            o.fork(p, nxt)
+            c.fork(p, nxt)
+            live.append(nxt)
+            nxt += 1
+        elif r < 0.45:
+            s = live.pop(rnd.randrange(len(live)))
+            o.free(s)
+            c.free(s)
+        elif r < 0.6 and resident:
+            s = rnd.choice(resident)
+            res = both(lambda: o.swap_out(s), lambda: c.swap_out(s))
+            if res:
+                assert [tuple(p) for p in res[1].tolist()] == res[0]
+        elif r < 0.75 and swapped:
+            s = rnd.choice(swapped)
+            res = both(lambda: o.swap_in(s), lambda: c.swap_in(s))
+            if res:
+                assert [tuple(p) for p in res[1].tolist()] == res[0]
+        elif resident:
+            s = rnd.choice(resident)
+            n = rnd.choice([1, 3])
+            res = both(lambda: o.append(s, n), lambda: c.append(s, n))
+            if res:
+                assert res[1][0].tolist() == res[0][0] and res[1][1] == res[0][1]
+        assert c.num_free() == o.num_free() and c.num_host_free() == o.num_host_free()
+        for s in live:
+            if o.is_swapped(s):
+                assert c.host_table(s) == o.host_table(s)
+            else:
+                assert c.block_table(s) == o.block_table(s)
+        assert c.evictable() == list(o._evictable)

@@ -443,3 +443,118 @@ def test_forks_of_forks_share_and_copy():
         m.check()
     assert len({m.a.block_table(s)[1] for s in range(4)}) == 4
     assert len({m.a.block_table(s)[0] for s in range(4)}) == 1
+
+
+# ---------------------------------------------------------------------------
+# swapping
+# ---------------------------------------------------------------------------
+
+class SwapModel(PrefixIsolationModel):
+    """Adds a host pool: swap_out copies device blocks to host blocks by the
+    reported pairs, swap_in copies them back; a swapped sequence must still
+    read back its own prefixes through its host blocks."""
+
+    def __init__(self, alloc, num_host):
+        super().__init__(alloc)
+        alloc.set_host_pool(num_host, list(range(num_host)))
+        self.host = [None] * (num_host * alloc.block_size)
+
+    def swap_out(self, s):
+        bs = self.a.block_size
+        pairs = self.a.swap_out(s)
+        for b, h in pairs:
+            self.host[h * bs:(h + 1) * bs] = self.phys[b * bs:(b + 1) * bs]
+        return pairs
+
+    def swap_in(self, s):
+        bs = self.a.block_size
+        pairs = self.a.swap_in(s)
+        for h, b in pairs:
+            self.phys[b * bs:(b + 1) * bs] = self.host[h * bs:(h + 1) * bs]
+        return pairs
+
+    def check(self):
+        self.a.check_invariants()
+        bs = self.a.block_size
+        for s, toks in self.logical.items():
+            want = [tuple(toks[:t + 1]) for t in range(len(toks))]
+            if self.a.is_swapped(s):
+                ht = self.a.host_table(s)
+                got = [self.host[ht[t // bs] * bs + t % bs] for t in range(self.a.length(s))]
+            else:
+                got = [self.phys[self.a.slot(s, t)] for t in range(self.a.length(s))]
+            assert got == want, f"sequence {s} reads a foreign prefix"
+
+
+def _swap_session(seed, alloc_cls=BlockAllocator, num_blocks=24, num_host=20, bs=4, steps=500):
+    rnd = random.Random(seed)
+    order = list(range(num_blocks))
+    rnd.shuffle(order)
+    m = SwapModel(alloc_cls(num_blocks, bs, order), num_host)
+    systems = [[rnd.randrange(3) for _ in range(rnd.choice([4, 8, 9]))] for _ in range(2)]
+    nxt, swaps = 0, 0
+    for _ in range(steps):
+        live = list(m.logical)
+        resident = [s for s in live if not m.a.is_swapped(s)]
+        swapped = [s for s in live if m.a.is_swapped(s)]
+        r = rnd.random()
+        try:
+            if r < 0.2 or not live:
+                prompt = rnd.choice(systems) + [rnd.randrange(3) for _ in range(rnd.randrange(0, 6))]
+                hit = m.add_prefix(nxt, prompt)
+                nxt += 1
+                m.append_tokens(nxt - 1, prompt[hit:])
+            elif r < 0.3 and resident:
+                m.fork(rnd.choice(resident), nxt)
+                nxt += 1
+            elif r < 0.45:
+                m.free(rnd.choice(live))
+            elif r < 0.6 and resident:
+                m.swap_out(rnd.choice(resident))
+                swaps += 1
+            elif r < 0.75 and swapped:
+                m.swap_in(rnd.choice(swapped))
+            elif resident:
+                s = rnd.choice(resident)
+                if m.a._tokens.get(s) is not None:
+                    m.append_tokens(s, [rnd.randrange(3) for _ in range(rnd.choice([1, 3, 5]))])
+                else:
+                    m.append(s, rnd.choice([1, 4]))
+        except OutOfBlocks:
+            pass
+        m.check()
+    return swaps
+
+
+@pytest.mark.parametrize("seed", range(10))
+def test_swap_sessions_keep_contents(seed):
+    assert _swap_session(seed) > 0
+
+
+def test_swapped_sequence_accepts_only_swap_in_or_free():
+    a = BlockAllocator(8, 4, list(range(8)))
+    a.set_host_pool(4)
+    a.add(0)
+    a.append(0, 6)
+    a.swap_out(0)
+    for fn, args in ((a.append, (0, 1)), (a.fork, (0, 1)), (a.swap_out, (0,)), (a.append_tokens, (0, [1]))):
+        with pytest.raises(AllocatorError):
+            fn(*args)
+    a.free(0)
+    assert a.num_host_free() == 4 and a.num_free() == 8
+    a.check_invariants()
+
+
+class _MutantSwapInReversed(BlockAllocator):
+    """Planted mistake: pairs host blocks with device blocks in reverse order."""
+
+    def swap_in(self, seq):
+        pairs = super().swap_in(seq)
+        hs = [h for h, _ in pairs]
+        return list(zip(reversed(hs), [b for _, b in pairs]))
+
+
+def test_swap_pins_catch_planted_mistake():
+    with pytest.raises(AssertionError):
+        for seed in range(10):
+            _swap_session(seed, alloc_cls=_MutantSwapInReversed)
