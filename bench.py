@@ -39,6 +39,7 @@ if ROOT not in sys.path:
 
 METRIC = "paged decode attention: KV-read GB/s (% of B200 HBM peak) and decode tok/s"
 WORKLOAD = "llama7b_bs64"
+PREFILL_METRIC = "chunked-prefill paged attention: TFLOP/s (causal QK^T and PV of every new token)"
 
 
 def parse():
@@ -95,6 +96,23 @@ def step_bytes(plan):
     return {"kv": kv, "decode": decode, "write": write, "step": decode + write}
 
 
+def is_prefill(plan):
+    """A multi-token step (some sequence brings more than one new token)."""
+    return bool((plan.query_lens != 1).any())
+
+
+def prefill_flops(plan):
+    """Algorithmic FLOPs of one multi-token step: the new token at position p
+    of a sequence attends p + 1 keys in every query head, 2 * D flops for its
+    QK^T dot product and 2 * D for its share of P V per key."""
+    w = plan.workload
+    total = 0
+    for c, n in zip(plan.context_lens.tolist(), plan.query_lens.tolist()):
+        prior = c - n
+        total += n * prior + n * (n + 1) // 2
+    return 4 * w.head_size * w.num_heads * total
+
+
 def measured_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -102,6 +120,16 @@ def measured_peaks():
         return float(d["hbm_gbs"]), "measured"
     except Exception:
         return 6650.0, "fallback"
+
+
+def measured_tensor_peak():
+    """Dense bf16 tensor peak (burst: the prefill kernel is timed alone)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
 
 
 def kernel_source_hash():
@@ -301,11 +329,62 @@ def oracle_timing(plan, seconds, max_rows=None):
             "tok_per_s": rows_done / el}
 
 
+def oracle_timing_prefill(plan, seconds):
+    """Time the multi-token oracle as it stands on whole sequences of the
+    workload (all their new tokens, all heads) until ``seconds`` have passed."""
+    from oracle.prefill import paged_prefill_seqs
+    from oracle.replay import block_table_array, replay
+    from workloads import query_values
+
+    alloc, cache, _ = replay(plan)
+    tables = block_table_array(alloc, plan.batch, plan.max_blocks_per_seq)
+    q = query_values(plan)
+    w = plan.workload
+    scale = 1.0 / math.sqrt(w.head_size)
+    order = sorted(range(plan.B), key=lambda i: int(plan.context_lens[i]))  # short sequences first
+    flops, seqs, k = 0, 0, 0
+    t0 = time.perf_counter()
+    while True:
+        i = order[k % plan.B]
+        paged_prefill_seqs(q, cache, tables, plan.context_lens, plan.query_start, scale, [i])
+        c, n = int(plan.context_lens[i]), int(plan.query_lens[i])
+        flops += 4 * w.head_size * w.num_heads * (n * (c - n) + n * (n + 1) // 2)
+        seqs += 1
+        k += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    try:
+        from threadpoolctl import threadpool_info
+
+        cores = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
+    except Exception:
+        cores = 1
+    return {"tflops": flops / el / 1e12, "seconds": el, "seqs": seqs, "cores": cores}
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     plan = workload_plan(args.workload)
+    if is_prefill(plan):
+        per = max(1.0, min(10.0, 120.0 / max(1, args.steps + args.warmup)))
+        res = [oracle_timing_prefill(plan, per) for _ in range(max(1, args.steps))]
+        tf = statistics.median(r["tflops"] for r in res)
+        tot_s = sum(r["seconds"] for r in res)
+        line = {
+            "impl": "reference", "metric": PREFILL_METRIC, "value": round(tf, 6), "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1000 * tot_s / max(1, args.steps), 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+            "config": {"workload": f"{plan.workload.name}: {plan.workload.description}", "sample": "whole sequences"},
+            "cpu_baseline": {"value": round(tf, 6), "unit": "TFLOP/s", "cores": res[0]["cores"], "kind": "oracle",
+                             "sample": f"{sum(r['seqs'] for r in res)} whole sequences, about {per:.1f} s per step"},
+            "e2e": {"value": round(tf, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }
+        print(json.dumps(line), flush=True)
+        return
     per = max(0.5, min(5.0, 120.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
         oracle_timing(plan, per / 4, max_rows=1)
@@ -354,6 +433,8 @@ def run_ours(args):
     if args.tuning:
         pa.pa_set_decode_tuning(*[int(x) for x in args.tuning.split(",")])
     plan = workload_plan(args.workload, args.pool_gb)
+    if is_prefill(plan):
+        return run_prefill(args, plan, device, world, rank)
     w = plan.workload
     nbytes = step_bytes(plan)
     kv, inp = setup_device(plan, device)
@@ -541,6 +622,159 @@ def run_ours(args):
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": launches_per_step * K,
+        "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_prefill(args, plan, device, world, rank):
+    """GPU arm for a multi-token (chunked-prefill) workload: a step writes
+    the new tokens' K/V into the cache (pa_reshape_and_cache) and runs
+    pa_prefill over them; value = the step's attention FLOPs / device time."""
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import paged_kv_cache_351_b200 as pa
+
+    w = plan.workload
+    flops = prefill_flops(plan)
+    kv, inp = setup_device(plan, device)
+    dev = inp["dev"]
+    q, key, value = dev(inp["query"]), dev(inp["key"]), dev(inp["value"])
+    slots = torch.from_numpy(inp["slots"]).to(device)
+    bt = torch.from_numpy(inp["tables"]).to(device)
+    cl = torch.from_numpy(inp["lens"]).to(device)
+    qs = torch.from_numpy(plan.query_start).to(device)
+    mq = int(plan.query_lens.max())
+    out = torch.empty_like(q)
+    scale = 1.0 / math.sqrt(w.head_size)
+    stream = torch.cuda.Stream(device)
+    T = plan.num_query_rows
+    write_bytes = T * w.num_kv_heads * w.head_size * 2 * (w.elem_bytes + w.cache_elem_bytes) + 8 * T
+
+    def attend(o, qq, b, c, s):
+        pa.pa_prefill(o, qq, kv.k_cache, kv.v_cache, b, c, s, mq, scale, w.num_kv_heads, stream=stream)
+
+    def step():
+        kv.write(slots, key, value, None, stream=stream)
+        attend(out, q, bt, cl, qs)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            step()
+    torch.cuda.synchronize()
+    st, bits = pa.pa_get_device_status(stream)
+    if st != 0:
+        raise RuntimeError(f"device status {st} bits {bits:#x} after warm-up")
+    K = args.steps
+    uuid = str(torch.cuda.get_device_properties(device).uuid)
+    uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+    sampler = ClockSampler(uuid)
+    time.sleep(0.25)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        for _ in range(K):
+            step()
+        ev1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    elapsed = ev0.elapsed_time(ev1)
+    ea = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    eb = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    with torch.cuda.stream(stream):
+        for k in range(K):
+            ea[k].record(stream)
+            attend(out, q, bt, cl, qs)
+            eb[k].record(stream)
+    torch.cuda.synchronize()
+    pf_ms = statistics.mean(ea[k].elapsed_time(eb[k]) for k in range(K))
+    t_soak = time.perf_counter()
+    with torch.cuda.stream(stream):
+        while time.perf_counter() - t_soak < max(0.0, 0.6 - elapsed / 1000):
+            for _ in range(20):
+                step()
+            torch.cuda.synchronize()
+    clocks = sampler.stop()
+    st, bits = pa.pa_get_device_status(stream)
+    if st != 0:
+        raise RuntimeError(f"device status {st} bits {bits:#x} after the timed region")
+    elapsed, pf_ms = max_over_ranks([elapsed, pf_ms], device, world)
+    ms_step = elapsed / K
+    value = flops * world / (ms_step * 1e-3) / 1e12
+    peak, peak_kind = measured_tensor_peak()
+
+    e2e = None
+    if not args.no_e2e:
+        pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()  # noqa: E731
+        h_in = (pin(inp["query"].view(np.int16)), pin(inp["key"].view(np.int16)), pin(inp["value"].view(np.int16)),
+                pin(inp["slots"]), pin(inp["tables"]), pin(inp["lens"]), pin(plan.query_start))
+        h_out = torch.empty(out.shape, dtype=torch.int16).pin_memory()
+        d_in = tuple(torch.empty(x.shape, dtype=x.dtype, device=device) for x in h_in)
+        h2d = sum(x.numel() * x.element_size() for x in h_in)
+        d2h = h_out.numel() * h_out.element_size()
+        bf = lambda t: t.view(torch.bfloat16)  # noqa: E731
+
+        def e2e_step():
+            for d, h in zip(d_in, h_in):
+                d.copy_(h, non_blocking=True)
+            d_q, d_k, d_v, d_s, d_bt, d_cl, d_qs = d_in
+            kv.write(d_s, bf(d_k), bf(d_v), None, stream=stream)
+            attend(out, bf(d_q), d_bt, d_cl, d_qs)
+            h_out.copy_(out.view(torch.int16), non_blocking=True)
+
+        with torch.cuda.stream(stream):
+            for _ in range(max(3, args.warmup)):
+                e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            f0.record(stream)
+            for _ in range(K):
+                e2e_step()
+            f1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = max_over_ranks([f0.elapsed_time(f1)], device, world)[0] / K
+        e2e = {"value": round(flops * world / (e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": round(e_ms, 5),
+               "overlap": "none: copies in, step, copy out, serialised on one stream"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        r = oracle_timing_prefill(plan, args.cpu_seconds)
+        cpu = {"value": round(r["tflops"], 6), "unit": "TFLOP/s", "cores": r["cores"], "kind": "oracle",
+               "sample": f"{r['seqs']} whole sequences (all new tokens, all heads) in {r['seconds']:.1f} s"}
+    achieved = flops / (pf_ms * 1e-3) / 1e12
+    line = {
+        "metric": PREFILL_METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded)",
+        "config": {"workload": f"{w.name}: {w.description}", "query_rows": T, "sequences": plan.B,
+                   "sum_context_tokens": int(plan.context_lens.sum()), "parallelism": f"replicas x{world}",
+                   "l2": "no flush: each step rewrites the new tokens' K/V and reads "
+                         f"{int(plan.context_lens.sum()) * 2 * w.num_kv_heads * w.head_size * 2 / 1e9:.2f} GB of "
+                         "cache per kv head group; the kernel is tensor-bound"},
+        "tokens_per_s": round(T * world / (ms_step * 1e-3), 1),
+        "flops_per_step": flops, "write_bytes_per_step": write_bytes,
+        "roofline": {"bound": "tensor", "kernel": "pa_prefill (prefill_kernel, tcgen05)", "achieved": round(achieved, 2),
+                     "peak": peak, "peak_kind": peak_kind + " bf16 dense (burst)", "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "traffic": None, "algorithmic_flops_per_launch": flops,
+                     "avg_launch_ms": round(pf_ms, 5),
+                     "timing": f"{K} prefill launches, each bracketed by CUDA events, after the timed region"},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": 2 * K,
         "clocks": clocks,
     }
     if rank == 0:

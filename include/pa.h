@@ -242,6 +242,48 @@ pa_status pa_decode_fp8(pa_tensor* out, const pa_tensor* query, const pa_tensor*
                         int32_t num_kv_heads, const pa_tensor* k_scale, const pa_tensor* v_scale,
                         const pa_opts* opts);
 
+/* ---------------------------------------------------------------------------
+ * Multi-token (chunked-prefill) paged attention.  The pages list chunked
+ * prefill among the serving-loop optimisations: a long prompt's prefill is
+ * cut into chunks that run in the same step as decode requests (gitcode
+ * walkthrough, section 2.2); the attention is the section 2.1 computation
+ * applied to every new token, causally:
+ *
+ *   sequence i has n_i = query_start[i+1] - query_start[i] new tokens at
+ *   positions c_i + j (c_i = context_lens[i] - n_i; their K/V must already
+ *   be in the cache, e.g. by pa_reshape_and_cache earlier on the stream);
+ *   for row r = query_start[i] + j and query head h, g = h / (H / H_kv):
+ *     s_t = scale * <query[r,h,:], K_i[t, g, :]>,  t = 0 .. c_i + j
+ *     out[r,h,:] = sum_t softmax(s)_t V_i[t, g, :]
+ *
+ * A decode request is n_i = 1; a whole prompt is n_i = context_lens[i];
+ * n_i = 0 writes nothing.  Runs on the tensor cores (tcgen05): QK^T and PV
+ * in bf16 with fp32 accumulation, the probabilities rounded to bf16 before
+ * the PV product (and the softmax denominator summed from the rounded
+ * values), output rounded to nearest even.
+ *
+ * out, query:   [T, H, 128] bf16, last dim contiguous, strides multiples of
+ *               16 bytes, 16-byte aligned (T = total new tokens).  Rows not
+ *               covered by any sequence are left unwritten.
+ * k_cache, v_cache: bf16 [num_blocks, H_kv, 16, 128] (layout above).
+ * block_tables: [B, max_blocks_per_seq] int32 (entries past
+ *               ceil(context_lens[i] / 16) are not read; bad ids set
+ *               PA_DEV_BAD_BLOCK and are replaced by block 0).
+ * context_lens: [B] int32, tokens of sequence i after the step.
+ * query_start:  [B + 1] int32 on the device, non-decreasing, query_start[0]
+ *               >= 0, query_start[B] <= T.  A sequence with n_i < 0,
+ *               n_i > context_lens[i], rows outside [0, T), context_lens[i]
+ *               above the table capacity, or n_i > max_query_len sets
+ *               PA_DEV_BAD_CONTEXT and is skipped.
+ * max_query_len: host-side bound on every n_i (sizes the grid).
+ * scale:        softmax scale, finite and > 0.
+ * H / H_kv in {1, 2, 4, 8}; B <= 65535.  No workspace.  Other dtypes or
+ * head sizes return PA_ERR_UNSUPPORTED.
+ * ------------------------------------------------------------------------- */
+pa_status pa_prefill(pa_tensor* out, const pa_tensor* query, const pa_tensor* k_cache, const pa_tensor* v_cache,
+                     const pa_tensor* block_tables, const pa_tensor* context_lens, const pa_tensor* query_start,
+                     int32_t max_query_len, float scale, int32_t num_kv_heads, const pa_opts* opts);
+
 /* Workspace bytes pa_decode needs on the current device for these sizes and
  * this partition_tokens setting (0 = auto/balanced, >0 = fixed, -1 = none).
  * Needs a CUDA device for the auto mode (it depends on the SM count). */

@@ -131,6 +131,17 @@ def pa_decode(out, query, k_cache, v_cache, block_tables, context_lens, scale: f
                                  ctypes.byref(o)), "pa_decode")
 
 
+def pa_prefill(out, query, k_cache, v_cache, block_tables, context_lens, query_start, max_query_len: int,
+               scale: float, num_kv_heads: int, stream=None, timeout_ms: int = 0) -> None:
+    """Multi-token (chunked-prefill) paged attention: writes out [T, H, D]
+    for the new tokens of every sequence (rows query_start[i] ..
+    query_start[i+1]), each attending causally over its sequence's cache."""
+    ts = [_tensor(x) for x in (out, query, k_cache, v_cache, block_tables, context_lens, query_start)]
+    o = _opts(stream, timeout_ms=timeout_ms)
+    _check(_lib_handle.pa_prefill(*[ctypes.byref(t) for t in ts], int(max_query_len), ctypes.c_float(scale),
+                                  int(num_kv_heads), ctypes.byref(o)), "pa_prefill")
+
+
 def pa_reshape_and_cache_fp8(key, value, k_cache, v_cache, slot_mapping, k_scale, v_scale, stream=None) -> None:
     """Quantizing cache write into an FP8 (torch.float8_e4m3fn) cache: each
     value is stored as the e4m3 code of value / scale[kv head]."""

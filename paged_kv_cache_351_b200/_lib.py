@@ -72,6 +72,7 @@ SIGNATURES = {
     "pa_decode_no_alloc": (c_int32, [_T, _T, _T, _T, _T, _T, c_float, c_int32, _O]),
     "pa_reshape_and_cache_fp8": (c_int32, [_T, _T, _T, _T, _T, _T, _T, _O]),
     "pa_decode_fp8": (c_int32, [_T, _T, _T, _T, _T, _T, c_float, c_int32, _T, _T, _O]),
+    "pa_prefill": (c_int32, [_T, _T, _T, _T, _T, _T, _T, c_int32, c_float, c_int32, _O]),
     "pa_decode_workspace_bytes": (c_int32, [c_int32, c_int32, c_int32, c_int32, c_int32, c_int32, POINTER(c_size_t)]),
     "pa_set_decode_tuning": (c_int32, [c_int32, c_int32, c_int32]),
     "pa_alloc_create": (c_int32, [c_int32, c_int32, _I32P, POINTER(_A)]),

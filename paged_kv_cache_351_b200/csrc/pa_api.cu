@@ -3,6 +3,8 @@
 // status word is a plain __device__ variable, no relocatable device code).
 // The host allocator is in pa_alloc.cpp.
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <unistd.h>
@@ -18,6 +20,7 @@
 #include "pa_cache.cuh"
 #include "pa_common.cuh"
 #include "pa_decode.cuh"
+#include "pa_prefill.cuh"
 
 namespace {
 
@@ -327,6 +330,54 @@ pa_status plan_decode(int32_t dtype, int64_t B, int64_t H, int64_t Hkv, int64_t 
   } else {
     return PA_ERR_INVALID_ARG;
   }
+  return PA_OK;
+}
+
+// ---------------------------------------------------------------------------
+// prefill launch plumbing: tensor maps for the tiled TMA loads
+// ---------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    cudaGetLastError();
+  });
+  return fn;
+}
+
+// bf16 tensor map with 128-byte swizzle; dims innermost first, strides in
+// bytes for dims 1.. (each a multiple of 16), out-of-range elements read 0.
+pa_status bf16_map(CUtensorMap* m, void* ptr, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
+                   const cuuint32_t* box) {
+  PFN_cuTensorMapEncodeTiled_v12000 fn = tensor_map_encoder();
+  if (fn == nullptr) return PA_ERR_CUDA;
+  const cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, cuuint32_t(rank), ptr, dims, strides, box, es,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? PA_OK : PA_ERR_INVALID_ARG;
+}
+
+template <int G>
+pa_status run_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const pa::PrefillArgs& a,
+                      int max_query_len, int Hkv, cudaStream_t st, int dev) {
+  static bool attr_set[kMaxDevices] = {};
+  auto kern = pa::prefill_kernel<G>;
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(pa::kPfSmemBytes)) !=
+        cudaSuccess)
+      return launch_status();
+    attr_set[dev] = true;
+  }
+  constexpr int TOK = 128 / G;
+  const dim3 grid(unsigned((max_query_len + TOK - 1) / TOK), unsigned(Hkv), unsigned(a.B));
+  if (launch_pdl(kern, grid, dim3(pa::kPfThreads), pa::kPfSmemBytes, st, true, tq, tk, tv, a) != cudaSuccess)
+    return launch_status();
   return PA_OK;
 }
 
@@ -681,6 +732,86 @@ pa_status pa_decode_fp8(pa_tensor* out, const pa_tensor* query, const pa_tensor*
   if (k_cache == nullptr || k_cache->dtype != PA_FP8_E4M3) return PA_ERR_INVALID_ARG;
   return decode_impl(out, query, k_cache, v_cache, block_tables, context_lens, scale, num_kv_heads, k_scale, v_scale,
                      opts);
+}
+
+pa_status pa_prefill(pa_tensor* out, const pa_tensor* query, const pa_tensor* k_cache, const pa_tensor* v_cache,
+                     const pa_tensor* block_tables, const pa_tensor* context_lens, const pa_tensor* query_start,
+                     int32_t max_query_len, float scale, int32_t num_kv_heads, const pa_opts* opts) {
+  pa_status st = check_pair(k_cache, v_cache);
+  if (st != PA_OK) return st;
+  const int64_t NB = k_cache->shape[0], Hkv = k_cache->shape[1], D = k_cache->shape[3];
+  if (k_cache->dtype != PA_BF16 || D != 128) return PA_ERR_UNSUPPORTED;
+  if (num_kv_heads != Hkv) return PA_ERR_INVALID_ARG;
+  if (query == nullptr || query->ndim != 3) return PA_ERR_INVALID_ARG;
+  const int64_t T = query->shape[0], H = query->shape[1];
+  if (T < 0 || H <= 0 || H % Hkv) return PA_ERR_INVALID_ARG;
+  if ((st = check_rows3(query, PA_BF16, T, H, D)) != PA_OK) return st;
+  if ((st = check_rows3(out, PA_BF16, T, H, D)) != PA_OK) return st;
+  if (context_lens == nullptr || context_lens->ndim != 1 || context_lens->dtype != PA_I32) return PA_ERR_INVALID_ARG;
+  const int64_t B = context_lens->shape[0];
+  if (B < 0 || (B > 0 && (context_lens->stride[0] != 1 || context_lens->data == nullptr))) return PA_ERR_INVALID_ARG;
+  if (query_start == nullptr || query_start->ndim != 1 || query_start->dtype != PA_I32 ||
+      query_start->shape[0] != B + 1 || query_start->stride[0] != 1 || query_start->data == nullptr)
+    return PA_ERR_INVALID_ARG;
+  if (block_tables == nullptr || block_tables->ndim != 2 || block_tables->dtype != PA_I32 ||
+      block_tables->shape[0] != B || block_tables->shape[1] < 0)
+    return PA_ERR_INVALID_ARG;
+  const int64_t max_nb = block_tables->shape[1];
+  if (B > 0 && max_nb > 0 &&
+      (block_tables->stride[1] != 1 || block_tables->stride[0] < max_nb || block_tables->data == nullptr))
+    return PA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return PA_ERR_INVALID_ARG;
+  if (max_query_len < 0 || (T > 0 && max_query_len == 0) || max_query_len > T) return PA_ERR_INVALID_ARG;
+  const int64_t G = H / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return PA_ERR_UNSUPPORTED;
+  if (B > 65535 || T >= (int64_t(1) << 31) || max_nb * 16 > INT32_MAX) return PA_ERR_UNSUPPORTED;
+  if (B == 0 || T == 0) return PA_OK;
+
+  DeviceInfo di;
+  int dev = 0;
+  if ((st = device_info(&di, &dev)) != PA_OK) return st;
+  if (di.smem_optin < int(pa::kPfSmemBytes)) return PA_ERR_UNSUPPORTED;
+
+  CUtensorMap tq, tk, tv;
+  {
+    const cuuint64_t dims[3] = {cuuint64_t(D), cuuint64_t(H), cuuint64_t(T)};
+    const cuuint64_t strides[2] = {cuuint64_t(query->stride[1]) * 2, cuuint64_t(query->stride[0]) * 2};
+    const cuuint32_t box[3] = {64, cuuint32_t(G), cuuint32_t(128 / G)};
+    if ((st = bf16_map(&tq, query->data, 3, dims, strides, box)) != PA_OK) return st;
+  }
+  {
+    const cuuint64_t dims[4] = {cuuint64_t(D), 16, cuuint64_t(Hkv), cuuint64_t(NB)};
+    const cuuint64_t strides[3] = {cuuint64_t(D) * 2, cuuint64_t(16 * D) * 2, cuuint64_t(Hkv * 16 * D) * 2};
+    const cuuint32_t box[4] = {64, 16, 1, 1};
+    if ((st = bf16_map(&tk, k_cache->data, 4, dims, strides, box)) != PA_OK) return st;
+    if ((st = bf16_map(&tv, v_cache->data, 4, dims, strides, box)) != PA_OK) return st;
+  }
+  pa::PrefillArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.out = static_cast<__nv_bfloat16*>(out->data);
+  a.o_st = out->stride[0];
+  a.o_sh = out->stride[1];
+  a.bt = static_cast<const int32_t*>(block_tables->data);
+  a.bt_stride = block_tables->stride[0];
+  a.ctx = static_cast<const int32_t*>(context_lens->data);
+  a.query_start = static_cast<const int32_t*>(query_start->data);
+  a.B = int32_t(B);
+  a.T = int32_t(T);
+  a.max_nb = int32_t(max_nb);
+  a.num_blocks = int32_t(NB);
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.timeout_ns = timeout_of(opts);
+  cudaStream_t s = stream_of(opts);
+  switch (G) {
+    case 1:
+      return run_prefill<1>(tq, tk, tv, a, max_query_len, int(Hkv), s, dev);
+    case 2:
+      return run_prefill<2>(tq, tk, tv, a, max_query_len, int(Hkv), s, dev);
+    case 4:
+      return run_prefill<4>(tq, tk, tv, a, max_query_len, int(Hkv), s, dev);
+    default:
+      return run_prefill<8>(tq, tk, tv, a, max_query_len, int(Hkv), s, dev);
+  }
 }
 
 pa_status pa_get_device_status(const pa_opts* opts, uint32_t* bits_out) {

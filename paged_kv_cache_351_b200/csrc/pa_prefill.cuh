@@ -1,0 +1,361 @@
+// Multi-token (chunked-prefill) paged attention on the tensor cores (sm_100a).
+//
+// What it computes (gitcode repo walkthrough, section 2.2: a long prompt's
+// prefill is cut into chunks that run in the same step as decode requests;
+// section 2.1: the attention itself is the QK dot product, softmax and
+// weighted sum of V over K/V gathered through the block table): sequence i
+// brings n_i new tokens at positions c_i .. c_i + n_i - 1 (c_i = ctx_i - n_i,
+// their K/V already in the cache); the query row of position p and head h
+// attends keys 0 .. p of kv head h / G.
+//
+// Design.  One CTA owns 128 query rows of one (sequence, kv head): 128 / G
+// consecutive new tokens times the G query heads of the kv head, so every
+// K/V page a CTA loads serves all heads of its group.  Keys stream in tiles
+// of 128 tokens (8 pages).  Per tile:
+//   S = Q K^T        tcgen05.mma, M = 128, N = 128, K = 128, fp32 in TMEM;
+//   P = exp(S - m)   4 softmax warps, one query row per thread, online max;
+//   O += P V         tcgen05.mma, P (bf16) from shared memory, O in TMEM.
+// Q, K and V reach shared memory through tiled TMA loads with 128-byte
+// swizzle: Q as one box of [128/G tokens][G heads][64 dims] per half of the
+// head dimension, each K/V page as a [16 tokens][64 dims] box per half (a
+// page is one (block, kv head) of the cache, its id from the block table).
+// Warp roles: warp 0 issues TMA loads, warp 1 owns TMEM and issues the MMAs
+// (one thread), warps 4-7 run the softmax and the epilogue.  S is double
+// buffered in TMEM, so the MMA of S for tile j + 1 runs while the softmax
+// of tile j does; K/V use two stages.  Every wait is bounded by the caller's
+// timeout (PA_DEV_TIMEOUT), after which each role stops, waits (bounded) for
+// its own copies and MMAs in flight, and TMEM is released.
+#pragma once
+
+#include "pa_common.cuh"
+#include "pa_tc.cuh"
+
+namespace pa {
+
+struct PrefillArgs {
+  __nv_bfloat16* out;  // [T, H, 128]
+  int64_t o_st, o_sh;  // element strides of out (token, head)
+  const int32_t* bt;   // block tables [B, max_nb]
+  int64_t bt_stride;
+  const int32_t* ctx;          // [B] tokens in the cache after the step
+  const int32_t* query_start;  // [B + 1] first query row of each sequence
+  int32_t B, T, max_nb, num_blocks;
+  float scale_log2;  // scale * log2(e), > 0
+  uint64_t timeout_ns;
+};
+
+constexpr int kPfThreads = 256;
+constexpr uint32_t kPfHalf = 16384;  // 128 rows x 128 bytes: one 64-dim half of a 128 x 128 bf16 tile
+constexpr uint32_t kPfTile = 2 * kPfHalf;
+constexpr uint32_t kSmQ = 0;
+constexpr uint32_t kSmK = kSmQ + kPfTile;      // two stages
+constexpr uint32_t kSmV = kSmK + 2 * kPfTile;  // two stages
+constexpr uint32_t kSmP = kSmV + 2 * kPfTile;
+constexpr uint32_t kSmBar = kSmP + kPfTile;
+constexpr uint32_t kPfSmemBytes = kSmBar + 128 + 1024;  // + barriers + alignment slack
+constexpr uint32_t kPfTmemCols = 512;                   // S0 [0,128), S1 [128,256), O [256,384)
+
+// Barrier slots (8 bytes each) after kSmBar.
+enum PfBar : int {
+  kBarQ = 0,
+  kBarKFull = 1,   // + stage
+  kBarVFull = 3,   // + stage
+  kBarKVFree = 5,  // + stage
+  kBarSFull = 7,   // + S buffer
+  kBarPFull = 9,
+  kBarODone = 10,
+  kBarDrain = 11,
+  kBarTmemSlot = 12,  // 4-byte TMEM base address
+};
+
+// All lanes wait; the warp agrees on the outcome so that warp-collective
+// tcgen05 instructions stay converged.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
+  const bool ok = mbar_wait_bounded(bar, parity, timeout_ns);
+  return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+template <int G>
+__global__ void __launch_bounds__(kPfThreads, 1)
+    prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const PrefillArgs a) {
+  constexpr int TOK = 128 / G;  // new tokens per CTA
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  auto bar = [&](int i) { return base + kSmBar + 8u * uint32_t(i); };
+
+  pdl_wait();
+  pdl_launch_dependents();
+
+  const int seq = blockIdx.z;
+  const int kvh = blockIdx.y;
+  const int qt = int(gridDim.x) - 1 - int(blockIdx.x);  // longest key ranges first
+  const int q0 = a.query_start[seq];
+  const int qlen = a.query_start[seq + 1] - q0;
+  const int ctx = a.ctx[seq];
+  if (q0 < 0 || qlen < 0 || q0 + qlen > a.T || qlen > ctx || ctx > a.max_nb * 16 ||
+      qlen > int(gridDim.x) * TOK) {
+    if (threadIdx.x == 0 && blockIdx.x == 0 && kvh == 0) flag(PA_DEV_BAD_CONTEXT);
+    return;
+  }
+  if (qt * TOK >= qlen) return;  // this tile holds no new token of the sequence
+  const int c0 = ctx - qlen;
+  const int tok_end = min(qlen, (qt + 1) * TOK);
+  const int kv_len = c0 + tok_end;  // keys seen by the tile's last token
+  const int nt = (kv_len + 127) / 128;
+  const int npages = (kv_len + 15) / 16;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(bar(kBarQ), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(kBarKFull + s), 1);
+      mbar_init(bar(kBarVFull + s), 1);
+      mbar_init(bar(kBarKVFree + s), 1);
+      mbar_init(bar(kBarSFull + s), 1);
+    }
+    mbar_init(bar(kBarPFull), 128);
+    mbar_init(bar(kBarODone), 1);
+    mbar_init(bar(kBarDrain), 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) tc::tmem_alloc(bar(kBarTmemSlot), kPfTmemCols);
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + kSmBar + 8 * kBarTmemSlot);
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    const int32_t* bt = a.bt + int64_t(seq) * a.bt_stride;
+    if (lane == 0) {
+      tc::tma_prefetch_desc(&tm_q);
+      tc::tma_prefetch_desc(&tm_k);
+      tc::tma_prefetch_desc(&tm_v);
+      mbar_arrive_expect_tx(bar(kBarQ), kPfTile);
+      tc::tma_load_3d(base + kSmQ, &tm_q, 0, kvh * G, q0 + qt * TOK, bar(kBarQ));
+      tc::tma_load_3d(base + kSmQ + kPfHalf, &tm_q, 64, kvh * G, q0 + qt * TOK, bar(kBarQ));
+    }
+    bool ok = true;
+    int issued = 0;  // tiles whose loads were issued
+    for (int j = 0; j < nt; ++j) {
+      const int s = j & 1;
+      if (j >= 2 && !(ok = warp_wait(bar(kBarKVFree + s), ((j >> 1) - 1) & 1, a.timeout_ns))) break;
+      const int p0 = j * 8;
+      const int np = min(8, npages - p0);
+      int blk = 0;
+      if (lane < np) {
+        blk = bt[p0 + lane];
+        if (blk < 0 || blk >= a.num_blocks) {
+          flag(PA_DEV_BAD_BLOCK);
+          blk = 0;
+        }
+      }
+      if (lane == 0) {
+        mbar_arrive_expect_tx(bar(kBarKFull + s), uint32_t(np) * 4096u);
+        mbar_arrive_expect_tx(bar(kBarVFull + s), uint32_t(np) * 4096u);
+      }
+      for (int p = 0; p < np; ++p) {
+        const int b = __shfl_sync(0xffffffffu, blk, p);
+        if (lane == 0) {
+          const uint32_t dk = base + kSmK + uint32_t(s) * kPfTile + uint32_t(p) * 2048u;
+          tc::tma_load_4d(dk, &tm_k, 0, 0, kvh, b, bar(kBarKFull + s));
+          tc::tma_load_4d(dk + kPfHalf, &tm_k, 64, 0, kvh, b, bar(kBarKFull + s));
+        }
+      }
+      for (int p = 0; p < np; ++p) {
+        const int b = __shfl_sync(0xffffffffu, blk, p);
+        if (lane == 0) {
+          const uint32_t dv = base + kSmV + uint32_t(s) * kPfTile + uint32_t(p) * 2048u;
+          tc::tma_load_4d(dv, &tm_v, 0, 0, kvh, b, bar(kBarVFull + s));
+          tc::tma_load_4d(dv + kPfHalf, &tm_v, 64, 0, kvh, b, bar(kBarVFull + s));
+        }
+      }
+      issued = j + 1;
+    }
+    // Before the CTA may exit, every copy it started must have landed.
+    mbar_wait_bounded(bar(kBarQ), 0, a.timeout_ns);
+    for (int j = max(0, issued - 2); j < issued; ++j) {
+      mbar_wait_bounded(bar(kBarKFull + (j & 1)), (j >> 1) & 1, a.timeout_ns);
+      mbar_wait_bounded(bar(kBarVFull + (j & 1)), (j >> 1) & 1, a.timeout_ns);
+    }
+    (void)ok;
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    constexpr uint32_t kIdQK = tc::idesc_bf16_f32(128, 128, false, false);
+    constexpr uint32_t kIdPV = tc::idesc_bf16_f32(128, 128, false, true);
+    auto issue_qk = [&](int j) {  // S[j & 1] = Q K_j^T
+      const uint32_t d = tmem + uint32_t(j & 1) * 128u;
+      const uint32_t kb = base + kSmK + uint32_t(j & 1) * kPfTile;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t off = uint32_t(kk >> 2) * kPfHalf + uint32_t(kk & 3) * 32u;
+        tc::mma_bf16_ss(d, tc::desc_kmajor(base + kSmQ + off), tc::desc_kmajor(kb + off), kIdQK, kk > 0);
+      }
+    };
+    bool ok = warp_wait(bar(kBarQ), 0, a.timeout_ns) && warp_wait(bar(kBarKFull), 0, a.timeout_ns);
+    if (ok) {
+      tc::fence_after_sync();
+      if (lane == 0) {
+        issue_qk(0);
+        tc::commit(bar(kBarSFull));
+      }
+      __syncwarp();
+    }
+    for (int j = 0; ok && j < nt; ++j) {
+      const int s = j & 1;
+      if (j + 1 < nt) {
+        if (!(ok = warp_wait(bar(kBarKFull + (s ^ 1)), ((j + 1) >> 1) & 1, a.timeout_ns))) break;
+        tc::fence_after_sync();
+        if (lane == 0) {
+          issue_qk(j + 1);
+          tc::commit(bar(kBarSFull + (s ^ 1)));
+        }
+        __syncwarp();
+      }
+      if (!(ok = warp_wait(bar(kBarPFull), j & 1, a.timeout_ns))) break;
+      if (!(ok = warp_wait(bar(kBarVFull + s), (j >> 1) & 1, a.timeout_ns))) break;
+      tc::fence_after_sync();
+      const int valid = kv_len - j * 128;
+      if (valid < 128) {
+        // Rows past the last key hold stale or never-written values (NaN
+        // would survive a zero probability): clear them before P V.
+        uint8_t* vs = gbase + kSmV + uint32_t(s) * kPfTile;
+        const int rows = 128 - valid;
+        for (int e = lane; e < rows * 16; e += 32) {
+          const int r = valid + (e >> 4), c = e & 15;
+          *reinterpret_cast<uint4*>(vs + uint32_t(c >> 3) * kPfHalf + uint32_t(r) * 128u + uint32_t(c & 7) * 16u) =
+              make_uint4(0u, 0u, 0u, 0u);
+        }
+        tc::fence_proxy_async_smem();
+        __syncwarp();
+      }
+      if (lane == 0) {
+        const uint32_t vb = base + kSmV + uint32_t(s) * kPfTile;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t pa_off = uint32_t(kk >> 2) * kPfHalf + uint32_t(kk & 3) * 32u;
+          tc::mma_bf16_ss(tmem + 256u, tc::desc_kmajor(base + kSmP + pa_off),
+                          tc::desc_mnmajor(vb + uint32_t(kk) * 2048u, kPfHalf), kIdPV, j > 0 || kk > 0);
+        }
+        tc::commit(bar(kBarODone));
+        tc::commit(bar(kBarKVFree + s));
+      }
+      __syncwarp();
+    }
+    // No MMA may still run when TMEM is released.
+    if (lane == 0) tc::commit(bar(kBarDrain));
+    __syncwarp();
+    mbar_wait_bounded(bar(kBarDrain), 0, a.timeout_ns);
+  } else if (warp >= 4) {
+    // ---------------- softmax + epilogue: one query row per thread ----------------
+    const int r = (warp - 4) * 32 + lane;
+    const int tok = r / G, g = r - (r / G) * G;
+    const int qi = qt * TOK + tok;
+    const bool row_valid = qi < qlen;
+    const int kmax = row_valid ? c0 + qi + 1 : 0;  // keys [0, kmax) are visible
+    const uint32_t tl = tmem + (uint32_t((warp - 4) * 32) << 16);
+    const float cl = a.scale_log2;
+    float m_raw = -INFINITY, l = 0.f;
+    bool ok = true;
+    uint8_t* sp = gbase + kSmP + uint32_t(r) * 128u;
+    for (int j = 0; j < nt; ++j) {
+      const int s = j & 1;
+      if (!(ok = warp_wait(bar(kBarSFull + s), (j >> 1) & 1, a.timeout_ns))) break;
+      tc::fence_after_sync();
+      float x[128];
+      __syncwarp();  // tcgen05.ld is warp-collective
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tc::tmem_ld32(tl + uint32_t(s) * 128u + uint32_t(c) * 32u, x + 32 * c);
+      const int lim = kmax - j * 128;  // columns [0, lim) are visible
+      if (lim < 128) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) x[c] = c < lim ? x[c] : -INFINITY;
+      }
+      float mt = x[0];
+#pragma unroll
+      for (int c = 1; c < 128; ++c) mt = fmaxf(mt, x[c]);
+      const float m_new = fmaxf(m_raw, mt);
+      float alpha = 1.f, m_use = 0.f;
+      if (m_new != -INFINITY) {
+        alpha = ex2((m_raw - m_new) * cl);  // 0 on the first visible tile
+        m_use = m_new * cl;
+      }
+      m_raw = m_new;
+#pragma unroll
+      for (int c = 0; c < 128; ++c) x[c] = ex2(fmaf(x[c], cl, -m_use));
+      // P V of the previous tile must be done before P and O are touched.
+      if (j > 0) {
+        if (!(ok = warp_wait(bar(kBarODone), (j - 1) & 1, a.timeout_ns))) break;
+        tc::fence_after_sync();
+      }
+      float rs = 0.f;
+#pragma unroll
+      for (int ch = 0; ch < 16; ++ch) {
+        uint32_t w[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          w[k] = pack_bf16x2(x[ch * 8 + 2 * k], x[ch * 8 + 2 * k + 1]);
+          // the row sum uses the rounded probabilities the MMA multiplies
+          rs += __uint_as_float(w[k] << 16) + __uint_as_float(w[k] & 0xFFFF0000u);
+        }
+        const uint32_t off = uint32_t(ch >> 3) * kPfHalf + (uint32_t((ch & 7) ^ (r & 7)) << 4);
+        *reinterpret_cast<uint4*>(sp + off) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      __syncwarp();
+      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          float o[32];
+          tc::tmem_ld32(tl + 256u + uint32_t(c) * 32u, o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] *= alpha;
+          tc::tmem_st32(tl + 256u + uint32_t(c) * 32u, o);
+        }
+        tc::tmem_wait_st();
+      }
+      l = l * alpha + rs;
+      tc::fence_proxy_async_smem();
+      tc::fence_before_sync();
+      mbar_arrive(bar(kBarPFull));
+    }
+    if (ok) ok = warp_wait(bar(kBarODone), (nt - 1) & 1, a.timeout_ns);
+    if (ok) {
+      tc::fence_after_sync();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      __nv_bfloat16* dst = a.out + int64_t(q0 + qi) * a.o_st + int64_t(kvh * G + g) * a.o_sh;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        float o[32];
+        __syncwarp();
+        tc::tmem_ld32(tl + 256u + uint32_t(c) * 32u, o);
+        if (row_valid) {
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            uint4 w;
+            w.x = pack_bf16x2(o[8 * v + 0] * inv, o[8 * v + 1] * inv);
+            w.y = pack_bf16x2(o[8 * v + 2] * inv, o[8 * v + 3] * inv);
+            w.z = pack_bf16x2(o[8 * v + 4] * inv, o[8 * v + 5] * inv);
+            w.w = pack_bf16x2(o[8 * v + 6] * inv, o[8 * v + 7] * inv);
+            *reinterpret_cast<uint4*>(dst + c * 32 + v * 8) = w;
+          }
+        }
+      }
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, kPfTmemCols);
+  }
+}
+
+}  // namespace pa

@@ -113,6 +113,38 @@ def test_decode_validation():
                  stream=0)
 
 
+def test_prefill_validation():
+    kc, vc = _cache(hk=2), _cache(hk=2)
+    B, T, H = 3, 10, 8
+    q = torch.empty(T, H, 128, dtype=torch.bfloat16)
+    out = torch.empty_like(q)
+    bt = torch.zeros(B, 4, dtype=torch.int32)
+    cl = torch.zeros(B, dtype=torch.int32)
+    qs = torch.zeros(B + 1, dtype=torch.int32)
+    f = pa.pa_prefill
+    _expect(INVALID, f, out, q, kc, vc, bt, cl, qs, 4, 0.1, 4, stream=0)  # num_kv_heads mismatch
+    _expect(INVALID, f, out, q, kc, vc, bt, cl, qs[:B], 4, 0.1, 2, stream=0)  # query_start not [B + 1]
+    _expect(INVALID, f, out, q, kc, vc, bt, cl, qs.long(), 4, 0.1, 2, stream=0)
+    _expect(INVALID, f, out, q, kc, vc, bt[:2], cl, qs, 4, 0.1, 2, stream=0)
+    _expect(INVALID, f, out, q, kc, vc, bt, cl, qs, 4, 0.0, 2, stream=0)  # scale must be > 0
+    _expect(INVALID, f, out, q, kc, vc, bt, cl, qs, 4, -0.1, 2, stream=0)
+    _expect(INVALID, f, out, q, kc, vc, bt, cl, qs, 0, 0.1, 2, stream=0)  # T > 0 needs max_query_len > 0
+    _expect(INVALID, f, out, q, kc, vc, bt, cl, qs, T + 1, 0.1, 2, stream=0)
+    _expect(INVALID, f, out[:5], q, kc, vc, bt, cl, qs, 4, 0.1, 2, stream=0)
+    _expect(UNSUPPORTED, f, out.float(), q.float(), _cache(hk=2, dtype=torch.float32),
+            _cache(hk=2, dtype=torch.float32), bt, cl, qs, 4, 0.1, 2, stream=0)  # tensor-core path is bf16 only
+    q64 = torch.empty(T, H, 64, dtype=torch.bfloat16)
+    _expect(UNSUPPORTED, f, torch.empty_like(q64), q64, _cache(hk=2, d=64), _cache(hk=2, d=64), bt, cl, qs, 4, 0.1,
+            2, stream=0)
+    q6 = torch.empty(T, 6, 128, dtype=torch.bfloat16)
+    _expect(UNSUPPORTED, f, torch.empty_like(q6), q6, kc, vc, bt, cl, qs, 4, 0.1, 2, stream=0)  # group of 3
+    # nothing to compute: valid, nothing launched
+    z = torch.empty(0, H, 128, dtype=torch.bfloat16)
+    f(z, z, kc, vc, bt, cl, qs, 0, 0.1, 2, stream=0)
+    f(out, q, kc, vc, torch.zeros(0, 4, dtype=torch.int32), torch.zeros(0, dtype=torch.int32),
+      torch.zeros(1, dtype=torch.int32), 4, 0.1, 2, stream=0)
+
+
 def test_fixed_workspace_size():
     n = pa.pa_decode_workspace_bytes(8, 32, 8, 128, 8192, 512)
     P = 8192 * 16 // 512
