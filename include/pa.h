@@ -258,9 +258,9 @@ pa_status pa_decode_fp8(pa_tensor* out, const pa_tensor* query, const pa_tensor*
  *
  * A decode request is n_i = 1; a whole prompt is n_i = context_lens[i];
  * n_i = 0 writes nothing.  Runs on the tensor cores (tcgen05): QK^T and PV
- * in bf16 with fp32 accumulation, the probabilities rounded to bf16 before
- * the PV product (and the softmax denominator summed from the rounded
- * values), output rounded to nearest even.
+ * in bf16 with fp32 accumulation; the softmax is fp32 (its denominator summed
+ * before rounding), the probabilities are rounded to bf16 for the PV
+ * product, and the output is rounded to nearest even.
  *
  * out, query:   [T, H, 128] bf16, last dim contiguous, strides multiples of
  *               16 bytes, 16-byte aligned (T = total new tokens).  Rows not

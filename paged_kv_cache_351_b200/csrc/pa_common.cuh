@@ -157,6 +157,45 @@ __device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, 
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
+// d = a + b on two fp32 lanes at once (packed add, sm_100), round to nearest.
+__device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+// 2^x for two values on the FMA pipe (a stand-in for the special-function
+// unit when that unit is the bottleneck).  Range reduction x = n + f with n
+// the nearest integer (adding 1.5 * 2^23 rounds to it) and |f| <= 1/2; 2^f
+// from a cubic whose coefficients were fitted here by iteratively reweighted
+// least squares on [-1/2, 1/2] for the smallest maximum relative error
+// (1.0e-4, below a bf16 rounding step of 3.9e-3); 2^n is added to the
+// exponent field.  Inputs are clamped to >= -126 (results below 2^-126 come
+// out as about 2^-126 instead of 0); inputs must be <= 127.
+__device__ __forceinline__ void ex2_poly2(float& a, float& b) {
+  constexpr float kRound = 12582912.0f;
+  constexpr float kC1 = 0.6932829022407532f, kC2 = 0.24221085011959076f, kC3 = 0.05500883609056473f;
+  a = fmaxf(a, -126.f);
+  b = fmaxf(b, -126.f);
+  float ta, tb, ra, rb;
+  fadd2(ta, tb, a, b, kRound, kRound);
+  fadd2(ra, rb, ta, tb, -kRound, -kRound);
+  float fa = a, fb = b;
+  ffma2(fa, fb, ra, rb, -1.f, -1.f);  // f = x - n
+  float pa = kC2, pb = kC2;
+  ffma2(pa, pb, fa, fb, kC3, kC3);
+  float qa = kC1, qb = kC1;
+  ffma2(qa, qb, fa, fb, pa, pb);
+  float ua = 1.f, ub = 1.f;
+  ffma2(ua, ub, fa, fb, qa, qb);
+  a = __int_as_float(__float_as_int(ua) + (__float_as_int(ta) << 23));
+  b = __int_as_float(__float_as_int(ub) + (__float_as_int(tb) << 23));
+}
+
 // Storage-type traits: a 16-byte vector holds EPV elements.
 template <typename T>
 struct Elem;

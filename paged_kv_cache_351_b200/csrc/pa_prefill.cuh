@@ -19,12 +19,14 @@
 // swizzle: Q as one box of [128/G tokens][G heads][64 dims] per half of the
 // head dimension, each K/V page as a [16 tokens][64 dims] box per half (a
 // page is one (block, kv head) of the cache, its id from the block table).
-// Warp roles: warp 0 issues TMA loads, warp 1 owns TMEM and issues the MMAs
-// (one thread), warps 4-7 run the softmax and the epilogue.  S is double
-// buffered in TMEM, so the MMA of S for tile j + 1 runs while the softmax
-// of tile j does; K/V use two stages.  Every wait is bounded by the caller's
-// timeout (PA_DEV_TIMEOUT), after which each role stops, waits (bounded) for
-// its own copies and MMAs in flight, and TMEM is released.
+// Warp roles: warp 0 issues the Q and K loads, warp 2 the V loads, warp 1
+// owns TMEM and issues the MMAs (one thread), warps 4-7 run the softmax and
+// the epilogue.  S is double buffered in TMEM, so the MMA of S for tile
+// j + 1 runs while the softmax of tile j does.  K has three stages, each
+// released as soon as QK^T of its tile is done; V has two, released after
+// PV.  Every wait is bounded by the caller's timeout (PA_DEV_TIMEOUT), after
+// which each role stops, waits (bounded) for its own copies and MMAs in
+// flight, and TMEM is released.
 #pragma once
 
 #include "pa_common.cuh"
@@ -47,26 +49,31 @@ struct PrefillArgs {
 constexpr int kPfThreads = 256;
 constexpr uint32_t kPfHalf = 16384;  // 128 rows x 128 bytes: one 64-dim half of a 128 x 128 bf16 tile
 constexpr uint32_t kPfTile = 2 * kPfHalf;
+constexpr int kKStages = 3;  // K is free again once QK^T of its tile is done
+constexpr int kVStages = 2;  // V is free again once PV of its tile is done
 constexpr uint32_t kSmQ = 0;
-constexpr uint32_t kSmK = kSmQ + kPfTile;      // two stages
-constexpr uint32_t kSmV = kSmK + 2 * kPfTile;  // two stages
-constexpr uint32_t kSmP = kSmV + 2 * kPfTile;
+constexpr uint32_t kSmK = kSmQ + kPfTile;
+constexpr uint32_t kSmV = kSmK + kKStages * kPfTile;
+constexpr uint32_t kSmP = kSmV + kVStages * kPfTile;
 constexpr uint32_t kSmBar = kSmP + kPfTile;
-constexpr uint32_t kPfSmemBytes = kSmBar + 128 + 1024;  // + barriers + alignment slack
+constexpr uint32_t kPfSmemBytes = kSmBar + 160 + 1024;  // + barriers + alignment slack (<= 227 KiB)
 constexpr uint32_t kPfTmemCols = 512;                   // S0 [0,128), S1 [128,256), O [256,384)
 
 // Barrier slots (8 bytes each) after kSmBar.
 enum PfBar : int {
   kBarQ = 0,
-  kBarKFull = 1,   // + stage
-  kBarVFull = 3,   // + stage
-  kBarKVFree = 5,  // + stage
-  kBarSFull = 7,   // + S buffer
-  kBarPFull = 9,
-  kBarODone = 10,
-  kBarDrain = 11,
-  kBarTmemSlot = 12,  // 4-byte TMEM base address
+  kBarKFull = 1,   // + K stage (3)
+  kBarKFree = 4,   // + K stage (3)
+  kBarVFull = 7,   // + V stage (2)
+  kBarVFree = 9,   // + V stage (2)
+  kBarSFull = 11,  // + S buffer (2)
+  kBarPFull = 13,
+  kBarODone = 14,
+  kBarDrain = 15,
+  kBarTmemSlot = 16,  // 4-byte TMEM base address
 };
+static_assert(kSmBar + 8 * kBarTmemSlot + 4 <= kSmBar + 160, "barrier area");
+static_assert(kPfSmemBytes <= 232448, "shared memory per block");
 
 // All lanes wait; the warp agrees on the outcome so that warp-collective
 // tcgen05 instructions stay converged.
@@ -115,12 +122,15 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     mbar_init(bar(kBarQ), 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(bar(kBarKFull + s), 1);
-      mbar_init(bar(kBarVFull + s), 1);
-      mbar_init(bar(kBarKVFree + s), 1);
-      mbar_init(bar(kBarSFull + s), 1);
+    for (int st = 0; st < kKStages; ++st) {
+      mbar_init(bar(kBarKFull + st), 1);
+      mbar_init(bar(kBarKFree + st), 1);
     }
+    for (int st = 0; st < kVStages; ++st) {
+      mbar_init(bar(kBarVFull + st), 1);
+      mbar_init(bar(kBarVFree + st), 1);
+    }
+    for (int b = 0; b < 2; ++b) mbar_init(bar(kBarSFull + b), 1);
     mbar_init(bar(kBarPFull), 128);
     mbar_init(bar(kBarODone), 1);
     mbar_init(bar(kBarDrain), 1);
@@ -132,22 +142,27 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   tc::fence_after_sync();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + kSmBar + 8 * kBarTmemSlot);
 
-  if (warp == 0) {
-    // ---------------- TMA producer ----------------
+  if (warp == 0 || warp == 2) {
+    // ---------------- TMA producers: warp 0 streams K (and Q), warp 2 streams V ----------------
+    const bool is_k = warp == 0;
+    const int nst = is_k ? kKStages : kVStages;
+    const CUtensorMap* tm = is_k ? &tm_k : &tm_v;
+    const uint32_t ring = base + (is_k ? kSmK : kSmV);
+    const int full0 = is_k ? kBarKFull : kBarVFull, free0 = is_k ? kBarKFree : kBarVFree;
     const int32_t* bt = a.bt + int64_t(seq) * a.bt_stride;
     if (lane == 0) {
-      tc::tma_prefetch_desc(&tm_q);
-      tc::tma_prefetch_desc(&tm_k);
-      tc::tma_prefetch_desc(&tm_v);
-      mbar_arrive_expect_tx(bar(kBarQ), kPfTile);
-      tc::tma_load_3d(base + kSmQ, &tm_q, 0, kvh * G, q0 + qt * TOK, bar(kBarQ));
-      tc::tma_load_3d(base + kSmQ + kPfHalf, &tm_q, 64, kvh * G, q0 + qt * TOK, bar(kBarQ));
+      tc::tma_prefetch_desc(tm);
+      if (is_k) {
+        tc::tma_prefetch_desc(&tm_q);
+        mbar_arrive_expect_tx(bar(kBarQ), kPfTile);
+        tc::tma_load_3d(base + kSmQ, &tm_q, 0, kvh * G, q0 + qt * TOK, bar(kBarQ));
+        tc::tma_load_3d(base + kSmQ + kPfHalf, &tm_q, 64, kvh * G, q0 + qt * TOK, bar(kBarQ));
+      }
     }
-    bool ok = true;
     int issued = 0;  // tiles whose loads were issued
     for (int j = 0; j < nt; ++j) {
-      const int s = j & 1;
-      if (j >= 2 && !(ok = warp_wait(bar(kBarKVFree + s), ((j >> 1) - 1) & 1, a.timeout_ns))) break;
+      const int st = j % nst, use = j / nst;
+      if (j >= nst && !warp_wait(bar(free0 + st), (use - 1) & 1, a.timeout_ns)) break;
       const int p0 = j * 8;
       const int np = min(8, npages - p0);
       int blk = 0;
@@ -158,76 +173,56 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           blk = 0;
         }
       }
-      if (lane == 0) {
-        mbar_arrive_expect_tx(bar(kBarKFull + s), uint32_t(np) * 4096u);
-        mbar_arrive_expect_tx(bar(kBarVFull + s), uint32_t(np) * 4096u);
-      }
+      if (lane == 0) mbar_arrive_expect_tx(bar(full0 + st), uint32_t(np) * 4096u);
       for (int p = 0; p < np; ++p) {
         const int b = __shfl_sync(0xffffffffu, blk, p);
         if (lane == 0) {
-          const uint32_t dk = base + kSmK + uint32_t(s) * kPfTile + uint32_t(p) * 2048u;
-          tc::tma_load_4d(dk, &tm_k, 0, 0, kvh, b, bar(kBarKFull + s));
-          tc::tma_load_4d(dk + kPfHalf, &tm_k, 64, 0, kvh, b, bar(kBarKFull + s));
-        }
-      }
-      for (int p = 0; p < np; ++p) {
-        const int b = __shfl_sync(0xffffffffu, blk, p);
-        if (lane == 0) {
-          const uint32_t dv = base + kSmV + uint32_t(s) * kPfTile + uint32_t(p) * 2048u;
-          tc::tma_load_4d(dv, &tm_v, 0, 0, kvh, b, bar(kBarVFull + s));
-          tc::tma_load_4d(dv + kPfHalf, &tm_v, 64, 0, kvh, b, bar(kBarVFull + s));
+          const uint32_t d = ring + uint32_t(st) * kPfTile + uint32_t(p) * 2048u;
+          tc::tma_load_4d(d, tm, 0, 0, kvh, b, bar(full0 + st));
+          tc::tma_load_4d(d + kPfHalf, tm, 64, 0, kvh, b, bar(full0 + st));
         }
       }
       issued = j + 1;
     }
     // Before the CTA may exit, every copy it started must have landed.
-    mbar_wait_bounded(bar(kBarQ), 0, a.timeout_ns);
-    for (int j = max(0, issued - 2); j < issued; ++j) {
-      mbar_wait_bounded(bar(kBarKFull + (j & 1)), (j >> 1) & 1, a.timeout_ns);
-      mbar_wait_bounded(bar(kBarVFull + (j & 1)), (j >> 1) & 1, a.timeout_ns);
-    }
-    (void)ok;
+    if (is_k) mbar_wait_bounded(bar(kBarQ), 0, a.timeout_ns);
+    for (int j = max(0, issued - nst); j < issued; ++j)
+      mbar_wait_bounded(bar(full0 + j % nst), (j / nst) & 1, a.timeout_ns);
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     constexpr uint32_t kIdQK = tc::idesc_bf16_f32(128, 128, false, false);
     constexpr uint32_t kIdPV = tc::idesc_bf16_f32(128, 128, false, true);
-    auto issue_qk = [&](int j) {  // S[j & 1] = Q K_j^T
-      const uint32_t d = tmem + uint32_t(j & 1) * 128u;
-      const uint32_t kb = base + kSmK + uint32_t(j & 1) * kPfTile;
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t off = uint32_t(kk >> 2) * kPfHalf + uint32_t(kk & 3) * 32u;
-        tc::mma_bf16_ss(d, tc::desc_kmajor(base + kSmQ + off), tc::desc_kmajor(kb + off), kIdQK, kk > 0);
-      }
-    };
-    bool ok = warp_wait(bar(kBarQ), 0, a.timeout_ns) && warp_wait(bar(kBarKFull), 0, a.timeout_ns);
-    if (ok) {
+    // S[j & 1] = Q K_j^T; K stage j % 3 is released when it completes.
+    auto qk = [&](int j) -> bool {
+      const int st = j % kKStages;
+      if (!warp_wait(bar(kBarKFull + st), (j / kKStages) & 1, a.timeout_ns)) return false;
       tc::fence_after_sync();
       if (lane == 0) {
-        issue_qk(0);
-        tc::commit(bar(kBarSFull));
+        const uint32_t d = tmem + uint32_t(j & 1) * 128u;
+        const uint32_t kb = base + kSmK + uint32_t(st) * kPfTile;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = uint32_t(kk >> 2) * kPfHalf + uint32_t(kk & 3) * 32u;
+          tc::mma_bf16_ss(d, tc::desc_kmajor(base + kSmQ + off), tc::desc_kmajor(kb + off), kIdQK, kk > 0);
+        }
+        tc::commit(bar(kBarSFull + (j & 1)));
+        tc::commit(bar(kBarKFree + st));
       }
       __syncwarp();
-    }
+      return true;
+    };
+    bool ok = warp_wait(bar(kBarQ), 0, a.timeout_ns) && qk(0);
     for (int j = 0; ok && j < nt; ++j) {
-      const int s = j & 1;
-      if (j + 1 < nt) {
-        if (!(ok = warp_wait(bar(kBarKFull + (s ^ 1)), ((j + 1) >> 1) & 1, a.timeout_ns))) break;
-        tc::fence_after_sync();
-        if (lane == 0) {
-          issue_qk(j + 1);
-          tc::commit(bar(kBarSFull + (s ^ 1)));
-        }
-        __syncwarp();
-      }
+      const int sv = j % kVStages;
+      if (j + 1 < nt && !(ok = qk(j + 1))) break;
       if (!(ok = warp_wait(bar(kBarPFull), j & 1, a.timeout_ns))) break;
-      if (!(ok = warp_wait(bar(kBarVFull + s), (j >> 1) & 1, a.timeout_ns))) break;
+      if (!(ok = warp_wait(bar(kBarVFull + sv), (j / kVStages) & 1, a.timeout_ns))) break;
       tc::fence_after_sync();
       const int valid = kv_len - j * 128;
       if (valid < 128) {
         // Rows past the last key hold stale or never-written values (NaN
         // would survive a zero probability): clear them before P V.
-        uint8_t* vs = gbase + kSmV + uint32_t(s) * kPfTile;
+        uint8_t* vs = gbase + kSmV + uint32_t(sv) * kPfTile;
         const int rows = 128 - valid;
         for (int e = lane; e < rows * 16; e += 32) {
           const int r = valid + (e >> 4), c = e & 15;
@@ -238,7 +233,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         __syncwarp();
       }
       if (lane == 0) {
-        const uint32_t vb = base + kSmV + uint32_t(s) * kPfTile;
+        const uint32_t vb = base + kSmV + uint32_t(sv) * kPfTile;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t pa_off = uint32_t(kk >> 2) * kPfHalf + uint32_t(kk & 3) * 32u;
@@ -246,7 +241,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                           tc::desc_mnmajor(vb + uint32_t(kk) * 2048u, kPfHalf), kIdPV, j > 0 || kk > 0);
         }
         tc::commit(bar(kBarODone));
-        tc::commit(bar(kBarKVFree + s));
+        tc::commit(bar(kBarVFree + sv));
       }
       __syncwarp();
     }
@@ -263,7 +258,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const int kmax = row_valid ? c0 + qi + 1 : 0;  // keys [0, kmax) are visible
     const uint32_t tl = tmem + (uint32_t((warp - 4) * 32) << 16);
     const float cl = a.scale_log2;
-    float m_raw = -INFINITY, l = 0.f;
+    // Lazy rescaling: the exponent offset m_used (raw logit units) moves only
+    // when a row's max exceeds it by more than kRescaleLog2 / cl, so
+    // probabilities stay below 2^kRescaleLog2 and O is rarely rescaled; the
+    // final division by l uses the same offset, so the result is unchanged.
+    constexpr float kRescaleLog2 = 8.f;
+    const float thr = kRescaleLog2 / cl;
+    float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     uint8_t* sp = gbase + kSmP + uint32_t(r) * 128u;
     for (int j = 0; j < nt; ++j) {
@@ -272,45 +273,58 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       tc::fence_after_sync();
       float x[128];
       __syncwarp();  // tcgen05.ld is warp-collective
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tc::tmem_ld32(tl + uint32_t(s) * 128u + uint32_t(c) * 32u, x + 32 * c);
+      tc::tmem_ld128(tl + uint32_t(s) * 128u, x);
       const int lim = kmax - j * 128;  // columns [0, lim) are visible
       if (lim < 128) {
 #pragma unroll
         for (int c = 0; c < 128; ++c) x[c] = c < lim ? x[c] : -INFINITY;
       }
-      float mt = x[0];
+      float m8[8];
 #pragma unroll
-      for (int c = 1; c < 128; ++c) mt = fmaxf(mt, x[c]);
-      const float m_new = fmaxf(m_raw, mt);
-      float alpha = 1.f, m_use = 0.f;
-      if (m_new != -INFINITY) {
-        alpha = ex2((m_raw - m_new) * cl);  // 0 on the first visible tile
-        m_use = m_new * cl;
+      for (int k = 0; k < 8; ++k) m8[k] = x[k];
+#pragma unroll
+      for (int c = 8; c < 128; ++c) m8[c & 7] = fmaxf(m8[c & 7], x[c]);
+      const float mt = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+      const bool moved = __any_sync(0xffffffffu, mt > m_used + thr);
+      float alpha = 1.f;
+      if (moved) {
+        const float m_new = fmaxf(m_used, mt);
+        alpha = m_new == -INFINITY ? 1.f : ex2((m_used - m_new) * cl);  // 0 on a row's first visible tile
+        m_used = m_new;
       }
-      m_raw = m_new;
+      const float mu = m_used == -INFINITY ? 0.f : m_used * cl;
 #pragma unroll
-      for (int c = 0; c < 128; ++c) x[c] = ex2(fmaf(x[c], cl, -m_use));
+      for (int c = 0; c < 128; c += 2) {
+        float e0 = -mu, e1 = -mu;
+        ffma2(e0, e1, x[c], x[c + 1], cl, cl);  // x * cl - mu
+        if (((c >> 3) & 3) == 3) {              // a quarter of the exponentials on the FMA pipe
+          ex2_poly2(e0, e1);
+        } else {
+          e0 = ex2(e0);
+          e1 = ex2(e1);
+        }
+        x[c] = e0;
+        x[c + 1] = e1;
+      }
       // P V of the previous tile must be done before P and O are touched.
       if (j > 0) {
         if (!(ok = warp_wait(bar(kBarODone), (j - 1) & 1, a.timeout_ns))) break;
         tc::fence_after_sync();
       }
-      float rs = 0.f;
+      float rs[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int ch = 0; ch < 16; ++ch) {
         uint32_t w[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          w[k] = pack_bf16x2(x[ch * 8 + 2 * k], x[ch * 8 + 2 * k + 1]);
-          // the row sum uses the rounded probabilities the MMA multiplies
-          rs += __uint_as_float(w[k] << 16) + __uint_as_float(w[k] & 0xFFFF0000u);
-        }
+        for (int k = 0; k < 4; ++k) w[k] = pack_bf16x2(x[ch * 8 + 2 * k], x[ch * 8 + 2 * k + 1]);
         const uint32_t off = uint32_t(ch >> 3) * kPfHalf + (uint32_t((ch & 7) ^ (r & 7)) << 4);
         *reinterpret_cast<uint4*>(sp + off) = make_uint4(w[0], w[1], w[2], w[3]);
+#pragma unroll
+        for (int k = 0; k < 8; k += 2) fadd2(rs[k], rs[k + 1], rs[k], rs[k + 1], x[ch * 8 + k], x[ch * 8 + k + 1]);
       }
       __syncwarp();
-      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+      if (j > 0 && moved) {
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           float o[32];
@@ -321,7 +335,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
         tc::tmem_wait_st();
       }
-      l = l * alpha + rs;
+      l = l * alpha + (((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7])));
       tc::fence_proxy_async_smem();
       tc::fence_before_sync();
       mbar_arrive(bar(kBarPFull));
