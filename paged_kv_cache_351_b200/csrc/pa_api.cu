@@ -374,7 +374,7 @@ pa_status run_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtens
       return launch_status();
     attr_set[dev] = true;
   }
-  constexpr int TOK = 128 / G;
+  constexpr int TOK = pa::kPfRows / G;  // new tokens per CTA
   const dim3 grid(unsigned((max_query_len + TOK - 1) / TOK), unsigned(Hkv), unsigned(a.B));
   if (launch_pdl(kern, grid, dim3(pa::kPfThreads), pa::kPfSmemBytes, st, true, tq, tk, tv, a) != cudaSuccess)
     return launch_status();

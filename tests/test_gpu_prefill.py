@@ -158,7 +158,7 @@ def test_prefill_reports_bad_query_start():
     c.run(qs=bad)
     st, bits = pa.pa_get_device_status()
     assert bits & 0x4
-    c2 = Case(52, [(10, 200)], 8, 8)
+    c2 = Case(52, [(10, 600)], 8, 8)
     c2.run(max_q=5)  # max_query_len so small that the grid misses rows of a sequence
     st, bits = pa.pa_get_device_status()
     assert bits & 0x4
