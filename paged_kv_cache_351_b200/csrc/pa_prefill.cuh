@@ -252,16 +252,17 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         tc::fence_proxy_async_smem();
         __syncwarp();
       }
-      if (more && !(ok = warp_wait(bar(kBarKFull + (j + 1) % kKStages), ((j + 1) / kKStages) & 1, a.timeout_ns)))
-        break;
       // half A: P V of this tile, then Q K^T of the next (S_A is free once P_A is consumed, in MMA order)
       if (!(ok = warp_wait(bar(kBarPFull + 0), j & 1, a.timeout_ns))) break;
       tc::fence_after_sync();
-      if (lane == 0) {
-        pv(j, 0);
-        if (more) qk(j + 1, 0);
-      }
+      if (lane == 0) pv(j, 0);
       __syncwarp();
+      if (more) {
+        if (!(ok = warp_wait(bar(kBarKFull + (j + 1) % kKStages), ((j + 1) / kKStages) & 1, a.timeout_ns))) break;
+        tc::fence_after_sync();
+        if (lane == 0) qk(j + 1, 0);
+        __syncwarp();
+      }
       // half B, then release the K and V stages
       if (!(ok = warp_wait(bar(kBarPFull + 1), j & 1, a.timeout_ns))) break;
       tc::fence_after_sync();
