@@ -132,19 +132,22 @@ def measured_tensor_peak():
         return 1590.0, "fallback"
 
 
-def kernel_source_hash():
+def kernel_source_hash(files=("pa_decode.cuh", "pa_common.cuh")):
     h = hashlib.sha256()
-    for f in ("pa_decode.cuh", "pa_common.cuh"):
+    for f in files:
         with open(os.path.join(ROOT, "paged_kv_cache_351_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(workload):
-    """DRAM bytes (read + write) per launch of the decode kernel from the
-    committed ncu summary of this workload, if it was taken on the current
-    kernel source; else None."""
-    p = os.path.join(ROOT, "profiles", f"decode_kernel_{workload}.md")
+PREFILL_SOURCES = ("pa_prefill.cuh", "pa_tc.cuh", "pa_common.cuh")
+
+
+def ncu_traffic(workload, kernel="decode_kernel", files=("pa_decode.cuh", "pa_common.cuh")):
+    """DRAM bytes (read + write) per launch of a kernel from the committed
+    ncu summary of this workload, if it was taken on the current kernel
+    source; else None."""
+    p = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
     try:
         vals = {}
         with open(p) as f:
@@ -152,7 +155,7 @@ def ncu_traffic(workload):
                 k, _, v = line.strip().partition(":")
                 if k in ("workload", "kernel_source_sha", "dram_bytes_per_launch"):
                     vals[k] = v.strip()
-        if vals.get("kernel_source_sha") != kernel_source_hash() or vals.get("workload") != workload:
+        if vals.get("kernel_source_sha") != kernel_source_hash(files) or vals.get("workload") != workload:
             return None
         return float(vals["dram_bytes_per_launch"])
     except Exception:
@@ -769,7 +772,9 @@ def run_prefill(args, plan, device, world, rank):
         "flops_per_step": flops, "write_bytes_per_step": write_bytes,
         "roofline": {"bound": "tensor", "kernel": "pa_prefill (prefill_kernel, tcgen05)", "achieved": round(achieved, 2),
                      "peak": peak, "peak_kind": peak_kind + " bf16 dense (burst)", "unit": "TFLOP/s",
-                     "frac": round(achieved / peak, 4), "traffic": None, "algorithmic_flops_per_launch": flops,
+                     "frac": round(achieved / peak, 4),
+                     "traffic": ncu_traffic(w.name, "prefill_kernel", PREFILL_SOURCES),
+                     "traffic_unit": "DRAM bytes per launch", "algorithmic_flops_per_launch": flops,
                      "avg_launch_ms": round(pf_ms, 5),
                      "timing": f"{K} prefill launches, each bracketed by CUDA events, after the timed region"},
         "cpu_baseline": cpu,
