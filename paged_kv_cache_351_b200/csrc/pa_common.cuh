@@ -196,6 +196,27 @@ __device__ __forceinline__ void ex2_poly2(float& a, float& b) {
   b = __int_as_float(__float_as_int(ub) + (__float_as_int(tb) << 23));
 }
 
+// The two e4m3 codes in the low (lo) or high (hi) half of w, low byte
+// first -> two f16 in one register (exact): one cvt.rn.f16x2.e4m3x2, the
+// half selected by register pairing.
+__device__ __forceinline__ uint32_t e4m3x2_lo_to_f16x2(uint32_t w) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, lo;\n\t}" : "=r"(r) : "r"(w));
+  return r;
+}
+__device__ __forceinline__ uint32_t e4m3x2_hi_to_f16x2(uint32_t w) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, hi;\n\t}" : "=r"(r) : "r"(w));
+  return r;
+}
+
+// Two f16 in one register -> two fp32 (exact).
+__device__ __forceinline__ void f16x2_to_f32(uint32_t h, float& lo, float& hi) {
+  asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\tcvt.f32.f16 %0, a;\n\tcvt.f32.f16 %1, b;\n\t}"
+      : "=f"(lo), "=f"(hi)
+      : "r"(h));
+}
+
 // Storage-type traits: a 16-byte vector holds EPV elements.
 template <typename T>
 struct Elem;
@@ -248,14 +269,8 @@ struct Elem<__nv_fp8_e4m3> {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[k] & 0xFFFFu), __NV_E4M3);
-      const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[k] >> 16), __NV_E4M3);
-      const float2 a = __half22float2(__half2(lo));
-      const float2 b = __half22float2(__half2(hi));
-      f[4 * k + 0] = a.x;
-      f[4 * k + 1] = a.y;
-      f[4 * k + 2] = b.x;
-      f[4 * k + 3] = b.y;
+      f16x2_to_f32(e4m3x2_lo_to_f16x2(w[k]), f[4 * k + 0], f[4 * k + 1]);
+      f16x2_to_f32(e4m3x2_hi_to_f16x2(w[k]), f[4 * k + 2], f[4 * k + 3]);
     }
   }
 };
@@ -264,6 +279,24 @@ struct Elem<__nv_fp8_e4m3> {
 // NaN stays NaN), first value in the low byte.
 __device__ __forceinline__ uint32_t quantize_e4m3x2(float a, float b) {
   return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3));
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// d += a * b on the tensor cores: m16n8k16, f16 inputs, fp32 accumulate.
+// Fragment layout (lane = 4 * gr + tig): a = {(row gr, k 2tig..+1),
+// (row gr + 8, k 2tig..+1), (row gr, k 2tig+8..+9), (row gr + 8, k 2tig+8..+9)},
+// b = {(k 2tig..+1, col gr), (k 2tig+8..+9, col gr)}, d = {(gr, 2tig),
+// (gr, 2tig+1), (gr + 8, 2tig), (gr + 8, 2tig+1)}.
+__device__ __forceinline__ void mma_16816_f16(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
 __device__ __forceinline__ uint4 ld_nc_v4(const uint4* p) {
