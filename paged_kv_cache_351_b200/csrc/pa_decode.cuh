@@ -48,10 +48,14 @@ namespace pa {
 constexpr int kBS = 16;        // tokens per block (block_size)
 constexpr int kMaxWarps = 12;  // workers per CTA (registers allow 12 at G <= 4)
 
-// Warps per CTA the register budget allows without spills: a lane keeps the
-// query and output of G heads x EPV dims in registers (2 G EPV floats); at
-// 128 or more (bf16 G = 8, FP8 G = 4) only 8 warps fit.
-__host__ __device__ constexpr int max_warps_for(int G, int EPV) { return 2 * G * EPV >= 128 ? 8 : kMaxWarps; }
+// Warps per CTA the register budget allows without spills: a lane of the
+// scalar path keeps the query and output of G heads x EPV dims in registers
+// (2 G EPV floats); at 128 or more (bf16 G = 8) only 8 warps fit.  The FP8
+// path (EPV = 16) keeps tensor-core fragments instead and fits 12 up to
+// G = 4 (its segment end still gathers G x 16 outputs per lane).
+__host__ __device__ constexpr int max_warps_for(int G, int EPV) {
+  return EPV == 16 ? (G >= 8 ? 8 : kMaxWarps) : (2 * G * EPV >= 128 ? 8 : kMaxWarps);
+}
 
 enum DecodeMode : int32_t { kBalanced = 0, kFixed = 1, kNoSplit = 2 };
 
@@ -314,17 +318,16 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
     float q[G][EPV];
     float o[G][EPV];
     float m[G], lpart[GH];
-    // FP8 cache with G >= 2: the page math runs on the tensor cores (mma.sync m16n8k16,
+    // FP8 cache: the page math runs on the tensor cores (mma.sync m16n8k16,
     // f16 operands, fp32 accumulation), lane = 4 gr + tig.  QK^T: the page's
     // 16 tokens are the M rows, the heads (padded to 8) the N columns, and
     // lane (gr, tig) feeds dims [32 tig, 32 tig + 32) of rows gr and gr + 8
     // (the contraction index is permuted the same way in both operands).
     // PV is computed as O^T = V^T P with the dims as M rows: lane (gr, tig)
     // accumulates dims [16 gr, 16 gr + 16) of heads 2 tig and 2 tig + 1.
-    // Measured on B200: at G = 1 the scalar path below is faster (0.083 vs
-    // 0.097 ms on the LLaMA-7B batch-64 shape); from G = 2 on the per-page
-    // FMAs it saves dominate (0.274 -> 0.209 ms at G = 4).
-    constexpr bool kMma = sizeof(Tkv) == 1 && G >= 2;
+    // Measured on B200 against the scalar path below: 0.274 -> 0.189 ms at
+    // G = 4 (GQA batch 256), 0.0843 -> 0.0826 ms at G = 1 (LLaMA-7B batch 64).
+    constexpr bool kMma = sizeof(Tkv) == 1;
     const int gr = lane >> 2, tig = lane & 3;
     uint32_t qf[16];     // query of head gr, f16 pairs of this lane's 32 dims
     float oacc[8][4];    // O^T fragments
