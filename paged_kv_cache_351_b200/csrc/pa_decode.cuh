@@ -51,8 +51,10 @@ constexpr int kMaxWarps = 12;  // workers per CTA (registers allow 12 at G <= 4)
 // Warps per CTA the register budget allows without spills: a lane of the
 // scalar path keeps the query and output of G heads x EPV dims in registers
 // (2 G EPV floats); at 128 or more (bf16 G = 8) only 8 warps fit.  The FP8
-// path (EPV = 16) keeps tensor-core fragments instead and fits 12 up to
-// G = 4 (its segment end still gathers G x 16 outputs per lane).
+// path (EPV = 16) keeps tensor-core fragments instead and runs 12 up to
+// G = 4 (its segment end gathers G x 16 outputs per lane).  Registers are
+// split per SM sub-partition: 9 to 12 warps put 3 on one and leave 168
+// registers per thread, 8 warps leave 255.
 __host__ __device__ constexpr int max_warps_for(int G, int EPV) {
   return EPV == 16 ? (G >= 8 ? 8 : kMaxWarps) : (2 * G * EPV >= 128 ? 8 : kMaxWarps);
 }
@@ -318,18 +320,20 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
     float q[G][EPV];
     float o[G][EPV];
     float m[G], lpart[GH];
-    // FP8 cache: the page math runs on the tensor cores (mma.sync m16n8k16,
+    // FP8 cache, G >= 2: the page math runs on the tensor cores (mma.sync m16n8k16,
     // f16 operands, fp32 accumulation), lane = 4 gr + tig.  QK^T: the page's
     // 16 tokens are the M rows, the heads (padded to 8) the N columns, and
     // lane (gr, tig) feeds dims [32 tig, 32 tig + 32) of rows gr and gr + 8
     // (the contraction index is permuted the same way in both operands).
     // PV is computed as O^T = V^T P with the dims as M rows: lane (gr, tig)
     // accumulates dims [16 gr, 16 gr + 16) of heads 2 tig and 2 tig + 1.
-    // Measured on B200 against the scalar path below: 0.274 -> 0.189 ms at
-    // G = 4 (GQA batch 256), 0.0843 -> 0.0826 ms at G = 1 (LLaMA-7B batch 64).
-    constexpr bool kMma = sizeof(Tkv) == 1;
+    // Measured on B200 against the scalar path below (fp32 query): 0.274 ->
+    // 0.191 ms at G = 4 (GQA batch 256); at G = 1 the scalar path is faster
+    // (0.084 vs 0.089 ms on LLaMA-7B batch 64) and stays.
+    constexpr bool kMma = sizeof(Tkv) == 1 && G >= 2;
     const int gr = lane >> 2, tig = lane & 3;
     uint32_t qf[16];     // query of head gr, f16 pairs of this lane's 32 dims
+    uint32_t ql[16];     // the f16 rounding error of qf (q = qf + ql to about 2^-22)
     float oacc[8][4];    // O^T fragments
     float mh[2], lh[2];  // running max and denominator of heads 2 tig, 2 tig + 1
     float sfac[2];       // power-of-two factor undoing the query's range normalisation
@@ -380,7 +384,13 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
           const int ex = mx > 0.f ? ilogbf(mx) - 14 : 0;
           const float down = ldexpf(1.f, -ex);
 #pragma unroll
-          for (int j2 = 0; j2 < 16; ++j2) qf[j2] = pack_f16x2(qv[2 * j2] * down, qv[2 * j2 + 1] * down);
+          for (int j2 = 0; j2 < 16; ++j2) {
+            const float a0 = qv[2 * j2] * down, a1 = qv[2 * j2 + 1] * down;
+            qf[j2] = pack_f16x2(a0, a1);
+            float h0, h1;
+            f16x2_to_f32(qf[j2], h0, h1);
+            ql[j2] = pack_f16x2(a0 - h0, a1 - h1);
+          }
           const float up = ldexpf(1.f, ex);
           sfac[0] = __shfl_sync(0xffffffffu, up, (2 * tig) * 4);
           sfac[1] = __shfl_sync(0xffffffffu, up, (2 * tig + 1) * 4);
@@ -419,7 +429,10 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
         const unsigned char* Kb = st;
         const unsigned char* Vb = st + C::PAGE;
         // ---- S = K q^T: rows = tokens, columns = heads ----
-        float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};  // two MMA chains (even, odd kk)
+        // four MMA chains: high and low query parts, even and odd kk (K codes are
+        // exact in f16, so both products are exact before fp32 accumulation)
+        float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+        float la[4] = {0.f, 0.f, 0.f, 0.f}, lb[4] = {0.f, 0.f, 0.f, 0.f};
         {
           const uint4 x0 = *reinterpret_cast<const uint4*>(Kb + gr * 128 + tig * 32);
           const uint4 x1 = *reinterpret_cast<const uint4*>(Kb + gr * 128 + tig * 32 + 16);
@@ -434,9 +447,10 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
             const uint32_t af[4] = {e4m3x2_lo_to_f16x2(r0[kk]), e4m3x2_lo_to_f16x2(r1[kk]),
                                     e4m3x2_hi_to_f16x2(r0[kk]), e4m3x2_hi_to_f16x2(r1[kk])};
             mma_16816_f16((kk & 1) ? sb : sa, af, qf[2 * kk], qf[2 * kk + 1]);
+            mma_16816_f16((kk & 1) ? lb : la, af, ql[2 * kk], ql[2 * kk + 1]);
           }
 #pragma unroll
-          for (int k = 0; k < 4; ++k) sa[k] += sb[k];
+          for (int k = 0; k < 4; ++k) sa[k] = (sa[k] + sb[k]) + (la[k] + lb[k]);
         }
         // sa = {S[gr][2tig], S[gr][2tig+1], S[gr+8][2tig], S[gr+8][2tig+1]} (log2 units)
         float sc4[4] = {sa[0] * sfac[0], sa[1] * sfac[1], sa[2] * sfac[0], sa[3] * sfac[1]};

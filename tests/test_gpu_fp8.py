@@ -62,7 +62,7 @@ def test_fp8_write_bit_exact(in_dtype):
 
 
 class Fp8Case:
-    def __init__(self, seed, ctxs, H, hk, spare=5):
+    def __init__(self, seed, ctxs, H, hk, spare=5, q_mult=1.0):
         rng = np.random.default_rng(seed)
         self.ctxs, self.H, self.hk = list(ctxs), H, hk
         nbs = [-(-c // 16) for c in ctxs]
@@ -91,7 +91,7 @@ class Fp8Case:
             pa.pa_reshape_and_cache_fp8(to_device_values(kx, "bf16", DEV), to_device_values(vx, "bf16", DEV),
                                         self.kc, self.vc, torch.tensor(slots, dtype=torch.int64, device=DEV),
                                         self.kst, self.vst)
-        self.q = to_bf16_bits(rng.standard_normal((len(ctxs), H, D)).astype(np.float32))
+        self.q = to_bf16_bits((rng.standard_normal((len(ctxs), H, D)) * q_mult).astype(np.float32))
         self.qd = to_device_values(self.q, "bf16", DEV)
         self.bt = torch.from_numpy(self.tables).to(DEV)
         self.cl = torch.tensor(ctxs, dtype=torch.int32, device=DEV)
@@ -122,6 +122,25 @@ def test_fp8_decode_parity(H, hk, mode):
     check_status_clean()
     assert not torch.isnan(out.float()).any()
     assert c.err(out) <= 1e-2
+
+
+@pytest.mark.parametrize("H,hk", [(8, 8), (16, 4), (16, 2)])
+@pytest.mark.parametrize("q_mult", [1e-3, 3e3])
+def test_fp8_decode_extreme_query_magnitudes(H, hk, q_mult):
+    """The tensor-core page math carries the query as f16 high and low parts
+    after scaling each head by a power of two; queries far larger (near
+    one-hot softmax) or far smaller (near uniform) than N(0, 1) must still
+    match the oracle.  In the one-hot regime an output is a single V value
+    (up to ~4 here), so the bound adds one bf16 rounding step of |ref|
+    (2^-8 relative) to the 1e-2 used elsewhere."""
+    c = Fp8Case(80 + H + hk, [1, 17, 100, 513, 2049], H, hk, q_mult=q_mult)
+    ref = paged_decode(c.q, c.cache, c.tables, c.ctxs, c.scale)
+    for mode in (0, -1):
+        out = c.run(mode)
+        got = widen(to_host_raw(out, "bf16"), "bf16")
+        assert not np.isnan(got).any()
+        assert np.all(np.abs(got - ref) <= 1e-2 + 2.0 ** -8 * np.abs(ref))
+    check_status_clean()
 
 
 def test_fp8_decode_random_batch():
