@@ -123,6 +123,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   if (tok0 >= qlen) return;       // this tile holds no new token of the sequence
   const int c0 = ctx - qlen;
   const int kv_len = c0 + min(qlen, tok0 + 2 * TOK);  // keys seen by the CTA's last token
+  const bool has_b = tok0 + TOK < qlen;  // half B holds a new token (else it is skipped by every role)
   const int nt = (kv_len + 127) / 128;
   const int npages = (kv_len + 15) / 16;
 
@@ -229,7 +230,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       tc::fence_after_sync();
       if (lane == 0) {
         qk(0, 0);
-        qk(0, 1);
+        if (has_b) qk(0, 1);
         tc::commit(bar(kBarKFree));
       }
       __syncwarp();
@@ -260,8 +261,16 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       if (more) {
         if (!(ok = warp_wait(bar(kBarKFull + (j + 1) % kKStages), ((j + 1) / kKStages) & 1, a.timeout_ns))) break;
         tc::fence_after_sync();
-        if (lane == 0) qk(j + 1, 0);
+        if (lane == 0) {
+          qk(j + 1, 0);
+          if (!has_b) tc::commit(bar(kBarKFree + (j + 1) % kKStages));
+        }
         __syncwarp();
+      }
+      if (!has_b) {
+        if (lane == 0) tc::commit(bar(kBarVFree + sv));
+        __syncwarp();
+        continue;
       }
       // half B, then release the K and V stages
       if (!(ok = warp_wait(bar(kBarPFull + 1), j & 1, a.timeout_ns))) break;
@@ -283,6 +292,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   } else if (warp >= 4) {
     // ---------------- softmax + epilogue: one query row per thread ----------------
     const int x = (warp - 4) >> 2;  // half
+    const bool active = x == 0 || has_b;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;  // row within the half = TMEM lane
     const int tok = r / G, g = r - (r / G) * G;
@@ -299,8 +309,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     constexpr float kRescaleLog2 = 8.f;
     const float thr = kRescaleLog2 / cl;
     float m_used = -INFINITY, l = 0.f;
-    bool ok = true;
-    for (int j = 0; j < nt; ++j) {
+    bool ok = active;
+    for (int j = 0; ok && j < nt; ++j) {
       if (!(ok = warp_wait(bar(kBarSFull + x), j & 1, a.timeout_ns))) break;
       tc::fence_after_sync();
       float s[128];
