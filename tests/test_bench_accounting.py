@@ -1,0 +1,53 @@
+"""The benchmark's algorithmic work counts, checked on CPU against brute
+force over the seeded plans: the decode step's bytes (every context token's
+K and V in the cache's element size, query and output, block-table entries,
+context lengths; the cache write reads the new tokens' K/V and writes them)
+and the chunked-prefill FLOPs (each new token at position p attends p + 1
+keys in every query head: 2 D flops for QK^T and 2 D for PV per key)."""
+
+import numpy as np
+import pytest
+
+import bench
+from workloads import AppendOp, make_plan
+
+
+@pytest.mark.parametrize("name", ["tiny_fp32", "llama7b_bs64", "gqa_bs256_fp8"])
+def test_decode_step_bytes_brute_force(name):
+    plan = make_plan(name)
+    w = plan.workload
+    got = bench.step_bytes(plan)
+    kv = 0
+    tables = 0
+    for c in plan.context_lens.tolist():
+        for _t in range(int(c)):
+            kv += 2 * w.num_kv_heads * w.head_size * w.cache_elem_bytes
+        tables += 4 * len(range(0, int(c), w.block_size))
+    qo = 2 * plan.B * w.num_heads * w.head_size * w.elem_bytes
+    assert got["kv"] == kv
+    assert got["decode"] == kv + qo + tables + 4 * plan.B
+    new_tokens = sum(op.n for op in plan.step_ops if isinstance(op, AppendOp))
+    assert new_tokens == len(plan.step_ops)  # one token per sequence in a decode step
+    per_token = w.num_kv_heads * w.head_size * 2 * (w.elem_bytes + w.cache_elem_bytes) + 8
+    assert got["write"] == new_tokens * per_token
+    assert got["step"] == got["decode"] + got["write"]
+
+
+@pytest.mark.parametrize("name", ["prefill_tiny", "prefill_mixed_gqa"])
+def test_prefill_flops_brute_force(name):
+    plan = make_plan(name)
+    w = plan.workload
+    total = 0
+    for c, n in zip(plan.context_lens.tolist(), plan.query_lens.tolist()):
+        for j in range(n):
+            pos = c - n + j
+            total += w.num_heads * (pos + 1) * 4 * w.head_size
+    assert bench.prefill_flops(plan) == total
+    assert bench.is_prefill(plan)
+    assert not bench.is_prefill(make_plan("llama7b_bs64"))
+
+
+def test_aggregate_value_scales_with_ranks():
+    assert bench.aggregate_value(1e9, 1.0, 1) == pytest.approx(1000.0)
+    assert bench.aggregate_value(1e9, 1.0, 4) == pytest.approx(4000.0)
+    assert np.allclose(bench.max_over_ranks([1.0, 2.5], None, 1), [1.0, 2.5])
