@@ -1,4 +1,4 @@
-"""Python binding of libpa.so — paged KV cache decode for B200 (sm_100a).
+"""Python binding of libpa.so — paged KV cache attention for B200 (sm_100a).
 
 Thin wrappers with the C ABI's names (include/pa.h).  They only turn torch
 tensors and numpy arrays into the ABI's plain pointers, shapes and strides;
@@ -21,7 +21,8 @@ from ._lib import (PA_DEV_BAD_BLOCK, PA_DEV_BAD_CONTEXT, PA_DEV_BAD_SLOT,  # noq
 
 __all__ = [
     "PagedAttentionError", "OutOfBlocksError", "pa_reshape_and_cache", "pa_copy_blocks", "pa_decode",
-    "pa_decode_workspace_bytes", "pa_decode_no_alloc", "pa_reshape_and_cache_fp8", "pa_decode_fp8", "pa_swap_blocks", "pa_set_decode_tuning", "pa_get_device_status", "pa_debug_wait_selftest",
+    "pa_decode_workspace_bytes", "pa_decode_no_alloc", "pa_reshape_and_cache_fp8", "pa_decode_fp8", "pa_prefill",
+    "pa_swap_blocks", "pa_set_decode_tuning", "pa_get_device_status", "pa_debug_wait_selftest",
     "Allocator", "library",
 ]
 
