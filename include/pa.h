@@ -1,5 +1,5 @@
 /*
- * pa.h — C ABI of the paged-KV-cache decode library (libpa.so), sm_100a.
+ * pa.h — C ABI of the paged-KV-cache attention library (libpa.so), sm_100a.
  *
  * The library implements the data-parallel hot path of PagedAttention: the
  * KV cache is cut into fixed-size blocks of BLOCK_SIZE tokens, a per-sequence
@@ -33,11 +33,12 @@
  * section 2.1) served per-thread-group 16-byte loads on older GPUs and is not
  * used.
  *
- * Supported: block_size 16; (bf16, head_size 128), (bf16, head_size 64),
- * (fp32, head_size 64), (fp32, head_size 128), and an FP8 e4m3 cache with
- * head_size 128 and bf16 query/output (pa_reshape_and_cache_fp8,
- * pa_decode_fp8); num_heads / num_kv_heads in {1, 2, 4, 8}.  Anything else
- * returns PA_ERR_UNSUPPORTED.
+ * Supported: block_size 16; for the cache write and decode (bf16, head_size
+ * 128), (bf16, head_size 64), (fp32, head_size 64), (fp32, head_size 128),
+ * and an FP8 e4m3 cache with head_size 128 and bf16 query/output
+ * (pa_reshape_and_cache_fp8, pa_decode_fp8); for multi-token attention
+ * (pa_prefill) bf16 with head_size 128; num_heads / num_kv_heads in
+ * {1, 2, 4, 8}.  Anything else returns PA_ERR_UNSUPPORTED.
  */
 #ifndef PA_H_
 #define PA_H_
@@ -89,7 +90,7 @@ typedef struct {
 /* Device status bits (pa_get_device_status). */
 #define PA_DEV_TIMEOUT 0x1u     /* a bounded wait gave up */
 #define PA_DEV_BAD_BLOCK 0x2u   /* block-table entry or copy pair outside [0, num_blocks) */
-#define PA_DEV_BAD_CONTEXT 0x4u /* context_len < 0 or > block-table row capacity */
+#define PA_DEV_BAD_CONTEXT 0x4u /* context_len < 0 or > block-table row capacity; pa_prefill: a query range that does not fit */
 #define PA_DEV_BAD_SLOT 0x8u    /* slot_mapping entry < -1 or >= num_blocks*block_size */
 
 /* ---------------------------------------------------------------------------
