@@ -74,7 +74,9 @@ typedef struct {
 
 typedef struct {
   void* stream;             /* cudaStream_t, NULL = legacy default stream */
-  void* workspace;          /* device scratch for split decode, 256-byte aligned, may be NULL */
+  void* workspace;          /* device scratch for split decode, 256-byte aligned, may be NULL; its
+                               contents need no initialisation (each call tags what it writes), but
+                               calls whose kernels may overlap on the GPU must not share it */
   size_t workspace_bytes;   /* size of workspace */
   int32_t partition_tokens; /* pa_decode context split:
                                  0  = auto: balanced split over all SMs when the
