@@ -185,6 +185,21 @@ def aggregate_value(bytes_per_step, ms_per_step, world):
 # device setup through the library
 # ---------------------------------------------------------------------------
 
+def step_kv(plan):
+    """K and V (storage form, [new tokens, H_kv, D]) of the step's new tokens,
+    request by request; empty arrays when the step appends nothing."""
+    import numpy as np
+
+    from workloads import stream_kv
+
+    w = plan.workload
+    parts = [stream_kv(plan, op.stream, op.start, op.n) for op in plan.step_ops]
+    if not parts:
+        empty = np.zeros((0, w.num_kv_heads, w.head_size), np.float32 if w.dtype == "f32" else np.uint16)
+        return empty, empty.copy()
+    return np.concatenate([k for k, _ in parts]), np.concatenate([v for _, v in parts])
+
+
 def setup_device(plan, device):
     """Replay the workload's setup requests through the host allocator and
     the library's copy/write kernels; return the runtime and the step's
@@ -235,14 +250,15 @@ def setup_device(plan, device):
             if sum(len(s) for s in pend["slots"]) > 200_000:
                 flush()
     flush()
-    # the step's allocator work (host): one new token per sequence
+    # the step's allocator work (host): the new tokens of the step (one per
+    # sequence for decode, none when every request was made before the step)
     seqs = [op.seq for op in plan.step_ops]
     slots, pairs = kv.append(seqs, [op.n for op in plan.step_ops])
     assert len(pairs) == 0
-    ks, vs = zip(*[stream_kv(plan, op.stream, op.start, op.n) for op in plan.step_ops])
+    key, value = step_kv(plan)
     tables, lens = kv.block_tables(plan.batch, plan.max_blocks_per_seq)
     inputs = {
-        "slots": slots, "key": np.concatenate(ks), "value": np.concatenate(vs),
+        "slots": slots, "key": key, "value": value,
         "query": query_values(plan), "tables": tables, "lens": lens, "tdt": tdt, "dev": dev,
     }
     torch.cuda.synchronize()
@@ -451,8 +467,9 @@ def run_ours(args):
     scale = 1.0 / math.sqrt(w.head_size)
     ws = kv.workspace(plan.B, w.num_heads, bt.shape[1], args.partition)
     stream = torch.cuda.Stream(device)
-    # cache write + decode; fixed partitions add the log-sum-exp merge kernel
-    launches_per_step = 2 + (1 if args.partition > 0 else 0)
+    # cache write (when the step appends tokens) + decode; fixed partitions add
+    # the log-sum-exp merge kernel
+    launches_per_step = (1 if len(inp["slots"]) else 0) + 1 + (1 if args.partition > 0 else 0)
 
     def step():
         kv.write(slots, key, value, None, stream=stream)

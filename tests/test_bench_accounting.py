@@ -51,3 +51,16 @@ def test_aggregate_value_scales_with_ranks():
     assert bench.aggregate_value(1e9, 1.0, 1) == pytest.approx(1000.0)
     assert bench.aggregate_value(1e9, 1.0, 4) == pytest.approx(4000.0)
     assert np.allclose(bench.max_over_ranks([1.0, 2.5], None, 1), [1.0, 2.5])
+
+
+def test_step_kv_shapes():
+    """The step's new-token K/V: one row per appended token, empty for a
+    step that appends nothing (all requests made before the step)."""
+    for name, rows in (("llama7b_bs64", 64), ("prefill_tiny", None), ("parallel_sampling_13b", 0)):
+        plan = make_plan(name)
+        w = plan.workload
+        k, v = bench.step_kv(plan)
+        n = sum(op.n for op in plan.step_ops)
+        assert k.shape == v.shape == (n, w.num_kv_heads, w.head_size)
+        if rows is not None:
+            assert n == rows
