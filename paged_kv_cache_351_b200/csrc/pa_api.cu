@@ -120,9 +120,13 @@ pa_status check_pair(const pa_tensor* k, const pa_tensor* v) {
 }
 
 // [n0, n1, D] rows: last dim contiguous, other strides multiples of 16 bytes.
+// An empty tensor (n0 or n1 zero) is never read or written, so its strides
+// and pointer are not checked (frameworks give empty tensors any strides).
 pa_status check_rows3(const pa_tensor* t, int32_t dtype, int64_t n0, int64_t n1, int64_t D) {
   if (t == nullptr || t->ndim != 3 || t->dtype != dtype) return PA_ERR_INVALID_ARG;
-  if (t->shape[0] != n0 || t->shape[1] != n1 || t->shape[2] != D || t->stride[2] != 1) return PA_ERR_INVALID_ARG;
+  if (t->shape[0] != n0 || t->shape[1] != n1 || t->shape[2] != D) return PA_ERR_INVALID_ARG;
+  if (n0 == 0 || n1 == 0) return PA_OK;
+  if (t->stride[2] != 1) return PA_ERR_INVALID_ARG;
   const int e = esize(dtype);
   if (t->stride[0] < 0 || t->stride[1] < 0 || (t->stride[0] * e) % 16 || (t->stride[1] * e) % 16)
     return PA_ERR_INVALID_ARG;

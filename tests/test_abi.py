@@ -145,6 +145,21 @@ def test_prefill_validation():
       torch.zeros(1, dtype=torch.int32), 4, 0.1, 2, stream=0)
 
 
+def test_empty_tensors_with_any_strides_are_accepted():
+    """An empty batch is never read: the strides numpy gives empty arrays
+    (all zero) must not be rejected, and nothing is launched."""
+    empty = lambda *shape: torch.from_numpy(np.zeros(shape, np.uint16).view(np.int16)).view(torch.bfloat16)  # noqa: E731
+    k = empty(0, 2, 128)
+    assert k.stride() == (0, 0, 0)
+    kc, vc = _cache(hk=2), _cache(hk=2)
+    pa.pa_reshape_and_cache(k, k, kc, vc, torch.from_numpy(np.zeros(0, np.int64)), stream=0)
+    q = empty(0, 4, 128)
+    pa.pa_decode(q, q, kc, vc, torch.zeros(0, 4, dtype=torch.int32), torch.zeros(0, dtype=torch.int32), 0.1, 2,
+                 stream=0)
+    pa.pa_prefill(q, q, kc, vc, torch.zeros(2, 4, dtype=torch.int32), torch.zeros(2, dtype=torch.int32),
+                  torch.zeros(3, dtype=torch.int32), 0, 0.1, 2, stream=0)
+
+
 def test_fixed_workspace_size():
     n = pa.pa_decode_workspace_bytes(8, 32, 8, 128, 8192, 512)
     P = 8192 * 16 // 512
