@@ -1,4 +1,4 @@
-"""CPU oracle for paged decode attention — TEST INFRASTRUCTURE ONLY.
+"""CPU oracle for paged KV cache attention — TEST INFRASTRUCTURE ONLY.
 
 Plain, slow, obviously-correct NumPy code (fp64 for all floating point) that
 states what the PagedAttention hot path computes, written from the pages'
@@ -17,6 +17,13 @@ definitions:
 * ``attention``  — single-query attention softmax(q K^T * scale) V over the
   tokens a block table names, walked logically, in fp64; and the
   log-sum-exp merge of per-partition partial results.
+* ``prefill``    — multi-token (chunked-prefill) attention: every new token
+  of a sequence attends causally over its cache (gitcode repo walkthrough,
+  section 2.2), in fp64.
+* ``replay``     — applies a seeded workload's requests to the allocator and
+  cache models.
+* the allocator also models prefix caching (hash-free keys: parent block and
+  token ids) and swapping to a host block pool.
 
 Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
 leg (and its ``--impl reference`` arm) may import this package.  It shares no
@@ -41,3 +48,4 @@ from .attention import (  # noqa: F401
     partition_partials,
     lse_merge,
 )
+from .prefill import paged_prefill, paged_prefill_seqs  # noqa: F401
