@@ -64,3 +64,27 @@ def test_step_kv_shapes():
         assert k.shape == v.shape == (n, w.num_kv_heads, w.head_size)
         if rows is not None:
             assert n == rows
+
+
+@pytest.mark.parametrize("name,unit", [("tiny_fp32", "GB/s"), ("prefill_tiny", "TFLOP/s")])
+def test_reference_arm_prints_the_contract_line(name, unit):
+    """`bench.py --impl reference` times the oracle on the host and prints one
+    JSON line with the contract's keys (CPU only)."""
+    import json
+    import os
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    res = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--workload", name,
+                          "--steps", "1", "--warmup", "0"], capture_output=True, text=True, timeout=300, cwd=root)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [l for l in res.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["unit"] == unit and d["value"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
