@@ -4,12 +4,14 @@ Thin wrappers with the C ABI's names (include/pa.h).  They only turn torch
 tensors and numpy arrays into the ABI's plain pointers, shapes and strides;
 all device work runs in the library's CUDA kernels.  PyTorch is used by
 callers for device memory and streams.  A non-OK status raises
-``PagedAttentionError``.  When no stream is given, the current torch CUDA
-stream is used.
+``PagedAttentionError``.  Each device call runs with the device that holds
+its CUDA tensors made current (tensors on two devices are refused); when no
+stream is given, that device's current torch stream is used.
 """
 
 from __future__ import annotations
 
+import contextlib
 import ctypes
 from typing import Optional, Sequence, Tuple
 
@@ -86,6 +88,37 @@ def _stream_ptr(stream) -> Optional[int]:
     return stream.cuda_stream or None
 
 
+def _device_index(tensors) -> Optional[int]:
+    """The CUDA device that holds the call's CUDA tensors (None when none is
+    on a CUDA device, e.g. pinned host pools only).  Tensors on two CUDA
+    devices are refused: one launch runs on one device."""
+    idx = None
+    for t in tensors:
+        d = getattr(t, "device", None)
+        if getattr(d, "type", None) != "cuda":  # host tensors, None, numpy's "cpu"
+            continue
+        i = 0 if d.index is None else int(d.index)
+        if idx is None:
+            idx = i
+        elif i != idx:
+            raise ValueError(f"tensors on cuda:{idx} and cuda:{i} in one call")
+    return idx
+
+
+def _on_device(tensors):
+    """The library launches on the current CUDA device: make it the one that
+    holds the tensors for the duration of the call (no switch when it already
+    is, which is the usual one-process-per-GPU case)."""
+    idx = _device_index(tensors)
+    if idx is None:
+        return contextlib.nullcontext()
+    import torch
+
+    if idx == torch.cuda.current_device():
+        return contextlib.nullcontext()
+    return torch.cuda.device(idx)
+
+
 def _opts(stream=None, workspace=None, partition_tokens: int = 0, timeout_ms: int = 0) -> PaOpts:
     o = PaOpts()
     o.stream = _stream_ptr(stream)
@@ -107,17 +140,20 @@ def _opts(stream=None, workspace=None, partition_tokens: int = 0, timeout_ms: in
 def pa_reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, stream=None) -> None:
     """Write each token's K/V [T, H_kv, D] into its slot of the paged cache."""
     tk, tv, kc, vc, sm = (_tensor(x) for x in (key, value, k_cache, v_cache, slot_mapping))
-    o = _opts(stream)
-    _check(_lib_handle.pa_reshape_and_cache(ctypes.byref(tk), ctypes.byref(tv), ctypes.byref(kc), ctypes.byref(vc),
-                                            ctypes.byref(sm), ctypes.byref(o)), "pa_reshape_and_cache")
+    with _on_device((key, value, k_cache, v_cache, slot_mapping)):
+        o = _opts(stream)
+        _check(_lib_handle.pa_reshape_and_cache(ctypes.byref(tk), ctypes.byref(tv), ctypes.byref(kc),
+                                                ctypes.byref(vc), ctypes.byref(sm), ctypes.byref(o)),
+               "pa_reshape_and_cache")
 
 
 def pa_copy_blocks(k_cache, v_cache, pairs, stream=None) -> None:
     """Copy whole blocks (K and V) for each (src, dst) row of the int64 [n, 2] device tensor."""
     kc, vc, pr = (_tensor(x) for x in (k_cache, v_cache, pairs))
-    o = _opts(stream)
-    _check(_lib_handle.pa_copy_blocks(ctypes.byref(kc), ctypes.byref(vc), ctypes.byref(pr), ctypes.byref(o)),
-           "pa_copy_blocks")
+    with _on_device((k_cache, v_cache, pairs)):
+        o = _opts(stream)
+        _check(_lib_handle.pa_copy_blocks(ctypes.byref(kc), ctypes.byref(vc), ctypes.byref(pr), ctypes.byref(o)),
+               "pa_copy_blocks")
 
 
 def pa_decode(out, query, k_cache, v_cache, block_tables, context_lens, scale: float, num_kv_heads: int,
@@ -126,10 +162,11 @@ def pa_decode(out, query, k_cache, v_cache, block_tables, context_lens, scale: f
     0 = auto (balanced split when ``workspace`` is large enough), >0 = fixed
     partitions, -1 = no split."""
     to, tq, kc, vc, bt, cl = (_tensor(x) for x in (out, query, k_cache, v_cache, block_tables, context_lens))
-    o = _opts(stream, workspace, partition_tokens, timeout_ms)
-    _check(_lib_handle.pa_decode(ctypes.byref(to), ctypes.byref(tq), ctypes.byref(kc), ctypes.byref(vc),
-                                 ctypes.byref(bt), ctypes.byref(cl), ctypes.c_float(scale), int(num_kv_heads),
-                                 ctypes.byref(o)), "pa_decode")
+    with _on_device((out, query, k_cache, v_cache, block_tables, context_lens, workspace)):
+        o = _opts(stream, workspace, partition_tokens, timeout_ms)
+        _check(_lib_handle.pa_decode(ctypes.byref(to), ctypes.byref(tq), ctypes.byref(kc), ctypes.byref(vc),
+                                     ctypes.byref(bt), ctypes.byref(cl), ctypes.c_float(scale), int(num_kv_heads),
+                                     ctypes.byref(o)), "pa_decode")
 
 
 def pa_prefill(out, query, k_cache, v_cache, block_tables, context_lens, query_start, max_query_len: int,
@@ -137,37 +174,45 @@ def pa_prefill(out, query, k_cache, v_cache, block_tables, context_lens, query_s
     """Multi-token (chunked-prefill) paged attention: writes out [T, H, D]
     for the new tokens of every sequence (rows query_start[i] ..
     query_start[i+1]), each attending causally over its sequence's cache."""
-    ts = [_tensor(x) for x in (out, query, k_cache, v_cache, block_tables, context_lens, query_start)]
-    o = _opts(stream, timeout_ms=timeout_ms)
-    _check(_lib_handle.pa_prefill(*[ctypes.byref(t) for t in ts], int(max_query_len), ctypes.c_float(scale),
-                                  int(num_kv_heads), ctypes.byref(o)), "pa_prefill")
+    args = (out, query, k_cache, v_cache, block_tables, context_lens, query_start)
+    ts = [_tensor(x) for x in args]
+    with _on_device(args):
+        o = _opts(stream, timeout_ms=timeout_ms)
+        _check(_lib_handle.pa_prefill(*[ctypes.byref(t) for t in ts], int(max_query_len), ctypes.c_float(scale),
+                                      int(num_kv_heads), ctypes.byref(o)), "pa_prefill")
 
 
 def pa_reshape_and_cache_fp8(key, value, k_cache, v_cache, slot_mapping, k_scale, v_scale, stream=None) -> None:
     """Quantizing cache write into an FP8 (torch.float8_e4m3fn) cache: each
     value is stored as the e4m3 code of value / scale[kv head]."""
-    ts = [_tensor(x) for x in (key, value, k_cache, v_cache, slot_mapping, k_scale, v_scale)]
-    o = _opts(stream)
-    _check(_lib_handle.pa_reshape_and_cache_fp8(*[ctypes.byref(t) for t in ts], ctypes.byref(o)),
-           "pa_reshape_and_cache_fp8")
+    args = (key, value, k_cache, v_cache, slot_mapping, k_scale, v_scale)
+    ts = [_tensor(x) for x in args]
+    with _on_device(args):
+        o = _opts(stream)
+        _check(_lib_handle.pa_reshape_and_cache_fp8(*[ctypes.byref(t) for t in ts], ctypes.byref(o)),
+               "pa_reshape_and_cache_fp8")
 
 
 def pa_decode_fp8(out, query, k_cache, v_cache, block_tables, context_lens, scale: float, num_kv_heads: int,
                   k_scale, v_scale, workspace=None, partition_tokens: int = 0, stream=None, timeout_ms: int = 0) -> None:
     """Paged decode over an FP8 cache with per-kv-head scales; bf16 query and output."""
-    ts = [_tensor(x) for x in (out, query, k_cache, v_cache, block_tables, context_lens)]
+    args = (out, query, k_cache, v_cache, block_tables, context_lens)
+    ts = [_tensor(x) for x in args]
     ks, vs = _tensor(k_scale), _tensor(v_scale)
-    o = _opts(stream, workspace, partition_tokens, timeout_ms)
-    _check(_lib_handle.pa_decode_fp8(*[ctypes.byref(t) for t in ts], ctypes.c_float(scale), int(num_kv_heads),
-                                     ctypes.byref(ks), ctypes.byref(vs), ctypes.byref(o)), "pa_decode_fp8")
+    with _on_device(args + (k_scale, v_scale, workspace)):
+        o = _opts(stream, workspace, partition_tokens, timeout_ms)
+        _check(_lib_handle.pa_decode_fp8(*[ctypes.byref(t) for t in ts], ctypes.c_float(scale), int(num_kv_heads),
+                                         ctypes.byref(ks), ctypes.byref(vs), ctypes.byref(o)), "pa_decode_fp8")
 
 
 def pa_swap_blocks(src_k, src_v, dst_k, dst_v, pairs, stream=None) -> None:
     """Copy whole blocks between a device pool and a pinned host pool (either
     direction) for each (src, dst) row of ``pairs``."""
-    ts = [_tensor(x) for x in (src_k, src_v, dst_k, dst_v, pairs)]
-    o = _opts(stream)
-    _check(_lib_handle.pa_swap_blocks(*[ctypes.byref(t) for t in ts], ctypes.byref(o)), "pa_swap_blocks")
+    args = (src_k, src_v, dst_k, dst_v, pairs)
+    ts = [_tensor(x) for x in args]
+    with _on_device(args):
+        o = _opts(stream)
+        _check(_lib_handle.pa_swap_blocks(*[ctypes.byref(t) for t in ts], ctypes.byref(o)), "pa_swap_blocks")
 
 
 NO_ALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
@@ -183,10 +228,11 @@ def pa_decode_no_alloc(out, query, k_cache, v_cache, block_tables, context_lens,
     on a device looks up that array's address, so make it before any stream
     capture.  Calls share the array: issue them on one stream."""
     to, tq, kc, vc, bt, cl = (_tensor(x) for x in (out, query, k_cache, v_cache, block_tables, context_lens))
-    o = _opts(stream, None, partition_tokens, timeout_ms)
-    _check(_lib_handle.pa_decode_no_alloc(ctypes.byref(to), ctypes.byref(tq), ctypes.byref(kc), ctypes.byref(vc),
-                                          ctypes.byref(bt), ctypes.byref(cl), ctypes.c_float(scale),
-                                          int(num_kv_heads), ctypes.byref(o)), "pa_decode_no_alloc")
+    with _on_device((out, query, k_cache, v_cache, block_tables, context_lens)):
+        o = _opts(stream, None, partition_tokens, timeout_ms)
+        _check(_lib_handle.pa_decode_no_alloc(ctypes.byref(to), ctypes.byref(tq), ctypes.byref(kc), ctypes.byref(vc),
+                                              ctypes.byref(bt), ctypes.byref(cl), ctypes.c_float(scale),
+                                              int(num_kv_heads), ctypes.byref(o)), "pa_decode_no_alloc")
 
 
 def pa_decode_workspace_bytes(num_seqs: int, num_heads: int, num_kv_heads: int, head_size: int,

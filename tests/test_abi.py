@@ -160,6 +160,26 @@ def test_empty_tensors_with_any_strides_are_accepted():
                   torch.zeros(3, dtype=torch.int32), 0, 0.1, 2, stream=0)
 
 
+def test_device_of_a_call():
+    """The binding makes the device holding a call's CUDA tensors current
+    (the library launches on the current device); tensors on two devices are
+    refused before anything runs, and host-only calls switch nothing."""
+    from types import SimpleNamespace
+
+    from paged_kv_cache_351_b200 import _device_index, _on_device
+
+    on = lambda i: SimpleNamespace(device=torch.device("cuda", i))  # noqa: E731
+    host = torch.empty(2)
+    assert _device_index([host, None, np.zeros(2)]) is None
+    assert _device_index([host, on(1), on(1), None]) == 1
+    with pytest.raises(ValueError):
+        _device_index([on(0), host, on(1)])
+    with _on_device([host, None]):
+        pass
+    with pytest.raises(ValueError):
+        _on_device([on(0), on(1)])
+
+
 def test_fixed_workspace_size():
     n = pa.pa_decode_workspace_bytes(8, 32, 8, 128, 8192, 512)
     P = 8192 * 16 // 512
