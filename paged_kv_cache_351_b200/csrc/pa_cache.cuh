@@ -1,6 +1,12 @@
 // Byte-moving kernels of the paged KV cache (sm_100a): the per-token cache
-// write by slot (plain, or quantizing into an FP8 cache) and the whole-block
-// copy of copy-on-write.
+// write by slot (plain, or quantizing into an FP8 cache), the whole-block
+// copy of copy-on-write, and the block swap between the device pool and a
+// pinned host pool.  The pages fix what these do without naming kernels: a
+// new token's K/V lands in the physical block its table names, at its
+// offset in that block, and a write into a block that several samples share
+// first copies the block (vLLM launch blog, "PagedAttention" section, as
+// summarised on the CSDN discovery note, item 2); blocks can be swapped out
+// (agientry.com overview, opening section).
 //
 // Both are pure HBM traffic.  Every (token, kv head) row of K or V is
 // head_size * elem bytes (256 B for bf16/128 and fp32/64) and contiguous on
