@@ -149,6 +149,25 @@ pa_status launch_status() {
   return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
+// Raise a kernel's dynamic shared-memory limit on the current device to at
+// least `bytes` (limit[dev] remembers what was set).  The limit only grows and
+// the check-and-set is serialised, so host threads launching the same kernel
+// cannot lower it under one another.  False if the runtime refused.
+std::mutex g_attr_mu;
+
+template <typename Kern>
+bool raise_smem_limit(Kern kern, size_t bytes, int dev, std::atomic<size_t>* limit) {
+  if (limit[dev].load(std::memory_order_acquire) >= bytes) return true;
+  std::lock_guard<std::mutex> lk(g_attr_mu);
+  if (limit[dev].load(std::memory_order_relaxed) >= bytes) return true;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes)) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return false;
+  }
+  limit[dev].store(bytes, std::memory_order_release);
+  return true;
+}
+
 template <typename Kern, typename... Args>
 cudaError_t launch_pdl(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl, Args... args) {
   cudaLaunchConfig_t cfg = {};
@@ -226,15 +245,9 @@ unsigned long long next_call_tag() {
 
 template <typename Tkv, typename Tq, int D, int G>
 pa_status run_decode(const pa::DecodeArgs& base, const DecodePlan& p, cudaStream_t st, int dev) {
-  static bool attr_set[kMaxDevices] = {};
-  static size_t attr_bytes[kMaxDevices] = {};
+  static std::atomic<size_t> smem_limit[kMaxDevices];
   auto kern = pa::decode_kernel<Tkv, Tq, D, G>;
-  if (!attr_set[dev] || attr_bytes[dev] < p.smem) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(p.smem)) != cudaSuccess)
-      return PA_ERR_CUDA;
-    attr_set[dev] = true;
-    attr_bytes[dev] = p.smem;
-  }
+  if (!raise_smem_limit(kern, p.smem, dev, smem_limit)) return PA_ERR_CUDA;
   pa::DecodeArgs a = base;
   a.stages = p.stages;
   a.mode = p.mode;
@@ -370,14 +383,9 @@ pa_status bf16_map(CUtensorMap* m, void* ptr, int rank, const cuuint64_t* dims, 
 template <int G>
 pa_status run_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const pa::PrefillArgs& a,
                       int max_query_len, int Hkv, cudaStream_t st, int dev) {
-  static bool attr_set[kMaxDevices] = {};
+  static std::atomic<size_t> smem_limit[kMaxDevices];
   auto kern = pa::prefill_kernel<G>;
-  if (!attr_set[dev]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(pa::kPfSmemBytes)) !=
-        cudaSuccess)
-      return launch_status();
-    attr_set[dev] = true;
-  }
+  if (!raise_smem_limit(kern, size_t(pa::kPfSmemBytes), dev, smem_limit)) return PA_ERR_CUDA;
   constexpr int TOK = pa::kPfRows / G;  // new tokens per CTA
   const dim3 grid(unsigned((max_query_len + TOK - 1) / TOK), unsigned(Hkv), unsigned(a.B));
   if (launch_pdl(kern, grid, dim3(pa::kPfThreads), pa::kPfSmemBytes, st, true, tq, tk, tv, a) != cudaSuccess)
@@ -710,7 +718,7 @@ static pa_status decode_impl(pa_tensor* out, const pa_tensor* query, const pa_te
     a.call_tag = next_call_tag();
   }
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PA_ERR_CUDA;
   cudaStream_t s = stream_of(opts);
   if (dt == PA_BF16 && D == 128) return dispatch_group<__nv_bfloat16, __nv_bfloat16, 128>(int(G), a, plan, s, dev);
   if (dt == PA_BF16 && D == 64) return dispatch_group<__nv_bfloat16, __nv_bfloat16, 64>(int(G), a, plan, s, dev);
