@@ -84,16 +84,38 @@ struct pa_allocator {
 
   int64_t available() const { return static_cast<int64_t>(free_stack.size()) + static_cast<int64_t>(lru.size()); }
 
-  void unregister(int32_t b) {
-    cache.erase(key_of[b]);
-    reg[b] = 0;
-    const int32_t parent = key_of[b].parent;
-    if (parent >= 0) children[parent].erase(b);
-    std::set<int32_t> kids;
-    kids.swap(children[b]);
-    for (int32_t c : kids) {  // increasing block order, depth first
-      unregister(c);
-      if (in_lru[c]) {
+  // Unregister block `root` and, below it, every registered descendant in
+  // increasing block order, depth first.  A descendant that nobody holds
+  // loses its key and goes back on the free stack once its own subtree is
+  // done.  Iterative: a registered chain is as deep as its sequence is long
+  // in blocks, far beyond what recursion on a thread's stack can take.
+  void unregister(int32_t root) {
+    struct Frame {
+      int32_t b;
+      std::vector<int32_t> kids;  // b's registered children, increasing
+      size_t next;
+    };
+    std::vector<Frame> stack;
+    auto enter = [&](int32_t b) {
+      cache.erase(key_of[b]);
+      reg[b] = 0;
+      const int32_t parent = key_of[b].parent;
+      if (parent >= 0) children[parent].erase(b);
+      Frame f{b, std::vector<int32_t>(children[b].begin(), children[b].end()), 0};
+      children[b].clear();
+      stack.push_back(std::move(f));
+    };
+    enter(root);
+    while (!stack.empty()) {
+      Frame& top = stack.back();
+      if (top.next < top.kids.size()) {
+        const int32_t c = top.kids[top.next++];
+        enter(c);  // may reallocate `stack`: `top` is not used after this
+        continue;
+      }
+      const int32_t c = top.b;
+      stack.pop_back();
+      if (!stack.empty() && in_lru[c]) {  // a descendant, not the root
         lru.erase(lru_pos[c]);
         in_lru[c] = 0;
         free_stack.push_back(c);

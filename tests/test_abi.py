@@ -403,6 +403,78 @@ def test_prefix_cache_matches_oracle_random(seed):
         assert c.stats()["num_cached"] == o.num_cached()
 
 
+def test_eviction_cascade_over_a_deep_branching_tree():
+    """Evicting the root of a registered tree 500 blocks deep, with side
+    branches at several depths, unregisters the descendants in the oracle's
+    order (increasing block id, depth first) as the pool is drained a few
+    blocks at a time."""
+    import sys
+
+    nb, bs, depth = 720, 4, 500
+    rnd = random.Random(77)
+    order = list(range(nb))
+    rnd.shuffle(order)
+    c, o = pa.Allocator(nb, bs, order), BlockAllocator(nb, bs, order)
+    base = [rnd.randrange(5) for _ in range(depth * bs)]
+    prompts = [base + [9]]
+    for k in (50, 120, 121, 300, 499):
+        prompts.append(base[: k * bs] + [5 + j % 3 for j in range(3 * bs)] + [9])
+    limit = sys.getrecursionlimit()
+    sys.setrecursionlimit(max(limit, 20 * depth))  # the oracle recurses once per tree level
+    try:
+        for s, prompt in enumerate(prompts):
+            hit = o.add_prefix(s, prompt)
+            assert c.add_prefix(s, prompt) == hit
+            so, co = o.append_tokens(s, prompt[hit:])
+            sc, cc = c.append_tokens(s, prompt[hit:])
+            assert sc.tolist() == so and cc == co
+        for s in (3, 0, 5, 1, 4, 2):
+            o.free(s)
+            c.free(s)
+        assert c.evictable() == list(o._evictable) and len(c.evictable()) == depth + 5 * 3
+        o.add(100)
+        c.add(100)
+        deepest = 0
+        while o.num_free() > 0:
+            n = min(37, o.num_free() * bs)
+            before = o.num_cached()
+            so, co = o.append(100, n)
+            sc, cc = c.append(100, n)
+            assert sc.tolist() == so and cc == co
+            deepest = max(deepest, before - o.num_cached())
+            _compare_state(c, o)
+            assert c.evictable() == list(o._evictable)
+            assert c.stats()["num_cached"] == o.num_cached()
+        assert deepest > 100  # at least one request unregistered a subtree of over 100 blocks
+    finally:
+        sys.setrecursionlimit(limit)
+
+
+def test_eviction_of_a_very_long_chain_keeps_the_host_stack():
+    """A sequence of 100,000 registered blocks (1.6M tokens) freed and then
+    evicted by one request: the cascade runs without recursion (a separate
+    process, so a stack overflow would fail this test, not the test run)."""
+    import subprocess
+    import sys
+
+    code = (
+        "import numpy as np, paged_kv_cache_351_b200 as pa\n"
+        "n, bs = 100000, 16\n"
+        "a = pa.Allocator(n + 4, bs)\n"
+        "toks = (np.arange(n * bs + 1) % 7 + 100 * (np.arange(n * bs + 1) // bs)).tolist()\n"
+        "hit = a.add_prefix(0, toks)\n"
+        "a.append_tokens(0, toks[hit:])\n"
+        "a.free(0)\n"
+        "assert len(a.evictable()) == n\n"
+        "a.add(1)\n"
+        "a.append(1, (n + 2) * bs)\n"
+        "print('free', a.num_free(), 'evictable', len(a.evictable()))\n"
+    )
+    res = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert res.returncode == 0, res.stderr[-2000:]
+    assert res.stdout.split() == ["free", "2", "evictable", "0"]
+
+
 @pytest.mark.parametrize("seed", range(6))
 def test_swap_matches_oracle_random(seed):
     """Swap-out/in requests (with prefix caching and forks) give identical
