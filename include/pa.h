@@ -58,7 +58,8 @@ typedef enum {
   PA_ERR_CUDA = 4,           /* a CUDA runtime call failed */
   PA_ERR_DEVICE_TIMEOUT = 5, /* a device-side bounded wait gave up */
   PA_ERR_DEVICE_BOUNDS = 6,  /* a device-side index check failed; element skipped */
-  PA_ERR_SCRATCH_LIMIT = 7   /* pa_decode_no_alloc: the call needs more scratch than the library's fixed buffer */
+  PA_ERR_SCRATCH_LIMIT = 7,  /* pa_decode_no_alloc: the call needs more scratch than the library's fixed buffer */
+  PA_ERR_HOST_ALLOC = 8      /* allocator: host memory ran out inside the call (see the allocator rules) */
 } pa_status;
 
 typedef enum { PA_F32 = 0, PA_BF16 = 1, PA_I32 = 2, PA_I64 = 3, PA_FP8_E4M3 = 4 } pa_dtype;
@@ -314,7 +315,10 @@ pa_status pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_heads, int32_t
  *    gains one reference;
  *  - free: blocks lose one reference in table order; a block reaching 0 is
  *    pushed on the free stack.
- * Sequence ids are arbitrary int64 values.
+ * Sequence ids are arbitrary int64 values.  No C++ exception leaves these
+ * calls: if host memory runs out inside one, it returns PA_ERR_HOST_ALLOC
+ * (pa_alloc_create then creates nothing; after any other call the
+ * allocator's state is unspecified and it should only be destroyed).
  * ------------------------------------------------------------------------- */
 typedef struct pa_allocator pa_allocator;
 

@@ -55,6 +55,7 @@ STATUS_NAMES = {
     5: "PA_ERR_DEVICE_TIMEOUT",
     6: "PA_ERR_DEVICE_BOUNDS",
     7: "PA_ERR_SCRATCH_LIMIT",
+    8: "PA_ERR_HOST_ALLOC",
 }
 PA_F32, PA_BF16, PA_I32, PA_I64, PA_FP8_E4M3 = 0, 1, 2, 3, 4
 PA_DEV_TIMEOUT, PA_DEV_BAD_BLOCK, PA_DEV_BAD_CONTEXT, PA_DEV_BAD_SLOT = 0x1, 0x2, 0x4, 0x8

@@ -14,7 +14,7 @@
 #include <cstdint>
 #include <cstring>
 #include <list>
-#include <new>
+#include <memory>
 #include <set>
 #include <unordered_map>
 #include <vector>
@@ -50,6 +50,18 @@ struct KeyHash {
     return static_cast<size_t>(h);
   }
 };
+
+// Runs the body of a C entry point: no C++ exception may cross the C ABI,
+// and the only ones this code can raise come from host allocation
+// (std::bad_alloc, or std::length_error for an impossible size).
+template <typename F>
+pa_status no_throw(F&& body) {
+  try {
+    return body();
+  } catch (...) {
+    return PA_ERR_HOST_ALLOC;
+  }
+}
 
 }  // namespace
 
@@ -227,151 +239,163 @@ extern "C" {
 pa_status pa_alloc_create(int32_t num_blocks, int32_t block_size, const int32_t* free_order, pa_allocator** out) {
   if (out == nullptr || num_blocks <= 0 || block_size <= 0) return PA_ERR_INVALID_ARG;
   *out = nullptr;
-  pa_allocator* a = new (std::nothrow) pa_allocator();
-  if (a == nullptr) return PA_ERR_INVALID_ARG;
-  a->num_blocks = num_blocks;
-  a->block_size = block_size;
-  a->ref.assign(num_blocks, 0);
-  a->init_cache_state();
-  a->free_stack.resize(num_blocks);
-  if (free_order != nullptr) {
-    std::vector<uint8_t> seen(num_blocks, 0);
-    for (int32_t k = 0; k < num_blocks; ++k) {
-      const int32_t b = free_order[k];
-      if (b < 0 || b >= num_blocks || seen[b]) {
-        delete a;
-        return PA_ERR_INVALID_ARG;
+  return no_throw([&]() -> pa_status {
+    std::unique_ptr<pa_allocator> a(new pa_allocator());
+    a->num_blocks = num_blocks;
+    a->block_size = block_size;
+    a->ref.assign(num_blocks, 0);
+    a->init_cache_state();
+    a->free_stack.resize(num_blocks);
+    if (free_order != nullptr) {
+      std::vector<uint8_t> seen(num_blocks, 0);
+      for (int32_t k = 0; k < num_blocks; ++k) {
+        const int32_t b = free_order[k];
+        if (b < 0 || b >= num_blocks || seen[b]) return PA_ERR_INVALID_ARG;
+        seen[b] = 1;
+        a->free_stack[num_blocks - 1 - k] = b;
       }
-      seen[b] = 1;
-      a->free_stack[num_blocks - 1 - k] = b;
+    } else {
+      for (int32_t k = 0; k < num_blocks; ++k) a->free_stack[num_blocks - 1 - k] = k;
     }
-  } else {
-    for (int32_t k = 0; k < num_blocks; ++k) a->free_stack[num_blocks - 1 - k] = k;
-  }
-  *out = a;
-  return PA_OK;
+    *out = a.release();
+    return PA_OK;
+  });
 }
 
 void pa_alloc_destroy(pa_allocator* a) { delete a; }
 
 pa_status pa_seq_add(pa_allocator* a, int64_t seq_id) {
-  if (a == nullptr) return PA_ERR_INVALID_ARG;
-  if (a->seqs.count(seq_id)) return PA_ERR_INVALID_ARG;
-  a->seqs.emplace(seq_id, Seq());
-  return PA_OK;
+  return no_throw([&]() -> pa_status {
+    if (a == nullptr) return PA_ERR_INVALID_ARG;
+    if (a->seqs.count(seq_id)) return PA_ERR_INVALID_ARG;
+    a->seqs.emplace(seq_id, Seq());
+    return PA_OK;
+  });
 }
 
 pa_status pa_seq_append(pa_allocator* a, int64_t seq_id, int32_t n_tokens, int64_t* slots_out,
                         int64_t* cow_pair_out, int32_t* n_cow_out) {
-  if (a == nullptr) return PA_ERR_INVALID_ARG;
-  return a->append(seq_id, n_tokens, nullptr, slots_out, cow_pair_out, n_cow_out);
+  return no_throw([&]() -> pa_status {
+    if (a == nullptr) return PA_ERR_INVALID_ARG;
+    return a->append(seq_id, n_tokens, nullptr, slots_out, cow_pair_out, n_cow_out);
+  });
 }
 
 pa_status pa_seq_add_prefix(pa_allocator* a, int64_t seq_id, const int64_t* tokens, int32_t n_tokens,
                             int32_t* n_cached_out) {
-  if (a == nullptr || n_tokens < 0 || (n_tokens > 0 && tokens == nullptr)) return PA_ERR_INVALID_ARG;
-  if (a->seqs.count(seq_id)) return PA_ERR_INVALID_ARG;
-  const int32_t bs = a->block_size;
-  std::vector<int32_t> hits;
-  int32_t parent = -1;
-  Key k{-1, std::vector<int64_t>(bs)};
-  for (int32_t j = 0; j < (n_tokens > 0 ? (n_tokens - 1) / bs : 0); ++j) {
-    k.parent = parent;
-    std::copy(tokens + static_cast<int64_t>(j) * bs, tokens + static_cast<int64_t>(j + 1) * bs, k.toks.begin());
-    auto it = a->cache.find(k);
-    if (it == a->cache.end()) break;
-    hits.push_back(it->second);
-    parent = it->second;
-  }
-  for (int32_t b : hits) {
-    if (a->ref[b] == 0 && a->in_lru[b]) {
-      a->lru.erase(a->lru_pos[b]);
-      a->in_lru[b] = 0;
+  return no_throw([&]() -> pa_status {
+    if (a == nullptr || n_tokens < 0 || (n_tokens > 0 && tokens == nullptr)) return PA_ERR_INVALID_ARG;
+    if (a->seqs.count(seq_id)) return PA_ERR_INVALID_ARG;
+    const int32_t bs = a->block_size;
+    std::vector<int32_t> hits;
+    int32_t parent = -1;
+    Key k{-1, std::vector<int64_t>(bs)};
+    for (int32_t j = 0; j < (n_tokens > 0 ? (n_tokens - 1) / bs : 0); ++j) {
+      k.parent = parent;
+      std::copy(tokens + static_cast<int64_t>(j) * bs, tokens + static_cast<int64_t>(j + 1) * bs, k.toks.begin());
+      auto it = a->cache.find(k);
+      if (it == a->cache.end()) break;
+      hits.push_back(it->second);
+      parent = it->second;
     }
-    a->ref[b] += 1;
-  }
-  Seq s;
-  s.table = hits;
-  s.len = static_cast<int32_t>(hits.size()) * bs;
-  s.tokens.assign(tokens, tokens + s.len);
-  a->seqs.emplace(seq_id, std::move(s));
-  if (n_cached_out != nullptr) *n_cached_out = static_cast<int32_t>(hits.size()) * bs;
-  return PA_OK;
+    for (int32_t b : hits) {
+      if (a->ref[b] == 0 && a->in_lru[b]) {
+        a->lru.erase(a->lru_pos[b]);
+        a->in_lru[b] = 0;
+      }
+      a->ref[b] += 1;
+    }
+    Seq s;
+    s.table = hits;
+    s.len = static_cast<int32_t>(hits.size()) * bs;
+    s.tokens.assign(tokens, tokens + s.len);
+    a->seqs.emplace(seq_id, std::move(s));
+    if (n_cached_out != nullptr) *n_cached_out = static_cast<int32_t>(hits.size()) * bs;
+    return PA_OK;
+  });
 }
 
 pa_status pa_seq_append_tokens(pa_allocator* a, int64_t seq_id, const int64_t* tokens, int32_t n_tokens,
                                int64_t* slots_out, int64_t* cow_pair_out, int32_t* n_cow_out) {
-  if (a == nullptr || (n_tokens > 0 && tokens == nullptr)) return PA_ERR_INVALID_ARG;
-  static const int64_t kNone = 0;
-  return a->append(seq_id, n_tokens, n_tokens > 0 ? tokens : &kNone, slots_out, cow_pair_out, n_cow_out);
+  return no_throw([&]() -> pa_status {
+    if (a == nullptr || (n_tokens > 0 && tokens == nullptr)) return PA_ERR_INVALID_ARG;
+    static const int64_t kNone = 0;
+    return a->append(seq_id, n_tokens, n_tokens > 0 ? tokens : &kNone, slots_out, cow_pair_out, n_cow_out);
+  });
 }
 
 pa_status pa_alloc_set_host_pool(pa_allocator* a, int32_t num_host_blocks, const int32_t* host_free_order) {
-  if (a == nullptr || num_host_blocks < 0) return PA_ERR_INVALID_ARG;
-  for (const auto& kv : a->seqs)
-    if (kv.second.swapped) return PA_ERR_INVALID_ARG;
-  std::vector<int32_t> st(num_host_blocks);
-  std::vector<uint8_t> seen(num_host_blocks, 0);
-  for (int32_t k = 0; k < num_host_blocks; ++k) {
-    const int32_t h = host_free_order ? host_free_order[k] : k;
-    if (h < 0 || h >= num_host_blocks || seen[h]) return PA_ERR_INVALID_ARG;
-    seen[h] = 1;
-    st[num_host_blocks - 1 - k] = h;
-  }
-  a->num_host_blocks = num_host_blocks;
-  a->host_free.swap(st);
-  return PA_OK;
+  return no_throw([&]() -> pa_status {
+    if (a == nullptr || num_host_blocks < 0) return PA_ERR_INVALID_ARG;
+    for (const auto& kv : a->seqs)
+      if (kv.second.swapped) return PA_ERR_INVALID_ARG;
+    std::vector<int32_t> st(num_host_blocks);
+    std::vector<uint8_t> seen(num_host_blocks, 0);
+    for (int32_t k = 0; k < num_host_blocks; ++k) {
+      const int32_t h = host_free_order ? host_free_order[k] : k;
+      if (h < 0 || h >= num_host_blocks || seen[h]) return PA_ERR_INVALID_ARG;
+      seen[h] = 1;
+      st[num_host_blocks - 1 - k] = h;
+    }
+    a->num_host_blocks = num_host_blocks;
+    a->host_free.swap(st);
+    return PA_OK;
+  });
 }
 
 pa_status pa_seq_swap_out(pa_allocator* a, int64_t seq_id, int64_t* pairs_out, int32_t cap, int32_t* n_out) {
-  if (a == nullptr || n_out == nullptr) return PA_ERR_INVALID_ARG;
-  auto it = a->seqs.find(seq_id);
-  if (it == a->seqs.end() || it->second.swapped) return PA_ERR_INVALID_ARG;
-  Seq& s = it->second;
-  const int32_t n = static_cast<int32_t>(s.table.size());
-  *n_out = n;
-  if (n > cap || (n > 0 && pairs_out == nullptr)) return PA_ERR_INVALID_ARG;
-  if (n > static_cast<int32_t>(a->host_free.size())) return PA_ERR_OUT_OF_BLOCKS;
-  s.host.resize(n);
-  for (int32_t k = 0; k < n; ++k) {
-    const int32_t h = a->host_free.back();
-    a->host_free.pop_back();
-    s.host[k] = h;
-    pairs_out[2 * k] = s.table[k];
-    pairs_out[2 * k + 1] = h;
-  }
-  for (int32_t b : s.table) a->release(b);
-  s.table.clear();
-  s.swapped = true;
-  return PA_OK;
+  return no_throw([&]() -> pa_status {
+    if (a == nullptr || n_out == nullptr) return PA_ERR_INVALID_ARG;
+    auto it = a->seqs.find(seq_id);
+    if (it == a->seqs.end() || it->second.swapped) return PA_ERR_INVALID_ARG;
+    Seq& s = it->second;
+    const int32_t n = static_cast<int32_t>(s.table.size());
+    *n_out = n;
+    if (n > cap || (n > 0 && pairs_out == nullptr)) return PA_ERR_INVALID_ARG;
+    if (n > static_cast<int32_t>(a->host_free.size())) return PA_ERR_OUT_OF_BLOCKS;
+    s.host.resize(n);
+    for (int32_t k = 0; k < n; ++k) {
+      const int32_t h = a->host_free.back();
+      a->host_free.pop_back();
+      s.host[k] = h;
+      pairs_out[2 * k] = s.table[k];
+      pairs_out[2 * k + 1] = h;
+    }
+    for (int32_t b : s.table) a->release(b);
+    s.table.clear();
+    s.swapped = true;
+    return PA_OK;
+  });
 }
 
 pa_status pa_seq_swap_in(pa_allocator* a, int64_t seq_id, int64_t* pairs_out, int32_t cap, int32_t* n_out) {
-  if (a == nullptr || n_out == nullptr) return PA_ERR_INVALID_ARG;
-  auto it = a->seqs.find(seq_id);
-  if (it == a->seqs.end() || !it->second.swapped) return PA_ERR_INVALID_ARG;
-  Seq& s = it->second;
-  const int32_t n = static_cast<int32_t>(s.host.size());
-  *n_out = n;
-  if (n > cap || (n > 0 && pairs_out == nullptr)) return PA_ERR_INVALID_ARG;
-  if (n > a->available()) return PA_ERR_OUT_OF_BLOCKS;
-  s.table.resize(n);
-  for (int32_t k = 0; k < n; ++k) {
-    const int32_t b = a->take_block();
-    a->ref[b] = 1;
-    s.table[k] = b;
-    pairs_out[2 * k] = s.host[k];
-    pairs_out[2 * k + 1] = b;
-  }
-  for (int32_t h : s.host) a->host_free.push_back(h);
-  s.host.clear();
-  s.swapped = false;
-  if (s.tracked) {
-    const int32_t bs = a->block_size;
-    for (int32_t j = 0; j < s.len / bs; ++j)
-      a->register_block(s.table[j], j ? s.table[j - 1] : -1, s.tokens.data() + static_cast<int64_t>(j) * bs);
-  }
-  return PA_OK;
+  return no_throw([&]() -> pa_status {
+    if (a == nullptr || n_out == nullptr) return PA_ERR_INVALID_ARG;
+    auto it = a->seqs.find(seq_id);
+    if (it == a->seqs.end() || !it->second.swapped) return PA_ERR_INVALID_ARG;
+    Seq& s = it->second;
+    const int32_t n = static_cast<int32_t>(s.host.size());
+    *n_out = n;
+    if (n > cap || (n > 0 && pairs_out == nullptr)) return PA_ERR_INVALID_ARG;
+    if (n > a->available()) return PA_ERR_OUT_OF_BLOCKS;
+    s.table.resize(n);
+    for (int32_t k = 0; k < n; ++k) {
+      const int32_t b = a->take_block();
+      a->ref[b] = 1;
+      s.table[k] = b;
+      pairs_out[2 * k] = s.host[k];
+      pairs_out[2 * k + 1] = b;
+    }
+    for (int32_t h : s.host) a->host_free.push_back(h);
+    s.host.clear();
+    s.swapped = false;
+    if (s.tracked) {
+      const int32_t bs = a->block_size;
+      for (int32_t j = 0; j < s.len / bs; ++j)
+        a->register_block(s.table[j], j ? s.table[j - 1] : -1, s.tokens.data() + static_cast<int64_t>(j) * bs);
+    }
+    return PA_OK;
+  });
 }
 
 int32_t pa_alloc_num_host_free(const pa_allocator* a) {
@@ -400,48 +424,54 @@ pa_status pa_alloc_evictable(const pa_allocator* a, int32_t* out, int32_t cap, i
 
 pa_status pa_seq_append_batch(pa_allocator* a, const int64_t* seq_ids, const int32_t* n_tokens, int32_t n,
                               int64_t* slots_out, int64_t* cow_pairs_out, int32_t* n_cow_out, int32_t* n_done_out) {
-  if (a == nullptr || n < 0 || (n > 0 && (seq_ids == nullptr || n_tokens == nullptr))) return PA_ERR_INVALID_ARG;
-  int64_t off = 0;
-  int32_t cows = 0;
-  pa_status st = PA_OK;
-  int32_t k = 0;
-  for (; k < n; ++k) {
-    int32_t c = 0;
-    int64_t pair[2] = {-1, -1};
-    st = a->append(seq_ids[k], n_tokens[k], nullptr, slots_out == nullptr ? nullptr : slots_out + off, pair, &c);
-    if (st != PA_OK) break;
-    off += n_tokens[k];
-    if (c) {
-      if (cow_pairs_out != nullptr) {
-        cow_pairs_out[2 * cows] = pair[0];
-        cow_pairs_out[2 * cows + 1] = pair[1];
+  return no_throw([&]() -> pa_status {
+    if (a == nullptr || n < 0 || (n > 0 && (seq_ids == nullptr || n_tokens == nullptr))) return PA_ERR_INVALID_ARG;
+    int64_t off = 0;
+    int32_t cows = 0;
+    pa_status st = PA_OK;
+    int32_t k = 0;
+    for (; k < n; ++k) {
+      int32_t c = 0;
+      int64_t pair[2] = {-1, -1};
+      st = a->append(seq_ids[k], n_tokens[k], nullptr, slots_out == nullptr ? nullptr : slots_out + off, pair, &c);
+      if (st != PA_OK) break;
+      off += n_tokens[k];
+      if (c) {
+        if (cow_pairs_out != nullptr) {
+          cow_pairs_out[2 * cows] = pair[0];
+          cow_pairs_out[2 * cows + 1] = pair[1];
+        }
+        ++cows;
       }
-      ++cows;
     }
-  }
-  if (n_cow_out != nullptr) *n_cow_out = cows;
-  if (n_done_out != nullptr) *n_done_out = k;
-  return st;
+    if (n_cow_out != nullptr) *n_cow_out = cows;
+    if (n_done_out != nullptr) *n_done_out = k;
+    return st;
+  });
 }
 
 pa_status pa_seq_fork(pa_allocator* a, int64_t parent, int64_t child) {
-  if (a == nullptr) return PA_ERR_INVALID_ARG;
-  auto it = a->seqs.find(parent);
-  if (it == a->seqs.end() || it->second.swapped || a->seqs.count(child)) return PA_ERR_INVALID_ARG;
-  Seq c = it->second;  // copy before emplace may rehash
-  for (int32_t b : c.table) a->ref[b] += 1;
-  a->seqs.emplace(child, std::move(c));
-  return PA_OK;
+  return no_throw([&]() -> pa_status {
+    if (a == nullptr) return PA_ERR_INVALID_ARG;
+    auto it = a->seqs.find(parent);
+    if (it == a->seqs.end() || it->second.swapped || a->seqs.count(child)) return PA_ERR_INVALID_ARG;
+    Seq c = it->second;  // copy before emplace may rehash
+    for (int32_t b : c.table) a->ref[b] += 1;
+    a->seqs.emplace(child, std::move(c));
+    return PA_OK;
+  });
 }
 
 pa_status pa_seq_free(pa_allocator* a, int64_t seq_id) {
-  if (a == nullptr) return PA_ERR_INVALID_ARG;
-  auto it = a->seqs.find(seq_id);
-  if (it == a->seqs.end()) return PA_ERR_INVALID_ARG;
-  for (int32_t b : it->second.table) a->release(b);
-  for (int32_t h : it->second.host) a->host_free.push_back(h);
-  a->seqs.erase(it);
-  return PA_OK;
+  return no_throw([&]() -> pa_status {
+    if (a == nullptr) return PA_ERR_INVALID_ARG;
+    auto it = a->seqs.find(seq_id);
+    if (it == a->seqs.end()) return PA_ERR_INVALID_ARG;
+    for (int32_t b : it->second.table) a->release(b);
+    for (int32_t h : it->second.host) a->host_free.push_back(h);
+    a->seqs.erase(it);
+    return PA_OK;
+  });
 }
 
 pa_status pa_seq_len(const pa_allocator* a, int64_t seq_id, int32_t* len_out) {
@@ -489,31 +519,33 @@ int32_t pa_block_refcount(const pa_allocator* a, int32_t block) {
 }
 
 pa_status pa_alloc_get_stats(const pa_allocator* a, pa_alloc_stats* out) {
-  if (a == nullptr || out == nullptr) return PA_ERR_INVALID_ARG;
-  const int32_t bs = a->block_size;
-  std::vector<int32_t> filled(a->num_blocks, 0);
-  int64_t tokens = 0;
-  for (const auto& kv : a->seqs) {
-    const Seq& s = kv.second;
-    tokens += s.len;
-    for (size_t k = 0; k < s.table.size(); ++k) {
-      const int64_t f = std::min<int64_t>(bs, s.len - static_cast<int64_t>(k) * bs);
-      int32_t& slot = filled[s.table[k]];
-      if (f > slot) slot = static_cast<int32_t>(f);
+  return no_throw([&]() -> pa_status {
+    if (a == nullptr || out == nullptr) return PA_ERR_INVALID_ARG;
+    const int32_t bs = a->block_size;
+    std::vector<int32_t> filled(a->num_blocks, 0);
+    int64_t tokens = 0;
+    for (const auto& kv : a->seqs) {
+      const Seq& s = kv.second;
+      tokens += s.len;
+      for (size_t k = 0; k < s.table.size(); ++k) {
+        const int64_t f = std::min<int64_t>(bs, s.len - static_cast<int64_t>(k) * bs);
+        int32_t& slot = filled[s.table[k]];
+        if (f > slot) slot = static_cast<int32_t>(f);
+      }
     }
-  }
-  int64_t waste = 0;
-  for (int32_t b = 0; b < a->num_blocks; ++b)
-    if (a->ref[b] > 0) waste += bs - filled[b];
-  out->num_blocks = a->num_blocks;
-  out->num_free = static_cast<int32_t>(a->available());
-  out->num_cached = static_cast<int32_t>(a->cache.size());
-  out->num_evictable = static_cast<int32_t>(a->lru.size());
-  out->num_seqs = static_cast<int32_t>(a->seqs.size());
-  out->block_size = bs;
-  out->num_tokens = tokens;
-  out->waste_slots = waste;
-  return PA_OK;
+    int64_t waste = 0;
+    for (int32_t b = 0; b < a->num_blocks; ++b)
+      if (a->ref[b] > 0) waste += bs - filled[b];
+    out->num_blocks = a->num_blocks;
+    out->num_free = static_cast<int32_t>(a->available());
+    out->num_cached = static_cast<int32_t>(a->cache.size());
+    out->num_evictable = static_cast<int32_t>(a->lru.size());
+    out->num_seqs = static_cast<int32_t>(a->seqs.size());
+    out->block_size = bs;
+    out->num_tokens = tokens;
+    out->waste_slots = waste;
+    return PA_OK;
+  });
 }
 
 }  // extern "C"

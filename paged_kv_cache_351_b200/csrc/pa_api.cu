@@ -417,6 +417,8 @@ const char* pa_status_string(pa_status s) {
       return "device index check failed";
     case PA_ERR_SCRATCH_LIMIT:
       return "needs more split scratch than the library's fixed no-alloc buffer holds";
+    case PA_ERR_HOST_ALLOC:
+      return "host memory allocation failed";
   }
   return "unknown status";
 }

@@ -38,8 +38,37 @@ def test_exports_every_declared_function():
 
 def test_status_strings():
     lib = pa.library()
-    for s in range(7):
-        assert lib.pa_status_string(s)
+    for s in range(9):
+        assert lib.pa_status_string(s) != b"unknown status"
+    assert lib.pa_status_string(99) == b"unknown status"
+
+
+def test_host_allocation_failure_is_a_status():
+    """Host memory running out inside the allocator returns PA_ERR_HOST_ALLOC
+    instead of letting a C++ exception cross the C ABI (which would end the
+    process).  A child process caps its address space so that a pool of 2^30
+    blocks cannot get its bookkeeping; a small pool in the same process keeps
+    working."""
+    import subprocess
+    import sys
+
+    code = (
+        "import resource\n"
+        "import paged_kv_cache_351_b200 as pa\n"
+        "vm = [int(l.split()[1]) * 1024 for l in open('/proc/self/status') if l.startswith('VmSize:')][0]\n"
+        "resource.setrlimit(resource.RLIMIT_AS, (vm + (1 << 30), resource.RLIM_INFINITY))\n"
+        "small = pa.Allocator(1000, 16)\n"
+        "try:\n"
+        "    pa.Allocator(1 << 30, 16)\n"
+        "except pa.PagedAttentionError as e:\n"
+        "    print('status', e.status)\n"
+        "small.add(0)\n"
+        "small.append(0, 40)\n"
+        "print('free', small.num_free())\n"
+    )
+    res = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=120, cwd=ROOT)
+    assert res.returncode == 0, res.stderr[-2000:]
+    assert res.stdout.split() == ["status", "8", "free", "997"]
 
 
 # ---------------------------------------------------------------------------
