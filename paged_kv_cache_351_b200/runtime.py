@@ -75,6 +75,9 @@ class PagedKVCacheGPU:
             pa_reshape_and_cache(key, value, self.k_cache, self.v_cache, slots, stream=stream)
 
     def workspace(self, num_seqs: int, num_heads: int, max_blocks: int, partition_tokens: int = 0):
+        """Split scratch for ``decode``, grown on demand and reused by every
+        call: decodes that may overlap on the GPU (different streams) must
+        each pass a workspace of their own."""
         n = pa_decode_workspace_bytes(num_seqs, num_heads, self.num_kv_heads, self.head_size, max_blocks,
                                       partition_tokens)
         if n == 0:
