@@ -96,6 +96,33 @@ def step_bytes(plan):
     return {"kv": kv, "decode": decode, "write": write, "step": decode + write}
 
 
+def allocator_report(plan):
+    """Memory use of the workload's paged cache after its step: the
+    workload's requests (setup and step) replayed on a fresh host block
+    allocator of the library.  Blocks in use, the slots they leave unused
+    (only a sequence's last block can hold any), that waste as a fraction of
+    the slots in use, tokens held per sequence (shared prompt tokens counted
+    once per holder) and the copy-on-write copies the requests caused."""
+    import paged_kv_cache_351_b200 as pa
+    from workloads import AddOp, ForkOp
+
+    w = plan.workload
+    alloc = pa.Allocator(plan.num_blocks, w.block_size, plan.free_order)
+    cows = 0
+    for op in list(plan.setup_ops) + list(plan.step_ops):
+        if isinstance(op, AddOp):
+            alloc.add(op.seq)
+        elif isinstance(op, ForkOp):
+            alloc.fork(op.parent, op.child)
+        else:
+            cows += len(alloc.append(op.seq, op.n)[1])
+    st = alloc.stats()
+    used = st["num_blocks"] - st["num_free"]
+    return {"blocks_used": used, "waste_slots": st["waste_slots"],
+            "waste_frac": round(st["waste_slots"] / max(1, used * w.block_size), 5),
+            "tokens_held": st["num_tokens"], "cow_copies": cows}
+
+
 def is_prefill(plan):
     """A multi-token step (some sequence brings more than one new token)."""
     return bool((plan.query_lens != 1).any())
@@ -634,6 +661,7 @@ def run_ours(args):
         "frac_of_hbm_peak": round(value / world / peak, 4),
         "frac_of_8tbs_spec": round(value / world / 8000.0, 4),
         "bytes_per_step": nbytes,
+        "allocator": allocator_report(plan),
         "roofline": {"bound": "hbm", "kernel": "pa_decode (decode_kernel, log-sum-exp merge fused)",
                      "achieved": round(achieved, 2), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
@@ -787,6 +815,7 @@ def run_prefill(args, plan, device, world, rank):
                          "cache per kv head group; the kernel is tensor-bound"},
         "tokens_per_s": round(T * world / (ms_step * 1e-3), 1),
         "flops_per_step": flops, "write_bytes_per_step": write_bytes,
+        "allocator": allocator_report(plan),
         "roofline": {"bound": "tensor", "kernel": "pa_prefill (prefill_kernel, tcgen05)", "achieved": round(achieved, 2),
                      "peak": peak, "peak_kind": peak_kind + " bf16 dense (burst)", "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4),

@@ -104,3 +104,38 @@ def test_reference_arm_runs_on_rank_zero_only():
                          env=env)
     assert res.returncode == 0, res.stderr[-2000:]
     assert not [l for l in res.stdout.splitlines() if l.startswith("{")]
+
+
+@pytest.mark.parametrize("name", ["tiny_fp32", "llama7b_bs64", "parallel_sampling_13b", "prefill_mixed_gqa"])
+def test_allocator_report_matches_the_oracle_replay(name):
+    """The benchmark's memory report (blocks in use, unused slots, tokens
+    held, copy-on-write copies) equals the oracle block manager's on the same
+    requests; only last blocks waste (at most bs - 1 slots per sequence); in
+    the sampling workload every prompt whose length is not a multiple of the
+    block size costs 3 copies (4 samples write into its shared last block)."""
+    from oracle.allocator import BlockAllocator
+    from workloads import AddOp, ForkOp
+
+    plan = make_plan(name)
+    w = plan.workload
+    rep = bench.allocator_report(plan)
+    o = BlockAllocator(plan.num_blocks, w.block_size, plan.free_order)
+    cows, prompts = 0, {}
+    for op in list(plan.setup_ops) + list(plan.step_ops):
+        if isinstance(op, AddOp):
+            o.add(op.seq)
+        elif isinstance(op, ForkOp):
+            o.fork(op.parent, op.child)
+        else:
+            prompts.setdefault(op.seq, op.n)
+            cows += len(o.append(op.seq, op.n)[1])
+    used = plan.num_blocks - o.num_free()
+    held = sum(o.length(s) for s in o.sequences())
+    assert rep == {"blocks_used": used, "waste_slots": o.waste_slots(),
+                   "waste_frac": round(o.waste_slots() / (used * w.block_size), 5), "tokens_held": held,
+                   "cow_copies": cows}
+    assert rep["waste_slots"] <= (w.block_size - 1) * len(o.sequences())
+    if name == "parallel_sampling_13b":
+        roots = [n for s, n in prompts.items() if s < 64]  # sequences 0..63 are the prompts
+        assert len(roots) == 64
+        assert rep["cow_copies"] == 3 * sum(1 for n in roots if n % w.block_size)
