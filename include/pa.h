@@ -333,10 +333,19 @@ typedef struct {
   int32_t num_evictable; /* registered blocks nobody holds */
 } pa_alloc_stats;
 
+/* A new allocator over blocks 0 .. num_blocks-1 of block_size tokens (both
+ * > 0).  free_order: NULL, or a permutation of 0 .. num_blocks-1 (anything
+ * else is PA_ERR_INVALID_ARG).  *out is the caller's, released with
+ * pa_alloc_destroy (NULL is a no-op); on any error (out not NULL) *out is
+ * NULL. */
 pa_status pa_alloc_create(int32_t num_blocks, int32_t block_size, const int32_t* free_order, pa_allocator** out);
 void pa_alloc_destroy(pa_allocator* a);
+/* A new empty sequence; an id already present is PA_ERR_INVALID_ARG. */
 pa_status pa_seq_add(pa_allocator* a, int64_t seq_id);
-/* slots_out: [n_tokens]; cow_pair_out: [2], written (src, dst) when *n_cow_out == 1. */
+/* Appends n_tokens (>= 0) tokens with unknown ids.  slots_out: [n_tokens]
+ * (may be NULL when n_tokens == 0); cow_pair_out: [2] (nullable), written
+ * (src, dst) when *n_cow_out (nullable) is 1.  An unknown or swapped-out
+ * sequence, or a length past INT32_MAX, is PA_ERR_INVALID_ARG. */
 pa_status pa_seq_append(pa_allocator* a, int64_t seq_id, int32_t n_tokens, int64_t* slots_out,
                         int64_t* cow_pair_out, int32_t* n_cow_out);
 /* Appends n_tokens[k] tokens to seq_ids[k] for k = 0..n-1 in order.  Each
@@ -346,6 +355,8 @@ pa_status pa_seq_append(pa_allocator* a, int64_t seq_id, int32_t n_tokens, int64
  * *n_cow_out copy pairs in order. */
 pa_status pa_seq_append_batch(pa_allocator* a, const int64_t* seq_ids, const int32_t* n_tokens, int32_t n,
                               int64_t* slots_out, int64_t* cow_pairs_out, int32_t* n_cow_out, int32_t* n_done_out);
+/* child (a new id) starts as a copy of parent (present, not swapped out):
+ * same table and length, one more reference on each block. */
 pa_status pa_seq_fork(pa_allocator* a, int64_t parent, int64_t child);
 
 /* Prefix caching.  The pages give the effect — requests reuse the computed
@@ -397,15 +408,24 @@ pa_status pa_alloc_set_host_pool(pa_allocator* a, int32_t num_host_blocks, const
 pa_status pa_seq_swap_out(pa_allocator* a, int64_t seq_id, int64_t* pairs_out, int32_t cap, int32_t* n_out);
 pa_status pa_seq_swap_in(pa_allocator* a, int64_t seq_id, int64_t* pairs_out, int32_t cap, int32_t* n_out);
 int32_t pa_alloc_num_host_free(const pa_allocator* a);
+/* Host blocks of a swapped-out sequence, in table order (else
+ * PA_ERR_INVALID_ARG). */
 pa_status pa_seq_host_table(const pa_allocator* a, int64_t seq_id, int32_t* out, int32_t cap, int32_t* n_out);
+/* Releases the sequence's blocks (device, or host if swapped out) and
+ * forgets the id; an unknown id (e.g. a second free) is PA_ERR_INVALID_ARG. */
 pa_status pa_seq_free(pa_allocator* a, int64_t seq_id);
 pa_status pa_seq_len(const pa_allocator* a, int64_t seq_id, int32_t* len_out);
+/* The sequence's block table.  For a known sequence *n_out is set to the
+ * table's length; if that exceeds cap the call is PA_ERR_INVALID_ARG and out
+ * is not written (the same holds for the other out/cap/n_out calls, so a
+ * caller can size its buffer from *n_out and call again). */
 pa_status pa_seq_block_table(const pa_allocator* a, int64_t seq_id, int32_t* out, int32_t cap, int32_t* n_out);
 /* Fills out [n, max_blocks] (row-major) with the tables of seq_ids, padding
  * with -1, and context_lens_out [n] (nullable) with their lengths.  A table
  * longer than max_blocks is PA_ERR_INVALID_ARG (nothing written). */
 pa_status pa_alloc_block_tables(const pa_allocator* a, const int64_t* seq_ids, int32_t n, int32_t* out,
                                 int32_t max_blocks, int32_t* context_lens_out);
+/* Blocks available to allocation (free plus evictable); -1 for NULL. */
 int32_t pa_alloc_num_free(const pa_allocator* a);
 int32_t pa_block_refcount(const pa_allocator* a, int32_t block); /* -1 if out of range */
 pa_status pa_alloc_get_stats(const pa_allocator* a, pa_alloc_stats* out);

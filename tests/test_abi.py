@@ -575,3 +575,20 @@ def test_swap_matches_oracle_random(seed):
             else:
                 assert c.block_table(s) == o.block_table(s)
         assert c.evictable() == list(o._evictable)
+
+
+def test_table_calls_report_the_size_they_need():
+    """A table call given too little room fails with PA_ERR_INVALID_ARG,
+    writes nothing, and reports the length it needs in *n_out."""
+    import ctypes
+
+    lib = pa.library()
+    a = pa.Allocator(16, 4)
+    a.add(3)
+    a.append(3, 10)  # 3 blocks
+    n = ctypes.c_int32(-1)
+    out = (ctypes.c_int32 * 8)(*([-7] * 8))
+    st = lib.pa_seq_block_table(a._h, 3, out, 2, ctypes.byref(n))
+    assert st == 1 and n.value == 3 and list(out) == [-7] * 8
+    st = lib.pa_seq_block_table(a._h, 3, out, n.value, ctypes.byref(n))
+    assert st == 0 and list(out[:3]) == a.block_table(3) and out[3] == -7
