@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-seconds", type=float, default=120.0,
+                    help="--impl reference: oracle time spread over the warm-up and timed steps")
     ap.add_argument("--tuning", default="", help="warps,stages,ctas_per_sm for pa_set_decode_tuning")
     return ap.parse_args()
 
@@ -339,74 +341,124 @@ class ClockSampler:
 # CPU oracle timing
 # ---------------------------------------------------------------------------
 
-def oracle_timing(plan, seconds, max_rows=None):
-    """Time the oracle as it stands (fp64 NumPy, walking the block tables)
-    on whole rows of the same workload until ``seconds`` have passed."""
-    import numpy as np
-
-    from oracle.attention import paged_decode_rows
+def oracle_state(plan):
+    """The oracle's own copy of the workload, built once and outside every
+    timed sample: its allocator and cache replayed from the requests, the
+    block tables and the queries; plus where the next sample starts."""
     from oracle.replay import block_table_array, replay
     from workloads import query_values
 
     alloc, cache, _ = replay(plan)
-    tables = block_table_array(alloc, plan.batch, plan.max_blocks_per_seq)
+    return {"cache": cache, "tables": block_table_array(alloc, plan.batch, plan.max_blocks_per_seq),
+            "q": query_values(plan), "next": (0, 0)}
+
+
+def _threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        return max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
+    except Exception:
+        return 1
+
+
+def oracle_timing(plan, seconds, max_rows=None, state=None):
+    """Time the oracle as it stands (fp64 NumPy, walking the block tables)
+    on whole rows (one sequence, all heads) of the same workload until
+    ``seconds`` have passed (at least one row).  With a ``state`` from
+    ``oracle_state`` the rows continue where its previous sample stopped."""
+    from oracle.attention import paged_decode_rows
+
+    st = state if state is not None else oracle_state(plan)
     lens = plan.context_lens
-    q = query_values(plan)
     scale = 1.0 / math.sqrt(plan.workload.head_size)
     w = plan.workload
     per_tok = 2 * w.num_kv_heads * w.head_size * w.cache_elem_bytes
-    done_bytes, rows_done, i = 0, 0, 0
+    done_bytes, rows_done, i = 0, 0, st["next"][0]
     t0 = time.perf_counter()
     while True:
-        paged_decode_rows(q, cache, tables, lens, scale, [i])
+        paged_decode_rows(st["q"], st["cache"], st["tables"], lens, scale, [i])
         done_bytes += int(lens[i]) * per_tok + 2 * w.num_heads * w.head_size * w.elem_bytes
         rows_done += 1
         i = (i + 1) % plan.B
         el = time.perf_counter() - t0
         if el >= seconds or (max_rows is not None and rows_done >= max_rows):
             break
-    try:
-        from threadpoolctl import threadpool_info
-
-        cores = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
-    except Exception:
-        cores = 1
-    return {"gbs": done_bytes / el / 1e9, "seconds": el, "rows": rows_done, "cores": cores,
+    st["next"] = (i, 0)
+    return {"gbs": done_bytes / el / 1e9, "seconds": el, "rows": rows_done, "cores": _threads(),
             "tok_per_s": rows_done / el}
 
 
-def oracle_timing_prefill(plan, seconds):
-    """Time the multi-token oracle as it stands on whole sequences of the
-    workload (all their new tokens, all heads) until ``seconds`` have passed."""
-    from oracle.prefill import paged_prefill_seqs
-    from oracle.replay import block_table_array, replay
-    from workloads import query_values
+def _prefix_sum(m):
+    return m * (m + 1) // 2
 
-    alloc, cache, _ = replay(plan)
-    tables = block_table_array(alloc, plan.batch, plan.max_blocks_per_seq)
-    q = query_values(plan)
+
+def prefill_rows_flops(plan, i, j0, j1):
+    """Causal QK^T and PV FLOPs of new tokens j0 .. j1-1 of sequence i: the
+    token at position p attends p + 1 keys in every query head."""
     w = plan.workload
-    scale = 1.0 / math.sqrt(w.head_size)
-    order = sorted(range(plan.B), key=lambda i: int(plan.context_lens[i]))  # short sequences first
-    flops, seqs, k = 0, 0, 0
+    c = int(plan.context_lens[i]) - int(plan.query_lens[i])
+    return 4 * w.head_size * w.num_heads * (_prefix_sum(c + j1) - _prefix_sum(c + j0))
+
+
+def prefill_row_request(plan, state, i, j0, j1):
+    """New tokens j0 .. j1-1 of sequence i as a request of their own: the
+    same query rows over the context that ends at token j1 - 1 (causal
+    attention gives them the rows of the whole request, up to fp64
+    summation order).  Returns
+    the oracle's arguments (query, block tables, context lengths,
+    query_start) for that one-sequence request."""
+    import numpy as np
+
+    a = int(plan.query_start[i])
+    c = int(plan.context_lens[i]) - int(plan.query_lens[i])
+    q = state["q"][a + j0:a + j1]
+    return (q, state["tables"][i:i + 1], np.array([c + j1], np.int32), np.array([0, j1 - j0], np.int32))
+
+
+def oracle_timing_prefill(plan, seconds, rows_per_sample=None, state=None):
+    """Time the multi-token oracle as it stands until ``seconds`` have
+    passed (at least one sample): on whole sequences (all their new tokens,
+    all heads), short ones first; or, with ``rows_per_sample``, on runs of
+    that many consecutive new tokens of a sequence, each run computed as the
+    request that ends at its last token (``prefill_row_request``; a run
+    re-gathers its sequence's context, so runs cost more per FLOP than whole
+    sequences).  With a
+    ``state`` from ``oracle_state`` the samples continue where its previous
+    sample stopped."""
+    from oracle.prefill import paged_prefill_seqs
+
+    st = state if state is not None else oracle_state(plan)
+    scale = 1.0 / math.sqrt(plan.workload.head_size)
+    order = [i for i in sorted(range(plan.B), key=lambda i: int(plan.context_lens[i]))  # short sequences first
+             if int(plan.query_lens[i]) > 0]
+    flops, seqs, rows = 0, 0, 0
+    k, j0 = st["next"]
     t0 = time.perf_counter()
     while True:
-        i = order[k % plan.B]
-        paged_prefill_seqs(q, cache, tables, plan.context_lens, plan.query_start, scale, [i])
-        c, n = int(plan.context_lens[i]), int(plan.query_lens[i])
-        flops += 4 * w.head_size * w.num_heads * (n * (c - n) + n * (n + 1) // 2)
-        seqs += 1
-        k += 1
+        i = order[k % len(order)]
+        n = int(plan.query_lens[i])
+        if rows_per_sample is None:
+            paged_prefill_seqs(st["q"], st["cache"], st["tables"], plan.context_lens, plan.query_start, scale, [i])
+            flops += prefill_rows_flops(plan, i, 0, n)
+            rows += n
+            seqs += 1
+            k += 1
+        else:
+            j1 = min(n, j0 + rows_per_sample)
+            q, tables, cl, qs = prefill_row_request(plan, st, i, j0, j1)
+            paged_prefill_seqs(q, st["cache"], tables, cl, qs, scale, [0])
+            flops += prefill_rows_flops(plan, i, j0, j1)
+            rows += j1 - j0
+            j0 = j1
+            if j0 >= n:
+                k, j0 = k + 1, 0
+                seqs += 1
         el = time.perf_counter() - t0
         if el >= seconds:
             break
-    try:
-        from threadpoolctl import threadpool_info
-
-        cores = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
-    except Exception:
-        cores = 1
-    return {"tflops": flops / el / 1e12, "seconds": el, "seqs": seqs, "cores": cores}
+    st["next"] = (k, j0)
+    return {"tflops": flops / el / 1e12, "seconds": el, "seqs": seqs, "rows": rows, "cores": _threads()}
 
 
 def run_reference(args):
@@ -414,9 +466,13 @@ def run_reference(args):
     if rank != 0:
         return
     plan = workload_plan(args.workload)
+    state = oracle_state(plan)  # untimed: the oracle's copy of the workload
+    # each step is a bounded sample, so that K steps take about ref_seconds
+    per = min(5.0, args.ref_seconds / max(1, args.steps + args.warmup))
     if is_prefill(plan):
-        per = max(1.0, min(10.0, 120.0 / max(1, args.steps + args.warmup)))
-        res = [oracle_timing_prefill(plan, per) for _ in range(max(1, args.steps))]
+        for _ in range(args.warmup):
+            oracle_timing_prefill(plan, per / 4, rows_per_sample=64, state=state)
+        res = [oracle_timing_prefill(plan, per, rows_per_sample=64, state=state) for _ in range(max(1, args.steps))]
         tf = statistics.median(r["tflops"] for r in res)
         tot_s = sum(r["seconds"] for r in res)
         line = {
@@ -424,17 +480,18 @@ def run_reference(args):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(1000 * tot_s / max(1, args.steps), 3), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
-            "config": {"workload": f"{plan.workload.name}: {plan.workload.description}", "sample": "whole sequences"},
+            "config": {"workload": f"{plan.workload.name}: {plan.workload.description}",
+                       "sample": "runs of 64 consecutive new tokens (all heads) of the step's sequences"},
             "cpu_baseline": {"value": round(tf, 6), "unit": "TFLOP/s", "cores": res[0]["cores"], "kind": "oracle",
-                             "sample": f"{sum(r['seqs'] for r in res)} whole sequences, about {per:.1f} s per step"},
+                             "sample": f"{sum(r['rows'] for r in res)} new tokens (all heads) in runs of 64, "
+                                       f"about {per:.3f} s per step"},
             "e2e": {"value": round(tf, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         }
         print(json.dumps(line), flush=True)
         return
-    per = max(0.5, min(5.0, 120.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
-        oracle_timing(plan, per / 4, max_rows=1)
-    res = [oracle_timing(plan, per) for _ in range(max(1, args.steps))]
+        oracle_timing(plan, per / 4, max_rows=1, state=state)
+    res = [oracle_timing(plan, per, state=state) for _ in range(max(1, args.steps))]
     gbs = statistics.median(r["gbs"] for r in res)
     tot_rows = sum(r["rows"] for r in res)
     tot_s = sum(r["seconds"] for r in res)
@@ -445,7 +502,7 @@ def run_reference(args):
         "data": "synthetic (seeded lognormal lengths standing in for ShareGPT)",
         "config": {"workload": f"{plan.workload.name}: {plan.workload.description}", "sample": "whole rows"},
         "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": res[0]["cores"], "kind": "oracle",
-                         "sample": f"{tot_rows} sequences (all heads) of the workload, about {per:.1f} s per step"},
+                         "sample": f"{tot_rows} sequences (all heads) of the workload, about {per:.3f} s per step"},
         "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "tok_per_s": round(tot_rows / tot_s, 3),
     }

@@ -139,3 +139,51 @@ def test_allocator_report_matches_the_oracle_replay(name):
         roots = [n for s, n in prompts.items() if s < 64]  # sequences 0..63 are the prompts
         assert len(roots) == 64
         assert rep["cow_copies"] == 3 * sum(1 for n in roots if n % w.block_size)
+
+
+def test_prefill_row_requests_reproduce_the_whole_request():
+    """The reference arm times the prefill oracle on runs of consecutive new
+    tokens, each asked as the request that ends at the run's last token.
+    Causal attention makes those rows equal to the whole request's (up to
+    fp64 summation order), and the runs' FLOPs add up to the step's."""
+    import numpy as np
+
+    from oracle.prefill import paged_prefill_seqs
+
+    plan = make_plan("prefill_tiny")
+    st = bench.oracle_state(plan)
+    scale = 1.0 / np.sqrt(plan.workload.head_size)
+    whole = paged_prefill_seqs(st["q"], st["cache"], st["tables"], plan.context_lens, plan.query_start, scale,
+                               range(plan.B))
+    total = 0
+    for i in range(plan.B):
+        n = int(plan.query_lens[i])
+        for j0 in range(0, n, 5):
+            j1 = min(n, j0 + 5)
+            q, tables, cl, qs = bench.prefill_row_request(plan, st, i, j0, j1)
+            part = paged_prefill_seqs(q, st["cache"], tables, cl, qs, scale, [0])[0]
+            # the same rows; only fp64 summation order differs (shorter masked key range)
+            assert np.max(np.abs(part - whole[i][j0:j1]), initial=0.0) <= 1e-12, (i, j0)
+            total += bench.prefill_rows_flops(plan, i, j0, j1)
+    assert total == bench.prefill_flops(plan)
+
+
+@pytest.mark.parametrize("name", ["tiny_fp32", "prefill_tiny"])
+def test_reference_arm_bounds_each_step(name):
+    """Many steps stay within the oracle time budget: the oracle's copy of
+    the workload is built once and each step is a bounded sample."""
+    import json
+    import os
+    import subprocess
+    import sys
+    import time
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    t0 = time.time()
+    res = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--workload", name,
+                          "--steps", "2000", "--warmup", "20", "--ref-seconds", "3"], capture_output=True, text=True,
+                         timeout=300, cwd=root)
+    assert res.returncode == 0, res.stderr[-2000:]
+    assert time.time() - t0 < 120
+    d = json.loads([l for l in res.stdout.splitlines() if l.startswith("{")][0])
+    assert d["steps"] == 2000 and d["value"] > 0
