@@ -120,14 +120,13 @@ def test_allocator_report_matches_the_oracle_replay(name):
     w = plan.workload
     rep = bench.allocator_report(plan)
     o = BlockAllocator(plan.num_blocks, w.block_size, plan.free_order)
-    cows, prompts = 0, {}
+    cows = 0
     for op in list(plan.setup_ops) + list(plan.step_ops):
         if isinstance(op, AddOp):
             o.add(op.seq)
         elif isinstance(op, ForkOp):
             o.fork(op.parent, op.child)
         else:
-            prompts.setdefault(op.seq, op.n)
             cows += len(o.append(op.seq, op.n)[1])
     used = plan.num_blocks - o.num_free()
     held = sum(o.length(s) for s in o.sequences())
@@ -136,9 +135,10 @@ def test_allocator_report_matches_the_oracle_replay(name):
                    "cow_copies": cows}
     assert rep["waste_slots"] <= (w.block_size - 1) * len(o.sequences())
     if name == "parallel_sampling_13b":
-        roots = [n for s, n in prompts.items() if s < 64]  # sequences 0..63 are the prompts
-        assert len(roots) == 64
-        assert rep["cow_copies"] == 3 * sum(1 for n in roots if n % w.block_size)
+        from workloads.synth import parallel_sampling_lengths
+
+        plen, _ = parallel_sampling_lengths(w)
+        assert rep["cow_copies"] == 3 * sum(1 for n in plen.tolist() if n % w.block_size)
 
 
 def test_prefill_row_requests_reproduce_the_whole_request():
