@@ -104,7 +104,9 @@ def allocator_report(plan):
     allocator of the library.  Blocks in use, the slots they leave unused
     (only a sequence's last block can hold any), that waste as a fraction of
     the slots in use, tokens held per sequence (shared prompt tokens counted
-    once per holder) and the copy-on-write copies the requests caused."""
+    once per holder) and the copy-on-write copies the requests caused.  For
+    comparison, the fraction of slots a contiguous layout would leave unused
+    if every sequence reserved the batch's longest context (no sharing)."""
     import paged_kv_cache_351_b200 as pa
     from workloads import AddOp, ForkOp
 
@@ -120,9 +122,11 @@ def allocator_report(plan):
             cows += len(alloc.append(op.seq, op.n)[1])
     st = alloc.stats()
     used = st["num_blocks"] - st["num_free"]
+    reserved = st["num_seqs"] * max([int(c) for c in plan.context_lens] + [1])
     return {"blocks_used": used, "waste_slots": st["waste_slots"],
             "waste_frac": round(st["waste_slots"] / max(1, used * w.block_size), 5),
-            "tokens_held": st["num_tokens"], "cow_copies": cows}
+            "tokens_held": st["num_tokens"], "cow_copies": cows,
+            "waste_frac_if_contiguous": round(1.0 - st["num_tokens"] / reserved, 5)}
 
 
 def is_prefill(plan):

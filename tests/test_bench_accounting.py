@@ -130,9 +130,11 @@ def test_allocator_report_matches_the_oracle_replay(name):
             cows += len(o.append(op.seq, op.n)[1])
     used = plan.num_blocks - o.num_free()
     held = sum(o.length(s) for s in o.sequences())
+    longest = max(int(c) for c in plan.context_lens)
     assert rep == {"blocks_used": used, "waste_slots": o.waste_slots(),
                    "waste_frac": round(o.waste_slots() / (used * w.block_size), 5), "tokens_held": held,
-                   "cow_copies": cows}
+                   "cow_copies": cows,
+                   "waste_frac_if_contiguous": round(1.0 - held / (len(o.sequences()) * longest), 5)}
     assert rep["waste_slots"] <= (w.block_size - 1) * len(o.sequences())
     if name == "parallel_sampling_13b":
         from workloads.synth import parallel_sampling_lengths
