@@ -28,7 +28,8 @@ op = st.one_of(
 
 def _same_state(c, o, live):
     assert c.num_free() == o.num_free()
-    for b in range(NB):
+    assert c.evictable() == list(o._evictable)
+    for b in range(o.num_blocks):
         assert c.refcount(b) == o.refcount(b), b
     for s in live:
         if not o.is_swapped(s):
@@ -101,3 +102,51 @@ def test_allocator_fuzz_matches_oracle(order, horder, ops):
         _same_state(c, o, live)
         o.check_invariants()
     assert c.num_host_free() == o.num_host_free()
+
+
+# Long prompts over a small alphabet: deep registered chains that branch
+# wherever two prompts diverge, so evictions unregister whole subtrees.
+deep_op = st.one_of(
+    st.tuples(st.just("prefix"), st.lists(st.integers(0, 1), min_size=1, max_size=90)),
+    st.tuples(st.just("append"), st.integers(0, 7), st.integers(1, 9)),
+    st.tuples(st.just("fork"), st.integers(0, 7)),
+    st.tuples(st.just("free"), st.integers(0, 7)),
+)
+
+
+@settings(max_examples=300, deadline=None, derandomize=True, suppress_health_check=[HealthCheck.too_slow])
+@given(order=st.permutations(list(range(48))), ops=st.lists(deep_op, min_size=1, max_size=40))
+def test_allocator_fuzz_deep_prefix_trees(order, ops):
+    nb, bs = 48, 2
+    c, o = pa.Allocator(nb, bs, order), BlockAllocator(nb, bs, order)
+    live, nxt = [], 0
+    for item in ops:
+        kind = item[0]
+        if kind == "prefix":
+            toks = item[1]
+            assert c.add_prefix(nxt, toks) == o.add_prefix(nxt, toks)
+            hit = o.length(nxt)
+            live.append(nxt)
+            res = _both(lambda: o.append_tokens(nxt, toks[hit:]), lambda: c.append_tokens(nxt, toks[hit:]))
+            if res:
+                assert res[1][0].tolist() == res[0][0] and res[1][1] == res[0][1]
+            nxt += 1
+        elif kind == "append" and live:
+            s = live[item[1] % len(live)]
+            toks = [(s + k) % 2 for k in range(item[2])]
+            res = _both(lambda: o.append_tokens(s, toks), lambda: c.append_tokens(s, toks))
+            if res:
+                assert res[1][0].tolist() == res[0][0] and res[1][1] == res[0][1]
+        elif kind == "fork" and live:
+            p = live[item[1] % len(live)]
+            o.fork(p, nxt)
+            c.fork(p, nxt)
+            live.append(nxt)
+            nxt += 1
+        elif kind == "free" and live:
+            s = live.pop(item[1] % len(live))
+            o.free(s)
+            c.free(s)
+        _same_state(c, o, live)
+        assert c.stats()["num_cached"] == o.num_cached()
+        o.check_invariants()
