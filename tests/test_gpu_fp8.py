@@ -100,7 +100,7 @@ class Fp8Case:
     def run(self, mode):
         out = torch.empty_like(self.qd)
         n = pa.pa_decode_workspace_bytes(len(self.ctxs), self.H, self.hk, D, self.max_nb, mode)
-        ws = torch.empty(n + 256, dtype=torch.uint8, device=DEV) if n else None
+        ws = torch.zeros(n + 256, dtype=torch.uint8, device=DEV) if n else None
         pa.pa_decode_fp8(out, self.qd, self.kc, self.vc, self.bt, self.cl, self.scale, self.hk, self.kst, self.vst,
                          workspace=ws, partition_tokens=mode)
         torch.cuda.synchronize()
@@ -124,22 +124,44 @@ def test_fp8_decode_parity(H, hk, mode):
     assert c.err(out) <= 1e-2
 
 
+def bf16_ulp(x: np.ndarray) -> np.ndarray:
+    """Spacing of bf16 values (8 significant bits) at |x| (normal range)."""
+    e = np.floor(np.log2(np.maximum(np.abs(x), 2.0 ** -126)))
+    return 2.0 ** (e - 7)
+
+
 @pytest.mark.parametrize("H,hk", [(8, 8), (16, 4), (16, 2)])
 @pytest.mark.parametrize("q_mult", [1e-3, 3e3])
 def test_fp8_decode_extreme_query_magnitudes(H, hk, q_mult):
     """The tensor-core page math carries the query as f16 high and low parts
     after scaling each head by a power of two; queries far larger (near
     one-hot softmax) or far smaller (near uniform) than N(0, 1) must still
-    match the oracle.  In the one-hot regime an output is a single V value
-    (up to ~4 here), so the bound adds one bf16 rounding step of |ref|
-    (2^-8 relative) to the 1e-2 used elsewhere."""
+    match the oracle at the plain bf16 bar: max-abs <= 1e-2 wherever
+    |ref| < 4.  At |ref| >= 4 half a bf16 step is already 0.0156, so no
+    bf16 output can promise 1e-2 there: those elements must be the correctly
+    rounded bf16 value of the exact result, or its neighbour on the other
+    side when the exact result lies within the fp32 computation's error
+    (2^-12 relative) of a rounding midpoint; their error is printed in bf16
+    steps."""
     c = Fp8Case(80 + H + hk, [1, 17, 100, 513, 2049], H, hk, q_mult=q_mult)
     ref = paged_decode(c.q, c.cache, c.tables, c.ctxs, c.scale)
+    small = np.abs(ref) < 4.0
+    ulp = bf16_ulp(ref)
     for mode in (0, -1):
         out = c.run(mode)
         got = widen(to_host_raw(out, "bf16"), "bf16")
         assert not np.isnan(got).any()
-        assert np.all(np.abs(got - ref) <= 1e-2 + 2.0 ** -8 * np.abs(ref))
+        err = np.abs(got - ref)
+        err_small = float(err[small].max()) if small.any() else 0.0
+        ulps = err[~small] / ulp[~small]
+        # distance from ref to the nearest rounding midpoint, in bf16 steps
+        frac = np.abs(ref[~small]) / ulp[~small]
+        mid_dist = np.abs(frac - np.floor(frac) - 0.5)
+        near_mid = mid_dist * ulp[~small] <= 2.0 ** -12 * np.abs(ref[~small])
+        print(f"H={H} hk={hk} q_mult={q_mult} mode={mode}: max abs err {err_small:.3e} where |ref| < 4; "
+              f"{int((~small).sum())} elements >= 4, max {float(ulps.max()) if ulps.size else 0.0:.3f} bf16 steps")
+        assert err_small <= 1e-2, err_small
+        assert np.all((ulps <= 0.5) | (near_mid & (ulps < 1.0))), ulps.max()
     check_status_clean()
 
 
