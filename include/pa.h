@@ -73,11 +73,19 @@ typedef struct {
   int64_t stride[5];
 } pa_tensor;
 
+/* Decode workspace header: the first PA_DECODE_WS_HEADER_BYTES of every
+ * workspace hold the balanced split's merge counters (one 32-bit counter per
+ * worker, at most PA_DECODE_WS_HEADER_BYTES / 4 workers).  They must be zero
+ * before a workspace is first used; every call leaves them zero again, in
+ * every split mode, including a call that times out, so a workspace
+ * zero-filled once (cudaMemset, torch.zeros) serves any sequence of calls. */
+#define PA_DECODE_WS_HEADER_BYTES (64u * 1024u)
+
 typedef struct {
   void* stream;             /* cudaStream_t, NULL = legacy default stream */
-  void* workspace;          /* device scratch for split decode, 256-byte aligned, may be NULL; its
-                               contents need no initialisation (each call tags what it writes), but
-                               calls whose kernels may overlap on the GPU must not share it */
+  void* workspace;          /* device scratch for split decode, 256-byte aligned, may be NULL; zero-filled
+                               once before its first use (see PA_DECODE_WS_HEADER_BYTES); calls whose
+                               kernels may overlap on the GPU must not share it */
   size_t workspace_bytes;   /* size of workspace */
   int32_t partition_tokens; /* pa_decode context split:
                                  0  = auto: balanced split over all SMs when the
@@ -89,12 +97,18 @@ typedef struct {
                                       reduced by one warp, no workspace needed */
   int32_t timeout_ms;       /* bound on every device-side wait; 0 = 1000 ms */
 } pa_opts;
+/* pa_opts departs from the survey's sketch of this struct in two fields:
+ * there is no force_split (a caller forces a split by choosing
+ * partition_tokens > 0, and the auto mode already splits whenever the
+ * workspace allows), and timeout_ms is added, because every device-side wait
+ * of this library is bounded and a caller may want a bound other than 1 s. */
 
 /* Device status bits (pa_get_device_status). */
 #define PA_DEV_TIMEOUT 0x1u     /* a bounded wait gave up */
 #define PA_DEV_BAD_BLOCK 0x2u   /* block-table entry or copy pair outside [0, num_blocks) */
 #define PA_DEV_BAD_CONTEXT 0x4u /* context_len < 0 or > block-table row capacity; pa_prefill: a query range that does not fit */
 #define PA_DEV_BAD_SLOT 0x8u    /* slot_mapping entry < -1 or >= num_blocks*block_size */
+#define PA_DEV_BAD_WORKSPACE 0x10u /* pa_decode: a merge counter of the workspace did not start at zero */
 
 /* ---------------------------------------------------------------------------
  * Cache write (the step that stores each new token's K/V at its slot).
@@ -175,10 +189,15 @@ pa_status pa_swap_blocks(const pa_tensor* src_k, const pa_tensor* src_v, pa_tens
  * Accumulation is fp32; the output is rounded to the cache dtype (bf16:
  * round-to-nearest-even).  Split modes (opts->partition_tokens) change only
  * fp32 rounding order.  Fixed-partition mode leaves its per-partition
- * results in the workspace: float o[B][H][P][head_size] (normalised) followed
- * by float lse[B][H][P] (natural log of the partition's softmax denominator
- * plus its max logit), P = ceil(max_blocks_per_seq*bs / partition_tokens);
- * entries of partitions past a sequence's end are left unwritten.
+ * results in the workspace after the header: at byte offset
+ * PA_DECODE_WS_HEADER_BYTES, float o[B][H][P][head_size] (normalised), then,
+ * at the next multiple of 256 bytes, float lse[B][H][P] (natural log of the
+ * partition's softmax denominator plus its max logit),
+ * P = ceil(max_blocks_per_seq*bs / partition_tokens); entries of partitions
+ * past a sequence's end are left unwritten.  The balanced split (auto mode)
+ * merges the shares of a row cut between workers inside the same launch:
+ * the worker whose pages complete the row merges it, so no worker waits for
+ * another and no assumption is made about which CTAs run at the same time.
  * B may be 0.  B must be < 2^20.
  * ------------------------------------------------------------------------- */
 pa_status pa_decode(pa_tensor* out, const pa_tensor* query, const pa_tensor* k_cache, const pa_tensor* v_cache,
@@ -212,15 +231,63 @@ pa_status pa_set_decode_tuning(int32_t warps_per_cta, int32_t stages, int32_t ct
  *  - A call whose split needs more scratch than PA_NO_ALLOC_SCRATCH_BYTES
  *    returns PA_ERR_SCRATCH_LIMIT before launching anything (use
  *    partition_tokens -1, no split, which needs none).
- *  - All calls share the array and it keeps the last call's contents.  No
- *    byte of it has to start at zero: every byte a call reads was written
- *    earlier in that same call.  Calls whose kernels overlap on the GPU (two
+ *  - In the auto mode (partition_tokens 0) a split that needs more than the
+ *    array holds (e.g. after pa_set_decode_tuning raised the worker count)
+ *    runs unsplit, as pa_decode does when its workspace is too small.
+ *  - All calls share the array and it keeps the last call's contents.  Its
+ *    header of merge counters is zero when the library is loaded and every
+ *    call leaves it zero; every other byte a call reads was written earlier
+ *    in that same call.  Calls whose kernels overlap on the GPU (two
  *    streams, or two host threads) race on it: issue them on one stream.
  * ------------------------------------------------------------------------- */
 #define PA_NO_ALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
 pa_status pa_decode_no_alloc(pa_tensor* out, const pa_tensor* query, const pa_tensor* k_cache,
                              const pa_tensor* v_cache, const pa_tensor* block_tables,
                              const pa_tensor* context_lens, float scale, int32_t num_kv_heads, const pa_opts* opts);
+
+/* ---------------------------------------------------------------------------
+ * Shared-prefix decode.  The pages state that reference counts and
+ * copy-on-write let parallel samples of one prompt share the prompt's memory
+ * and its computation (CSDN discovery note, item 2, on the vLLM launch
+ * blog's "PagedAttention" section).  pa_decode shares the memory only: each
+ * sample still reads every prompt block.  This call also shares the reads:
+ * the batch is cut into groups of consecutive sequences whose block tables
+ * begin with the same group_blocks[v] blocks; each shared page is read once
+ * for all of a group's members and query heads, each member then runs over
+ * the rest of its own context, and the two partial results are merged by
+ * log-sum-exp.  The output is pa_decode's (the same formula; only fp32
+ * rounding order differs).
+ *
+ * group_start:  [n_groups + 1] int32 on the device: group v holds sequences
+ *               group_start[v] .. group_start[v+1] - 1; group_start[0] = 0,
+ *               non-decreasing, group_start[n_groups] = B (else
+ *               PA_DEV_BAD_CONTEXT and every sequence is decoded in full).
+ * group_blocks: [n_groups] int32 on the device: leading blocks every member
+ *               of the group holds (the same block ids at the same table
+ *               indices; not checked).  Values above a member's number of
+ *               full blocks are capped (PA_DEV_BAD_CONTEXT).  0 = no
+ *               sharing.  pa_alloc_prefix_groups computes both from the
+ *               allocator.
+ * max_group_size: most members a group may have; (num_heads / num_kv_heads)
+ *               * max_group_size must be 1, 2, 4 or 8 (else
+ *               PA_ERR_UNSUPPORTED).  Larger groups are decoded in full
+ *               (PA_DEV_BAD_CONTEXT).
+ * Other arguments as pa_decode; bf16 with head_size 128 or fp32 with
+ * head_size 64.  A workspace of pa_decode_cascade_workspace_bytes is
+ * required (zero-filled before first use, as for pa_decode): it also holds
+ * the prefix's partial results, fp32 [B][H][head_size] + [B][H].
+ * opts->partition_tokens: 0 (balanced split in both passes) or -1 (none);
+ * fixed partitions are PA_ERR_UNSUPPORTED.  Two kernel launches.
+ * ------------------------------------------------------------------------- */
+pa_status pa_decode_cascade(pa_tensor* out, const pa_tensor* query, const pa_tensor* k_cache,
+                            const pa_tensor* v_cache, const pa_tensor* block_tables, const pa_tensor* context_lens,
+                            const pa_tensor* group_start, const pa_tensor* group_blocks, int32_t max_group_size,
+                            float scale, int32_t num_kv_heads, const pa_opts* opts);
+/* Workspace bytes of pa_decode_cascade for these sizes on the current
+ * device (partition_tokens 0 or -1). */
+pa_status pa_decode_cascade_workspace_bytes(int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
+                                            int32_t head_size, int32_t max_group_size, int32_t partition_tokens,
+                                            size_t* bytes_out);
 
 /* ---------------------------------------------------------------------------
  * FP8 (e4m3) KV cache.  The pages say only that the KV cache itself can be
@@ -289,8 +356,17 @@ pa_status pa_prefill(pa_tensor* out, const pa_tensor* query, const pa_tensor* k_
                      int32_t max_query_len, float scale, int32_t num_kv_heads, const pa_opts* opts);
 
 /* Workspace bytes pa_decode needs on the current device for these sizes and
- * this partition_tokens setting (0 = auto/balanced, >0 = fixed, -1 = none).
- * Needs a CUDA device for the auto mode (it depends on the SM count). */
+ * this partition_tokens setting (0 = auto/balanced, >0 = fixed, -1 = none),
+ * header included; 0 for -1.  Departs from the survey's sketch
+ * (num_seqs, num_heads, head_size, max_context_len, partition_tokens) ->
+ * size_t: it takes num_kv_heads, because the balanced split's shares hold
+ * one row per query head of a kv-head group, and max_blocks_per_seq (the
+ * block-table width the decode call will get) instead of a token count, and
+ * it returns a status with the size in *bytes_out, so that bad arguments and
+ * a missing device are reported rather than folded into a size.  The auto
+ * mode's size depends on the current device's SM count and on
+ * pa_set_decode_tuning: it is per device, so size a workspace on the device
+ * that will run the decode. */
 pa_status pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
                                     int32_t head_size, int32_t max_blocks_per_seq, int32_t partition_tokens,
                                     size_t* bytes_out);
@@ -425,6 +501,22 @@ pa_status pa_seq_block_table(const pa_allocator* a, int64_t seq_id, int32_t* out
  * longer than max_blocks is PA_ERR_INVALID_ARG (nothing written). */
 pa_status pa_alloc_block_tables(const pa_allocator* a, const int64_t* seq_ids, int32_t n, int32_t* out,
                                 int32_t max_blocks, int32_t* context_lens_out);
+/* Groups for pa_decode_cascade: cuts the batch seq_ids[0..n) (in that
+ * order) into runs of consecutive sequences that share their leading blocks
+ * (forks of one prompt, placed next to each other).  Greedy: a run starts at
+ * a sequence with its full blocks as the shared count; the next sequence
+ * joins while the run has fewer than max_group_size members, the two tables
+ * begin with at least one common full block, and joining keeps at least half
+ * of the run's shared count (which becomes the common count).  A run of one
+ * sequence gets 0 shared blocks.  Writes group_start_out [n_groups + 1]
+ * (first member of each run, then n), group_blocks_out [n_groups] (shared
+ * full blocks, each a block every member's table holds at the same index)
+ * and *n_groups_out (<= n).  An unknown or swapped-out id is
+ * PA_ERR_INVALID_ARG.  The grouping affects only speed: any grouping whose
+ * members really share their first group_blocks blocks decodes to the same
+ * result. */
+pa_status pa_alloc_prefix_groups(const pa_allocator* a, const int64_t* seq_ids, int32_t n, int32_t max_group_size,
+                                 int32_t* group_start_out, int32_t* group_blocks_out, int32_t* n_groups_out);
 /* Blocks available to allocation (free plus evictable); -1 for NULL. */
 int32_t pa_alloc_num_free(const pa_allocator* a);
 int32_t pa_block_refcount(const pa_allocator* a, int32_t block); /* -1 if out of range */
@@ -435,8 +527,9 @@ pa_status pa_alloc_get_stats(const pa_allocator* a, pa_alloc_stats* out);
  * ------------------------------------------------------------------------- */
 /* Synchronises opts->stream, then reads and clears the current device's
  * status word into *bits_out (nullable).  Returns PA_ERR_DEVICE_TIMEOUT if the
- * timeout bit was set, else PA_ERR_DEVICE_BOUNDS if any bounds bit was set,
- * else PA_OK. */
+ * timeout bit was set, else PA_ERR_DEVICE_BOUNDS if any other bit was set,
+ * else PA_OK.  Departs from the survey's sketch (opts only) by the bits_out
+ * out-parameter, so a caller can tell which check fired. */
 pa_status pa_get_device_status(const pa_opts* opts, uint32_t* bits_out);
 
 /* Launches one warp that waits, with the same bounded wait the decode

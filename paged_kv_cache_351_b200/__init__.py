@@ -18,12 +18,14 @@ from typing import Optional, Sequence, Tuple
 import numpy as np
 
 from . import _lib
-from ._lib import (PA_DEV_BAD_BLOCK, PA_DEV_BAD_CONTEXT, PA_DEV_BAD_SLOT,  # noqa: F401
-                   PA_DEV_TIMEOUT, PaAllocStats, PaOpts, PaTensor)
+from ._lib import (PA_DECODE_WS_HEADER_BYTES, PA_DEV_BAD_BLOCK, PA_DEV_BAD_CONTEXT,  # noqa: F401
+                   PA_DEV_BAD_SLOT, PA_DEV_BAD_WORKSPACE, PA_DEV_TIMEOUT, PaAllocStats, PaOpts, PaTensor)
 
 __all__ = [
     "PagedAttentionError", "OutOfBlocksError", "pa_reshape_and_cache", "pa_copy_blocks", "pa_decode",
     "pa_decode_workspace_bytes", "pa_decode_no_alloc", "pa_reshape_and_cache_fp8", "pa_decode_fp8", "pa_prefill",
+    "pa_decode_cascade", "pa_decode_cascade_workspace_bytes", "PreparedCall", "prepare_reshape_and_cache",
+    "prepare_decode", "prepare_decode_cascade", "prepare_reshape_and_cache_fp8", "prepare_decode_fp8",
     "pa_swap_blocks", "pa_set_decode_tuning", "pa_get_device_status", "pa_debug_wait_selftest",
     "Allocator", "library",
 ]
@@ -169,6 +171,31 @@ def pa_decode(out, query, k_cache, v_cache, block_tables, context_lens, scale: f
                                      ctypes.byref(o)), "pa_decode")
 
 
+def pa_decode_cascade(out, query, k_cache, v_cache, block_tables, context_lens, group_start, group_blocks,
+                      max_group_size: int, scale: float, num_kv_heads: int, workspace, partition_tokens: int = 0,
+                      stream=None, timeout_ms: int = 0) -> None:
+    """Shared-prefix decode: pa_decode's result, with each group's shared
+    leading blocks (int32 device tensors ``group_start`` [n_groups + 1] and
+    ``group_blocks`` [n_groups], e.g. from ``Allocator.prefix_groups``) read
+    once for all of the group's members.  ``workspace``: at least
+    ``pa_decode_cascade_workspace_bytes`` bytes, zero-filled before first use."""
+    args = (out, query, k_cache, v_cache, block_tables, context_lens, group_start, group_blocks)
+    ts = [_tensor(x) for x in args]
+    with _on_device(args + (workspace,)):
+        o = _opts(stream, workspace, partition_tokens, timeout_ms)
+        _check(_lib_handle.pa_decode_cascade(*[ctypes.byref(t) for t in ts], int(max_group_size), ctypes.c_float(scale),
+                                             int(num_kv_heads), ctypes.byref(o)), "pa_decode_cascade")
+
+
+def pa_decode_cascade_workspace_bytes(num_seqs: int, num_heads: int, num_kv_heads: int, head_size: int,
+                                      max_group_size: int, partition_tokens: int = 0) -> int:
+    n = ctypes.c_size_t(0)
+    _check(_lib_handle.pa_decode_cascade_workspace_bytes(num_seqs, num_heads, num_kv_heads, head_size, max_group_size,
+                                                         partition_tokens, ctypes.byref(n)),
+           "pa_decode_cascade_workspace_bytes")
+    return int(n.value)
+
+
 def pa_prefill(out, query, k_cache, v_cache, block_tables, context_lens, query_start, max_query_len: int,
                scale: float, num_kv_heads: int, stream=None, timeout_ms: int = 0) -> None:
     """Multi-token (chunked-prefill) paged attention: writes out [T, H, D]
@@ -237,6 +264,9 @@ def pa_decode_no_alloc(out, query, k_cache, v_cache, block_tables, context_lens,
 
 def pa_decode_workspace_bytes(num_seqs: int, num_heads: int, num_kv_heads: int, head_size: int,
                               max_blocks_per_seq: int, partition_tokens: int = 0) -> int:
+    """Bytes of decode workspace for these sizes on the current device (0
+    for no split).  A workspace must be zero-filled before its first use
+    (its header holds merge counters that every call leaves at zero)."""
     n = ctypes.c_size_t(0)
     _check(_lib_handle.pa_decode_workspace_bytes(num_seqs, num_heads, num_kv_heads, head_size, max_blocks_per_seq,
                                                  partition_tokens, ctypes.byref(n)), "pa_decode_workspace_bytes")
@@ -258,6 +288,82 @@ def pa_get_device_status(stream=None) -> Tuple[int, int]:
 def pa_debug_wait_selftest(timeout_ms: int, stream=None) -> None:
     o = _opts(stream, timeout_ms=timeout_ms)
     _check(_lib_handle.pa_debug_wait_selftest(ctypes.byref(o)), "pa_debug_wait_selftest")
+
+
+# ---------------------------------------------------------------------------
+# prepared calls: descriptors built once, for serving loops
+# ---------------------------------------------------------------------------
+
+class PreparedCall:
+    """One library call whose descriptors (pa_tensor, pa_opts and scalars)
+    are built once.  Calling it issues the same C call again, on ``stream``
+    if given (else the stream it was prepared with), with no other Python
+    work per call: for a serving loop that reuses the same buffers every
+    step.  The tensors must stay alive and keep their storage, shapes and
+    strides; their contents may change between calls.  Call it with the
+    tensors' device current (as the preparing call had)."""
+
+    def __init__(self, name: str, tensors, scalars, opts: PaOpts, keep):
+        self._name = name
+        self._fn = getattr(_lib_handle, name)
+        self._structs = [_tensor(t) for t in tensors]
+        self._opts = opts
+        self._args = [ctypes.byref(t) for t in self._structs] + list(scalars) + [ctypes.byref(opts)]
+        self._keep = keep  # the tensors, so their storage outlives this object
+
+    def __call__(self, stream=None) -> None:
+        if stream is not None:
+            self._opts.stream = _stream_ptr(stream)
+        _check(self._fn(*self._args), self._name)
+
+
+def prepare_reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, stream=None) -> PreparedCall:
+    """pa_reshape_and_cache, prepared (see PreparedCall)."""
+    args = (key, value, k_cache, v_cache, slot_mapping)
+    _device_index(args)
+    return PreparedCall("pa_reshape_and_cache", args, [], _opts(stream), args)
+
+
+def prepare_decode(out, query, k_cache, v_cache, block_tables, context_lens, scale: float, num_kv_heads: int,
+                   workspace=None, partition_tokens: int = 0, stream=None, timeout_ms: int = 0) -> PreparedCall:
+    """pa_decode, prepared (see PreparedCall)."""
+    args = (out, query, k_cache, v_cache, block_tables, context_lens)
+    _device_index(args + (workspace,))
+    return PreparedCall("pa_decode", args, [ctypes.c_float(scale), ctypes.c_int32(int(num_kv_heads))],
+                        _opts(stream, workspace, partition_tokens, timeout_ms), args + (workspace,))
+
+
+def prepare_reshape_and_cache_fp8(key, value, k_cache, v_cache, slot_mapping, k_scale, v_scale,
+                                  stream=None) -> PreparedCall:
+    """pa_reshape_and_cache_fp8, prepared (see PreparedCall)."""
+    args = (key, value, k_cache, v_cache, slot_mapping, k_scale, v_scale)
+    _device_index(args)
+    return PreparedCall("pa_reshape_and_cache_fp8", args, [], _opts(stream), args)
+
+
+def prepare_decode_fp8(out, query, k_cache, v_cache, block_tables, context_lens, scale: float, num_kv_heads: int,
+                       k_scale, v_scale, workspace=None, partition_tokens: int = 0, stream=None,
+                       timeout_ms: int = 0) -> PreparedCall:
+    """pa_decode_fp8, prepared (see PreparedCall)."""
+    args = (out, query, k_cache, v_cache, block_tables, context_lens)
+    _device_index(args + (k_scale, v_scale, workspace))
+    call = PreparedCall("pa_decode_fp8", args, [ctypes.c_float(scale), ctypes.c_int32(int(num_kv_heads))],
+                        _opts(stream, workspace, partition_tokens, timeout_ms), args + (k_scale, v_scale, workspace))
+    # the two scale descriptors go between num_kv_heads and opts
+    call._scales = [_tensor(k_scale), _tensor(v_scale)]
+    call._args = call._args[:-1] + [ctypes.byref(t) for t in call._scales] + call._args[-1:]
+    return call
+
+
+def prepare_decode_cascade(out, query, k_cache, v_cache, block_tables, context_lens, group_start, group_blocks,
+                           max_group_size: int, scale: float, num_kv_heads: int, workspace,
+                           partition_tokens: int = 0, stream=None, timeout_ms: int = 0) -> PreparedCall:
+    """pa_decode_cascade, prepared (see PreparedCall)."""
+    args = (out, query, k_cache, v_cache, block_tables, context_lens, group_start, group_blocks)
+    _device_index(args + (workspace,))
+    return PreparedCall("pa_decode_cascade", args,
+                        [ctypes.c_int32(int(max_group_size)), ctypes.c_float(scale), ctypes.c_int32(int(num_kv_heads))],
+                        _opts(stream, workspace, partition_tokens, timeout_ms), args + (workspace,))
 
 
 # ---------------------------------------------------------------------------
@@ -408,6 +514,19 @@ class Allocator:
         _check(_lib_handle.pa_alloc_block_tables(self._h, _i64p(ids), len(ids), _i32p(out), max_blocks,
                                                  _i32p(lens)), "pa_alloc_block_tables")
         return out[:, :max_blocks], lens[: len(ids)]
+
+    def prefix_groups(self, seqs: Sequence[int], max_group_size: int):
+        """(group_start int32 [n_groups + 1], group_blocks int32 [n_groups]):
+        runs of consecutive batch sequences that share leading blocks, for
+        ``pa_decode_cascade`` (pa_alloc_prefix_groups)."""
+        ids = np.ascontiguousarray(np.asarray(seqs, np.int64))
+        n = len(ids)
+        gs = np.zeros(n + 1, np.int32)
+        gb = np.zeros(max(n, 1), np.int32)
+        ng = ctypes.c_int32(0)
+        _check(_lib_handle.pa_alloc_prefix_groups(self._h, _i64p(ids) if n else None, n, int(max_group_size),
+                                                  _i32p(gs), _i32p(gb), ctypes.byref(ng)), "pa_alloc_prefix_groups")
+        return gs[: ng.value + 1], gb[: ng.value]
 
     def num_free(self) -> int:
         return int(_lib_handle.pa_alloc_num_free(self._h))

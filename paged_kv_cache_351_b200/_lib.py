@@ -59,6 +59,8 @@ STATUS_NAMES = {
 }
 PA_F32, PA_BF16, PA_I32, PA_I64, PA_FP8_E4M3 = 0, 1, 2, 3, 4
 PA_DEV_TIMEOUT, PA_DEV_BAD_BLOCK, PA_DEV_BAD_CONTEXT, PA_DEV_BAD_SLOT = 0x1, 0x2, 0x4, 0x8
+PA_DEV_BAD_WORKSPACE = 0x10
+PA_DECODE_WS_HEADER_BYTES = 64 * 1024
 
 _T = POINTER(PaTensor)
 _O = POINTER(PaOpts)
@@ -75,6 +77,10 @@ SIGNATURES = {
     "pa_decode_fp8": (c_int32, [_T, _T, _T, _T, _T, _T, c_float, c_int32, _T, _T, _O]),
     "pa_prefill": (c_int32, [_T, _T, _T, _T, _T, _T, _T, c_int32, c_float, c_int32, _O]),
     "pa_decode_workspace_bytes": (c_int32, [c_int32, c_int32, c_int32, c_int32, c_int32, c_int32, POINTER(c_size_t)]),
+    "pa_decode_cascade": (c_int32, [_T, _T, _T, _T, _T, _T, _T, _T, c_int32, c_float, c_int32, _O]),
+    "pa_decode_cascade_workspace_bytes": (c_int32, [c_int32, c_int32, c_int32, c_int32, c_int32, c_int32,
+                                                    POINTER(c_size_t)]),
+    "pa_alloc_prefix_groups": (c_int32, [_A, _I64P, c_int32, c_int32, _I32P, _I32P, _I32P]),
     "pa_set_decode_tuning": (c_int32, [c_int32, c_int32, c_int32]),
     "pa_alloc_create": (c_int32, [c_int32, c_int32, _I32P, POINTER(_A)]),
     "pa_alloc_destroy": (None, [_A]),

@@ -511,6 +511,42 @@ pa_status pa_alloc_block_tables(const pa_allocator* a, const int64_t* seq_ids, i
   return PA_OK;
 }
 
+pa_status pa_alloc_prefix_groups(const pa_allocator* a, const int64_t* seq_ids, int32_t n, int32_t max_group_size,
+                                 int32_t* group_start_out, int32_t* group_blocks_out, int32_t* n_groups_out) {
+  if (a == nullptr || n < 0 || max_group_size < 1 || group_start_out == nullptr || n_groups_out == nullptr ||
+      (n > 0 && (seq_ids == nullptr || group_blocks_out == nullptr)))
+    return PA_ERR_INVALID_ARG;
+  std::vector<const Seq*> ss(static_cast<size_t>(n));
+  for (int32_t r = 0; r < n; ++r) {
+    auto it = a->seqs.find(seq_ids[r]);
+    if (it == a->seqs.end() || it->second.swapped) return PA_ERR_INVALID_ARG;
+    ss[r] = &it->second;
+  }
+  const int32_t bs = a->block_size;
+  int32_t g = 0, k = 0;
+  while (k < n) {
+    const int32_t start = k;
+    const Seq& lead = *ss[k];
+    int32_t common = lead.len / bs;  // the leader's full blocks
+    ++k;
+    while (k < n && k - start < max_group_size) {
+      const Seq& s = *ss[k];
+      const int32_t cap = std::min(common, s.len / bs);
+      int32_t c = 0;
+      while (c < cap && s.table[c] == lead.table[c]) ++c;
+      if (c == 0 || 2 * c < common) break;  // joining would give up more than half the shared blocks
+      common = c;
+      ++k;
+    }
+    group_start_out[g] = start;
+    group_blocks_out[g] = (k - start > 1) ? common : 0;
+    ++g;
+  }
+  group_start_out[g] = n;
+  *n_groups_out = g;
+  return PA_OK;
+}
+
 int32_t pa_alloc_num_free(const pa_allocator* a) { return a == nullptr ? -1 : static_cast<int32_t>(a->available()); }
 
 int32_t pa_block_refcount(const pa_allocator* a, int32_t block) {

@@ -7,10 +7,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
-#include <unistd.h>
-
 #include <atomic>
-#include <chrono>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -197,11 +194,14 @@ struct DecodePlan {
   size_t ws_need;
 };
 
+// Shared-memory bytes of a decode launch: the row-sequence prefix (U row
+// sequences, X extra ints) and one ring per warp, with the deepest ring (at
+// most `want` stages) that fits.
 template <typename Tkv, typename Tq, int D, int G>
-size_t stage_fit(int B, int warps, int want, int optin, int* stages_out) {
+size_t stage_fit(int U, int X, int warps, int want, int optin, int* stages_out) {
   using C = pa::DecodeCfg<Tkv, Tq, D, G>;
   for (int st = want; st >= 1; --st) {
-    const size_t bytes = pa::decode_prefix_bytes(B) + size_t(warps) * C::warp_bytes(st);
+    const size_t bytes = pa::decode_prefix_bytes(U, X) + size_t(warps) * C::warp_bytes(st);
     if (bytes <= size_t(optin)) {
       *stages_out = st;
       return bytes;
@@ -212,41 +212,36 @@ size_t stage_fit(int B, int warps, int want, int optin, int* stages_out) {
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-size_t fixed_ws_bytes(int64_t B, int64_t H, int64_t D, int64_t P) {
+// Every decode workspace starts with the same header: one 32-bit merge
+// counter per worker of the balanced split (PA_DECODE_WS_HEADER_BYTES,
+// enough for kMaxWorkers).  Every mode leaves it alone or leaves it zero, so
+// one zero-filled workspace serves every mode and launch shape in turn.
+constexpr size_t kWsHeader = PA_DECODE_WS_HEADER_BYTES;
+constexpr int64_t kMaxWorkers = int64_t(PA_DECODE_WS_HEADER_BYTES / 4);
+
+// Fixed mode, after the header: the documented per-partition partials
+// (o, then lse); the shares of partitions cut between workers follow.
+size_t fixed_partials_bytes(int64_t B, int64_t H, int64_t D, int64_t P) {
   return align_up(size_t(B * H * P * D) * 4, 256) + align_up(size_t(B * H * P) * 4, 256);
 }
 
-// Balanced mode: per worker one published share [G][D] + [G] and its flag.
-size_t balanced_ws_bytes(int64_t workers, int64_t G, int64_t D) {
-  return align_up(size_t(workers * G * D) * 4, 256) + align_up(size_t(workers * G) * 4, 256) +
-         align_up(size_t(workers) * 8, 256);
+// Shares of units cut between workers: per worker two slots ([G][D]
+// outputs + [G] lse): one for a cut unit its range begins in, one for a cut
+// unit it ends in.
+size_t shares_bytes(int64_t workers, int64_t G, int64_t D) {
+  return align_up(size_t(2 * workers * G * D) * 4, 256) + align_up(size_t(2 * workers * G) * 4, 256);
 }
 
-// Tags that mark one call's published shares.  Consecutive calls differ, so
-// a flag left by an earlier call (or by whatever the memory held before) is
-// not mistaken for this call's; the start value is mixed from the clock and
-// the process id.
-std::atomic<unsigned long long> g_call_tag{0};
-std::once_flag g_call_tag_once;
-
-unsigned long long next_call_tag() {
-  std::call_once(g_call_tag_once, [] {
-    unsigned long long x = static_cast<unsigned long long>(
-        std::chrono::high_resolution_clock::now().time_since_epoch().count());
-    x ^= static_cast<unsigned long long>(getpid()) << 32;
-    x += 0x9E3779B97F4A7C15ull;  // splitmix64 finaliser
-    x = (x ^ (x >> 30)) * 0xBF58476D1CE4E5B9ull;
-    x = (x ^ (x >> 27)) * 0x94D049BB133111EBull;
-    x ^= x >> 31;
-    g_call_tag.store(x | 1ull);
-  });
-  return g_call_tag.fetch_add(2ull);
+size_t fixed_ws_bytes(int64_t B, int64_t H, int64_t D, int64_t P, int64_t workers, int64_t G) {
+  return kWsHeader + fixed_partials_bytes(B, H, D, P) + shares_bytes(workers, G, D);
 }
 
-template <typename Tkv, typename Tq, int D, int G>
+size_t balanced_ws_bytes(int64_t workers, int64_t G, int64_t D) { return kWsHeader + shares_bytes(workers, G, D); }
+
+template <typename Tkv, typename Tq, int D, int G, int CK>
 pa_status run_decode(const pa::DecodeArgs& base, const DecodePlan& p, cudaStream_t st, int dev) {
   static std::atomic<size_t> smem_limit[kMaxDevices];
-  auto kern = pa::decode_kernel<Tkv, Tq, D, G>;
+  auto kern = pa::decode_kernel<Tkv, Tq, D, G, CK>;
   if (!raise_smem_limit(kern, p.smem, dev, smem_limit)) return PA_ERR_CUDA;
   pa::DecodeArgs a = base;
   a.stages = p.stages;
@@ -254,74 +249,73 @@ pa_status run_decode(const pa::DecodeArgs& base, const DecodePlan& p, cudaStream
   a.part_pages = p.part_pages;
   a.P_max = p.P_max;
   if (launch_pdl(kern, dim3(p.grid), dim3(p.warps * 32), p.smem, st, true, a) != cudaSuccess) return launch_status();
-  const int64_t nworkers = int64_t(p.grid) * p.warps;
   if (p.mode == pa::kFixed) {
-    const int64_t tasks = int64_t(a.B) * a.H;
-    const int blocks = int((tasks + 7) / 8);
-    if (launch_pdl(pa::merge_fixed_kernel<Tq, D>, dim3(blocks), dim3(256), 0, st, true, a,
+    const int64_t rows = int64_t(a.B) * a.H;  // one CTA per (sequence, query head)
+    if (launch_pdl(pa::merge_fixed_kernel<Tq, D>, dim3(unsigned(rows)), dim3(pa::kMergeWarps * 32), 0, st, true, a,
                    p.part_pages * pa::kBS) != cudaSuccess)
       return launch_status();
   }
-  (void)nworkers;
   return launch_status();
 }
 
-template <typename Tkv, typename Tq, int D>
+template <typename Tkv, typename Tq, int D, int CK>
 pa_status dispatch_group(int G, const pa::DecodeArgs& a, const DecodePlan& p, cudaStream_t st, int dev) {
   switch (G) {
     case 1:
-      return run_decode<Tkv, Tq, D, 1>(a, p, st, dev);
+      return run_decode<Tkv, Tq, D, 1, CK>(a, p, st, dev);
     case 2:
-      return run_decode<Tkv, Tq, D, 2>(a, p, st, dev);
+      return run_decode<Tkv, Tq, D, 2, CK>(a, p, st, dev);
     case 4:
-      return run_decode<Tkv, Tq, D, 4>(a, p, st, dev);
+      return run_decode<Tkv, Tq, D, 4, CK>(a, p, st, dev);
     case 8:
-      return run_decode<Tkv, Tq, D, 8>(a, p, st, dev);
+      return run_decode<Tkv, Tq, D, 8, CK>(a, p, st, dev);
     default:
       return PA_ERR_UNSUPPORTED;
   }
 }
 
 template <typename Tkv, typename Tq, int D>
-size_t fit_for_group(int G, int B, int warps, int want, int optin, int* stages) {
+size_t fit_for_group(int G, int U, int X, int warps, int want, int optin, int* stages) {
   switch (G) {
     case 1:
-      return stage_fit<Tkv, Tq, D, 1>(B, warps, want, optin, stages);
+      return stage_fit<Tkv, Tq, D, 1>(U, X, warps, want, optin, stages);
     case 2:
-      return stage_fit<Tkv, Tq, D, 2>(B, warps, want, optin, stages);
+      return stage_fit<Tkv, Tq, D, 2>(U, X, warps, want, optin, stages);
     case 4:
-      return stage_fit<Tkv, Tq, D, 4>(B, warps, want, optin, stages);
+      return stage_fit<Tkv, Tq, D, 4>(U, X, warps, want, optin, stages);
     case 8:
-      return stage_fit<Tkv, Tq, D, 8>(B, warps, want, optin, stages);
+      return stage_fit<Tkv, Tq, D, 8>(U, X, warps, want, optin, stages);
     default:
       return 0;
   }
 }
 
 // The (cache type, query/output type, head size) combinations built.
-size_t fit_stages(int32_t kv_dtype, int D, int G, int B, int warps, int want, int optin, int* stages) {
+size_t fit_stages(int32_t kv_dtype, int D, int G, int U, int X, int warps, int want, int optin, int* stages) {
   if (kv_dtype == PA_BF16 && D == 128)
-    return fit_for_group<__nv_bfloat16, __nv_bfloat16, 128>(G, B, warps, want, optin, stages);
+    return fit_for_group<__nv_bfloat16, __nv_bfloat16, 128>(G, U, X, warps, want, optin, stages);
   if (kv_dtype == PA_BF16 && D == 64)
-    return fit_for_group<__nv_bfloat16, __nv_bfloat16, 64>(G, B, warps, want, optin, stages);
-  if (kv_dtype == PA_F32 && D == 64) return fit_for_group<float, float, 64>(G, B, warps, want, optin, stages);
-  if (kv_dtype == PA_F32 && D == 128) return fit_for_group<float, float, 128>(G, B, warps, want, optin, stages);
+    return fit_for_group<__nv_bfloat16, __nv_bfloat16, 64>(G, U, X, warps, want, optin, stages);
+  if (kv_dtype == PA_F32 && D == 64) return fit_for_group<float, float, 64>(G, U, X, warps, want, optin, stages);
+  if (kv_dtype == PA_F32 && D == 128) return fit_for_group<float, float, 128>(G, U, X, warps, want, optin, stages);
   if (kv_dtype == PA_FP8_E4M3 && D == 128)
-    return fit_for_group<__nv_fp8_e4m3, __nv_bfloat16, 128>(G, B, warps, want, optin, stages);
+    return fit_for_group<__nv_fp8_e4m3, __nv_bfloat16, 128>(G, U, X, warps, want, optin, stages);
   return 0;
 }
 
-// Mode, grid, smem and workspace of one decode call.
-pa_status plan_decode(int32_t dtype, int64_t B, int64_t H, int64_t Hkv, int64_t D, int64_t max_nb, int32_t part_tokens,
-                      size_t ws_bytes, bool ws_given, DecodePlan* p) {
+// Mode, grid and smem of one decode launch whose rows carry G query rows
+// each, over U row sequences (X extra prefix ints); ws_need = the workspace
+// bytes its split uses (header included).  Shares of a balanced split need
+// share_room bytes after the header.
+pa_status plan_decode(int32_t dtype, int G, int64_t U, int64_t X, int64_t B, int64_t H, int64_t D, int64_t max_nb,
+                      int32_t part_tokens, size_t share_room, bool ws_given, DecodePlan* p) {
   DeviceInfo di;
   int dev = 0;
   pa_status s = device_info(&di, &dev);
   if (s != PA_OK) return s;
-  const int G = int(H / Hkv);
   p->warps = warps_for(G, dtype);
   p->grid = di.sms * g_tuning.ctas_per_sm;
-  p->smem = fit_stages(dtype, int(D), G, int(B), p->warps, g_tuning.stages, di.smem_optin, &p->stages);
+  p->smem = fit_stages(dtype, int(D), G, int(U), int(X), p->warps, g_tuning.stages, di.smem_optin, &p->stages);
   if (p->smem == 0) return PA_ERR_UNSUPPORTED;
   p->part_pages = 0;
   p->P_max = 0;
@@ -333,12 +327,13 @@ pa_status plan_decode(int32_t dtype, int64_t B, int64_t H, int64_t Hkv, int64_t 
     p->part_pages = part_tokens / pa::kBS;
     p->P_max = int((max_nb + p->part_pages - 1) / p->part_pages);
     if (p->P_max < 1) p->P_max = 1;
-    p->ws_need = fixed_ws_bytes(B, H, D, p->P_max);
+    if (nworkers > kMaxWorkers) return PA_ERR_UNSUPPORTED;
+    p->ws_need = fixed_ws_bytes(B, H, D, p->P_max, nworkers, G);
   } else if (part_tokens == 0) {
-    const size_t need = balanced_ws_bytes(nworkers, G, D);
-    if (ws_given && ws_bytes >= need) {
+    const size_t need = shares_bytes(nworkers, G, D);
+    if (ws_given && share_room >= need && nworkers <= kMaxWorkers) {
       p->mode = pa::kBalanced;
-      p->ws_need = need;
+      p->ws_need = kWsHeader + need;
     } else {
       p->mode = pa::kNoSplit;
     }
@@ -610,30 +605,42 @@ pa_status pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_heads, int32_t
     return PA_ERR_INVALID_ARG;
   *bytes_out = 0;
   if (partition_tokens == -1) return PA_OK;
-  if (partition_tokens > 0) {
-    if (partition_tokens % pa::kBS) return PA_ERR_INVALID_ARG;
-    const int64_t pp = partition_tokens / pa::kBS;
-    int64_t P = (max_blocks_per_seq + pp - 1) / pp;
-    if (P < 1) P = 1;
-    *bytes_out = fixed_ws_bytes(num_seqs, num_heads, head_size, P);
-    return PA_OK;
-  }
-  if (partition_tokens != 0) return PA_ERR_INVALID_ARG;
+  if (partition_tokens < -1 || (partition_tokens > 0 && partition_tokens % pa::kBS)) return PA_ERR_INVALID_ARG;
   DeviceInfo di;
   pa_status st = device_info(&di, nullptr);
   if (st != PA_OK) return st;
   const int G = num_heads / num_kv_heads;
   // an upper bound over cache types (FP8 may cap the warps lower)
   const int64_t workers = int64_t(di.sms) * g_tuning.ctas_per_sm * (g_tuning.warps ? g_tuning.warps : default_warps(G, true));
+  if (partition_tokens > 0) {
+    const int64_t pp = partition_tokens / pa::kBS;
+    int64_t P = (max_blocks_per_seq + pp - 1) / pp;
+    if (P < 1) P = 1;
+    *bytes_out = fixed_ws_bytes(num_seqs, num_heads, head_size, P, workers, G);
+    return PA_OK;
+  }
   *bytes_out = balanced_ws_bytes(workers, G, head_size);
   return PA_OK;
 }
 
-// Both decode entry points: k_scale/v_scale are null unless the cache is FP8.
-static pa_status decode_impl(pa_tensor* out, const pa_tensor* query, const pa_tensor* k_cache,
-                             const pa_tensor* v_cache, const pa_tensor* block_tables, const pa_tensor* context_lens,
-                             float scale, int32_t num_kv_heads, const pa_tensor* k_scale, const pa_tensor* v_scale,
-                             const pa_opts* opts) {
+}  // extern "C"
+
+namespace {
+
+// What every decode entry point checks and passes on: sizes, layouts and the
+// kernel arguments that do not depend on the launch plan.
+struct DecodeCall {
+  int64_t B, H, Hkv, D, G, max_nb;
+  int32_t dt;
+  pa::DecodeArgs a;
+};
+
+// k_scale/v_scale are null unless the cache is FP8.
+static pa_status decode_prepare(pa_tensor* out, const pa_tensor* query, const pa_tensor* k_cache,
+                                const pa_tensor* v_cache, const pa_tensor* block_tables,
+                                const pa_tensor* context_lens, float scale, int32_t num_kv_heads,
+                                const pa_tensor* k_scale, const pa_tensor* v_scale, const pa_opts* opts,
+                                DecodeCall* dc) {
   pa_status st = check_pair(k_cache, v_cache);
   if (st != PA_OK) return st;
   const int64_t NB = k_cache->shape[0], Hkv = k_cache->shape[1], D = k_cache->shape[3];
@@ -669,19 +676,13 @@ static pa_status decode_impl(pa_tensor* out, const pa_tensor* query, const pa_te
   if (B >= (int64_t(1) << 20) || B > kMaxBatch) return PA_ERR_UNSUPPORTED;
   if (B * Hkv * max_nb >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
   if (max_nb * 16 > INT32_MAX) return PA_ERR_UNSUPPORTED;
-  if (B == 0) return PA_OK;
-
   const int32_t part = opts ? opts->partition_tokens : 0;
   if (part < -1 || (part > 0 && part % pa::kBS)) return PA_ERR_INVALID_ARG;
-  const bool ws_given = opts && opts->workspace != nullptr;
-  const size_t ws_bytes = ws_given ? opts->workspace_bytes : 0;
-  if (ws_given && (reinterpret_cast<uintptr_t>(opts->workspace) & 255u)) return PA_ERR_INVALID_ARG;
-  DecodePlan plan;
-  st = plan_decode(dt, B, H, Hkv, D, max_nb, part, ws_bytes, ws_given, &plan);
-  if (st != PA_OK) return st;
-  if (plan.mode != pa::kNoSplit && (!ws_given || ws_bytes < plan.ws_need)) return PA_ERR_INVALID_ARG;
+  if (opts && opts->workspace != nullptr && (reinterpret_cast<uintptr_t>(opts->workspace) & 255u))
+    return PA_ERR_INVALID_ARG;
 
-  pa::DecodeArgs a;
+  dc->B = B, dc->H = H, dc->Hkv = Hkv, dc->D = D, dc->G = G, dc->max_nb = max_nb, dc->dt = dt;
+  pa::DecodeArgs& a = dc->a;
   std::memset(&a, 0, sizeof(a));
   a.out = out->data;
   a.q = query->data;
@@ -705,31 +706,108 @@ static pa_status decode_impl(pa_tensor* out, const pa_tensor* query, const pa_te
     a.k_scale = static_cast<const float*>(k_scale->data);
     a.v_scale = static_cast<const float*>(v_scale->data);
   }
-  if (plan.mode == pa::kFixed) {
-    char* w = static_cast<char*>(opts->workspace);
-    a.ws_o = reinterpret_cast<float*>(w);
-    a.ws_lse = reinterpret_cast<float*>(w + align_up(size_t(B * H * plan.P_max * D) * 4, 256));
-  } else if (plan.mode == pa::kBalanced) {
-    const int64_t workers = int64_t(plan.grid) * plan.warps;
-    char* w = static_cast<char*>(opts->workspace);
-    const size_t o_bytes = align_up(size_t(workers * G * D) * 4, 256);
-    const size_t l_bytes = align_up(size_t(workers * G) * 4, 256);
-    a.ws_o = reinterpret_cast<float*>(w);
-    a.ws_lse = reinterpret_cast<float*>(w + o_bytes);
-    a.ws_flag = reinterpret_cast<unsigned long long*>(w + o_bytes + l_bytes);
-    a.call_tag = next_call_tag();
-  }
+  return PA_OK;
+}
+
+// Points a launch's counters (the header) and shares (at byte offset
+// shares_off) into the workspace.
+static void place_shares(pa::DecodeArgs* a, void* workspace, size_t shares_off, const DecodePlan& plan, int64_t G,
+                         int64_t D) {
+  const int64_t workers = int64_t(plan.grid) * plan.warps;
+  char* w = static_cast<char*>(workspace);
+  a->ws_cnt = reinterpret_cast<unsigned int*>(w);
+  w += shares_off;
+  a->sh_o = reinterpret_cast<float*>(w);
+  a->sh_lse = reinterpret_cast<float*>(w + align_up(size_t(2 * workers * G * D) * 4, 256));
+}
+
+template <int CK>
+static pa_status launch_kind(const DecodeCall& dc, int G, const pa::DecodeArgs& a, const DecodePlan& plan,
+                             cudaStream_t s) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PA_ERR_CUDA;
-  cudaStream_t s = stream_of(opts);
-  if (dt == PA_BF16 && D == 128) return dispatch_group<__nv_bfloat16, __nv_bfloat16, 128>(int(G), a, plan, s, dev);
-  if (dt == PA_BF16 && D == 64) return dispatch_group<__nv_bfloat16, __nv_bfloat16, 64>(int(G), a, plan, s, dev);
-  if (dt == PA_F32 && D == 64) return dispatch_group<float, float, 64>(int(G), a, plan, s, dev);
-  if (dt == PA_F32 && D == 128) return dispatch_group<float, float, 128>(int(G), a, plan, s, dev);
-  if (dt == PA_FP8_E4M3 && D == 128)
-    return dispatch_group<__nv_fp8_e4m3, __nv_bfloat16, 128>(int(G), a, plan, s, dev);
+  const int32_t dt = dc.dt;
+  const int64_t D = dc.D;
+  if constexpr (CK == pa::kPlain) {
+    if (dt == PA_BF16 && D == 128) return dispatch_group<__nv_bfloat16, __nv_bfloat16, 128, CK>(G, a, plan, s, dev);
+    if (dt == PA_BF16 && D == 64) return dispatch_group<__nv_bfloat16, __nv_bfloat16, 64, CK>(G, a, plan, s, dev);
+    if (dt == PA_F32 && D == 64) return dispatch_group<float, float, 64, CK>(G, a, plan, s, dev);
+    if (dt == PA_F32 && D == 128) return dispatch_group<float, float, 128, CK>(G, a, plan, s, dev);
+    if (dt == PA_FP8_E4M3 && D == 128)
+      return dispatch_group<__nv_fp8_e4m3, __nv_bfloat16, 128, CK>(G, a, plan, s, dev);
+  } else {
+    // shared-prefix passes: bf16 head size 128 and fp32 head size 64
+    if (dt == PA_BF16 && D == 128) return dispatch_group<__nv_bfloat16, __nv_bfloat16, 128, CK>(G, a, plan, s, dev);
+    if (dt == PA_F32 && D == 64) return dispatch_group<float, float, 64, CK>(G, a, plan, s, dev);
+  }
   return PA_ERR_UNSUPPORTED;
 }
+
+static pa_status decode_impl(pa_tensor* out, const pa_tensor* query, const pa_tensor* k_cache,
+                             const pa_tensor* v_cache, const pa_tensor* block_tables, const pa_tensor* context_lens,
+                             float scale, int32_t num_kv_heads, const pa_tensor* k_scale, const pa_tensor* v_scale,
+                             const pa_opts* opts) {
+  DecodeCall dc;
+  pa_status st = decode_prepare(out, query, k_cache, v_cache, block_tables, context_lens, scale, num_kv_heads,
+                                k_scale, v_scale, opts, &dc);
+  if (st != PA_OK) return st;
+  if (dc.B == 0) return PA_OK;
+  const int32_t part = opts ? opts->partition_tokens : 0;
+  const bool ws_given = opts && opts->workspace != nullptr;
+  const size_t ws_bytes = ws_given ? opts->workspace_bytes : 0;
+  DecodePlan plan;
+  st = plan_decode(dc.dt, int(dc.G), dc.B, 0, dc.B, dc.H, dc.D, dc.max_nb, part,
+                   ws_bytes > kWsHeader ? ws_bytes - kWsHeader : 0, ws_given, &plan);
+  if (st != PA_OK) return st;
+  if (plan.mode != pa::kNoSplit && (!ws_given || ws_bytes < plan.ws_need)) return PA_ERR_INVALID_ARG;
+  pa::DecodeArgs a = dc.a;
+  if (plan.mode == pa::kFixed) {
+    char* w = static_cast<char*>(opts->workspace) + kWsHeader;
+    a.ws_o = reinterpret_cast<float*>(w);
+    a.ws_lse = reinterpret_cast<float*>(w + align_up(size_t(dc.B * dc.H * plan.P_max * dc.D) * 4, 256));
+    place_shares(&a, opts->workspace, kWsHeader + fixed_partials_bytes(dc.B, dc.H, dc.D, plan.P_max), plan, dc.G,
+                 dc.D);
+  } else if (plan.mode == pa::kBalanced) {
+    place_shares(&a, opts->workspace, kWsHeader, plan, dc.G, dc.D);
+  }
+  return launch_kind<pa::kPlain>(dc, int(dc.G), a, plan, stream_of(opts));
+}
+
+// ---------------------------------------------------------------------------
+// shared-prefix (cascade) decode
+// ---------------------------------------------------------------------------
+// Workspace: [header][shares of the larger pass][pre_o: B*H*D fp32][pre_lse: B*H fp32].
+struct CascadeLayout {
+  size_t shares;  // bytes after the header for the balanced shares (0: no split)
+  size_t pre_o_off, pre_lse_off, total;
+};
+
+static CascadeLayout cascade_layout(int64_t B, int64_t H, int64_t D, size_t shares) {
+  CascadeLayout L;
+  L.shares = shares;
+  L.pre_o_off = kWsHeader + align_up(shares, 256);
+  L.pre_lse_off = L.pre_o_off + align_up(size_t(B * H * D) * 4, 256);
+  L.total = L.pre_lse_off + align_up(size_t(B * H) * 4, 256);
+  return L;
+}
+
+// Bytes of balanced shares the two passes need (the larger), on the current
+// device under the current tuning.
+static pa_status cascade_shares_bytes(int32_t dt, int64_t G, int64_t members, int64_t D, size_t* out) {
+  DeviceInfo di;
+  pa_status st = device_info(&di, nullptr);
+  if (st != PA_OK) return st;
+  const int64_t grid = int64_t(di.sms) * g_tuning.ctas_per_sm;
+  const int64_t gp = G * members;
+  const size_t pre = shares_bytes(grid * warps_for(int(gp), dt), gp, D);
+  const size_t suf = shares_bytes(grid * warps_for(int(G), dt), G, D);
+  *out = pre > suf ? pre : suf;
+  return PA_OK;
+}
+
+}  // namespace
+
+extern "C" {
 
 pa_status pa_decode(pa_tensor* out, const pa_tensor* query, const pa_tensor* k_cache, const pa_tensor* v_cache,
                     const pa_tensor* block_tables, const pa_tensor* context_lens, float scale, int32_t num_kv_heads,
@@ -746,6 +824,101 @@ pa_status pa_decode_fp8(pa_tensor* out, const pa_tensor* query, const pa_tensor*
   if (k_cache == nullptr || k_cache->dtype != PA_FP8_E4M3) return PA_ERR_INVALID_ARG;
   return decode_impl(out, query, k_cache, v_cache, block_tables, context_lens, scale, num_kv_heads, k_scale, v_scale,
                      opts);
+}
+
+}  // extern "C"
+
+namespace {
+
+// Checks the group tensors and the group width of a shared-prefix decode.
+static pa_status cascade_groups(const pa_tensor* group_start, const pa_tensor* group_blocks, int64_t G,
+                                int32_t max_group_size, int64_t* n_groups) {
+  if (group_blocks == nullptr || group_blocks->ndim != 1 || group_blocks->dtype != PA_I32 ||
+      group_start == nullptr || group_start->ndim != 1 || group_start->dtype != PA_I32)
+    return PA_ERR_INVALID_ARG;
+  const int64_t n = group_blocks->shape[0];
+  if (n < 1 || n > kMaxBatch || group_start->shape[0] != n + 1) return PA_ERR_INVALID_ARG;
+  if (group_start->stride[0] != 1 || group_blocks->stride[0] != 1 || group_start->data == nullptr ||
+      group_blocks->data == nullptr)
+    return PA_ERR_INVALID_ARG;
+  if (max_group_size < 1) return PA_ERR_INVALID_ARG;
+  const int64_t gp = G * max_group_size;
+  if (gp != 1 && gp != 2 && gp != 4 && gp != 8) return PA_ERR_UNSUPPORTED;
+  *n_groups = n;
+  return PA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+pa_status pa_decode_cascade_workspace_bytes(int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
+                                            int32_t head_size, int32_t max_group_size, int32_t partition_tokens,
+                                            size_t* bytes_out) {
+  if (bytes_out == nullptr || num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_size <= 0 ||
+      num_heads % num_kv_heads || max_group_size < 1)
+    return PA_ERR_INVALID_ARG;
+  if (partition_tokens != 0 && partition_tokens != -1) return PA_ERR_UNSUPPORTED;
+  const int64_t G = num_heads / num_kv_heads;
+  const int64_t gp = G * max_group_size;
+  if (gp != 1 && gp != 2 && gp != 4 && gp != 8) return PA_ERR_UNSUPPORTED;
+  size_t shares = 0;
+  if (partition_tokens == 0) {
+    // an upper bound over cache types (as for pa_decode_workspace_bytes)
+    const pa_status st = cascade_shares_bytes(PA_FP8_E4M3, G, max_group_size, head_size, &shares);
+    if (st != PA_OK) return st;
+    size_t b16 = 0;
+    cascade_shares_bytes(PA_BF16, G, max_group_size, head_size, &b16);
+    if (b16 > shares) shares = b16;
+  }
+  *bytes_out = cascade_layout(num_seqs, num_heads, head_size, shares).total;
+  return PA_OK;
+}
+
+pa_status pa_decode_cascade(pa_tensor* out, const pa_tensor* query, const pa_tensor* k_cache,
+                            const pa_tensor* v_cache, const pa_tensor* block_tables, const pa_tensor* context_lens,
+                            const pa_tensor* group_start, const pa_tensor* group_blocks, int32_t max_group_size,
+                            float scale, int32_t num_kv_heads, const pa_opts* opts) {
+  if (k_cache != nullptr && k_cache->dtype == PA_FP8_E4M3) return PA_ERR_UNSUPPORTED;
+  DecodeCall dc;
+  pa_status st = decode_prepare(out, query, k_cache, v_cache, block_tables, context_lens, scale, num_kv_heads,
+                                nullptr, nullptr, opts, &dc);
+  if (st != PA_OK) return st;
+  if (!((dc.dt == PA_BF16 && dc.D == 128) || (dc.dt == PA_F32 && dc.D == 64))) return PA_ERR_UNSUPPORTED;
+  int64_t n_groups = 0;
+  if ((st = cascade_groups(group_start, group_blocks, dc.G, max_group_size, &n_groups)) != PA_OK) return st;
+  const int32_t part = opts ? opts->partition_tokens : 0;
+  if (part != 0 && part != -1) return PA_ERR_UNSUPPORTED;
+  if (dc.B == 0) return PA_OK;
+  const int64_t gp = dc.G * max_group_size;
+  size_t shares = 0;
+  if (part == 0 && (st = cascade_shares_bytes(dc.dt, dc.G, max_group_size, dc.D, &shares)) != PA_OK) return st;
+  const CascadeLayout L = cascade_layout(dc.B, dc.H, dc.D, shares);
+  if (opts == nullptr || opts->workspace == nullptr || opts->workspace_bytes < L.total) return PA_ERR_INVALID_ARG;
+  char* ws = static_cast<char*>(opts->workspace);
+
+  DecodePlan pp, ps;
+  if ((st = plan_decode(dc.dt, int(gp), n_groups, 0, dc.B, dc.H, dc.D, dc.max_nb, part, L.shares, true, &pp)) !=
+      PA_OK)
+    return st;
+  if ((st = plan_decode(dc.dt, int(dc.G), dc.B, dc.B, dc.B, dc.H, dc.D, dc.max_nb, part, L.shares, true, &ps)) !=
+      PA_OK)
+    return st;
+  pa::DecodeArgs a = dc.a;
+  a.grp_start = static_cast<const int32_t*>(group_start->data);
+  a.grp_blocks = static_cast<const int32_t*>(group_blocks->data);
+  a.n_groups = int32_t(n_groups);
+  a.grp_members = max_group_size;
+  a.g_real = int32_t(dc.G);
+  a.pre_o = reinterpret_cast<float*>(ws + L.pre_o_off);
+  a.pre_lse = reinterpret_cast<float*>(ws + L.pre_lse_off);
+  const cudaStream_t s = stream_of(opts);
+  pa::DecodeArgs ap = a;
+  if (pp.mode == pa::kBalanced) place_shares(&ap, ws, kWsHeader, pp, gp, dc.D);
+  if ((st = launch_kind<pa::kPrefixPass>(dc, int(gp), ap, pp, s)) != PA_OK) return st;
+  pa::DecodeArgs as = a;
+  if (ps.mode == pa::kBalanced) place_shares(&as, ws, kWsHeader, ps, dc.G, dc.D);
+  return launch_kind<pa::kSuffixPass>(dc, int(dc.G), as, ps, s);
 }
 
 pa_status pa_prefill(pa_tensor* out, const pa_tensor* query, const pa_tensor* k_cache, const pa_tensor* v_cache,
@@ -890,8 +1063,10 @@ pa_status pa_decode_no_alloc(pa_tensor* out, const pa_tensor* query, const pa_te
   if (B < 0 || H <= 0 || num_kv_heads <= 0 || H % num_kv_heads || B > INT32_MAX || max_nb < 0 || max_nb > INT32_MAX ||
       D <= 0 || D > INT32_MAX || H > INT32_MAX)
     return PA_ERR_INVALID_ARG;
-  size_t need = 0;
-  if (part != -1 && B > 0) {
+  // Fixed partitions need their whole layout; the auto mode, like pa_decode
+  // given too small a workspace, falls back to no split by itself.
+  if (part > 0 && B > 0) {
+    size_t need = 0;
     const pa_status st = pa_decode_workspace_bytes(int32_t(B), int32_t(H), num_kv_heads, int32_t(D),
                                                    int32_t(max_nb), part, &need);
     if (st != PA_OK) return st;

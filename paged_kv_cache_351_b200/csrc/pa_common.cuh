@@ -82,35 +82,6 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
   }
 }
 
-// ---- flags between CTAs of one grid ---------------------------------------
-__device__ __forceinline__ void st_release_u64(unsigned long long* p, unsigned long long v) {
-  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-
-__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
-  unsigned long long v;
-  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-  return v;
-}
-
-// Wait until *p == want, giving up after timeout_ns (sets PA_DEV_TIMEOUT).
-__device__ __forceinline__ bool wait_flag_bounded(const unsigned long long* p, unsigned long long want,
-                                                  uint64_t timeout_ns) {
-  if (ld_acquire_u64(p) == want) return true;
-  const uint64_t t0 = globaltimer_ns();
-  while (true) {
-#pragma unroll 1
-    for (int k = 0; k < 32; ++k) {
-      __nanosleep(64);
-      if (ld_acquire_u64(p) == want) return true;
-    }
-    if (globaltimer_ns() - t0 > timeout_ns) {
-      flag(PA_DEV_TIMEOUT);
-      return false;
-    }
-  }
-}
-
 // ---- bulk copy (TMA engine, 1-D, no tensor map, no multicast) --------------
 // dst and src 16-byte aligned, bytes a multiple of 16.
 __device__ __forceinline__ void bulk_g2s(uint32_t dst_smem, const void* src, uint32_t bytes, uint32_t bar,

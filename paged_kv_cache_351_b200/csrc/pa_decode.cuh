@@ -13,14 +13,15 @@
 //    workers of a persistent grid (one CTA per SM) take equal, contiguous
 //    ranges of the flattened page list, so every SM streams the same number
 //    of bytes whatever the length mix.  A row cut by a range boundary yields
-//    per-worker partial results (normalised output and log-sum-exp).  The
-//    worker holding the row's first page merges them at the end of its own
-//    range: the later workers publish their share with a per-call tag, and
-//    the merging warp waits (bounded) for the tags, so no separate merge
-//    kernel and no zeroed workspace are needed.  Fixed-size partitions (each
-//    partition its own partial, merged by a small log-sum-exp kernel) and an
-//    unsplit mode are the same loop with boundaries snapped to partitions or
-//    rows.
+//    per-worker partial results (normalised output and log-sum-exp).  Each
+//    worker publishes its share, then adds its page count to the row's
+//    counter; the worker whose pages complete the row merges the shares (in
+//    worker order) and writes it, then resets the counter.  No worker waits
+//    for another, so nothing depends on which CTAs are resident at once,
+//    and the counters are zero again when the launch ends.  Fixed-size
+//    partitions (each partition its own partial, merged by a small
+//    log-sum-exp kernel) and an unsplit mode are the same loop with
+//    boundaries snapped to partitions or rows.
 //  * Each page of a row — 16 tokens x head_size for one kv head, 4 KiB for
 //    bf16/128 — is one contiguous run in the cache layout
 //    [num_blocks, num_kv_heads, 16, head_size], so a worker moves it with a
@@ -77,14 +78,32 @@ struct DecodeArgs {
   int32_t part_pages;  // fixed mode: pages per partition
   int32_t P_max;       // fixed mode: partition capacity per (seq, head)
   int32_t stages;      // ring depth per warp
-  float* ws_o;         // partial outputs (normalised)
-  float* ws_lse;       // partial log-sum-exp (natural log)
-  unsigned long long* ws_flag;  // balanced mode: per worker, the call tag once its partial is published
-  unsigned long long call_tag;  // distinct per call, so no flag has to start at zero
+  float* ws_o;         // fixed mode: one partial output per partition (normalised)
+  float* ws_lse;       // fixed mode: its log-sum-exp (natural log)
+  float* sh_o;         // shares of units cut between workers: two slots per worker, [G][D] outputs
+  float* sh_lse;       // and [G] log-sum-exp
+  unsigned int* ws_cnt;  // per cut unit (indexed by its first worker), pages counted in so far;
+                         // zero before the launch, and zero again after it
   uint64_t timeout_ns;
   const float* k_scale;  // FP8 cache: per-kv-head dequantization scales (else null)
   const float* v_scale;
+  // Shared-prefix (cascade) decode: the batch is cut into groups of
+  // consecutive sequences whose block tables begin with the same blocks.
+  const int32_t* grp_start;   // [n_groups + 1]: group v = sequences grp_start[v] .. grp_start[v+1] - 1
+  const int32_t* grp_blocks;  // [n_groups]: leading blocks every member shares
+  int32_t n_groups;
+  int32_t grp_members;  // most members a group may have (the prefix pass reads members x g_real query rows)
+  int32_t g_real;       // query heads per kv head
+  float* pre_o;         // [B][H][D]: the prefix's partial output of each (sequence, head), normalised
+  float* pre_lse;       // [B][H]: its log-sum-exp (natural log)
 };
+
+// Decode kinds: a plain decode, or one of the two passes of a shared-prefix
+// decode.  The prefix pass treats each group's shared blocks as one row of
+// members x g_real query rows (each page is read once for the whole group)
+// and leaves partial results; the suffix pass runs every sequence over the
+// rest of its context and merges the prefix's partial into its output.
+enum DecodeKind : int { kPlain = 0, kPrefixPass = 1, kSuffixPass = 2 };
 
 // Tkv: cache element type (fp32, bf16 or e4m3 codes); Tq: query/output type.
 template <typename Tkv, typename Tq, int D, int G>
@@ -113,9 +132,57 @@ struct DecodeCfg {
   }
 };
 
-// smem carve-up: [scan scratch: 32 int32][S: (B+1) int32], padded to 128 bytes,
-// then one region per warp (DecodeCfg::warp_bytes).
-__host__ __device__ inline size_t decode_prefix_bytes(int B) { return (size_t(B + 1 + 32) * 4 + 127) / 128 * 128; }
+// smem carve-up: [scan scratch: 32 int32][S: (U+1) int32][first page: X int32],
+// padded to 128 bytes, then one region per warp (DecodeCfg::warp_bytes).  U
+// is the number of row sequences (the batch, or the groups of a prefix
+// pass); X is B for a suffix pass (each sequence's first block after its
+// group's shared prefix), else 0.
+__host__ __device__ inline size_t decode_prefix_bytes(int U, int X = 0) {
+  return (size_t(U + 1 + 32 + X) * 4 + 127) / 128 * 128;
+}
+
+// Groups of a shared-prefix decode must tile the batch in order:
+// grp_start[0] = 0, non-decreasing, grp_start[n_groups] = B.  Block-wide
+// check (every CTA reaches the same verdict); anything else disables the
+// shared prefix for the whole call (every sequence then runs in full in the
+// suffix pass) and sets PA_DEV_BAD_CONTEXT.
+__device__ __forceinline__ bool groups_tile_batch(const DecodeArgs& a) {
+  int ok = 1;
+  const int n = a.n_groups;
+  for (int v = threadIdx.x; v <= n; v += blockDim.x) {
+    const int x = __ldg(a.grp_start + v);
+    if (v == 0 && x != 0) ok = 0;
+    if (v == n && x != a.B) ok = 0;
+    if (v < n && __ldg(a.grp_start + v + 1) < x) ok = 0;
+  }
+  ok = __syncthreads_and(ok);
+  if (!ok && blockIdx.x == 0 && threadIdx.x == 0) flag(PA_DEV_BAD_CONTEXT);
+  return ok != 0;
+}
+
+// Shared leading blocks of group v as both passes use them: 0 for an empty
+// group or one with more members than the prefix pass has query rows for;
+// else grp_blocks[v] capped at every member's count of full blocks (a cap
+// sets PA_DEV_BAD_CONTEXT).
+__device__ __forceinline__ int group_prefix_blocks(const DecodeArgs& a, int v, int ctx_cap) {
+  const int s0 = __ldg(a.grp_start + v), s1 = __ldg(a.grp_start + v + 1);
+  const int n = s1 - s0;
+  int b = __ldg(a.grp_blocks + v);
+  if (n <= 0 || b <= 0) return 0;
+  if (n > a.grp_members) {
+    if (blockIdx.x == 0) flag(PA_DEV_BAD_CONTEXT);
+    return 0;
+  }
+  for (int m = s0; m < s1; ++m) {
+    const int raw = __ldg(a.ctx + m);
+    const int full = (raw < 0 ? 0 : (raw > ctx_cap ? ctx_cap : raw)) / 16;
+    if (b > full) {
+      if (blockIdx.x == 0) flag(PA_DEV_BAD_CONTEXT);
+      b = full;
+    }
+  }
+  return b;
+}
 
 // Block-wide exclusive scan of one int per thread; returns the prefix and
 // writes the total to *total.  scratch: >= 32 ints of shared memory.
@@ -171,14 +238,28 @@ __device__ __forceinline__ RowPos locate(const int* S, int B, int Hkv, int64_t x
   return r;
 }
 
-// Snap a range boundary down to the start of its partition (fixed mode) or
-// row (unsplit mode); balanced mode keeps page granularity.
-__device__ __forceinline__ int64_t snap_boundary(const int* S, int B, int Hkv, int64_t b, int64_t W, int mode,
-                                                 int part_pages) {
-  if (b >= W || mode == kBalanced) return b < W ? b : W;
+// Snap a range boundary down to the start of its row (unsplit mode); the
+// balanced and fixed modes keep page granularity.
+__device__ __forceinline__ int64_t snap_boundary(const int* S, int B, int Hkv, int64_t b, int64_t W, int mode) {
+  if (b >= W || mode != kNoSplit) return b < W ? b : W;
   const RowPos r = locate(S, B, Hkv, b);
-  const int p0 = mode == kNoSplit ? 0 : (r.p / part_pages) * part_pages;
-  return int64_t(S[r.i]) + int64_t(r.g) * r.np + p0;
+  return int64_t(S[r.i]) + int64_t(r.g) * r.np;
+}
+
+// The unit a page belongs to: its row, or in fixed mode its partition of the
+// row.  A unit cut by a worker boundary is merged from its pieces by the
+// worker that completes it.  Returns the unit's first flat page and size.
+__device__ __forceinline__ void unit_of(const RowPos& r, const int* S, int mode, int part_pages, int64_t* first,
+                                        int* np) {
+  const int64_t rf = int64_t(S[r.i]) + int64_t(r.g) * r.np;
+  if (mode == kFixed) {
+    const int u0 = (r.p / part_pages) * part_pages;
+    *first = rf + u0;
+    *np = min(part_pages, r.np - u0);
+  } else {
+    *first = rf;
+    *np = r.np;
+  }
 }
 
 // Writes one lane's EPV output values of a row (QV 16-byte vectors of Tq).
@@ -189,7 +270,145 @@ __device__ __forceinline__ void store_out(Tq* dst, const float* f) {
   for (int v = 0; v < EPV / EPQ; ++v) *reinterpret_cast<uint4*>(dst + v * EPQ) = Elem<Tq>::pack(f + v * EPQ);
 }
 
-template <typename Tkv, typename Tq, int D, int G>
+// Writes PER consecutive output values (PER = 2 or 4; 8 or 16 bytes).
+template <typename Tq, int PER>
+__device__ __forceinline__ void store_out_small(Tq* dst, const float* f) {
+  if constexpr (sizeof(Tq) == 4) {
+    if constexpr (PER == 4)
+      *reinterpret_cast<float4*>(dst) = make_float4(f[0], f[1], f[2], f[3]);
+    else
+      *reinterpret_cast<float2*>(dst) = make_float2(f[0], f[1]);
+  } else {
+    uint32_t w[PER / 2];
+#pragma unroll
+    for (int k = 0; k < PER / 2; ++k) {
+      __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * k], f[2 * k + 1]);
+      w[k] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    if constexpr (PER == 4)
+      *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
+    else
+      *reinterpret_cast<uint32_t*>(dst) = w[0];
+  }
+}
+
+// ---- balanced split: shares of a row cut by worker boundaries --------------
+// Worker k owns the flat pages [ceil(k W / N), ceil((k+1) W / N)); page x
+// belongs to worker floor(x N / W).  A cut row leaves one share per worker
+// that holds some of its pages: the row's first worker wa publishes in its
+// "tail" slot (2 wa + 1), every later one in its "head" slot (2 k), since a
+// worker's range can begin inside one cut row and end inside another.
+__device__ __forceinline__ bool worker_empty(int64_t k, int64_t W, int64_t N) {
+  return (k * W + N - 1) / N == ((k + 1) * W + N - 1) / N;
+}
+
+__device__ __forceinline__ int64_t share_slot(int64_t k, int64_t wa) { return 2 * k + (k == wa ? 1 : 0); }
+
+// Counts `mine` pages of a row into its counter (one lane; every lane of the
+// warp has published its part of the share and fenced before).  True for
+// the worker whose pages complete the row: it resets the counter, so every
+// counter is zero again when the launch ends, and it alone merges the row.
+// Nobody waits for anybody.  A counter that overshoots the row (a workspace
+// whose counters did not start at zero) sets PA_DEV_BAD_WORKSPACE.
+__device__ __forceinline__ bool count_in(unsigned int* cnt, unsigned int mine, unsigned int total) {
+  const unsigned int now = atomicAdd(cnt, mine) + mine;
+  if (now < total) return false;
+  atomicExch(cnt, 0u);
+  if (now > total) {
+    flag(PA_DEV_BAD_WORKSPACE);
+    return false;
+  }
+  return true;
+}
+
+// Warp-collective: publish-then-count for this warp's share of a cut row.
+// Returns (in every lane) whether this worker completes the row.
+__device__ __forceinline__ bool share_done(unsigned int* cnt, int mine, int total) {
+  __threadfence();  // each lane's share stores, before the count
+  __syncwarp();
+  int last = 0;
+  if ((threadIdx.x & 31) == 0) last = count_in(cnt, unsigned(mine), unsigned(total));
+  last = __shfl_sync(0xffffffffu, last, 0);
+  if (last) __threadfence();  // the count, before reading the other shares
+  return last != 0;
+}
+
+// Warp-collective log-sum-exp merge of the shares of one cut row (workers
+// wa .. wb, in that order, so the result does not depend on which worker
+// finished last).  Lane l ends with dims [l PER, l PER + PER) of each of the
+// G query rows (normalised) and the rows' natural-log lse.  The shares are
+// taken 32 at a time: lane t loads the lse values of share k0 + t and turns
+// them into weights, which are then broadcast while every lane streams its
+// dims of each share's outputs; the output loads of several shares are in
+// flight at once (a long row can have tens of shares, and the merge sits at
+// the end of the launch).
+template <int D, int G>
+__device__ __forceinline__ void merge_shares(const float* ws_o, const float* ws_lse, int64_t wa, int64_t wb,
+                                             int64_t W, int64_t N, float (&acc)[G][D / 32], float (&lse)[G]) {
+  constexpr int PER = D / 32;
+  constexpr float kLog2e = 1.4426950408889634f;
+  const int lane = threadIdx.x & 31;
+  float mx[G], wsum[G];
+#pragma unroll
+  for (int j = 0; j < G; ++j) mx[j] = -INFINITY;
+  for (int64_t k = wa + lane; k <= wb; k += 32) {
+    if (worker_empty(k, W, N)) continue;
+    const int64_t slot = share_slot(k, wa);
+#pragma unroll
+    for (int j = 0; j < G; ++j) mx[j] = fmaxf(mx[j], __ldcg(ws_lse + slot * G + j));
+  }
+#pragma unroll
+  for (int j = 0; j < G; ++j) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx[j] = fmaxf(mx[j], __shfl_xor_sync(0xffffffffu, mx[j], o));
+    wsum[j] = 0.f;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) acc[j][e] = 0.f;
+  }
+  for (int64_t k0 = wa; k0 <= wb; k0 += 32) {
+    // this lane's share of the chunk: its weights (0 for none)
+    const int64_t kl = k0 + lane;
+    const bool mine = kl <= wb && !worker_empty(kl, W, N);
+    float wl[G];
+#pragma unroll
+    for (int j = 0; j < G; ++j)
+      wl[j] = mine ? ex2((__ldcg(ws_lse + share_slot(kl, wa) * G + j) - mx[j]) * kLog2e) : 0.f;
+    const int n = int(wb - k0 + 1 < 32 ? wb - k0 + 1 : 32);
+#pragma unroll 4
+    for (int t = 0; t < n; ++t) {
+      float w[G];
+#pragma unroll
+      for (int j = 0; j < G; ++j) w[j] = __shfl_sync(0xffffffffu, wl[j], t);
+      // an empty worker's slot was never written: skip it (its weight is 0)
+      const int64_t slot = share_slot(k0 + t, wa);
+      if (w[0] == 0.f && worker_empty(k0 + t, W, N)) continue;
+#pragma unroll
+      for (int j = 0; j < G; ++j) {
+        wsum[j] += w[j];
+        const float* src = ws_o + (slot * G + j) * D + lane * PER;
+        float v[PER];
+        if constexpr (PER == 4) {
+          const float4 v4 = __ldcg(reinterpret_cast<const float4*>(src));
+          v[0] = v4.x, v[1] = v4.y, v[2] = v4.z, v[3] = v4.w;
+        } else {
+          const float2 v2 = __ldcg(reinterpret_cast<const float2*>(src));
+          v[0] = v2.x, v[1] = v2.y;
+        }
+#pragma unroll
+        for (int e = 0; e < PER; ++e) acc[j][e] = fmaf(w[j], v[e], acc[j][e]);
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < G; ++j) {
+    const float inv = 1.f / wsum[j];
+#pragma unroll
+    for (int e = 0; e < PER; ++e) acc[j][e] *= inv;
+    lse[j] = mx[j] + logf(wsum[j]);
+  }
+}
+
+template <typename Tkv, typename Tq, int D, int G, int CK = kPlain>
 __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 1) decode_kernel(const DecodeArgs a) {
   using C = DecodeCfg<Tkv, Tq, D, G>;
   using T = Tkv;
@@ -200,12 +419,16 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
   const int warp = threadIdx.x >> 5;
   const int nwarps = blockDim.x >> 5;
   const int tg = lane / LPT, c = lane % LPT;
-  const int B = a.B, Hkv = a.Hkv, H = a.H;
+  // U row sequences: the groups in a prefix pass, else the batch's sequences
+  const int U = CK == kPrefixPass ? a.n_groups : a.B;
+  const int Hkv = a.Hkv, H = a.H;
   const int ctx_cap = a.max_nb * kBS;
 
   int* scan_scratch = reinterpret_cast<int*>(smem);
   int* S = scan_scratch + 32;
-  unsigned char* wbase = smem + decode_prefix_bytes(B) + size_t(warp) * C::warp_bytes(a.stages);
+  int* ST = S + U + 1;  // suffix pass: each sequence's first block after its group's shared prefix
+  unsigned char* wbase =
+      smem + decode_prefix_bytes(U, CK == kSuffixPass ? a.B : 0) + size_t(warp) * C::warp_bytes(a.stages);
   unsigned char* ring = wbase;
   float* pbuf = reinterpret_cast<float*>(wbase + size_t(a.stages) * C::STAGE);
   uint64_t* bars = reinterpret_cast<uint64_t*>(wbase + size_t(a.stages) * C::STAGE + C::PBUF);
@@ -219,44 +442,90 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
   pdl_wait();
   pdl_launch_dependents();
 
-  // ---- prologue: page prefix over sequences (every CTA computes it) ------
+  // ---- prologue: page prefix over row sequences (every CTA computes it) ----
   {
+    bool groups_ok = false;
+    if constexpr (CK != kPlain) groups_ok = groups_tile_batch(a);
+    if constexpr (CK == kSuffixPass) {
+      for (int i = threadIdx.x; i < U; i += blockDim.x) ST[i] = 0;
+      __syncthreads();
+      if (groups_ok)
+        for (int v = threadIdx.x; v < a.n_groups; v += blockDim.x) {
+          const int b = group_prefix_blocks(a, v, ctx_cap);
+          if (b)
+            for (int i = __ldg(a.grp_start + v); i < __ldg(a.grp_start + v + 1); ++i) ST[i] = b;
+        }
+      __syncthreads();
+    }
     const int nt = blockDim.x;
-    const int per = (B + nt - 1) / nt;
+    const int per = (U + nt - 1) / nt;
     const int i0 = threadIdx.x * per;
-    const int i1 = min(B, i0 + per);
+    const int i1 = min(U, i0 + per);
     int local = 0;
     for (int i = i0; i < i1; ++i) {
-      const int raw = a.ctx[i];
-      if ((raw < 0 || raw > ctx_cap) && blockIdx.x == 0) flag(PA_DEV_BAD_CONTEXT);
-      local += (clamp_ctx(raw, ctx_cap) + kBS - 1) / kBS * Hkv;
+      int np;
+      if constexpr (CK == kPrefixPass) {
+        np = groups_ok ? group_prefix_blocks(a, i, ctx_cap) : 0;
+      } else {
+        const int raw = a.ctx[i];
+        if ((raw < 0 || raw > ctx_cap) && blockIdx.x == 0) flag(PA_DEV_BAD_CONTEXT);
+        np = (clamp_ctx(raw, ctx_cap) + kBS - 1) / kBS;
+        if constexpr (CK == kSuffixPass) np -= ST[i];
+      }
+      S[i] = np;  // this thread's own entries: pages first, prefix below
+      local += np * Hkv;
     }
     int total;
     int run = block_exclusive_scan(local, scan_scratch, &total);
     for (int i = i0; i < i1; ++i) {
+      const int np = S[i];
       S[i] = run;
-      run += (clamp_ctx(a.ctx[i], ctx_cap) + kBS - 1) / kBS * Hkv;
+      run += np * Hkv;
     }
-    if (threadIdx.x == 0) S[B] = total;
+    if (threadIdx.x == 0) S[U] = total;
     __syncthreads();
   }
   __syncwarp();
 
-  const int64_t W = S[B];
+  const int64_t W = S[U];
   const int64_t nworkers = int64_t(gridDim.x) * nwarps;
   const int64_t wid = int64_t(blockIdx.x) * nwarps + warp;
   int64_t lo = (wid * W + nworkers - 1) / nworkers;
   int64_t hi = ((wid + 1) * W + nworkers - 1) / nworkers;
-  lo = snap_boundary(S, B, Hkv, lo, W, a.mode, a.part_pages);
-  hi = snap_boundary(S, B, Hkv, hi, W, a.mode, a.part_pages);
+  lo = snap_boundary(S, U, Hkv, lo, W, a.mode);
+  hi = snap_boundary(S, U, Hkv, hi, W, a.mode);
   const uint64_t pol = policy_evict_first();
   const Tq* qg = reinterpret_cast<const Tq*>(a.q);
   const unsigned char* kcb = reinterpret_cast<const unsigned char*>(a.kc);
   const unsigned char* vcb = reinterpret_cast<const unsigned char*>(a.vc);
 
   if (lo < hi) {
+    // The cut units this worker holds pages of (at most two: one that began
+    // in an earlier worker, one that continues in a later one), so that a
+    // worker giving up early still counts its pages in and leaves every
+    // counter at zero.
+    int64_t head_wa = -1, tail_wa = -1;
+    int head_pages = 0, head_np = 0, tail_pages = 0, tail_np = 0;
+    if (a.mode != kNoSplit) {
+      int64_t f0, f1;
+      int n0, n1;
+      unit_of(locate(S, U, Hkv, lo), S, a.mode, a.part_pages, &f0, &n0);
+      if (lo != f0) {
+        head_wa = f0 * nworkers / W;
+        head_np = n0;
+        head_pages = int((hi < f0 + n0 ? hi : f0 + n0) - lo);
+      }
+      unit_of(locate(S, U, Hkv, hi - 1), S, a.mode, a.part_pages, &f1, &n1);
+      if (hi != f1 + n1 && f1 >= lo) {
+        tail_wa = wid;
+        tail_np = n1;
+        tail_pages = int(hi - f1);
+      }
+    }
+    bool head_in = false, tail_in = false;  // counted in already
+
     // ---- producer cursor (warp-uniform) ----
-    RowPos pc = locate(S, B, Hkv, lo);
+    RowPos pc = locate(S, U, Hkv, lo);
     int64_t px = lo;
     int win_seq = -1, win_base = 0, win_blk = 0;  // lane-held window of 32 block ids
     int p_seg_first = 1;                          // next issued page opens a segment
@@ -267,7 +536,11 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
         win_seq = pc.i;
         win_base = pc.p & ~31;
         const int pp = win_base + lane;
-        win_blk = pp < pc.np ? a.bt[int64_t(pc.i) * a.bt_stride + pp] : 0;
+        // a group's pages are read through its first member's table; a
+        // suffix starts after its group's shared blocks
+        const int trow = CK == kPrefixPass ? __ldg(a.grp_start + pc.i) : pc.i;
+        const int toff = CK == kSuffixPass ? ST[pc.i] : 0;
+        win_blk = pp < pc.np ? a.bt[int64_t(trow) * a.bt_stride + toff + pp] : 0;
       }
       int blk = __shfl_sync(0xffffffffu, win_blk, pc.p - win_base);
       if (unsigned(blk) >= unsigned(a.num_blocks)) {
@@ -280,14 +553,27 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
         const int64_t page_off = (int64_t(blk) * Hkv + pc.g) * C::PAGE;
         // order this warp's earlier shared-memory reads of the stage before the async-proxy refill
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        mbar_arrive_expect_tx(bar, 2 * C::PAGE + (p_seg_first ? C::QBYTES : 0));
-        bulk_g2s(smem_u32(st), kcb + page_off, C::PAGE, bar, pol);
-        bulk_g2s(smem_u32(st + C::PAGE), vcb + page_off, C::PAGE, bar, pol);
-        if (p_seg_first) {
+        if constexpr (CK == kPrefixPass) {
+          // query rows of the group's members (rows past the last member are not loaded)
+          const int s0 = __ldg(a.grp_start + pc.i);
+          const int nq = p_seg_first ? (__ldg(a.grp_start + pc.i + 1) - s0) * a.g_real : 0;
+          mbar_arrive_expect_tx(bar, 2 * C::PAGE + nq * C::QROWB);
+          bulk_g2s(smem_u32(st), kcb + page_off, C::PAGE, bar, pol);
+          bulk_g2s(smem_u32(st + C::PAGE), vcb + page_off, C::PAGE, bar, pol);
+          for (int r = 0; r < nq; ++r)
+            bulk_g2s(smem_u32(st + 2 * C::PAGE + r * C::QROWB),
+                     qg + int64_t(s0 + r / a.g_real) * a.q_sb + int64_t(pc.g * a.g_real + r % a.g_real) * a.q_sh,
+                     C::QROWB, bar, pol);
+        } else {
+          mbar_arrive_expect_tx(bar, 2 * C::PAGE + (p_seg_first ? C::QBYTES : 0));
+          bulk_g2s(smem_u32(st), kcb + page_off, C::PAGE, bar, pol);
+          bulk_g2s(smem_u32(st + C::PAGE), vcb + page_off, C::PAGE, bar, pol);
+          if (p_seg_first) {
 #pragma unroll
-          for (int j = 0; j < G; ++j)
-            bulk_g2s(smem_u32(st + 2 * C::PAGE + j * C::QROWB),
-                     qg + int64_t(pc.i) * a.q_sb + int64_t(pc.g * G + j) * a.q_sh, C::QROWB, bar, pol);
+            for (int j = 0; j < G; ++j)
+              bulk_g2s(smem_u32(st + 2 * C::PAGE + j * C::QROWB),
+                       qg + int64_t(pc.i) * a.q_sb + int64_t(pc.g * G + j) * a.q_sh, C::QROWB, bar, pol);
+          }
         }
       }
       // advance the producer cursor
@@ -301,8 +587,8 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
           pc.g = 0;
           do {
             ++pc.i;
-          } while (pc.i < B && S[pc.i + 1] == S[pc.i]);
-          if (pc.i < B) pc.np = (S[pc.i + 1] - S[pc.i]) / Hkv;
+          } while (pc.i < U && S[pc.i + 1] == S[pc.i]);
+          if (pc.i < U) pc.np = (S[pc.i + 1] - S[pc.i]) / Hkv;
         }
       } else if (a.mode == kFixed && pc.p % a.part_pages == 0) {
         p_seg_first = 1;
@@ -313,7 +599,7 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
     for (int s = 0; s < npre; ++s) issue(s);
 
     // ---- consumer state ----
-    RowPos cc = locate(S, B, Hkv, lo);
+    RowPos cc = locate(S, U, Hkv, lo);
     int64_t cx = lo;
     int seg_p0 = cc.p;
     bool seg_first = true;
@@ -339,6 +625,7 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
     float sfac[2];       // power-of-two factor undoing the query's range normalisation
     float vscale = 1.f;
     int ctx_i = 0;
+    int nreal = G;       // query rows that belong to a sequence (prefix pass: members x g_real)
     uint32_t phase = 0;  // bit s = parity of the next wait on stage s
     int s = 0;
 
@@ -352,6 +639,12 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
           const int s2 = int((s + (y - cx)) % a.stages);
           mbar_wait_bounded(smem_u32(&bars[s2]), (phase >> s2) & 1u, a.timeout_ns);
         }
+        // count the unfinished shares in (their rows are left unwritten; the
+        // status word reports the timeout) so the counters end at zero
+        if (lane == 0) {
+          if (head_wa >= 0 && !head_in) count_in(a.ws_cnt + head_wa, unsigned(head_pages), unsigned(head_np));
+          if (tail_wa >= 0 && !tail_in) count_in(a.ws_cnt + tail_wa, unsigned(tail_pages), unsigned(tail_np));
+        }
         return;
       }
       phase ^= 1u << s;
@@ -361,9 +654,10 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
         // FP8 cache: fold the K dequantization scale into the query
         const float qscale = a.scale_log2 * (a.k_scale ? __ldg(a.k_scale + cc.g) : 1.f);
         vscale = a.v_scale ? __ldg(a.v_scale + cc.g) : 1.f;
+        if constexpr (CK == kPrefixPass) nreal = (__ldg(a.grp_start + cc.i + 1) - __ldg(a.grp_start + cc.i)) * a.g_real;
         if constexpr (kMma) {
           float qv[32];
-          if (gr < G) {
+          if (gr < nreal) {
 #pragma unroll
             for (int v = 0; v < 4; ++v) Elem<Tq>::unpack(qs[gr * (C::QROWB / 16) + tig * 4 + v], qv + 8 * v);
           } else {
@@ -404,8 +698,13 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
 #pragma unroll
         for (int j = 0; j < G; ++j) {
           float f[EPV];
+          if (CK != kPrefixPass || j < nreal) {
 #pragma unroll
-          for (int v = 0; v < QV; ++v) Elem<Tq>::unpack(qs[j * (C::QROWB / 16) + c * QV + v], f + v * EPQ);
+            for (int v = 0; v < QV; ++v) Elem<Tq>::unpack(qs[j * (C::QROWB / 16) + c * QV + v], f + v * EPQ);
+          } else {
+#pragma unroll
+            for (int e = 0; e < EPV; ++e) f[e] = 0.f;  // a row past the group's last member
+          }
 #pragma unroll
           for (int e = 0; e < EPV; ++e) {
             q[j][e] = f[e] * qscale;
@@ -416,7 +715,13 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
 #pragma unroll
         for (int jj = 0; jj < GH; ++jj) lpart[jj] = 0.f;
         }
-        ctx_i = clamp_ctx(a.ctx[cc.i], ctx_cap);  // consumed at the row's last page
+        // tokens of the row, consumed at its last page
+        if constexpr (CK == kPrefixPass)
+          ctx_i = cc.np * kBS;  // shared blocks are full
+        else if constexpr (CK == kSuffixPass)
+          ctx_i = clamp_ctx(a.ctx[cc.i], ctx_cap) - ST[cc.i] * kBS;
+        else
+          ctx_i = clamp_ctx(a.ctx[cc.i], ctx_cap);
         seg_p0 = cc.p;
       }
       const bool last_of_row = (cc.p == cc.np - 1);
@@ -703,21 +1008,60 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
           }
         }
         }
-        const bool whole_row = (seg_p0 == 0) && last_of_row;
-        if (whole_row) {
-          if (tg == 0) {
-            Tq* ob = reinterpret_cast<Tq*>(a.out) + int64_t(cc.i) * a.o_sb;
+        // This segment's unit: the row, or in fixed mode its partition.  A
+        // unit that spans the whole row gives the row's output; a partition
+        // of a longer row gives a partial for the merge kernel.
+        const int up0 = a.mode == kFixed ? (cc.p / a.part_pages) * a.part_pages : 0;
+        const int unp = a.mode == kFixed ? min(a.part_pages, cc.np - up0) : cc.np;
+        const bool row_unit = unp == cc.np;
+        const bool whole_unit = seg_p0 == up0 && cc.p == up0 + unp - 1;
+        if (whole_unit && row_unit) {
+          if constexpr (CK == kPrefixPass) {
+            // the group's partial result for each member's heads
+            const int s0 = __ldg(a.grp_start + cc.i);
 #pragma unroll
             for (int j = 0; j < G; ++j) {
-              const float inv = vscale / lall[j];
-              float f[EPV];
+              if (j >= nreal) continue;
+              const int64_t rowx = int64_t(s0 + j / a.g_real) * H + cc.g * a.g_real + j % a.g_real;
+              if (tg == 0) {
+                const float inv = vscale / lall[j];
+                float4* dst = reinterpret_cast<float4*>(a.pre_o + rowx * D + c * EPV);
 #pragma unroll
-              for (int e = 0; e < EPV; ++e) f[e] = o[j][e] * inv;
-              store_out<Tq, EPV>(ob + int64_t(cc.g * G + j) * a.o_sh + c * EPV, f);
+                for (int e4 = 0; e4 < EPV / 4; ++e4)
+                  dst[e4] = make_float4(o[j][4 * e4] * inv, o[j][4 * e4 + 1] * inv, o[j][4 * e4 + 2] * inv,
+                                        o[j][4 * e4 + 3] * inv);
+              }
+              if (lane == 0) a.pre_lse[rowx] = (m[j] + log2f(lall[j])) * 0.69314718055994530942f;
+            }
+          } else {
+            const bool has_pre = CK == kSuffixPass && ST[cc.i] > 0;
+            if (tg == 0) {
+              Tq* ob = reinterpret_cast<Tq*>(a.out) + int64_t(cc.i) * a.o_sb;
+#pragma unroll
+              for (int j = 0; j < G; ++j) {
+                const float inv = vscale / lall[j];
+                float f[EPV];
+                if (has_pre) {
+                  // merge with the shared prefix's partial by log-sum-exp
+                  const int64_t rowx = int64_t(cc.i) * H + cc.g * G + j;
+                  const float lr = (m[j] + log2f(lall[j])) * 0.69314718055994530942f;
+                  const float lp = a.pre_lse[rowx];
+                  const float mx = fmaxf(lr, lp);
+                  const float wr = ex2((lr - mx) * 1.4426950408889634f), wp = ex2((lp - mx) * 1.4426950408889634f);
+                  const float r = 1.f / (wr + wp);
+                  const float* po = a.pre_o + rowx * D + c * EPV;
+#pragma unroll
+                  for (int e = 0; e < EPV; ++e) f[e] = (wr * (o[j][e] * inv) + wp * po[e]) * r;
+                } else {
+#pragma unroll
+                  for (int e = 0; e < EPV; ++e) f[e] = o[j][e] * inv;
+                }
+                store_out<Tq, EPV>(ob + int64_t(cc.g * G + j) * a.o_sh + c * EPV, f);
+              }
             }
           }
-        } else if (a.mode == kFixed) {
-          // one partial per partition; a separate kernel merges them
+        } else if (whole_unit) {
+          // fixed mode: one partial per partition; a separate kernel merges them
           const int64_t base = (int64_t(cc.i) * H + int64_t(cc.g) * G) * a.P_max + cc.p / a.part_pages;
           if (tg == 0) {
 #pragma unroll
@@ -740,14 +1084,21 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
               }
             a.ws_lse[base + lane * a.P_max] = (mj + log2f(lj)) * 0.69314718055994530942f;
           }
-        } else if (seg_p0 != 0) {
-          // Balanced mode, a row that began in an earlier worker: publish this
-          // share (normalised output + log-sum-exp), then the call tag.
+        } else {
+          // A unit cut by a worker boundary: publish this worker's share
+          // (normalised output + log-sum-exp) in its slot, then count its
+          // pages in.  The worker whose pages complete the unit merges all
+          // shares in worker order and writes the row (or the partition's
+          // partial).
+          const int64_t unit_first = int64_t(S[cc.i]) + int64_t(cc.g) * cc.np + up0;
+          const int64_t wa = unit_first * nworkers / W;
+          const bool is_tail = (seg_p0 == up0);
+          const int64_t slot = 2 * wid + (is_tail ? 1 : 0);
           if (tg == 0) {
 #pragma unroll
             for (int j = 0; j < G; ++j) {
               const float inv = vscale / lall[j];
-              float4* dst = reinterpret_cast<float4*>(a.ws_o + (wid * G + j) * D + c * EPV);
+              float4* dst = reinterpret_cast<float4*>(a.sh_o + (slot * G + j) * D + c * EPV);
 #pragma unroll
               for (int e4 = 0; e4 < EPV / 4; ++e4)
                 dst[e4] = make_float4(o[j][4 * e4] * inv, o[j][4 * e4 + 1] * inv, o[j][4 * e4 + 2] * inv,
@@ -762,66 +1113,57 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
                 mj = m[j];
                 lj = lall[j];
               }
-            a.ws_lse[wid * G + lane] = (mj + log2f(lj)) * 0.69314718055994530942f;
+            a.sh_lse[slot * G + lane] = (mj + log2f(lj)) * 0.69314718055994530942f;
           }
-          __syncwarp();
-          if (lane == 0) {
-            __threadfence();
-            st_release_u64(a.ws_flag + wid, a.call_tag);
-          }
-        } else {
-          // Balanced mode, a row that began here and continues in later
-          // workers.  This is the last segment of this worker's range; the
-          // later workers published their shares at the start (or, for a
-          // range inside the row, the end) of theirs.  Merge them into this
-          // share by log-sum-exp and write the row.
-          const int64_t row_last = int64_t(S[cc.i]) + int64_t(cc.g) * cc.np + cc.np - 1;
-          const int64_t wb = row_last * nworkers / W;
-          float mx[G], wsum[G], acc[G][EPV];
+          const bool last = share_done(a.ws_cnt + wa, cc.p - seg_p0 + 1, unp);
+          if (is_tail)
+            tail_in = true;
+          else
+            head_in = true;
+          if (last) {
+            constexpr int PER = D / 32;
+            const int64_t wb = (unit_first + unp - 1) * nworkers / W;
+            float acc[G][PER], lse_m[G];
+            merge_shares<D, G>(a.sh_o, a.sh_lse, wa, wb, W, nworkers, acc, lse_m);
+            if (!row_unit) {
+              // the partition's partial, as if one worker had reduced it
+              const int64_t base = (int64_t(cc.i) * H + int64_t(cc.g) * G) * a.P_max + up0 / a.part_pages;
 #pragma unroll
-          for (int j = 0; j < G; ++j) {
-            mx[j] = (m[j] + log2f(lall[j])) * 0.69314718055994530942f;
-            wsum[j] = 1.f;
-            const float inv = vscale / lall[j];
+              for (int j = 0; j < G; ++j) {
+                float* dst = a.ws_o + (base + j * a.P_max) * D + lane * PER;
 #pragma unroll
-            for (int e = 0; e < EPV; ++e) acc[j][e] = o[j][e] * inv;
-          }
-          for (int64_t k = wid + 1; k <= wb; ++k) {
-            const int64_t klo = (k * W + nworkers - 1) / nworkers;
-            const int64_t khi = ((k + 1) * W + nworkers - 1) / nworkers;
-            if (klo == khi) continue;  // an empty worker holds no share
-            if (lane == 0) wait_flag_bounded(a.ws_flag + k, a.call_tag, a.timeout_ns);
-            __syncwarp();
-#pragma unroll
-            for (int j = 0; j < G; ++j) {
-              const float lk = __ldcg(a.ws_lse + k * G + j);
-              const float mn = fmaxf(mx[j], lk);
-              const float sc = ex2((mx[j] - mn) * 1.4426950408889634f);
-              const float wk = ex2((lk - mn) * 1.4426950408889634f);
-              mx[j] = mn;
-              wsum[j] = wsum[j] * sc + wk;
-              if (tg == 0) {
-                const float4* src = reinterpret_cast<const float4*>(a.ws_o + (k * G + j) * D + c * EPV);
-#pragma unroll
-                for (int e4 = 0; e4 < EPV / 4; ++e4) {
-                  const float4 v = __ldcg(src + e4);
-                  acc[j][4 * e4 + 0] = fmaf(wk, v.x, acc[j][4 * e4 + 0] * sc);
-                  acc[j][4 * e4 + 1] = fmaf(wk, v.y, acc[j][4 * e4 + 1] * sc);
-                  acc[j][4 * e4 + 2] = fmaf(wk, v.z, acc[j][4 * e4 + 2] * sc);
-                  acc[j][4 * e4 + 3] = fmaf(wk, v.w, acc[j][4 * e4 + 3] * sc);
-                }
+                for (int e = 0; e < PER; ++e) dst[e] = acc[j][e];
+                if (lane == 0) a.ws_lse[base + j * a.P_max] = lse_m[j];
               }
-            }
-          }
-          if (tg == 0) {
-            Tq* ob = reinterpret_cast<Tq*>(a.out) + int64_t(cc.i) * a.o_sb;
+            } else if constexpr (CK == kPrefixPass) {
+              const int s0 = __ldg(a.grp_start + cc.i);
 #pragma unroll
-            for (int j = 0; j < G; ++j) {
-              const float inv = 1.f / wsum[j];
-              float f[EPV];
+              for (int j = 0; j < G; ++j) {
+                if (j >= nreal) continue;
+                const int64_t rowx = int64_t(s0 + j / a.g_real) * H + cc.g * a.g_real + j % a.g_real;
+                float* dst = a.pre_o + rowx * D + lane * PER;
 #pragma unroll
-              for (int e = 0; e < EPV; ++e) f[e] = acc[j][e] * inv;
-              store_out<Tq, EPV>(ob + int64_t(cc.g * G + j) * a.o_sh + c * EPV, f);
+                for (int e = 0; e < PER; ++e) dst[e] = acc[j][e];
+                if (lane == 0) a.pre_lse[rowx] = lse_m[j];
+              }
+            } else {
+              const bool has_pre = CK == kSuffixPass && ST[cc.i] > 0;
+              Tq* ob = reinterpret_cast<Tq*>(a.out) + int64_t(cc.i) * a.o_sb + lane * PER;
+#pragma unroll
+              for (int j = 0; j < G; ++j) {
+                if (has_pre) {
+                  const int64_t rowx = int64_t(cc.i) * H + cc.g * G + j;
+                  const float lp = a.pre_lse[rowx];
+                  const float mx = fmaxf(lse_m[j], lp);
+                  const float wr = ex2((lse_m[j] - mx) * 1.4426950408889634f);
+                  const float wp = ex2((lp - mx) * 1.4426950408889634f);
+                  const float r = 1.f / (wr + wp);
+                  const float* po = a.pre_o + rowx * D + lane * PER;
+#pragma unroll
+                  for (int e = 0; e < PER; ++e) acc[j][e] = (wr * acc[j][e] + wp * po[e]) * r;
+                }
+                store_out_small<Tq, PER>(ob + int64_t(cc.g * G + j) * a.o_sh, acc[j]);
+              }
             }
           }
         }
@@ -836,83 +1178,123 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
           cc.g = 0;
           do {
             ++cc.i;
-          } while (cc.i < B && S[cc.i + 1] == S[cc.i]);
-          if (cc.i < B) cc.np = (S[cc.i + 1] - S[cc.i]) / Hkv;
+          } while (cc.i < U && S[cc.i + 1] == S[cc.i]);
+          if (cc.i < U) cc.np = (S[cc.i + 1] - S[cc.i]) / Hkv;
         }
       }
       if (++s == a.stages) s = 0;
     }
   }
 
-  // ---- sequences with no context: zero output rows ----
-  for (int64_t i = wid; i < B; i += nworkers) {
-    if (S[i + 1] != S[i]) continue;
-    Tq* ob = reinterpret_cast<Tq*>(a.out) + i * a.o_sb;
-    constexpr int OVR = C::QROWB / 16;  // 16-byte vectors per output row
-    for (int idx = lane; idx < H * OVR; idx += 32) {
-      const int h = idx / OVR, cc2 = idx % OVR;
-      *reinterpret_cast<uint4*>(ob + int64_t(h) * a.o_sh + cc2 * EPQ) = make_uint4(0, 0, 0, 0);
+  // ---- sequences with no pages in this launch: zero output rows (no
+  // context), or, after a shared prefix with nothing past it, its result ----
+  if constexpr (CK != kPrefixPass) {
+    for (int64_t i = wid; i < a.B; i += nworkers) {
+      if (S[i + 1] != S[i]) continue;
+      const bool has_pre = CK == kSuffixPass && ST[i] > 0;
+      Tq* ob = reinterpret_cast<Tq*>(a.out) + i * a.o_sb;
+      constexpr int OVR = C::QROWB / 16;  // 16-byte vectors per output row
+      for (int idx = lane; idx < H * OVR; idx += 32) {
+        const int h = idx / OVR, cc2 = idx % OVR;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (has_pre) {
+          float f[EPQ];
+          const float* po = a.pre_o + (i * H + h) * D + cc2 * EPQ;
+#pragma unroll
+          for (int e = 0; e < EPQ; ++e) f[e] = po[e];
+          v = Elem<Tq>::pack(f);
+        }
+        *reinterpret_cast<uint4*>(ob + int64_t(h) * a.o_sh + cc2 * EPQ) = v;
+      }
     }
   }
 }
 
 // ---- log-sum-exp merge of partial results ----------------------------------
 // out = sum_p exp(lse_p - LSE) o_p, LSE = log sum_p exp(lse_p), with o_p the
-// normalised partial outputs.  One warp merges one (sequence, query head).
-// Fixed partitions: one warp per (sequence, query head) with > 1 partition.
-// Each lane walks the partitions with a running max (one pass).
+// normalised partial outputs of fixed partitions.  One CTA of kMergeWarps
+// warps per (sequence, query head) with more than one partition: warp w
+// takes partitions w, w + kMergeWarps, ...; lanes first find the warp's
+// largest lse, then weight 32 partitions at a time and broadcast the
+// weights while every lane streams its dims (several partitions' loads in
+// flight); the warps' results are combined through shared memory in warp
+// order (a fixed order, so the result does not depend on timing).
+constexpr int kMergeWarps = 8;
+
 template <typename T, int D>
-__global__ void __launch_bounds__(256) merge_fixed_kernel(const DecodeArgs a, int part_tokens) {
+__global__ void __launch_bounds__(kMergeWarps * 32) merge_fixed_kernel(const DecodeArgs a, int part_tokens) {
   pdl_wait();
   constexpr int PER = D / 32;
-  const int lane = threadIdx.x & 31;
-  const int64_t task = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (task >= int64_t(a.B) * a.H) return;
-  const int i = int(task / a.H), h = int(task % a.H);
+  constexpr int NW = kMergeWarps;
+  constexpr float kLog2e = 1.4426950408889634f;
+  __shared__ float sm_m[NW], sm_w[NW];
+  __shared__ __align__(16) float sm_acc[NW][D];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t row = blockIdx.x;  // (sequence, query head)
+  if (row >= int64_t(a.B) * a.H) return;
+  const int i = int(row / a.H), h = int(row % a.H);
   const int ctx = clamp_ctx(a.ctx[i], a.max_nb * kBS);
   const int np = (ctx + part_tokens - 1) / part_tokens;
-  if (np <= 1) return;
-  const int64_t row = int64_t(i) * a.H + h;
+  if (np <= 1) return;  // the decode kernel wrote this row itself
   const float* lse = a.ws_lse + row * a.P_max;
   const float* ob = a.ws_o + row * a.P_max * D;
-  float mx = -INFINITY, wsum = 0.f;
-  float acc[PER];
+  const int mine = np > warp ? (np - warp + NW - 1) / NW : 0;  // partitions of this warp
+  float mw = -INFINITY;
+  for (int t = lane; t < mine; t += 32) mw = fmaxf(mw, __ldcg(lse + warp + NW * t));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mw = fmaxf(mw, __shfl_xor_sync(0xffffffffu, mw, o));
+  float acc[PER], wsum = 0.f;
 #pragma unroll
   for (int e = 0; e < PER; ++e) acc[e] = 0.f;
-  for (int p = 0; p < np; ++p) {
-    const float l = lse[p];
-    const float mn = fmaxf(mx, l);
-    const float sc = ex2((mx - mn) * 1.4426950408889634f);
-    const float w = ex2((l - mn) * 1.4426950408889634f);
-    mx = mn;
-    wsum = wsum * sc + w;
-    const float* src = ob + int64_t(p) * D + lane * PER;
-    float v[PER];
-    if constexpr (PER == 4) {
-      const float4 v4 = *reinterpret_cast<const float4*>(src);
-      v[0] = v4.x, v[1] = v4.y, v[2] = v4.z, v[3] = v4.w;
-    } else {
-      const float2 v2 = *reinterpret_cast<const float2*>(src);
-      v[0] = v2.x, v[1] = v2.y;
-    }
+  for (int c0 = 0; c0 < mine; c0 += 32) {
+    const int tl = c0 + lane;
+    const float wl = tl < mine ? ex2((__ldcg(lse + warp + NW * tl) - mw) * kLog2e) : 0.f;
+    const int n = mine - c0 < 32 ? mine - c0 : 32;
+#pragma unroll 4
+    for (int t = 0; t < n; ++t) {
+      const float w = __shfl_sync(0xffffffffu, wl, t);
+      const float* src = ob + int64_t(warp + NW * (c0 + t)) * D + lane * PER;
+      float v[PER];
+      if constexpr (PER == 4) {
+        const float4 v4 = __ldcg(reinterpret_cast<const float4*>(src));
+        v[0] = v4.x, v[1] = v4.y, v[2] = v4.z, v[3] = v4.w;
+      } else {
+        const float2 v2 = __ldcg(reinterpret_cast<const float2*>(src));
+        v[0] = v2.x, v[1] = v2.y;
+      }
+      wsum += w;
 #pragma unroll
-    for (int e = 0; e < PER; ++e) acc[e] = fmaf(w, v[e], acc[e] * sc);
+      for (int e = 0; e < PER; ++e) acc[e] = fmaf(w, v[e], acc[e]);
+    }
   }
-  const float inv = 1.f / wsum;
+  if (lane == 0) {
+    sm_m[warp] = mw;
+    sm_w[warp] = wsum;
+  }
+#pragma unroll
+  for (int e = 0; e < PER; ++e) sm_acc[warp][lane * PER + e] = acc[e];
+  __syncthreads();
+  if (warp != 0) return;
+  float M = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < NW; ++w)
+    if (sm_w[w] > 0.f) M = fmaxf(M, sm_m[w]);
+  float tot = 0.f, f[PER];
+#pragma unroll
+  for (int e = 0; e < PER; ++e) f[e] = 0.f;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) {
+    if (!(sm_w[w] > 0.f)) continue;
+    const float sc = ex2((sm_m[w] - M) * kLog2e);
+    tot += sc * sm_w[w];
+#pragma unroll
+    for (int e = 0; e < PER; ++e) f[e] = fmaf(sc, sm_acc[w][lane * PER + e], f[e]);
+  }
+  const float inv = 1.f / tot;
+#pragma unroll
+  for (int e = 0; e < PER; ++e) f[e] *= inv;
   T* dst = reinterpret_cast<T*>(a.out) + int64_t(i) * a.o_sb + int64_t(h) * a.o_sh + lane * PER;
-  float f[PER];
-#pragma unroll
-  for (int e = 0; e < PER; ++e) f[e] = acc[e] * inv;
-  if constexpr (sizeof(T) == 4) {
-#pragma unroll
-    for (int e = 0; e < PER; ++e) reinterpret_cast<float*>(dst)[e] = f[e];
-  } else {
-#pragma unroll
-    for (int e = 0; e < PER; e += 2) {
-      __nv_bfloat162 hh = __floats2bfloat162_rn(f[e], f[e + 1]);
-      *reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(dst) + e) = hh;
-    }
-  }
+  store_out_small<T, PER>(dst, f);
 }
 
 }  // namespace pa
