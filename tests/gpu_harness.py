@@ -151,7 +151,7 @@ def decode_on_device(st: DeviceState, query: torch.Tensor, partition_tokens: int
         out = torch.empty_like(query)
     n = pa.pa_decode_workspace_bytes(st.plan.B, w.num_heads, w.num_kv_heads, w.head_size,
                                      st.block_tables.shape[1], partition_tokens)
-    ws = torch.empty(max(n, 256), dtype=torch.uint8, device=query.device) if n else None
+    ws = torch.zeros(max(n, 256), dtype=torch.uint8, device=query.device) if n else None
     if st.k_scale is not None:
         pa.pa_decode_fp8(out, query, st.k_cache, st.v_cache, st.block_tables, st.context_lens,
                          1.0 / np.sqrt(w.head_size), w.num_kv_heads, st.k_scale, st.v_scale, workspace=ws,

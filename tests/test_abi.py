@@ -142,6 +142,37 @@ def test_decode_validation():
                  stream=0)
 
 
+def test_decode_cascade_validation():
+    """Shared-prefix decode: argument errors are reported before any CUDA
+    call (the group tensors, the group width, the split mode, the dtype)."""
+    kc, vc = _cache(hk=2), _cache(hk=2)
+    B, H = 4, 2
+    q = torch.empty(B, H, 128, dtype=torch.bfloat16)
+    out = torch.empty_like(q)
+    bt = torch.zeros(B, 4, dtype=torch.int32)
+    cl = torch.zeros(B, dtype=torch.int32)
+    gs = torch.tensor([0, 2, 4], dtype=torch.int32)
+    gb = torch.tensor([1, 0], dtype=torch.int32)
+    raw = torch.zeros((1 << 20) + 256, dtype=torch.uint8)
+    ws = raw[(-raw.data_ptr()) % 256:][: 1 << 20]  # 256-byte aligned, as the workspace must be
+    f = pa.pa_decode_cascade
+    _expect(UNSUPPORTED, f, out, q, kc, vc, bt, cl, gs, gb, 3, 0.1, 2, ws, stream=0)  # G x 3 = 3 rows
+    _expect(INVALID, f, out, q, kc, vc, bt, cl, gs, gb, 0, 0.1, 2, ws, stream=0)  # no member
+    _expect(INVALID, f, out, q, kc, vc, bt, cl, gs[:2], gb, 2, 0.1, 2, ws, stream=0)  # [n_groups + 1]
+    _expect(INVALID, f, out, q, kc, vc, bt, cl, gs.long(), gb, 2, 0.1, 2, ws, stream=0)
+    _expect(INVALID, f, out, q, kc, vc, bt, cl, gs, gb[:0], 2, 0.1, 2, ws, stream=0)  # no group
+    _expect(UNSUPPORTED, f, out, q, kc, vc, bt, cl, gs, gb, 2, 0.1, 2, ws, partition_tokens=512, stream=0)
+    _expect(INVALID, f, out, q, kc, vc, bt, cl, gs, gb, 2, 0.1, 4, ws, stream=0)  # num_kv_heads mismatch
+    k8, v8 = _cache(hk=2, dtype=torch.float8_e4m3fn), _cache(hk=2, dtype=torch.float8_e4m3fn)
+    _expect(UNSUPPORTED, f, out, q, k8, v8, bt, cl, gs, gb, 2, 0.1, 2, ws, stream=0)
+    q64 = torch.empty(B, H, 64, dtype=torch.bfloat16)
+    _expect(UNSUPPORTED, f, torch.empty_like(q64), q64, _cache(hk=2, d=64), _cache(hk=2, d=64), bt, cl, gs, gb, 2,
+            0.1, 2, ws, stream=0)  # bf16 at head size 64 has no shared-prefix kernels
+    _expect(UNSUPPORTED, pa.pa_decode_cascade_workspace_bytes, B, H, 2, 128, 3)
+    _expect(UNSUPPORTED, pa.pa_decode_cascade_workspace_bytes, B, H, 2, 128, 2, 512)
+    _expect(INVALID, pa.pa_decode_cascade_workspace_bytes, B, H, 2, 128, 0)
+
+
 def test_prefill_validation():
     kc, vc = _cache(hk=2), _cache(hk=2)
     B, T, H = 3, 10, 8
@@ -209,11 +240,17 @@ def test_device_of_a_call():
         _on_device([on(0), on(1)])
 
 
-def test_fixed_workspace_size():
-    n = pa.pa_decode_workspace_bytes(8, 32, 8, 128, 8192, 512)
-    P = 8192 * 16 // 512
-    assert n == 8 * 32 * P * 128 * 4 + 8 * 32 * P * 4
+def test_workspace_size_without_a_device():
+    """No split needs no workspace; the split modes size their share slots
+    by the device's SM count, so without a device they report PA_ERR_CUDA
+    (and bad arguments are still reported first)."""
+    assert pa.PA_DECODE_WS_HEADER_BYTES == 64 * 1024
     assert pa.pa_decode_workspace_bytes(8, 32, 8, 128, 8192, -1) == 0
+    _expect(INVALID, pa.pa_decode_workspace_bytes, 8, 32, 8, 128, 8192, 100)
+    _expect(INVALID, pa.pa_decode_workspace_bytes, 8, 30, 8, 128, 8192, 0)
+    if not torch.cuda.is_available():
+        _expect(4, pa.pa_decode_workspace_bytes, 8, 32, 8, 128, 8192, 512)
+        _expect(4, pa.pa_decode_workspace_bytes, 8, 32, 8, 128, 8192, 0)
 
 
 # ---------------------------------------------------------------------------

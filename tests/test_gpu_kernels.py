@@ -82,7 +82,7 @@ class Case:
         if out is None:
             out = torch.empty(len(self.ctxs), self.H, self.D, dtype=TORCH_DTYPE[self.dtype], device=DEV)
         n = pa.pa_decode_workspace_bytes(len(self.ctxs), self.H, self.Hkv, self.D, self.max_nb, partition_tokens)
-        self.ws = torch.empty(n + ws_extra + 256, dtype=torch.uint8, device=DEV) if n else None
+        self.ws = torch.zeros(n + ws_extra + 256, dtype=torch.uint8, device=DEV) if n else None
         pa.pa_decode(out, self.qd, self.kc, self.vc, self.bt, self.cl, self.scale, self.Hkv, workspace=self.ws,
                      partition_tokens=partition_tokens)
         torch.cuda.synchronize()
@@ -236,7 +236,7 @@ def test_fixed_partitions_leave_oracle_partials():
     P = -(-c.max_nb * 16 // part)
     nbytes_o = B * H * P * D * 4
     off_lse = (nbytes_o + 255) // 256 * 256
-    ws = c.ws
+    ws = c.ws[pa.PA_DECODE_WS_HEADER_BYTES:]  # after the header of merge counters
     o = ws[:nbytes_o].view(torch.float32).view(B, H, P, D).cpu().numpy()
     lse = ws[off_lse:off_lse + B * H * P * 4].view(torch.float32).view(B, H, P).cpu().numpy()
     for i, ctx in enumerate(ctxs):
@@ -249,6 +249,18 @@ def test_fixed_partitions_leave_oracle_partials():
         oo, ll = partition_partials(widen(c.q[i], "bf16"), k, v, c.scale, part)
         assert np.max(np.abs(o[i, :, :npart].transpose(1, 0, 2) - oo)) < 2e-5
         assert np.max(np.abs(lse[i, :, :npart].T - ll)) < 2e-5
+
+
+def test_fixed_workspace_layout():
+    """The fixed-partition workspace: the merge-counter header, o[B][H][P][D]
+    and lse[B][H][P] (fp32, each rounded up to 256 bytes), then two share
+    slots per worker for partitions cut between workers."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    n = pa.pa_decode_workspace_bytes(8, 32, 8, 128, 8192, 512)
+    P = 8192 * 16 // 512
+    workers = sms * 12  # G = 4: 12 warps per SM
+    shares = 2 * workers * 4 * 128 * 4 + (2 * workers * 4 * 4 + 255) // 256 * 256
+    assert n == pa.PA_DECODE_WS_HEADER_BYTES + 8 * 32 * P * 128 * 4 + 8 * 32 * P * 4 + shares
 
 
 def test_nosplit_is_bitwise_invariant_to_launch_shape():
@@ -265,14 +277,54 @@ def test_nosplit_is_bitwise_invariant_to_launch_shape():
 
 
 def test_balanced_split_under_other_launch_shapes():
+    """The balanced split under other launch shapes, including grids of 4 and
+    8 CTAs per SM that cannot all be resident at once (each CTA takes most of
+    an SM's shared memory, so they run in waves): no worker waits for
+    another, so every shape gives a correct result, the same bits on a second
+    call, and leaves the workspace's merge counters at zero."""
     c = Case(42, [3000, 5, 900, 4096, 1], 32, 8, 128, "bf16")
     try:
-        for warps, stages, ctas in ((8, 3, 1), (4, 2, 2), (1, 1, 1), (8, 1, 4)):
+        for warps, stages, ctas in ((8, 3, 1), (4, 2, 2), (1, 1, 1), (8, 1, 4), (12, 2, 8)):
             pa.pa_set_decode_tuning(warps, stages, ctas)
-            assert c.err(c.run(0)) <= TOL["bf16"], (warps, stages, ctas)
+            first = c.run(0).clone()
+            assert c.err(first) <= TOL["bf16"], (warps, stages, ctas)
+            assert torch.equal(c.run(0).view(torch.int16), first.view(torch.int16)), (warps, stages, ctas)
             check_status_clean()
+            assert int(c.ws[:pa.PA_DECODE_WS_HEADER_BYTES].count_nonzero()) == 0
     finally:
         pa.pa_set_decode_tuning(0, 0, 0)
+
+
+def test_balanced_split_replays_from_a_cuda_graph():
+    """A captured balanced-split decode replayed with new queries: each
+    replay must equal a direct call on the same query (the merge counters
+    are reset by the worker that completes each row, so a replay starts
+    from zero like a fresh call)."""
+    c = Case(45, [3000, 5, 900, 4096, 1, 700], 32, 8, 128, "bf16")
+    n = pa.pa_decode_workspace_bytes(len(c.ctxs), c.H, c.Hkv, c.D, c.max_nb, 0)
+    ws = torch.zeros(n, dtype=torch.uint8, device=DEV)
+    q_static = c.qd.clone()
+    out = torch.empty_like(q_static)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        pa.pa_decode(out, q_static, c.kc, c.vc, c.bt, c.cl, c.scale, c.Hkv, workspace=ws, stream=s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        pa.pa_decode(out, q_static, c.kc, c.vc, c.bt, c.cl, c.scale, c.Hkv, workspace=ws, stream=s)
+    gen = torch.Generator(device="cpu").manual_seed(3)
+    for _ in range(3):
+        q_new = torch.randn(q_static.shape, generator=gen).to(torch.bfloat16).to(DEV)
+        q_static.copy_(q_new)
+        g.replay()
+        torch.cuda.synchronize()
+        ref = torch.empty_like(out)
+        ws2 = torch.zeros(n, dtype=torch.uint8, device=DEV)
+        pa.pa_decode(ref, q_new, c.kc, c.vc, c.bt, c.cl, c.scale, c.Hkv, workspace=ws2)
+        torch.cuda.synchronize()
+        assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+    check_status_clean()
+    assert int(ws[:pa.PA_DECODE_WS_HEADER_BYTES].count_nonzero()) == 0
 
 
 def test_more_workers_than_pages():

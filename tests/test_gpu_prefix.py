@@ -93,7 +93,7 @@ def test_prefix_cache_reuse_and_eviction():
     q = to_bf16_bits(rng.standard_normal((len(seqs), H, D)).astype(np.float32))
     out = torch.empty(len(seqs), H, D, dtype=torch.bfloat16, device=DEV)
     n = pa.pa_decode_workspace_bytes(len(seqs), H, HK, D, max_nb, 0)
-    ws = torch.empty(n, dtype=torch.uint8, device=DEV)
+    ws = torch.zeros(n, dtype=torch.uint8, device=DEV)
     pa.pa_decode(out, to_device_values(q, "bf16", DEV), kc, vc, torch.from_numpy(tables).to(DEV),
                  torch.from_numpy(lens).to(DEV), 1 / math.sqrt(D), HK, workspace=ws)
     check_status_clean()

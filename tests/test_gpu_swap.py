@@ -84,7 +84,7 @@ def test_swap_out_reuse_swap_in_decode():
                                                                                         dev_o.v_page(b)[:, wr])
     q = to_bf16_bits(rng.standard_normal((len(live), H, D)).astype(np.float32))
     out = torch.empty(len(live), H, D, dtype=torch.bfloat16, device=DEV)
-    ws = torch.empty(pa.pa_decode_workspace_bytes(len(live), H, HK, D, max_nb, 0), dtype=torch.uint8, device=DEV)
+    ws = torch.zeros(pa.pa_decode_workspace_bytes(len(live), H, HK, D, max_nb, 0), dtype=torch.uint8, device=DEV)
     pa.pa_decode(out, to_device_values(q, "bf16", DEV), kc, vc, torch.from_numpy(tables).to(DEV),
                  torch.from_numpy(lens).to(DEV), 1 / math.sqrt(D), HK, workspace=ws)
     check_status_clean()

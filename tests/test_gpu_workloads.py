@@ -91,6 +91,31 @@ def test_parallel_sampling_13b():
     assert len(st.cow_pairs) == 3 * sum(1 for n in plen if n % 16)
 
 
+def test_parallel_sampling_13b_shared_prefix():
+    """The sampling workload through the shared-prefix decode: groups from
+    the library's allocator (each prompt's 4 samples share its full
+    blocks), every row against the oracle, in both split modes."""
+    plan = make_plan("parallel_sampling_13b")
+    st = build_device_state(plan)
+    w = plan.workload
+    gs, gb = st.alloc.prefix_groups(plan.batch, 4)
+    assert len(gb) == 64 and list(np.diff(gs)) == [4] * 64 and (gb > 0).all()
+    _, cache_o, _ = replay(plan)
+    q = device_query(plan)
+    ref = paged_decode_rows(query_values(plan), cache_o, st.tables_host, st.lens_host,
+                            1.0 / math.sqrt(w.head_size), range(plan.B))
+    gsd, gbd = torch.from_numpy(gs).cuda(), torch.from_numpy(gb).cuda()
+    for mode in (0, -1):
+        n = pa.pa_decode_cascade_workspace_bytes(plan.B, w.num_heads, w.num_kv_heads, w.head_size, 4, mode)
+        ws = torch.zeros(n, dtype=torch.uint8, device="cuda")
+        out = torch.empty_like(q)
+        pa.pa_decode_cascade(out, q, st.k_cache, st.v_cache, st.block_tables, st.context_lens, gsd, gbd, 4,
+                             1.0 / math.sqrt(w.head_size), w.num_kv_heads, ws, partition_tokens=mode)
+        torch.cuda.synchronize()
+        check_status_clean()
+        assert max_abs_err(out, ref, w.dtype) <= TOL[w.dtype], mode
+
+
 def test_llama7b_bs64_fp8():
     _run_workload("llama7b_bs64_fp8", modes=(0, -1, 512))
 
