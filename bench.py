@@ -57,6 +57,8 @@ def parse():
     ap.add_argument("--ref-seconds", type=float, default=120.0,
                     help="--impl reference: oracle time spread over the warm-up and timed steps")
     ap.add_argument("--tuning", default="", help="warps,stages,ctas_per_sm for pa_set_decode_tuning")
+    ap.add_argument("--cascade", choices=["auto", "on", "off"], default="auto",
+                    help="shared-prefix decode (pa_decode_cascade) when forks of one prompt share blocks")
     return ap.parse_args()
 
 
@@ -80,22 +82,31 @@ def workload_plan(name, pool_gb=None):
     return plan
 
 
-def step_bytes(plan):
+def step_bytes(plan, groups=None):
     """Algorithmic bytes: the decode reads every context token's K and V (in
     the cache's element size), the query and writes the output (in the
     query's), plus block tables and lengths; the write reads the new tokens'
-    K/V and writes them into the cache."""
+    K/V and writes them into the cache.  With ``groups`` (group_start,
+    group_blocks of a shared-prefix decode) a group's shared blocks count
+    once, not once per member: ``kv`` is then the unique bytes and
+    ``kv_logical`` what a per-sequence decode reads."""
     w = plan.workload
     e, ec, bs = w.elem_bytes, w.cache_elem_bytes, w.block_size
     ctx = [int(c) for c in plan.context_lens]
-    kv = sum(ctx) * 2 * w.num_kv_heads * w.head_size * ec
+    per_tok = 2 * w.num_kv_heads * w.head_size * ec
+    kv_logical = sum(ctx) * per_tok
+    saved_blocks = 0
+    if groups is not None:
+        gs, gb = groups
+        saved_blocks = sum((int(gs[v + 1]) - int(gs[v]) - 1) * int(gb[v]) for v in range(len(gb)))
+    kv = kv_logical - saved_blocks * bs * per_tok
     qo = 2 * plan.B * w.num_heads * w.head_size * e
-    tables = sum(4 * (-(-c // bs)) for c in ctx)
+    tables = sum(4 * (-(-c // bs)) for c in ctx) - 4 * saved_blocks
     lens = 4 * plan.B
     decode = kv + qo + tables + lens
     n_new = len(plan.step_ops)
     write = n_new * w.num_kv_heads * w.head_size * 2 * (e + ec) + 8 * n_new
-    return {"kv": kv, "decode": decode, "write": write, "step": decode + write}
+    return {"kv": kv, "kv_logical": kv_logical, "decode": decode, "write": write, "step": decode + write}
 
 
 def allocator_report(plan):
@@ -543,9 +554,15 @@ def run_ours(args):
     if is_prefill(plan):
         return run_prefill(args, plan, device, world, rank)
     w = plan.workload
-    nbytes = step_bytes(plan)
     kv, inp = setup_device(plan, device)
     dev, tdt = inp["dev"], inp["tdt"]
+    # shared-prefix decode when forks of one prompt share leading blocks
+    groups = None
+    if args.cascade != "off":
+        gs_h, gb_h, max_group = kv.prefix_groups(plan.batch, w.num_heads)
+        if (gb_h > 0).any() or args.cascade == "on":
+            groups = (gs_h, gb_h, max_group)
+    nbytes = step_bytes(plan, groups[:2] if groups else None)
     q = dev(inp["query"])
     key, value = dev(inp["key"]), dev(inp["value"])
     slots = torch.from_numpy(inp["slots"]).to(device)
@@ -553,15 +570,27 @@ def run_ours(args):
     cl = torch.from_numpy(inp["lens"]).to(device)
     out = torch.empty_like(q)
     scale = 1.0 / math.sqrt(w.head_size)
-    ws = kv.workspace(plan.B, w.num_heads, bt.shape[1], args.partition)
     stream = torch.cuda.Stream(device)
-    # cache write (when the step appends tokens) + decode; fixed partitions add
-    # the log-sum-exp merge kernel
-    launches_per_step = (1 if len(inp["slots"]) else 0) + 1 + (1 if args.partition > 0 else 0)
+    if groups:
+        gs_d, gb_d = torch.from_numpy(groups[0]).to(device), torch.from_numpy(groups[1]).to(device)
+        ws = kv.shared_workspace(plan.B, w.num_heads, groups[2], args.partition)
+    else:
+        ws = kv.workspace(plan.B, w.num_heads, bt.shape[1], args.partition)
+
+    def decode(o_, q_, bt_, cl_, gs_=None, gb_=None):
+        if groups:
+            kv.decode_shared(o_, q_, bt_, cl_, gs_d if gs_ is None else gs_, gb_d if gb_ is None else gb_, groups[2],
+                             scale, partition_tokens=args.partition, stream=stream, workspace=ws)
+        else:
+            kv.decode(o_, q_, bt_, cl_, scale, partition_tokens=args.partition, stream=stream, workspace=ws)
+
+    # cache write (when the step appends tokens) + decode (two passes for a
+    # shared-prefix decode); fixed partitions add the log-sum-exp merge kernel
+    launches_per_step = (1 if len(inp["slots"]) else 0) + (2 if groups else 1) + (1 if args.partition > 0 else 0)
 
     def step():
         kv.write(slots, key, value, None, stream=stream)
-        kv.decode(out, q, bt, cl, scale, partition_tokens=args.partition, stream=stream, workspace=ws)
+        decode(out, q, bt, cl)
 
     with torch.cuda.stream(stream):
         for _ in range(max(3, args.warmup)):
@@ -598,7 +627,7 @@ def run_ours(args):
     with torch.cuda.stream(stream):
         for k in range(K):
             ea[k].record(stream)
-            kv.decode(out, q, bt, cl, scale, partition_tokens=args.partition, stream=stream, workspace=ws)
+            decode(out, q, bt, cl)
             eb[k].record(stream)
     torch.cuda.synchronize()
     dec_ms = statistics.mean(ea[k].elapsed_time(eb[k]) for k in range(K))
@@ -625,80 +654,7 @@ def run_ours(args):
     # computes, as a serving loop would.
     e2e = None
     if not args.no_e2e:
-        pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()  # noqa: E731
-        raw = (lambda r: r if w.dtype == "f32" else r.view(np.int16))
-        view = (lambda t: t if w.dtype == "f32" else t.view(torch.bfloat16))
-        hosts = [(pin(raw(inp["query"])), pin(raw(inp["key"])), pin(raw(inp["value"])), pin(inp["slots"]),
-                  pin(inp["tables"]), pin(inp["lens"])) for _ in range(2)]
-        h_out = [torch.empty(out.shape, dtype=torch.int16 if w.dtype == "bf16" else torch.float32).pin_memory()
-                 for _ in range(2)]
-        devs = [tuple(torch.empty(x.shape, dtype=x.dtype, device=device) for x in hosts[b]) for b in range(2)]
-        d_out = [torch.empty_like(out) for _ in range(2)]
-        h2d = sum(x.numel() * x.element_size() for x in hosts[0])
-        d2h = h_out[0].numel() * h_out[0].element_size()
-        s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
-        ev_in = [torch.cuda.Event() for _ in range(2)]
-        ev_done = [torch.cuda.Event() for _ in range(2)]
-        ev_read = [torch.cuda.Event() for _ in range(2)]
-
-        def copy_in(k):
-            b = k % 2
-            with torch.cuda.stream(s_in):
-                if k >= 2:
-                    s_in.wait_event(ev_done[b])  # step k-2 no longer reads buffer set b
-                for d, h in zip(devs[b], hosts[b]):
-                    d.copy_(h, non_blocking=True)
-                ev_in[b].record(s_in)
-
-        def compute(k):
-            b = k % 2
-            d_q, d_k, d_v, d_s, d_bt, d_cl = devs[b]
-            stream.wait_event(ev_in[b])
-            if k >= 2:
-                stream.wait_event(ev_read[b])  # step k-2's output has been read back
-            kv.write(d_s, view(d_k), view(d_v), None, stream=stream)
-            kv.decode(d_out[b], view(d_q), d_bt, d_cl, scale, partition_tokens=args.partition, stream=stream,
-                      workspace=ws)
-            ev_done[b].record(stream)
-
-        def copy_out(k):
-            b = k % 2
-            with torch.cuda.stream(s_out):
-                s_out.wait_event(ev_done[b])
-                h_out[b].copy_(d_out[b].view(h_out[b].dtype), non_blocking=True)
-                ev_read[b].record(s_out)
-
-        def run_e2e(n):
-            copy_in(0)
-            for k in range(n):
-                if k + 1 < n:
-                    copy_in(k + 1)
-                compute(k)
-                copy_out(k)
-
-        run_e2e(max(3, args.warmup))
-        torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
-        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        f0.record(s_in)
-        stream.wait_event(f0)
-        s_out.wait_event(f0)
-        run_e2e(K)
-        s_out.wait_stream(stream)
-        s_out.wait_stream(s_in)
-        f1.record(s_out)
-        torch.cuda.synchronize()
-        e_ms = max_over_ranks([f0.elapsed_time(f1)], device, world)[0]
-        e_step = e_ms / K
-        got = h_out[(K - 1) % 2].view(torch.bfloat16 if w.dtype == "bf16" else torch.float32)
-        if not torch.equal(got.view(torch.int16 if w.dtype == "bf16" else torch.int32),
-                           out.view(torch.int16 if w.dtype == "bf16" else torch.int32).cpu()):
-            raise RuntimeError("end-to-end output differs from the device-resident step's output")
-        e2e = {"value": round(aggregate_value(nbytes["step"], e_step, world), 3), "unit": "GB/s",
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "ms_per_step": round(e_step, 5), "tok_per_s": round(plan.B * world / (e_step * 1e-3), 1),
-               "overlap": "double-buffered: copies of steps k+1 (in) and k-1 (out) overlap step k"}
+        e2e = run_e2e_decode(args, plan, kv, inp, out, scale, groups, nbytes, stream, device, world)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -719,11 +675,20 @@ def run_ours(args):
                    "l2": f"no flush: the KV read per step ({nbytes['kv'] / 1e9:.2f} GB) exceeds the 126 MB L2"},
         "tok_per_s": round(tok_s, 1),
         "kv_read_gbs": round(nbytes["kv"] * world / (ms_step * 1e-3) / 1e9, 3),
+        "shared_prefix": ({"groups": int(len(groups[1])), "groups_sharing": int((groups[1] > 0).sum()),
+                           "max_group_size": groups[2], "kv_logical_bytes": nbytes["kv_logical"],
+                           "kv_unique_bytes": nbytes["kv"],
+                           "kv_logical_gbs": round(nbytes["kv_logical"] * world / (ms_step * 1e-3) / 1e9, 3),
+                           "note": "value, kv_read_gbs and the roofline count each group's shared blocks once "
+                                   "(the bytes the step must move); kv_logical_gbs counts them per member"}
+                          if groups else None),
         "frac_of_hbm_peak": round(value / world / peak, 4),
         "frac_of_8tbs_spec": round(value / world / 8000.0, 4),
         "bytes_per_step": nbytes,
         "allocator": allocator_report(plan),
-        "roofline": {"bound": "hbm", "kernel": "pa_decode (decode_kernel, log-sum-exp merge fused)",
+        "roofline": {"bound": "hbm",
+                     "kernel": ("pa_decode_cascade (decode_kernel prefix pass + suffix pass)" if groups
+                                else "pa_decode (decode_kernel, log-sum-exp merge fused)"),
                      "achieved": round(achieved, 2), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
                      "algorithmic_bytes_per_launch": nbytes["decode"], "avg_launch_ms": round(dec_ms, 5),
@@ -738,6 +703,124 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def pack_inputs(arrays, device):
+    """One pinned host staging buffer holding the step's input arrays back
+    to back (each at a 256-byte boundary), a device buffer of the same
+    layout, and per array a function that views a buffer's segment as that
+    array's dtype and shape."""
+    import numpy as np
+    import torch
+
+    offs, off = [], 0
+    for a in arrays:
+        offs.append(off)
+        off = (off + a.nbytes + 255) // 256 * 256
+    host = torch.empty(max(off, 256), dtype=torch.uint8).pin_memory()
+    hv = host.numpy()
+    for a, o in zip(arrays, offs):
+        hv[o:o + a.nbytes] = np.ascontiguousarray(a).reshape(-1).view(np.uint8)
+    dev = torch.empty_like(host, device=device)
+    tdt = {np.dtype(np.float32): torch.float32, np.dtype(np.uint16): torch.int16, np.dtype(np.int16): torch.int16,
+           np.dtype(np.int32): torch.int32, np.dtype(np.int64): torch.int64}
+
+    def viewer(a, o):
+        return lambda buf: buf[o:o + a.nbytes].view(tdt[a.dtype]).view(a.shape)
+
+    return host, dev, [viewer(a, o) for a, o in zip(arrays, offs)], off
+
+
+def run_e2e_decode(args, plan, kv, inp, out, scale, groups, nbytes, stream, device, world):
+    """End to end through the public API: each step copies its inputs from
+    pinned host memory (one staging buffer: query, new K/V, slots, block
+    tables, lengths and, for a shared-prefix decode, the groups) to the
+    device, runs the step (cache write + decode, as prepared calls of the
+    runtime helper) and copies the output back.  Two buffer sets let the
+    copies of steps k+1 (in) and k-1 (out) run on copy streams while step k
+    computes, as a serving loop would."""
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    w = plan.workload
+    arrays = [inp["query"], inp["key"], inp["value"], inp["slots"], inp["tables"], inp["lens"]]
+    if groups:
+        arrays += [groups[0], groups[1]]
+    bf = w.dtype == "bf16"
+    view = (lambda t: t.view(torch.bfloat16)) if bf else (lambda t: t)
+    sets = []
+    for _ in range(2):
+        host, dbuf, viewers, nbytes_in = pack_inputs(arrays, device)
+        d = [f(dbuf) for f in viewers]
+        d_out = torch.empty_like(out)
+        grp = (d[6], d[7], groups[2]) if groups else None
+        step = kv.prepare_step(d[3], view(d[1]), view(d[2]), d_out, view(d[0]), d[4], d[5], scale,
+                               partition_tokens=args.partition, stream=stream, groups=grp)
+        h_out = torch.empty(out.shape, dtype=torch.int16 if bf else torch.float32).pin_memory()
+        sets.append({"host": host, "dev": dbuf, "out": d_out, "h_out": h_out, "step": step, "n_in": nbytes_in})
+    h2d = sets[0]["n_in"]  # the packed staging buffer copied each step
+    d2h = sets[0]["h_out"].numel() * sets[0]["h_out"].element_size()
+    s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_done = [torch.cuda.Event() for _ in range(2)]
+    ev_read = [torch.cuda.Event() for _ in range(2)]
+
+    def copy_in(k):
+        b = k % 2
+        if k >= 2:
+            s_in.wait_event(ev_done[b])  # step k-2 no longer reads buffer set b
+        with torch.cuda.stream(s_in):
+            sets[b]["dev"].copy_(sets[b]["host"], non_blocking=True)
+        ev_in[b].record(s_in)
+
+    def compute(k):
+        b = k % 2
+        stream.wait_event(ev_in[b])
+        if k >= 2:
+            stream.wait_event(ev_read[b])  # step k-2's output has been read back
+        sets[b]["step"]()
+        ev_done[b].record(stream)
+
+    def copy_out(k):
+        b = k % 2
+        s_out.wait_event(ev_done[b])
+        with torch.cuda.stream(s_out):
+            sets[b]["h_out"].copy_(sets[b]["out"].view(sets[b]["h_out"].dtype), non_blocking=True)
+        ev_read[b].record(s_out)
+
+    def run(n):
+        copy_in(0)
+        for k in range(n):
+            if k + 1 < n:
+                copy_in(k + 1)
+            compute(k)
+            copy_out(k)
+
+    run(max(3, args.warmup))
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    K = args.steps
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(s_in)
+    stream.wait_event(f0)
+    s_out.wait_event(f0)
+    run(K)
+    s_out.wait_stream(stream)
+    s_out.wait_stream(s_in)
+    f1.record(s_out)
+    torch.cuda.synchronize()
+    e_ms = max_over_ranks([f0.elapsed_time(f1)], device, world)[0]
+    e_step = e_ms / K
+    iv = torch.int16 if bf else torch.int32
+    if not torch.equal(sets[(K - 1) % 2]["h_out"].view(iv), out.view(iv).cpu()):
+        raise RuntimeError("end-to-end output differs from the device-resident step's output")
+    return {"value": round(aggregate_value(nbytes["step"], e_step, world), 3), "unit": "GB/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "ms_per_step": round(e_step, 5), "tok_per_s": round(plan.B * world / (e_step * 1e-3), 1),
+            "overlap": "double-buffered: one packed copy in (step k+1) and one copy out (step k-1) overlap step k",
+            "host_calls": "prepared library calls (descriptors built once per buffer set)"}
 
 
 def run_prefill(args, plan, device, world, rank):
