@@ -252,16 +252,19 @@ pa_status pa_decode_no_alloc(pa_tensor* out, const pa_tensor* query, const pa_te
  * blog's "PagedAttention" section).  pa_decode shares the memory only: each
  * sample still reads every prompt block.  This call also shares the reads:
  * the batch is cut into groups of consecutive sequences whose block tables
- * begin with the same group_blocks[v] blocks; each shared page is read once
- * for all of a group's members and query heads, each member then runs over
- * the rest of its own context, and the two partial results are merged by
- * log-sum-exp.  The output is pa_decode's (the same formula; only fp32
- * rounding order differs).
+ * begin with the same group_blocks[v] blocks; one kernel row per (group, kv
+ * head) carries the query heads of every member, attends the shared pages
+ * with all of them (each shared page is read once for the whole group), then
+ * each member's own remaining pages with that member's heads only.  The
+ * output is pa_decode's (the same formula; only fp32 rounding order
+ * differs).  One kernel launch.
  *
  * group_start:  [n_groups + 1] int32 on the device: group v holds sequences
  *               group_start[v] .. group_start[v+1] - 1; group_start[0] = 0,
- *               non-decreasing, group_start[n_groups] = B (else
- *               PA_DEV_BAD_CONTEXT and every sequence is decoded in full).
+ *               non-decreasing, group_start[n_groups] = B, at most
+ *               max_group_size members each (else PA_DEV_BAD_CONTEXT and
+ *               every sequence is decoded on its own: the output stays
+ *               right).
  * group_blocks: [n_groups] int32 on the device: leading blocks every member
  *               of the group holds (the same block ids at the same table
  *               indices; not checked).  Values above a member's number of
@@ -270,21 +273,19 @@ pa_status pa_decode_no_alloc(pa_tensor* out, const pa_tensor* query, const pa_te
  *               allocator.
  * max_group_size: most members a group may have; (num_heads / num_kv_heads)
  *               * max_group_size must be 1, 2, 4 or 8 (else
- *               PA_ERR_UNSUPPORTED).  Larger groups are decoded in full
- *               (PA_DEV_BAD_CONTEXT).
+ *               PA_ERR_UNSUPPORTED).
  * Other arguments as pa_decode; bf16 with head_size 128 or fp32 with
- * head_size 64.  A workspace of pa_decode_cascade_workspace_bytes is
- * required (zero-filled before first use, as for pa_decode): it also holds
- * the prefix's partial results, fp32 [B][H][head_size] + [B][H].
- * opts->partition_tokens: 0 (balanced split in both passes) or -1 (none);
- * fixed partitions are PA_ERR_UNSUPPORTED.  Two kernel launches.
+ * head_size 64.  opts->partition_tokens: 0 (balanced split: needs a
+ * workspace of pa_decode_cascade_workspace_bytes, zero-filled before first
+ * use, as for pa_decode) or -1 (no split, no workspace); fixed partitions
+ * are PA_ERR_UNSUPPORTED.
  * ------------------------------------------------------------------------- */
 pa_status pa_decode_cascade(pa_tensor* out, const pa_tensor* query, const pa_tensor* k_cache,
                             const pa_tensor* v_cache, const pa_tensor* block_tables, const pa_tensor* context_lens,
                             const pa_tensor* group_start, const pa_tensor* group_blocks, int32_t max_group_size,
                             float scale, int32_t num_kv_heads, const pa_opts* opts);
 /* Workspace bytes of pa_decode_cascade for these sizes on the current
- * device (partition_tokens 0 or -1). */
+ * device (partition_tokens 0; 0 bytes for -1). */
 pa_status pa_decode_cascade_workspace_bytes(int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
                                             int32_t head_size, int32_t max_group_size, int32_t partition_tokens,
                                             size_t* bytes_out);

@@ -776,32 +776,14 @@ static pa_status decode_impl(pa_tensor* out, const pa_tensor* query, const pa_te
 // ---------------------------------------------------------------------------
 // shared-prefix (cascade) decode
 // ---------------------------------------------------------------------------
-// Workspace: [header][shares of the larger pass][pre_o: B*H*D fp32][pre_lse: B*H fp32].
-struct CascadeLayout {
-  size_t shares;  // bytes after the header for the balanced shares (0: no split)
-  size_t pre_o_off, pre_lse_off, total;
-};
-
-static CascadeLayout cascade_layout(int64_t B, int64_t H, int64_t D, size_t shares) {
-  CascadeLayout L;
-  L.shares = shares;
-  L.pre_o_off = kWsHeader + align_up(shares, 256);
-  L.pre_lse_off = L.pre_o_off + align_up(size_t(B * H * D) * 4, 256);
-  L.total = L.pre_lse_off + align_up(size_t(B * H) * 4, 256);
-  return L;
-}
-
-// Bytes of balanced shares the two passes need (the larger), on the current
-// device under the current tuning.
-static pa_status cascade_shares_bytes(int32_t dt, int64_t G, int64_t members, int64_t D, size_t* out) {
+// Workspace: [header][shares of the group rows' launch] (the balanced split);
+// none without a split.
+static pa_status cascade_ws_bytes(int32_t dt, int64_t gp, int64_t D, size_t* out) {
   DeviceInfo di;
   pa_status st = device_info(&di, nullptr);
   if (st != PA_OK) return st;
-  const int64_t grid = int64_t(di.sms) * g_tuning.ctas_per_sm;
-  const int64_t gp = G * members;
-  const size_t pre = shares_bytes(grid * warps_for(int(gp), dt), gp, D);
-  const size_t suf = shares_bytes(grid * warps_for(int(G), dt), G, D);
-  *out = pre > suf ? pre : suf;
+  const int64_t workers = int64_t(di.sms) * g_tuning.ctas_per_sm * warps_for(int(gp), dt);
+  *out = balanced_ws_bytes(workers, gp, D);
   return PA_OK;
 }
 
@@ -862,16 +844,14 @@ pa_status pa_decode_cascade_workspace_bytes(int32_t num_seqs, int32_t num_heads,
   const int64_t G = num_heads / num_kv_heads;
   const int64_t gp = G * max_group_size;
   if (gp != 1 && gp != 2 && gp != 4 && gp != 8) return PA_ERR_UNSUPPORTED;
-  size_t shares = 0;
-  if (partition_tokens == 0) {
-    // an upper bound over cache types (as for pa_decode_workspace_bytes)
-    const pa_status st = cascade_shares_bytes(PA_FP8_E4M3, G, max_group_size, head_size, &shares);
-    if (st != PA_OK) return st;
-    size_t b16 = 0;
-    cascade_shares_bytes(PA_BF16, G, max_group_size, head_size, &b16);
-    if (b16 > shares) shares = b16;
-  }
-  *bytes_out = cascade_layout(num_seqs, num_heads, head_size, shares).total;
+  *bytes_out = 0;
+  if (partition_tokens == -1) return PA_OK;
+  // an upper bound over the cache types built
+  size_t a = 0, b = 0;
+  pa_status st = cascade_ws_bytes(PA_BF16, gp, head_size, &a);
+  if (st != PA_OK) return st;
+  if ((st = cascade_ws_bytes(PA_F32, gp, head_size, &b)) != PA_OK) return st;
+  *bytes_out = a > b ? a : b;
   return PA_OK;
 }
 
@@ -891,34 +871,24 @@ pa_status pa_decode_cascade(pa_tensor* out, const pa_tensor* query, const pa_ten
   if (part != 0 && part != -1) return PA_ERR_UNSUPPORTED;
   if (dc.B == 0) return PA_OK;
   const int64_t gp = dc.G * max_group_size;
-  size_t shares = 0;
-  if (part == 0 && (st = cascade_shares_bytes(dc.dt, dc.G, max_group_size, dc.D, &shares)) != PA_OK) return st;
-  const CascadeLayout L = cascade_layout(dc.B, dc.H, dc.D, shares);
-  if (opts == nullptr || opts->workspace == nullptr || opts->workspace_bytes < L.total) return PA_ERR_INVALID_ARG;
-  char* ws = static_cast<char*>(opts->workspace);
-
-  DecodePlan pp, ps;
-  if ((st = plan_decode(dc.dt, int(gp), n_groups, 0, dc.B, dc.H, dc.D, dc.max_nb, part, L.shares, true, &pp)) !=
-      PA_OK)
-    return st;
-  if ((st = plan_decode(dc.dt, int(dc.G), dc.B, dc.B, dc.B, dc.H, dc.D, dc.max_nb, part, L.shares, true, &ps)) !=
-      PA_OK)
-    return st;
+  const bool ws_given = opts && opts->workspace != nullptr;
+  const size_t ws_bytes = ws_given ? opts->workspace_bytes : 0;
+  // one launch over the group rows; the row sequences are the groups, or
+  // the sequences when the groups turn out malformed on the device
+  const int64_t umax = n_groups > dc.B ? n_groups : dc.B;
+  DecodePlan plan;
+  st = plan_decode(dc.dt, int(gp), umax, umax, dc.B, dc.H, dc.D, dc.max_nb, part,
+                   ws_bytes > kWsHeader ? ws_bytes - kWsHeader : 0, ws_given, &plan);
+  if (st != PA_OK) return st;
+  if (part == 0 && plan.mode != pa::kBalanced) return PA_ERR_INVALID_ARG;  // the workspace is too small
   pa::DecodeArgs a = dc.a;
   a.grp_start = static_cast<const int32_t*>(group_start->data);
   a.grp_blocks = static_cast<const int32_t*>(group_blocks->data);
   a.n_groups = int32_t(n_groups);
   a.grp_members = max_group_size;
   a.g_real = int32_t(dc.G);
-  a.pre_o = reinterpret_cast<float*>(ws + L.pre_o_off);
-  a.pre_lse = reinterpret_cast<float*>(ws + L.pre_lse_off);
-  const cudaStream_t s = stream_of(opts);
-  pa::DecodeArgs ap = a;
-  if (pp.mode == pa::kBalanced) place_shares(&ap, ws, kWsHeader, pp, gp, dc.D);
-  if ((st = launch_kind<pa::kPrefixPass>(dc, int(gp), ap, pp, s)) != PA_OK) return st;
-  pa::DecodeArgs as = a;
-  if (ps.mode == pa::kBalanced) place_shares(&as, ws, kWsHeader, ps, dc.G, dc.D);
-  return launch_kind<pa::kSuffixPass>(dc, int(dc.G), as, ps, s);
+  if (plan.mode == pa::kBalanced) place_shares(&a, opts->workspace, kWsHeader, plan, gp, dc.D);
+  return launch_kind<pa::kGroup>(dc, int(gp), a, plan, stream_of(opts));
 }
 
 pa_status pa_prefill(pa_tensor* out, const pa_tensor* query, const pa_tensor* k_cache, const pa_tensor* v_cache,

@@ -92,18 +92,18 @@ struct DecodeArgs {
   const int32_t* grp_start;   // [n_groups + 1]: group v = sequences grp_start[v] .. grp_start[v+1] - 1
   const int32_t* grp_blocks;  // [n_groups]: leading blocks every member shares
   int32_t n_groups;
-  int32_t grp_members;  // most members a group may have (the prefix pass reads members x g_real query rows)
+  int32_t grp_members;  // most members a group may have (a group row carries members x g_real query rows)
   int32_t g_real;       // query heads per kv head
-  float* pre_o;         // [B][H][D]: the prefix's partial output of each (sequence, head), normalised
-  float* pre_lse;       // [B][H]: its log-sum-exp (natural log)
 };
 
-// Decode kinds: a plain decode, or one of the two passes of a shared-prefix
-// decode.  The prefix pass treats each group's shared blocks as one row of
-// members x g_real query rows (each page is read once for the whole group)
-// and leaves partial results; the suffix pass runs every sequence over the
-// rest of its context and merges the prefix's partial into its output.
-enum DecodeKind : int { kPlain = 0, kPrefixPass = 1, kSuffixPass = 2 };
+// Decode kinds: a plain decode, or a shared-prefix decode.  In the latter a
+// row is (group, kv head) and carries the G query heads of every member of
+// the group (members x g_real query rows); its pages are the group's shared
+// blocks, which every member's rows attend, followed by each member's own
+// remaining blocks, which only that member's rows attend (the other rows are
+// masked).  A shared page is thus read once for the whole group, and each
+// member's output is complete at the row's end: no second pass.
+enum DecodeKind : int { kPlain = 0, kGroup = 1 };
 
 // Tkv: cache element type (fp32, bf16 or e4m3 codes); Tq: query/output type.
 template <typename Tkv, typename Tq, int D, int G>
@@ -141,11 +141,11 @@ __host__ __device__ inline size_t decode_prefix_bytes(int U, int X = 0) {
   return (size_t(U + 1 + 32 + X) * 4 + 127) / 128 * 128;
 }
 
-// Groups of a shared-prefix decode must tile the batch in order:
-// grp_start[0] = 0, non-decreasing, grp_start[n_groups] = B.  Block-wide
-// check (every CTA reaches the same verdict); anything else disables the
-// shared prefix for the whole call (every sequence then runs in full in the
-// suffix pass) and sets PA_DEV_BAD_CONTEXT.
+// Groups of a shared-prefix decode must tile the batch in order
+// (grp_start[0] = 0, non-decreasing, grp_start[n_groups] = B) with at most
+// grp_members members each.  Block-wide check (every CTA reaches the same
+// verdict); anything else sets PA_DEV_BAD_CONTEXT and the call decodes every
+// sequence on its own (each its own group, nothing shared).
 __device__ __forceinline__ bool groups_tile_batch(const DecodeArgs& a) {
   int ok = 1;
   const int n = a.n_groups;
@@ -153,26 +153,23 @@ __device__ __forceinline__ bool groups_tile_batch(const DecodeArgs& a) {
     const int x = __ldg(a.grp_start + v);
     if (v == 0 && x != 0) ok = 0;
     if (v == n && x != a.B) ok = 0;
-    if (v < n && __ldg(a.grp_start + v + 1) < x) ok = 0;
+    if (v < n) {
+      const int y = __ldg(a.grp_start + v + 1);
+      if (y < x || y - x > a.grp_members) ok = 0;
+    }
   }
   ok = __syncthreads_and(ok);
   if (!ok && blockIdx.x == 0 && threadIdx.x == 0) flag(PA_DEV_BAD_CONTEXT);
   return ok != 0;
 }
 
-// Shared leading blocks of group v as both passes use them: 0 for an empty
-// group or one with more members than the prefix pass has query rows for;
-// else grp_blocks[v] capped at every member's count of full blocks (a cap
-// sets PA_DEV_BAD_CONTEXT).
+// Shared leading blocks of group v: grp_blocks[v] (0 for a group of one),
+// capped at every member's count of full blocks (a cap sets
+// PA_DEV_BAD_CONTEXT).
 __device__ __forceinline__ int group_prefix_blocks(const DecodeArgs& a, int v, int ctx_cap) {
   const int s0 = __ldg(a.grp_start + v), s1 = __ldg(a.grp_start + v + 1);
-  const int n = s1 - s0;
   int b = __ldg(a.grp_blocks + v);
-  if (n <= 0 || b <= 0) return 0;
-  if (n > a.grp_members) {
-    if (blockIdx.x == 0) flag(PA_DEV_BAD_CONTEXT);
-    return 0;
-  }
+  if (s1 - s0 <= 1 || b <= 0) return 0;
   for (int m = s0; m < s1; ++m) {
     const int raw = __ldg(a.ctx + m);
     const int full = (raw < 0 ? 0 : (raw > ctx_cap ? ctx_cap : raw)) / 16;
@@ -182,6 +179,50 @@ __device__ __forceinline__ int group_prefix_blocks(const DecodeArgs& a, int v, i
     }
   }
   return b;
+}
+
+// Where page p of a group row lies: in the shared part (m = -1) or in member
+// m's own pages (its table from index pb on); q = page within that part,
+// e = pages of that part.  Members are walked in order, skipping those with
+// no page of their own.
+struct GroupCursor {
+  int s0, n, pb;  // first member, members, shared blocks
+  int m, q, e;
+};
+
+__device__ __forceinline__ int member_pages(const DecodeArgs& a, int seq, int pb, int ctx_cap) {
+  const int raw = __ldg(a.ctx + seq);
+  return ((raw < 0 ? 0 : (raw > ctx_cap ? ctx_cap : raw)) + 15) / 16 - pb;
+}
+
+__device__ __forceinline__ void group_seek(GroupCursor& g, const DecodeArgs& a, bool groups_ok, const int* PB, int v,
+                                           int p, int ctx_cap) {
+  g.s0 = groups_ok ? __ldg(a.grp_start + v) : v;
+  g.n = groups_ok ? __ldg(a.grp_start + v + 1) - g.s0 : 1;
+  g.pb = PB[v];
+  if (p < g.pb) {
+    g.m = -1, g.q = p, g.e = g.pb;
+    return;
+  }
+  int q = p - g.pb;
+  for (int m = 0; m < g.n; ++m) {
+    const int e = member_pages(a, g.s0 + m, g.pb, ctx_cap);
+    if (q < e) {
+      g.m = m, g.q = q, g.e = e;
+      return;
+    }
+    q -= e;
+  }
+  g.m = g.n, g.q = 0, g.e = 0;  // past the row (not reached for pages of the row)
+}
+
+__device__ __forceinline__ void group_next(GroupCursor& g, const DecodeArgs& a, int ctx_cap) {
+  if (++g.q < g.e) return;
+  g.q = 0;
+  do {
+    ++g.m;
+    g.e = g.m < g.n ? member_pages(a, g.s0 + g.m, g.pb, ctx_cap) : 0;
+  } while (g.e == 0 && g.m < g.n);
 }
 
 // Block-wide exclusive scan of one int per thread; returns the prefix and
@@ -371,8 +412,9 @@ __device__ __forceinline__ void merge_shares(const float* ws_o, const float* ws_
     const bool mine = kl <= wb && !worker_empty(kl, W, N);
     float wl[G];
 #pragma unroll
-    for (int j = 0; j < G; ++j)
-      wl[j] = mine ? ex2((__ldcg(ws_lse + share_slot(kl, wa) * G + j) - mx[j]) * kLog2e) : 0.f;
+    for (int j = 0; j < G; ++j)  // (a row with no weight anywhere: a row of a group that attended nothing)
+      wl[j] = (mine && mx[j] != -INFINITY) ? ex2((__ldcg(ws_lse + share_slot(kl, wa) * G + j) - mx[j]) * kLog2e)
+                                            : 0.f;
     const int n = int(wb - k0 + 1 < 32 ? wb - k0 + 1 : 32);
 #pragma unroll 4
     for (int t = 0; t < n; ++t) {
@@ -401,10 +443,10 @@ __device__ __forceinline__ void merge_shares(const float* ws_o, const float* ws_
   }
 #pragma unroll
   for (int j = 0; j < G; ++j) {
-    const float inv = 1.f / wsum[j];
+    const float inv = wsum[j] > 0.f ? 1.f / wsum[j] : 0.f;
 #pragma unroll
     for (int e = 0; e < PER; ++e) acc[j][e] *= inv;
-    lse[j] = mx[j] + logf(wsum[j]);
+    lse[j] = wsum[j] > 0.f ? mx[j] + logf(wsum[j]) : -INFINITY;
   }
 }
 
@@ -419,16 +461,18 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
   const int warp = threadIdx.x >> 5;
   const int nwarps = blockDim.x >> 5;
   const int tg = lane / LPT, c = lane % LPT;
-  // U row sequences: the groups in a prefix pass, else the batch's sequences
-  const int U = CK == kPrefixPass ? a.n_groups : a.B;
+  // Row sequences: the batch's sequences, or in a shared-prefix decode its
+  // groups (each sequence its own group if the groups are malformed).  The
+  // shared-memory layout is sized for the larger of the two.
   const int Hkv = a.Hkv, H = a.H;
   const int ctx_cap = a.max_nb * kBS;
+  const int Umax = CK == kGroup ? max(a.n_groups, a.B) : a.B;
 
   int* scan_scratch = reinterpret_cast<int*>(smem);
   int* S = scan_scratch + 32;
-  int* ST = S + U + 1;  // suffix pass: each sequence's first block after its group's shared prefix
+  int* PB = S + Umax + 1;  // shared-prefix decode: each group's shared blocks
   unsigned char* wbase =
-      smem + decode_prefix_bytes(U, CK == kSuffixPass ? a.B : 0) + size_t(warp) * C::warp_bytes(a.stages);
+      smem + decode_prefix_bytes(Umax, CK == kGroup ? Umax : 0) + size_t(warp) * C::warp_bytes(a.stages);
   unsigned char* ring = wbase;
   float* pbuf = reinterpret_cast<float*>(wbase + size_t(a.stages) * C::STAGE);
   uint64_t* bars = reinterpret_cast<uint64_t*>(wbase + size_t(a.stages) * C::STAGE + C::PBUF);
@@ -443,20 +487,10 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
   pdl_launch_dependents();
 
   // ---- prologue: page prefix over row sequences (every CTA computes it) ----
+  bool groups_ok = false;
+  if constexpr (CK == kGroup) groups_ok = groups_tile_batch(a);
+  const int U = groups_ok ? a.n_groups : a.B;
   {
-    bool groups_ok = false;
-    if constexpr (CK != kPlain) groups_ok = groups_tile_batch(a);
-    if constexpr (CK == kSuffixPass) {
-      for (int i = threadIdx.x; i < U; i += blockDim.x) ST[i] = 0;
-      __syncthreads();
-      if (groups_ok)
-        for (int v = threadIdx.x; v < a.n_groups; v += blockDim.x) {
-          const int b = group_prefix_blocks(a, v, ctx_cap);
-          if (b)
-            for (int i = __ldg(a.grp_start + v); i < __ldg(a.grp_start + v + 1); ++i) ST[i] = b;
-        }
-      __syncthreads();
-    }
     const int nt = blockDim.x;
     const int per = (U + nt - 1) / nt;
     const int i0 = threadIdx.x * per;
@@ -464,13 +498,22 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
     int local = 0;
     for (int i = i0; i < i1; ++i) {
       int np;
-      if constexpr (CK == kPrefixPass) {
-        np = groups_ok ? group_prefix_blocks(a, i, ctx_cap) : 0;
+      if constexpr (CK == kGroup) {
+        // shared blocks, then every member's own
+        const int pb = groups_ok ? group_prefix_blocks(a, i, ctx_cap) : 0;
+        const int s0 = groups_ok ? __ldg(a.grp_start + i) : i;
+        const int n = groups_ok ? __ldg(a.grp_start + i + 1) - s0 : 1;
+        PB[i] = pb;
+        np = pb;
+        for (int m = 0; m < n; ++m) {
+          const int raw = a.ctx[s0 + m];
+          if ((raw < 0 || raw > ctx_cap) && blockIdx.x == 0) flag(PA_DEV_BAD_CONTEXT);
+          np += (clamp_ctx(raw, ctx_cap) + kBS - 1) / kBS - pb;
+        }
       } else {
         const int raw = a.ctx[i];
         if ((raw < 0 || raw > ctx_cap) && blockIdx.x == 0) flag(PA_DEV_BAD_CONTEXT);
         np = (clamp_ctx(raw, ctx_cap) + kBS - 1) / kBS;
-        if constexpr (CK == kSuffixPass) np -= ST[i];
       }
       S[i] = np;  // this thread's own entries: pages first, prefix below
       local += np * Hkv;
@@ -527,22 +570,26 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
     // ---- producer cursor (warp-uniform) ----
     RowPos pc = locate(S, U, Hkv, lo);
     int64_t px = lo;
-    int win_seq = -1, win_base = 0, win_blk = 0;  // lane-held window of 32 block ids
+    int win_seq = -1, win_base = 0, win_blk = 0;  // lane-held window of 32 block ids of one table row
     int p_seg_first = 1;                          // next issued page opens a segment
+    GroupCursor pg;                               // shared-prefix decode: where page pc.p lies
+    if constexpr (CK == kGroup) group_seek(pg, a, groups_ok, PB, pc.i, pc.p, ctx_cap);
 
     auto issue = [&](int s) {
-      // block id of page pc.p of sequence pc.i (warp-collective)
-      if (pc.i != win_seq || pc.p < win_base || pc.p >= win_base + 32) {
-        win_seq = pc.i;
-        win_base = pc.p & ~31;
-        const int pp = win_base + lane;
-        // a group's pages are read through its first member's table; a
-        // suffix starts after its group's shared blocks
-        const int trow = CK == kPrefixPass ? __ldg(a.grp_start + pc.i) : pc.i;
-        const int toff = CK == kSuffixPass ? ST[pc.i] : 0;
-        win_blk = pp < pc.np ? a.bt[int64_t(trow) * a.bt_stride + toff + pp] : 0;
+      // block id of the page (warp-collective): page pc.p of sequence pc.i,
+      // or in a group row the shared page or the member's own page
+      int trow = pc.i, tpage = pc.p;
+      if constexpr (CK == kGroup) {
+        trow = pg.m < 0 ? pg.s0 : pg.s0 + pg.m;
+        tpage = pg.m < 0 ? pg.q : pg.pb + pg.q;
       }
-      int blk = __shfl_sync(0xffffffffu, win_blk, pc.p - win_base);
+      if (trow != win_seq || tpage < win_base || tpage >= win_base + 32) {
+        win_seq = trow;
+        win_base = tpage & ~31;
+        const int pp = win_base + lane;
+        win_blk = pp < a.max_nb ? a.bt[int64_t(trow) * a.bt_stride + pp] : 0;
+      }
+      int blk = __shfl_sync(0xffffffffu, win_blk, tpage - win_base);
       if (unsigned(blk) >= unsigned(a.num_blocks)) {
         if (lane == 0) flag(PA_DEV_BAD_BLOCK);
         blk = 0;
@@ -553,16 +600,15 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
         const int64_t page_off = (int64_t(blk) * Hkv + pc.g) * C::PAGE;
         // order this warp's earlier shared-memory reads of the stage before the async-proxy refill
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        if constexpr (CK == kPrefixPass) {
+        if constexpr (CK == kGroup) {
           // query rows of the group's members (rows past the last member are not loaded)
-          const int s0 = __ldg(a.grp_start + pc.i);
-          const int nq = p_seg_first ? (__ldg(a.grp_start + pc.i + 1) - s0) * a.g_real : 0;
+          const int nq = p_seg_first ? pg.n * a.g_real : 0;
           mbar_arrive_expect_tx(bar, 2 * C::PAGE + nq * C::QROWB);
           bulk_g2s(smem_u32(st), kcb + page_off, C::PAGE, bar, pol);
           bulk_g2s(smem_u32(st + C::PAGE), vcb + page_off, C::PAGE, bar, pol);
           for (int r = 0; r < nq; ++r)
             bulk_g2s(smem_u32(st + 2 * C::PAGE + r * C::QROWB),
-                     qg + int64_t(s0 + r / a.g_real) * a.q_sb + int64_t(pc.g * a.g_real + r % a.g_real) * a.q_sh,
+                     qg + int64_t(pg.s0 + r / a.g_real) * a.q_sb + int64_t(pc.g * a.g_real + r % a.g_real) * a.q_sh,
                      C::QROWB, bar, pol);
         } else {
           mbar_arrive_expect_tx(bar, 2 * C::PAGE + (p_seg_first ? C::QBYTES : 0));
@@ -590,8 +636,11 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
           } while (pc.i < U && S[pc.i + 1] == S[pc.i]);
           if (pc.i < U) pc.np = (S[pc.i + 1] - S[pc.i]) / Hkv;
         }
-      } else if (a.mode == kFixed && pc.p % a.part_pages == 0) {
-        p_seg_first = 1;
+        if constexpr (CK == kGroup)
+          if (pc.i < U) group_seek(pg, a, groups_ok, PB, pc.i, 0, ctx_cap);
+      } else {
+        if constexpr (CK == kGroup) group_next(pg, a, ctx_cap);
+        if (a.mode == kFixed && pc.p % a.part_pages == 0) p_seg_first = 1;
       }
     };
 
@@ -603,6 +652,8 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
     int64_t cx = lo;
     int seg_p0 = cc.p;
     bool seg_first = true;
+    GroupCursor cg;  // shared-prefix decode: where page cc.p lies
+    if constexpr (CK == kGroup) group_seek(cg, a, groups_ok, PB, cc.i, cc.p, ctx_cap);
     float q[G][EPV];
     float o[G][EPV];
     float m[G], lpart[GH];
@@ -616,6 +667,12 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
     // Measured on B200 against the scalar path below (fp32 query): 0.274 ->
     // 0.191 ms at G = 4 (GQA batch 256); at G = 1 the scalar path is faster
     // (0.084 vs 0.089 ms on LLaMA-7B batch 64) and stays.
+    // (A bf16 variant of this layout for G >= 4 — bf16 operands straight
+    // from shared memory, P as bf16 high and low parts — was measured slower
+    // than the CUDA-core path below: 0.241 vs 0.219 ms on the GQA batch-256
+    // decode; its 16-byte operand loads hit 4x the shared-memory wavefronts
+    // of the conflict-free scalar layout, since the page rows are 256 bytes
+    // apart.  Not kept.)
     constexpr bool kMma = sizeof(Tkv) == 1 && G >= 2;
     const int gr = lane >> 2, tig = lane & 3;
     uint32_t qf[16];     // query of head gr, f16 pairs of this lane's 32 dims
@@ -654,7 +711,7 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
         // FP8 cache: fold the K dequantization scale into the query
         const float qscale = a.scale_log2 * (a.k_scale ? __ldg(a.k_scale + cc.g) : 1.f);
         vscale = a.v_scale ? __ldg(a.v_scale + cc.g) : 1.f;
-        if constexpr (CK == kPrefixPass) nreal = (__ldg(a.grp_start + cc.i + 1) - __ldg(a.grp_start + cc.i)) * a.g_real;
+        if constexpr (CK == kGroup) nreal = cg.n * a.g_real;
         if constexpr (kMma) {
           float qv[32];
           if (gr < nreal) {
@@ -698,7 +755,7 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
 #pragma unroll
         for (int j = 0; j < G; ++j) {
           float f[EPV];
-          if (CK != kPrefixPass || j < nreal) {
+          if (CK != kGroup || j < nreal) {
 #pragma unroll
             for (int v = 0; v < QV; ++v) Elem<Tq>::unpack(qs[j * (C::QROWB / 16) + c * QV + v], f + v * EPQ);
           } else {
@@ -716,16 +773,24 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
         for (int jj = 0; jj < GH; ++jj) lpart[jj] = 0.f;
         }
         // tokens of the row, consumed at its last page
-        if constexpr (CK == kPrefixPass)
-          ctx_i = cc.np * kBS;  // shared blocks are full
-        else if constexpr (CK == kSuffixPass)
-          ctx_i = clamp_ctx(a.ctx[cc.i], ctx_cap) - ST[cc.i] * kBS;
-        else
-          ctx_i = clamp_ctx(a.ctx[cc.i], ctx_cap);
+        if constexpr (CK != kGroup) ctx_i = clamp_ctx(a.ctx[cc.i], ctx_cap);
         seg_p0 = cc.p;
       }
       const bool last_of_row = (cc.p == cc.np - 1);
-      const int valid = last_of_row ? ctx_i - cc.p * kBS : kBS;
+      int valid = last_of_row ? ctx_i - cc.p * kBS : kBS;
+      // group row: shared pages are full and attended by every member's rows;
+      // a member's own pages only by that member's rows [alo, ahi)
+      int alo = 0, ahi = G;
+      if constexpr (CK == kGroup) {
+        if (cg.m < 0) {
+          valid = kBS;
+          ahi = nreal;
+        } else {
+          valid = cg.q == cg.e - 1 ? clamp_ctx(a.ctx[cg.s0 + cg.m], ctx_cap) - (cg.pb + cg.q) * kBS : kBS;
+          alo = cg.m * a.g_real;
+          ahi = alo + a.g_real;
+        }
+      }
 
       const uint4* Ks = reinterpret_cast<const uint4*>(st);
       const uint4* Vs = reinterpret_cast<const uint4*>(st + C::PAGE);
@@ -761,19 +826,29 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
         float sc4[4] = {sa[0] * sfac[0], sa[1] * sfac[1], sa[2] * sfac[0], sa[3] * sfac[1]};
         if (gr >= valid) sc4[0] = sc4[1] = -INFINITY;
         if (gr + 8 >= valid) sc4[2] = sc4[3] = -INFINITY;
+        if constexpr (CK == kGroup) {  // rows (heads) that do not attend this page
+          if (2 * tig < alo || 2 * tig >= ahi) sc4[0] = sc4[2] = -INFINITY;
+          if (2 * tig + 1 < alo || 2 * tig + 1 >= ahi) sc4[1] = sc4[3] = -INFINITY;
+        }
         float pm0 = fmaxf(sc4[0], sc4[2]), pm1 = fmaxf(sc4[1], sc4[3]);
 #pragma unroll
         for (int msk = 4; msk < 32; msk <<= 1) {
           pm0 = fmaxf(pm0, __shfl_xor_sync(0xffffffffu, pm0, msk));
           pm1 = fmaxf(pm1, __shfl_xor_sync(0xffffffffu, pm1, msk));
         }
-        // token 0 of every page is valid, so the maxima are finite
+        // token 0 of every page is valid, so the maxima are finite; in a
+        // group row a row that has attended nothing yet keeps -inf (no
+        // rescale, zero probabilities)
         const float mn0 = fmaxf(mh[0], pm0), mn1 = fmaxf(mh[1], pm1);
-        const float al0 = ex2(mh[0] - mn0), al1 = ex2(mh[1] - mn1);
+        float al0 = ex2(mh[0] - mn0), al1 = ex2(mh[1] - mn1);
         const bool grew = __any_sync(0xffffffffu, mn0 != mh[0] || mn1 != mh[1]);
         mh[0] = mn0;
         mh[1] = mn1;
-        const float p0 = ex2(sc4[0] - mn0), p1 = ex2(sc4[1] - mn1), p2 = ex2(sc4[2] - mn0), p3 = ex2(sc4[3] - mn1);
+        float p0 = ex2(sc4[0] - mn0), p1 = ex2(sc4[1] - mn1), p2 = ex2(sc4[2] - mn0), p3 = ex2(sc4[3] - mn1);
+        if constexpr (CK == kGroup) {
+          if (mn0 == -INFINITY) al0 = 1.f, p0 = p2 = 0.f;
+          if (mn1 == -INFINITY) al1 = 1.f, p1 = p3 = 0.f;
+        }
         lh[0] = lh[0] * al0 + (p0 + p2);
         lh[1] = lh[1] * al1 + (p1 + p3);
         if (grew) {
@@ -876,6 +951,13 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
 #pragma unroll
         for (int jj = 0; jj < GH; ++jj) sc[jj] = -INFINITY;
       }
+      if constexpr (CK == kGroup) {  // rows (heads) that do not attend this page
+#pragma unroll
+        for (int jj = 0; jj < GH; ++jj) {
+          const int j = (G >= 2 && hi_half) ? jj + GH : jj;
+          if (j < alo || j >= ahi) sc[jj] = -INFINITY;
+        }
+      }
 
       // ---- page max, new running max, rescale factors ----
       float pm[GH];
@@ -902,7 +984,7 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
 #pragma unroll
       for (int j = 0; j < G; ++j) {
         const float mn = fmaxf(m[j], pmall[j]);
-        alpha[j] = ex2(m[j] - mn);
+        alpha[j] = (CK == kGroup && mn == -INFINITY) ? 1.f : ex2(m[j] - mn);  // a row that attended nothing yet
         grew |= (mn != m[j]);
         m[j] = mn;
       }
@@ -912,7 +994,7 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
       for (int jj = 0; jj < GH; ++jj) {
         const float mj = (G >= 2 && hi_half) ? m[(jj + GH) % G] : m[jj];
         const float aj = (G >= 2 && hi_half) ? alpha[(jj + GH) % G] : alpha[jj];
-        const float p = ex2(sc[jj] - mj);
+        const float p = (CK == kGroup && mj == -INFINITY) ? 0.f : ex2(sc[jj] - mj);
         const bool own = (G >= 2) || !hi_half;
         lpart[jj] = lpart[jj] * aj + (own ? p : 0.f);
         if (own) {
@@ -1016,48 +1098,24 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
         const bool row_unit = unp == cc.np;
         const bool whole_unit = seg_p0 == up0 && cc.p == up0 + unp - 1;
         if (whole_unit && row_unit) {
-          if constexpr (CK == kPrefixPass) {
-            // the group's partial result for each member's heads
-            const int s0 = __ldg(a.grp_start + cc.i);
+          if (tg == 0) {
 #pragma unroll
             for (int j = 0; j < G; ++j) {
-              if (j >= nreal) continue;
-              const int64_t rowx = int64_t(s0 + j / a.g_real) * H + cc.g * a.g_real + j % a.g_real;
-              if (tg == 0) {
-                const float inv = vscale / lall[j];
-                float4* dst = reinterpret_cast<float4*>(a.pre_o + rowx * D + c * EPV);
-#pragma unroll
-                for (int e4 = 0; e4 < EPV / 4; ++e4)
-                  dst[e4] = make_float4(o[j][4 * e4] * inv, o[j][4 * e4 + 1] * inv, o[j][4 * e4 + 2] * inv,
-                                        o[j][4 * e4 + 3] * inv);
+              // query row j -> (sequence, head); a group row's rows past its
+              // last member are dropped, and a member that attended nothing
+              // (no context) gets a zero row
+              int seq = cc.i, head = cc.g * G + j;
+              if constexpr (CK == kGroup) {
+                if (j >= nreal) continue;
+                seq = cg.s0 + j / a.g_real;
+                head = cc.g * a.g_real + j % a.g_real;
               }
-              if (lane == 0) a.pre_lse[rowx] = (m[j] + log2f(lall[j])) * 0.69314718055994530942f;
-            }
-          } else {
-            const bool has_pre = CK == kSuffixPass && ST[cc.i] > 0;
-            if (tg == 0) {
-              Tq* ob = reinterpret_cast<Tq*>(a.out) + int64_t(cc.i) * a.o_sb;
+              const float inv = (CK != kGroup || lall[j] > 0.f) ? vscale / lall[j] : 0.f;
+              float f[EPV];
 #pragma unroll
-              for (int j = 0; j < G; ++j) {
-                const float inv = vscale / lall[j];
-                float f[EPV];
-                if (has_pre) {
-                  // merge with the shared prefix's partial by log-sum-exp
-                  const int64_t rowx = int64_t(cc.i) * H + cc.g * G + j;
-                  const float lr = (m[j] + log2f(lall[j])) * 0.69314718055994530942f;
-                  const float lp = a.pre_lse[rowx];
-                  const float mx = fmaxf(lr, lp);
-                  const float wr = ex2((lr - mx) * 1.4426950408889634f), wp = ex2((lp - mx) * 1.4426950408889634f);
-                  const float r = 1.f / (wr + wp);
-                  const float* po = a.pre_o + rowx * D + c * EPV;
-#pragma unroll
-                  for (int e = 0; e < EPV; ++e) f[e] = (wr * (o[j][e] * inv) + wp * po[e]) * r;
-                } else {
-#pragma unroll
-                  for (int e = 0; e < EPV; ++e) f[e] = o[j][e] * inv;
-                }
-                store_out<Tq, EPV>(ob + int64_t(cc.g * G + j) * a.o_sh + c * EPV, f);
-              }
+              for (int e = 0; e < EPV; ++e) f[e] = o[j][e] * inv;
+              store_out<Tq, EPV>(reinterpret_cast<Tq*>(a.out) + int64_t(seq) * a.o_sb + int64_t(head) * a.o_sh + c * EPV,
+                                 f);
             }
           }
         } else if (whole_unit) {
@@ -1097,7 +1155,9 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
           if (tg == 0) {
 #pragma unroll
             for (int j = 0; j < G; ++j) {
-              const float inv = vscale / lall[j];
+              // (a group row's row that attended nothing in this segment: a
+              // zero share of weight 0)
+              const float inv = (CK != kGroup || lall[j] > 0.f) ? vscale / lall[j] : 0.f;
               float4* dst = reinterpret_cast<float4*>(a.sh_o + (slot * G + j) * D + c * EPV);
 #pragma unroll
               for (int e4 = 0; e4 < EPV / 4; ++e4)
@@ -1113,7 +1173,8 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
                 mj = m[j];
                 lj = lall[j];
               }
-            a.sh_lse[slot * G + lane] = (mj + log2f(lj)) * 0.69314718055994530942f;
+            a.sh_lse[slot * G + lane] =
+                (CK == kGroup && !(lj > 0.f)) ? -INFINITY : (mj + log2f(lj)) * 0.69314718055994530942f;
           }
           const bool last = share_done(a.ws_cnt + wa, cc.p - seg_p0 + 1, unp);
           if (is_tail)
@@ -1135,34 +1196,17 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
                 for (int e = 0; e < PER; ++e) dst[e] = acc[j][e];
                 if (lane == 0) a.ws_lse[base + j * a.P_max] = lse_m[j];
               }
-            } else if constexpr (CK == kPrefixPass) {
-              const int s0 = __ldg(a.grp_start + cc.i);
-#pragma unroll
-              for (int j = 0; j < G; ++j) {
-                if (j >= nreal) continue;
-                const int64_t rowx = int64_t(s0 + j / a.g_real) * H + cc.g * a.g_real + j % a.g_real;
-                float* dst = a.pre_o + rowx * D + lane * PER;
-#pragma unroll
-                for (int e = 0; e < PER; ++e) dst[e] = acc[j][e];
-                if (lane == 0) a.pre_lse[rowx] = lse_m[j];
-              }
             } else {
-              const bool has_pre = CK == kSuffixPass && ST[cc.i] > 0;
-              Tq* ob = reinterpret_cast<Tq*>(a.out) + int64_t(cc.i) * a.o_sb + lane * PER;
 #pragma unroll
               for (int j = 0; j < G; ++j) {
-                if (has_pre) {
-                  const int64_t rowx = int64_t(cc.i) * H + cc.g * G + j;
-                  const float lp = a.pre_lse[rowx];
-                  const float mx = fmaxf(lse_m[j], lp);
-                  const float wr = ex2((lse_m[j] - mx) * 1.4426950408889634f);
-                  const float wp = ex2((lp - mx) * 1.4426950408889634f);
-                  const float r = 1.f / (wr + wp);
-                  const float* po = a.pre_o + rowx * D + lane * PER;
-#pragma unroll
-                  for (int e = 0; e < PER; ++e) acc[j][e] = (wr * acc[j][e] + wp * po[e]) * r;
+                int seq = cc.i, head = cc.g * G + j;
+                if constexpr (CK == kGroup) {
+                  if (j >= nreal) continue;
+                  seq = cg.s0 + j / a.g_real;
+                  head = cc.g * a.g_real + j % a.g_real;
                 }
-                store_out_small<Tq, PER>(ob + int64_t(cc.g * G + j) * a.o_sh, acc[j]);
+                store_out_small<Tq, PER>(
+                    reinterpret_cast<Tq*>(a.out) + int64_t(seq) * a.o_sb + int64_t(head) * a.o_sh + lane * PER, acc[j]);
               }
             }
           }
@@ -1181,30 +1225,32 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
           } while (cc.i < U && S[cc.i + 1] == S[cc.i]);
           if (cc.i < U) cc.np = (S[cc.i + 1] - S[cc.i]) / Hkv;
         }
+        if constexpr (CK == kGroup)
+          if (cc.i < U) group_seek(cg, a, groups_ok, PB, cc.i, 0, ctx_cap);
+      } else {
+        if constexpr (CK == kGroup) group_next(cg, a, ctx_cap);
       }
       if (++s == a.stages) s = 0;
     }
   }
 
-  // ---- sequences with no pages in this launch: zero output rows (no
-  // context), or, after a shared prefix with nothing past it, its result ----
-  if constexpr (CK != kPrefixPass) {
-    for (int64_t i = wid; i < a.B; i += nworkers) {
-      if (S[i + 1] != S[i]) continue;
-      const bool has_pre = CK == kSuffixPass && ST[i] > 0;
-      Tq* ob = reinterpret_cast<Tq*>(a.out) + i * a.o_sb;
-      constexpr int OVR = C::QROWB / 16;  // 16-byte vectors per output row
+  // ---- row sequences with no pages: zero output rows (no context; in a
+  // shared-prefix decode, every member of such a group) ----
+  for (int64_t i = wid; i < U; i += nworkers) {
+    if (S[i + 1] != S[i]) continue;
+    int s0 = int(i), n = 1;
+    if constexpr (CK == kGroup) {
+      if (groups_ok) {
+        s0 = __ldg(a.grp_start + i);
+        n = __ldg(a.grp_start + i + 1) - s0;
+      }
+    }
+    constexpr int OVR = C::QROWB / 16;  // 16-byte vectors per output row
+    for (int mm = 0; mm < n; ++mm) {
+      Tq* ob = reinterpret_cast<Tq*>(a.out) + int64_t(s0 + mm) * a.o_sb;
       for (int idx = lane; idx < H * OVR; idx += 32) {
         const int h = idx / OVR, cc2 = idx % OVR;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (has_pre) {
-          float f[EPQ];
-          const float* po = a.pre_o + (i * H + h) * D + cc2 * EPQ;
-#pragma unroll
-          for (int e = 0; e < EPQ; ++e) f[e] = po[e];
-          v = Elem<Tq>::pack(f);
-        }
-        *reinterpret_cast<uint4*>(ob + int64_t(h) * a.o_sh + cc2 * EPQ) = v;
+        *reinterpret_cast<uint4*>(ob + int64_t(h) * a.o_sh + cc2 * EPQ) = make_uint4(0, 0, 0, 0);
       }
     }
   }
@@ -1213,13 +1259,14 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
 // ---- log-sum-exp merge of partial results ----------------------------------
 // out = sum_p exp(lse_p - LSE) o_p, LSE = log sum_p exp(lse_p), with o_p the
 // normalised partial outputs of fixed partitions.  One CTA of kMergeWarps
-// warps per (sequence, query head) with more than one partition: warp w
+// warps per (sequence, query head) with more than one partition (the merge
+// is bound by load latency, so many warps each keep loads in flight): warp w
 // takes partitions w, w + kMergeWarps, ...; lanes first find the warp's
 // largest lse, then weight 32 partitions at a time and broadcast the
 // weights while every lane streams its dims (several partitions' loads in
 // flight); the warps' results are combined through shared memory in warp
 // order (a fixed order, so the result does not depend on timing).
-constexpr int kMergeWarps = 8;
+constexpr int kMergeWarps = 16;
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kMergeWarps * 32) merge_fixed_kernel(const DecodeArgs a, int part_tokens) {
@@ -1250,7 +1297,7 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_fixed_kernel(const Dec
     const int tl = c0 + lane;
     const float wl = tl < mine ? ex2((__ldcg(lse + warp + NW * tl) - mw) * kLog2e) : 0.f;
     const int n = mine - c0 < 32 ? mine - c0 : 32;
-#pragma unroll 4
+#pragma unroll 8
     for (int t = 0; t < n; ++t) {
       const float w = __shfl_sync(0xffffffffu, wl, t);
       const float* src = ob + int64_t(warp + NW * (c0 + t)) * D + lane * PER;

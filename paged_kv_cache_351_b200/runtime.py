@@ -173,11 +173,20 @@ class PagedKVCacheGPU:
             else:
                 dec = prepare_decode(out, query, self.k_cache, self.v_cache, block_tables, context_lens, scale,
                                      self.num_kv_heads, workspace, partition_tokens, stream=stream)
-        has_new = slots.numel() > 0
+        return PreparedStep(write if slots.numel() > 0 else None, dec)
 
-        def step():
-            if has_new:
-                write()
-            dec()
 
-        return step
+class PreparedStep:
+    """A serving step as prepared library calls: ``write`` (the new tokens'
+    cache write, None when the step appends nothing) and ``decode``; calling
+    the step runs both, in that order, on the stream they were prepared
+    with."""
+
+    def __init__(self, write, decode):
+        self.write = write
+        self.decode = decode
+
+    def __call__(self) -> None:
+        if self.write is not None:
+            self.write()
+        self.decode()
