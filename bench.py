@@ -577,20 +577,14 @@ def run_ours(args):
     else:
         ws = kv.workspace(plan.B, w.num_heads, bt.shape[1], args.partition)
 
-    def decode(o_, q_, bt_, cl_, gs_=None, gb_=None):
-        if groups:
-            kv.decode_shared(o_, q_, bt_, cl_, gs_d if gs_ is None else gs_, gb_d if gb_ is None else gb_, groups[2],
-                             scale, partition_tokens=args.partition, stream=stream, workspace=ws)
-        else:
-            kv.decode(o_, q_, bt_, cl_, scale, partition_tokens=args.partition, stream=stream, workspace=ws)
-
     # cache write (when the step appends tokens) + decode (two passes for a
     # shared-prefix decode); fixed partitions add the log-sum-exp merge kernel
     launches_per_step = (1 if len(inp["slots"]) else 0) + (2 if groups else 1) + (1 if args.partition > 0 else 0)
 
-    def step():
-        kv.write(slots, key, value, None, stream=stream)
-        decode(out, q, bt, cl)
+    # the step as prepared library calls (descriptors built once), so that
+    # per-step Python work does not leave the GPU idle between launches
+    step = kv.prepare_step(slots, key, value, out, q, bt, cl, scale, partition_tokens=args.partition, stream=stream,
+                           workspace=ws, groups=(gs_d, gb_d, groups[2]) if groups else None)
 
     with torch.cuda.stream(stream):
         for _ in range(max(3, args.warmup)):
@@ -627,7 +621,7 @@ def run_ours(args):
     with torch.cuda.stream(stream):
         for k in range(K):
             ea[k].record(stream)
-            decode(out, q, bt, cl)
+            step.decode()
             eb[k].record(stream)
     torch.cuda.synchronize()
     dec_ms = statistics.mean(ea[k].elapsed_time(eb[k]) for k in range(K))
