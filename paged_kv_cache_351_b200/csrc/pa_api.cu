@@ -47,7 +47,9 @@ Tuning g_tuning;
 // registers.
 // An FP8 cache doubles the dequantization and math per byte, so it wants 12
 // warps even at G = 1 (+20% on the LLaMA-7B shape).
-int default_warps(int G, bool fp8 = false) { return (G == 2 || G == 4 || fp8) ? 12 : 8; }
+// An FP8 cache at G = 1 (scalar page math, 126 registers) is latency-bound
+// per page and takes 16.
+int default_warps(int G, bool fp8 = false) { return (fp8 && G == 1) ? 16 : (G == 2 || G == 4 || fp8) ? 12 : 8; }
 
 // Cache elements per 16-byte vector (dims per lane) of a cache dtype.
 int epv_of(int32_t kv_dtype) { return kv_dtype == PA_F32 ? 4 : kv_dtype == PA_FP8_E4M3 ? 16 : 8; }

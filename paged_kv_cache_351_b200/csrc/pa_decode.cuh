@@ -47,17 +47,18 @@
 namespace pa {
 
 constexpr int kBS = 16;        // tokens per block (block_size)
-constexpr int kMaxWarps = 12;  // workers per CTA (registers allow 12 at G <= 4)
+constexpr int kMaxWarps = 16;  // workers per CTA (the most any shape allows)
 
 // Warps per CTA the register budget allows without spills: a lane of the
 // scalar path keeps the query and output of G heads x EPV dims in registers
 // (2 G EPV floats); at 128 or more (bf16 G = 8) only 8 warps fit.  The FP8
-// path (EPV = 16) keeps tensor-core fragments instead and runs 12 up to
-// G = 4 (its segment end gathers G x 16 outputs per lane).  Registers are
-// split per SM sub-partition: 9 to 12 warps put 3 on one and leave 168
-// registers per thread, 8 warps leave 255.
+// path (EPV = 16) keeps tensor-core fragments instead and runs 12 at G = 2
+// or 4 (its segment end gathers G x 16 outputs per lane); its G = 1 scalar
+// path fits 126 registers and runs 16.  Registers are split per SM
+// sub-partition: 13 to 16 warps leave 128 registers per thread, 9 to 12 warps
+// 168, 8 warps 255.
 __host__ __device__ constexpr int max_warps_for(int G, int EPV) {
-  return EPV == 16 ? (G >= 8 ? 8 : kMaxWarps) : (2 * G * EPV >= 128 ? 8 : kMaxWarps);
+  return EPV == 16 ? (G >= 8 ? 8 : (G == 1 ? 16 : 12)) : (2 * G * EPV >= 128 ? 8 : 12);
 }
 
 enum DecodeMode : int32_t { kBalanced = 0, kFixed = 1, kNoSplit = 2 };
