@@ -33,6 +33,33 @@ def test_decode_step_bytes_brute_force(name):
     assert got["step"] == got["decode"] + got["write"]
 
 
+def test_shared_prefix_unique_bytes_brute_force():
+    """The sampling workload under a shared-prefix decode: the unique KV
+    bytes are the distinct (physical block, kv head, slot) entries the step
+    attends, found by replaying the requests on the oracle allocator and
+    walking every sequence's table; the groups come from the oracle's model
+    of the grouping rule."""
+    from oracle.cascade import prefix_groups
+    from oracle.replay import replay
+
+    plan = make_plan("parallel_sampling_13b")
+    w = plan.workload
+    alloc, _, _ = replay(plan, write_values=False)
+    tables = [alloc.block_table(int(s)) for s in plan.batch]
+    lens = [int(c) for c in plan.context_lens]
+    gs, gb = prefix_groups(tables, lens, 4, w.block_size)
+    assert all(b > 0 for b in gb)
+    got = bench.step_bytes(plan, (np.array(gs), np.array(gb)))
+    read = set()
+    for t, c in zip(tables, lens):
+        for pos in range(c):
+            read.add((t[pos // w.block_size], pos % w.block_size))
+    per_slot = 2 * w.num_kv_heads * w.head_size * w.cache_elem_bytes
+    assert got["kv"] == len(read) * per_slot
+    assert got["kv_logical"] == sum(lens) * per_slot
+    assert got["kv"] < got["kv_logical"] / 3
+
+
 @pytest.mark.parametrize("name", ["prefill_tiny", "prefill_mixed_gqa"])
 def test_prefill_flops_brute_force(name):
     plan = make_plan(name)
