@@ -219,6 +219,22 @@ def max_over_ranks(values, device, world):
     return [float(v) for v in t.tolist()]
 
 
+def warm(step, stream, warmup, min_busy_s=0.05):
+    """Untimed warm-up: at least max(3, warmup) steps, continued in bursts
+    until the GPU has been kept busy for min_busy_s of wall time, then a
+    synchronize."""
+    import torch
+
+    t0 = time.perf_counter()
+    n = 0
+    with torch.cuda.stream(stream):
+        while n < max(3, warmup) or time.perf_counter() - t0 < min_busy_s:
+            for _ in range(max(3, warmup)):
+                step()
+            n += max(3, warmup)
+            torch.cuda.synchronize()
+
+
 def aggregate_value(bytes_per_step, ms_per_step, world):
     """Whole-job GB/s: every replica moves bytes_per_step per step; the step
     time is the max over ranks."""
@@ -586,20 +602,19 @@ def run_ours(args):
     step = kv.prepare_step(slots, key, value, out, q, bt, cl, scale, partition_tokens=args.partition, stream=stream,
                            workspace=ws, groups=(gs_d, gb_d, groups[2]) if groups else None)
 
-    with torch.cuda.stream(stream):
-        for _ in range(max(3, args.warmup)):
-            step()
-    torch.cuda.synchronize()
-    st, bits = pa.pa_get_device_status(stream)
-    if st != 0:
-        raise RuntimeError(f"device status {st} bits {bits:#x} after warm-up")
-
     K = args.steps
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     uuid = str(torch.cuda.get_device_properties(device).uuid)
     uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
     sampler = ClockSampler(uuid)
     time.sleep(0.25)
+    # Warm-up right before the timed region (the sampler's start leaves the
+    # GPU idle, and clocks drop when idle): W steps, continued until the GPU
+    # has been busy for at least 50 ms.
+    warm(step, stream, args.warmup)
+    st, bits = pa.pa_get_device_status(stream)
+    if st != 0:
+        raise RuntimeError(f"device status {st} bits {bits:#x} after warm-up")
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -850,18 +865,15 @@ def run_prefill(args, plan, device, world, rank):
         kv.write(slots, key, value, None, stream=stream)
         attend(out, q, bt, cl, qs)
 
-    with torch.cuda.stream(stream):
-        for _ in range(max(3, args.warmup)):
-            step()
-    torch.cuda.synchronize()
-    st, bits = pa.pa_get_device_status(stream)
-    if st != 0:
-        raise RuntimeError(f"device status {st} bits {bits:#x} after warm-up")
     K = args.steps
     uuid = str(torch.cuda.get_device_properties(device).uuid)
     uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
     sampler = ClockSampler(uuid)
     time.sleep(0.25)
+    warm(step, stream, args.warmup)
+    st, bits = pa.pa_get_device_status(stream)
+    if st != 0:
+        raise RuntimeError(f"device status {st} bits {bits:#x} after warm-up")
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
