@@ -206,6 +206,15 @@ def ncu_traffic(workload, kernel="decode_kernel", files=("pa_decode.cuh", "pa_co
         return None
 
 
+def profile_key(name, partition, shared, groupable):
+    """Workload key of the ncu summary that matches the launch bench times:
+    the workload name, plus the partition size in fixed-partition mode, plus
+    "_no_prefix_groups" when a workload with shared prompts is decoded
+    without the shared-prefix path."""
+    key = name if partition <= 0 else f"{name}_{partition}"
+    return key + "_no_prefix_groups" if groupable and not shared else key
+
+
 def max_over_ranks(values, device, world):
     """Each rank's device-timed values -> their maximum over all ranks (the
     job is as slow as its slowest replica)."""
@@ -574,10 +583,10 @@ def run_ours(args):
     dev, tdt = inp["dev"], inp["tdt"]
     # shared-prefix decode when forks of one prompt share leading blocks
     groups = None
-    if args.cascade != "off":
-        gs_h, gb_h, max_group = kv.prefix_groups(plan.batch, w.num_heads)
-        if (gb_h > 0).any() or args.cascade == "on":
-            groups = (gs_h, gb_h, max_group)
+    gs_h, gb_h, max_group = kv.prefix_groups(plan.batch, w.num_heads)
+    grouped = bool((gb_h > 0).any())
+    if args.cascade == "on" or (args.cascade == "auto" and grouped):
+        groups = (gs_h, gb_h, max_group)
     nbytes = step_bytes(plan, groups[:2] if groups else None)
     q = dev(inp["query"])
     key, value = dev(inp["key"]), dev(inp["value"])
@@ -593,9 +602,9 @@ def run_ours(args):
     else:
         ws = kv.workspace(plan.B, w.num_heads, bt.shape[1], args.partition)
 
-    # cache write (when the step appends tokens) + decode (two passes for a
-    # shared-prefix decode); fixed partitions add the log-sum-exp merge kernel
-    launches_per_step = (1 if len(inp["slots"]) else 0) + (2 if groups else 1) + (1 if args.partition > 0 else 0)
+    # cache write (when the step appends tokens) + decode (one launch, also
+    # for a shared-prefix decode); fixed partitions add the merge kernel
+    launches_per_step = (1 if len(inp["slots"]) else 0) + 1 + (1 if args.partition > 0 else 0)
 
     # the step as prepared library calls (descriptors built once), so that
     # per-step Python work does not leave the GPU idle between launches
@@ -672,7 +681,7 @@ def run_ours(args):
                "sample": f"{r['rows']} whole sequences (all 32 heads) of the same workload in {r['seconds']:.1f} s"}
 
     achieved = nbytes["decode"] / (dec_ms * 1e-3) / 1e9
-    traffic = ncu_traffic(w.name)
+    traffic = ncu_traffic(profile_key(w.name, args.partition, groups is not None, grouped))
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
@@ -696,8 +705,9 @@ def run_ours(args):
         "bytes_per_step": nbytes,
         "allocator": allocator_report(plan),
         "roofline": {"bound": "hbm",
-                     "kernel": ("pa_decode_cascade (decode_kernel prefix pass + suffix pass)" if groups
-                                else "pa_decode (decode_kernel, log-sum-exp merge fused)"),
+                     "kernel": ("pa_decode_cascade (decode_kernel, shared-prefix groups, one launch)" if groups
+                                else "pa_decode (decode_kernel + merge_fixed_kernel, fixed partitions)"
+                                if args.partition > 0 else "pa_decode (decode_kernel, log-sum-exp merge fused)"),
                      "achieved": round(achieved, 2), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
                      "algorithmic_bytes_per_launch": nbytes["decode"], "avg_launch_ms": round(dec_ms, 5),
