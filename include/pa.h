@@ -206,10 +206,12 @@ pa_status pa_decode(pa_tensor* out, const pa_tensor* query, const pa_tensor* k_c
 
 /* Launch shape of pa_decode on the current process (a tuning knob; 0 keeps
  * the default): warps per CTA (each warp is one worker with its own page
- * ring; default 8 for G = 1 or 8 and 12 for G = 2 or 4, where G = num_heads /
- * num_kv_heads; at most 12, and 8 at G = 8), ring stages per warp (default 2; lowered
- * automatically to fit shared memory), CTAs per SM (default 1).  Changes
- * the workspace size of the auto mode.  Not thread-safe. */
+ * ring; G = num_heads / num_kv_heads.  bf16 or fp32 cache: default 8 for
+ * G = 1 or 8 and 12 for G = 2 or 4, at most 12 (8 for bf16 at G = 8).  FP8
+ * cache: default and most 16 up to G = 4, 8 at G = 8), ring stages per warp
+ * (default 2; lowered automatically to fit shared memory), CTAs per SM
+ * (default 1).  Changes the workspace size of the auto mode.  Not
+ * thread-safe. */
 pa_status pa_set_decode_tuning(int32_t warps_per_cta, int32_t stages, int32_t ctas_per_sm);
 
 /* ---------------------------------------------------------------------------

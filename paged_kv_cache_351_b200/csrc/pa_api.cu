@@ -7,6 +7,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
@@ -45,11 +46,11 @@ Tuning g_tuning;
 // pages in flight; grouped heads (G = 2, 4) do more math per page and need
 // 12 warps to hide it (+15% on the GQA workload); G = 8 is capped at 8 by
 // registers.
-// An FP8 cache doubles the dequantization and math per byte, so it wants 12
-// warps even at G = 1 (+20% on the LLaMA-7B shape).
-// An FP8 cache at G = 1 (scalar page math, 126 registers) is latency-bound
-// per page and takes 16.
-int default_warps(int G, bool fp8 = false) { return (fp8 && G == 1) ? 16 : (G == 2 || G == 4 || fp8) ? 12 : 8; }
+// An FP8 cache doubles the dequantization and math per byte and takes 16
+// warps up to G = 4 (at G = 1 the scalar page math in 126 registers, at
+// G = 2 and 4 the tensor-core page math with the query in shared memory);
+// G = 8 keeps 8.
+int default_warps(int G, bool fp8 = false) { return (fp8 && G <= 4) ? 16 : (G == 2 || G == 4 || fp8) ? 12 : 8; }
 
 // Cache elements per 16-byte vector (dims per lane) of a cache dtype.
 int epv_of(int32_t kv_dtype) { return kv_dtype == PA_F32 ? 4 : kv_dtype == PA_FP8_E4M3 ? 16 : 8; }
@@ -612,8 +613,9 @@ pa_status pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_heads, int32_t
   pa_status st = device_info(&di, nullptr);
   if (st != PA_OK) return st;
   const int G = num_heads / num_kv_heads;
-  // an upper bound over cache types (FP8 may cap the warps lower)
-  const int64_t workers = int64_t(di.sms) * g_tuning.ctas_per_sm * (g_tuning.warps ? g_tuning.warps : default_warps(G, true));
+  // an upper bound over cache types (the warps per CTA differ by cache type)
+  const int64_t workers = int64_t(di.sms) * g_tuning.ctas_per_sm *
+                          (g_tuning.warps ? g_tuning.warps : std::max(default_warps(G, false), default_warps(G, true)));
   if (partition_tokens > 0) {
     const int64_t pp = partition_tokens / pa::kBS;
     int64_t P = (max_blocks_per_seq + pp - 1) / pp;

@@ -52,14 +52,19 @@ constexpr int kMaxWarps = 16;  // workers per CTA (the most any shape allows)
 // Warps per CTA the register budget allows without spills: a lane of the
 // scalar path keeps the query and output of G heads x EPV dims in registers
 // (2 G EPV floats); at 128 or more (bf16 G = 8) only 8 warps fit.  The FP8
-// path (EPV = 16) keeps tensor-core fragments instead and runs 12 at G = 2
-// or 4 (its segment end gathers G x 16 outputs per lane); its G = 1 scalar
-// path fits 126 registers and runs 16.  Registers are split per SM
-// sub-partition: 13 to 16 warps leave 128 registers per thread, 9 to 12 warps
-// 168, 8 warps 255.
+// path (EPV = 16) runs 16 warps up to G = 4: its G = 1 scalar path fits 126
+// registers, and its tensor-core path (G >= 2) keeps the query's f16 parts
+// in shared memory and writes its results straight from the MMA fragments
+// (measured on the GQA batch-256 FP8 decode: 0.186 ms with 12 warps and the
+// query in registers, 0.169 ms with 12 warps and 0.161 ms with 16 after the
+// change).  Registers are split per SM sub-partition: 13 to 16 warps leave
+// 128 registers per thread, 9 to 12 warps 168, 8 warps 255.
 __host__ __device__ constexpr int max_warps_for(int G, int EPV) {
-  return EPV == 16 ? (G >= 8 ? 8 : (G == 1 ? 16 : 12)) : (2 * G * EPV >= 128 ? 8 : 12);
+  return EPV == 16 ? (G >= 8 ? 8 : 16) : (2 * G * EPV >= 128 ? 8 : 12);
 }
+
+// Smallest group size whose FP8 page math runs on the tensor cores.
+constexpr int kFp8MmaMinG = 2;
 
 enum DecodeMode : int32_t { kBalanced = 0, kFixed = 1, kNoSplit = 2 };
 
@@ -121,7 +126,12 @@ struct DecodeCfg {
   static constexpr int QBYTES = G * QROWB;           // the group's query rows
   static constexpr int STAGE = 2 * PAGE + QBYTES;  // K page, V page, query rows
   static constexpr int GH = G >= 2 ? G / 2 : 1;    // heads a lane holds after the butterfly
-  static constexpr int PBUF = G * kBS * 4;         // probabilities of one page
+  // FP8 cache, G >= kFp8MmaMinG: tensor-core page math, whose f16 query
+  // parts (high and low, 2 x 16 words for each of the 4 G lanes that hold a
+  // real head) live in shared memory after the probabilities
+  static constexpr bool MMA = sizeof(Tkv) == 1 && G >= kFp8MmaMinG;
+  static constexpr int QLO = MMA ? 4 * G * 128 : 0;
+  static constexpr int PBUF = G * kBS * 4 + QLO;   // probabilities of one page (+ low query parts)
   static constexpr int LOG2_NT = NT == 16 ? 4 : NT == 8 ? 3 : NT == 4 ? 2 : NT == 2 ? 1 : 0;
   static_assert(LPT >= 8 && LPT <= 32 && (LPT & (LPT - 1)) == 0, "row of 128, 256 or 512 bytes");
   static_assert(2 * NT == LPT, "lane layout");
@@ -133,11 +143,11 @@ struct DecodeCfg {
   }
 };
 
-// smem carve-up: [scan scratch: 32 int32][S: (U+1) int32][first page: X int32],
+// smem carve-up: [scan scratch: 32 int32][S: (U+1) int32][PB: X int32],
 // padded to 128 bytes, then one region per warp (DecodeCfg::warp_bytes).  U
-// is the number of row sequences (the batch, or the groups of a prefix
-// pass); X is B for a suffix pass (each sequence's first block after its
-// group's shared prefix), else 0.
+// is the number of row sequences (the batch, or the groups of a
+// shared-prefix decode); X is U for a shared-prefix decode (each group's
+// shared block count), else 0.
 __host__ __device__ inline size_t decode_prefix_bytes(int U, int X = 0) {
   return (size_t(U + 1 + 32 + X) * 4 + 127) / 128 * 128;
 }
@@ -674,10 +684,14 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
     // decode; its 16-byte operand loads hit 4x the shared-memory wavefronts
     // of the conflict-free scalar layout, since the page rows are 256 bytes
     // apart.  Not kept.)
-    constexpr bool kMma = sizeof(Tkv) == 1 && G >= 2;
+    constexpr bool kMma = C::MMA;
     const int gr = lane >> 2, tig = lane & 3;
-    uint32_t qf[16];     // query of head gr, f16 pairs of this lane's 32 dims
-    uint32_t ql[16];     // the f16 rounding error of qf (q = qf + ql to about 2^-22)
+    // query of head gr as f16 pairs of this lane's 32 dims (qf) and the f16
+    // rounding error of qf (ql; q = qf + ql to about 2^-22), kept in shared
+    // memory for the lanes of real heads (lane = 4 gr + tig < 4 G; the other
+    // lanes' query is zero): vector v (4 words) of lane l at qhl[v * 4 G + l],
+    // qf in v = 0..3, ql in v = 4..7
+    uint4* const qhl = reinterpret_cast<uint4*>(pbuf + G * kBS);
     float oacc[8][4];    // O^T fragments
     float mh[2], lh[2];  // running max and denominator of heads 2 tig, 2 tig + 1
     float sfac[2];       // power-of-two factor undoing the query's range normalisation
@@ -735,6 +749,7 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
           mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
           const int ex = mx > 0.f ? ilogbf(mx) - 14 : 0;
           const float down = ldexpf(1.f, -ex);
+          uint32_t qf[16], ql[16];
 #pragma unroll
           for (int j2 = 0; j2 < 16; ++j2) {
             const float a0 = qv[2 * j2] * down, a1 = qv[2 * j2 + 1] * down;
@@ -742,6 +757,13 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
             float h0, h1;
             f16x2_to_f32(qf[j2], h0, h1);
             ql[j2] = pack_f16x2(a0 - h0, a1 - h1);
+          }
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            if (gr < G) {
+              qhl[v * 4 * G + lane] = make_uint4(qf[4 * v], qf[4 * v + 1], qf[4 * v + 2], qf[4 * v + 3]);
+              qhl[(v + 4) * 4 * G + lane] = make_uint4(ql[4 * v], ql[4 * v + 1], ql[4 * v + 2], ql[4 * v + 3]);
+            }
           }
           const float up = ldexpf(1.f, ex);
           sfac[0] = __shfl_sync(0xffffffffu, up, (2 * tig) * 4);
@@ -817,8 +839,11 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
             // dims + {2, 3} -> k 2 tig + 8, 2 tig + 9
             const uint32_t af[4] = {e4m3x2_lo_to_f16x2(r0[kk]), e4m3x2_lo_to_f16x2(r1[kk]),
                                     e4m3x2_hi_to_f16x2(r0[kk]), e4m3x2_hi_to_f16x2(r1[kk])};
-            mma_16816_f16((kk & 1) ? sb : sa, af, qf[2 * kk], qf[2 * kk + 1]);
-            mma_16816_f16((kk & 1) ? lb : la, af, ql[2 * kk], ql[2 * kk + 1]);
+            const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+            const uint4 hw = gr < G ? qhl[(kk >> 1) * 4 * G + lane] : z4;
+            const uint4 lw = gr < G ? qhl[(4 + (kk >> 1)) * 4 * G + lane] : z4;
+            mma_16816_f16((kk & 1) ? sb : sa, af, (kk & 1) ? hw.z : hw.x, (kk & 1) ? hw.w : hw.y);
+            mma_16816_f16((kk & 1) ? lb : la, af, (kk & 1) ? lw.z : lw.x, (kk & 1) ? lw.w : lw.y);
           }
 #pragma unroll
           for (int k = 0; k < 4; ++k) sa[k] = (sa[k] + sb[k]) + (la[k] + lb[k]);
@@ -1051,23 +1076,22 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
       // ---- segment end: combine lanes and write ----
       const bool seg_last = (cx == hi - 1) || last_of_row || (a.mode == kFixed && (cc.p + 1) % a.part_pages == 0);
       if (seg_last) {
+        // Each lane owns some (query row j, chunk of EPV dims) pieces of the
+        // segment's result and calls put(j, chunk, values, max, denominator,
+        // writes_lse) for each.  Scalar path: lanes 0..LPT-1 (tg = 0) own
+        // chunk c of every row, lane 0 writes the rows' lse.  Tensor-core
+        // path: lane (gr, tig) already holds dims [16 gr, 16 gr + 16) of rows
+        // 2 tig and 2 tig + 1 in its O^T fragments and writes them from
+        // there (no gather into a per-lane copy of every row).
         float lall[G];
+        float lrow[2];
         if constexpr (kMma) {
-          // Back to the layout below: lanes 0..LPT-1 (tg = 0) hold dims
-          // [EPV c, EPV c + EPV) of every head; m and lall in every lane.
-          float lr0 = lh[0], lr1 = lh[1];
+          lrow[0] = lh[0];
+          lrow[1] = lh[1];
 #pragma unroll
           for (int msk = 4; msk < 32; msk <<= 1) {
-            lr0 += __shfl_xor_sync(0xffffffffu, lr0, msk);
-            lr1 += __shfl_xor_sync(0xffffffffu, lr1, msk);
-          }
-#pragma unroll
-          for (int j = 0; j < G; ++j) {
-            m[j] = __shfl_sync(0xffffffffu, (j & 1) ? mh[1] : mh[0], j >> 1);
-            lall[j] = __shfl_sync(0xffffffffu, (j & 1) ? lr1 : lr0, j >> 1);
-#pragma unroll
-            for (int e = 0; e < EPV; ++e)
-              o[j][e] = __shfl_sync(0xffffffffu, oacc[e >> 1][(j & 1) + 2 * (e & 1)], (lane % LPT) * 4 + (j >> 1));
+            lrow[0] += __shfl_xor_sync(0xffffffffu, lrow[0], msk);
+            lrow[1] += __shfl_xor_sync(0xffffffffu, lrow[1], msk);
           }
         } else {
 #pragma unroll
@@ -1091,6 +1115,25 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
           }
         }
         }
+        auto for_owned = [&](auto&& put) {
+          if constexpr (kMma) {
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              const int j = 2 * tig + hh;
+              if (j < G) {
+                float f[EPV];
+#pragma unroll
+                for (int e = 0; e < EPV; ++e) f[e] = oacc[e >> 1][hh + 2 * (e & 1)];
+                put(j, gr, f, mh[hh], lrow[hh], gr == 0);
+              }
+            }
+          } else {
+            if (tg == 0) {
+#pragma unroll
+              for (int j = 0; j < G; ++j) put(j, c, o[j], m[j], lall[j], c == 0);
+            }
+          }
+        };
         // This segment's unit: the row, or in fixed mode its partition.  A
         // unit that spans the whole row gives the row's output; a partition
         // of a longer row gives a partial for the merge kernel.
@@ -1099,50 +1142,34 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
         const bool row_unit = unp == cc.np;
         const bool whole_unit = seg_p0 == up0 && cc.p == up0 + unp - 1;
         if (whole_unit && row_unit) {
-          if (tg == 0) {
-#pragma unroll
-            for (int j = 0; j < G; ++j) {
-              // query row j -> (sequence, head); a group row's rows past its
-              // last member are dropped, and a member that attended nothing
-              // (no context) gets a zero row
-              int seq = cc.i, head = cc.g * G + j;
-              if constexpr (CK == kGroup) {
-                if (j >= nreal) continue;
-                seq = cg.s0 + j / a.g_real;
-                head = cc.g * a.g_real + j % a.g_real;
-              }
-              const float inv = (CK != kGroup || lall[j] > 0.f) ? vscale / lall[j] : 0.f;
-              float f[EPV];
-#pragma unroll
-              for (int e = 0; e < EPV; ++e) f[e] = o[j][e] * inv;
-              store_out<Tq, EPV>(reinterpret_cast<Tq*>(a.out) + int64_t(seq) * a.o_sb + int64_t(head) * a.o_sh + c * EPV,
-                                 f);
+          for_owned([&](int j, int ch, const float* f, float, float l, bool) {
+            // query row j -> (sequence, head); a group row's rows past its
+            // last member are dropped, and a member that attended nothing
+            // (no context) gets a zero row
+            int seq = cc.i, head = cc.g * G + j;
+            if constexpr (CK == kGroup) {
+              if (j >= nreal) return;
+              seq = cg.s0 + j / a.g_real;
+              head = cc.g * a.g_real + j % a.g_real;
             }
-          }
+            const float inv = (CK != kGroup || l > 0.f) ? vscale / l : 0.f;
+            float y[EPV];
+#pragma unroll
+            for (int e = 0; e < EPV; ++e) y[e] = f[e] * inv;
+            store_out<Tq, EPV>(reinterpret_cast<Tq*>(a.out) + int64_t(seq) * a.o_sb + int64_t(head) * a.o_sh + ch * EPV,
+                               y);
+          });
         } else if (whole_unit) {
           // fixed mode: one partial per partition; a separate kernel merges them
           const int64_t base = (int64_t(cc.i) * H + int64_t(cc.g) * G) * a.P_max + cc.p / a.part_pages;
-          if (tg == 0) {
+          for_owned([&](int j, int ch, const float* f, float mj, float l, bool lse_lane) {
+            const float inv = vscale / l;
+            float4* dst = reinterpret_cast<float4*>(a.ws_o + (base + j * a.P_max) * D + ch * EPV);
 #pragma unroll
-            for (int j = 0; j < G; ++j) {
-              const float inv = vscale / lall[j];
-              float4* dst = reinterpret_cast<float4*>(a.ws_o + (base + j * a.P_max) * D + c * EPV);
-#pragma unroll
-              for (int e4 = 0; e4 < EPV / 4; ++e4)
-                dst[e4] = make_float4(o[j][4 * e4] * inv, o[j][4 * e4 + 1] * inv, o[j][4 * e4 + 2] * inv,
-                                      o[j][4 * e4 + 3] * inv);
-            }
-          }
-          if (lane < G) {
-            float mj = m[0], lj = lall[0];
-#pragma unroll
-            for (int j = 1; j < G; ++j)
-              if (lane == j) {
-                mj = m[j];
-                lj = lall[j];
-              }
-            a.ws_lse[base + lane * a.P_max] = (mj + log2f(lj)) * 0.69314718055994530942f;
-          }
+            for (int e4 = 0; e4 < EPV / 4; ++e4)
+              dst[e4] = make_float4(f[4 * e4] * inv, f[4 * e4 + 1] * inv, f[4 * e4 + 2] * inv, f[4 * e4 + 3] * inv);
+            if (lse_lane) a.ws_lse[base + j * a.P_max] = (mj + log2f(l)) * 0.69314718055994530942f;
+          });
         } else {
           // A unit cut by a worker boundary: publish this worker's share
           // (normalised output + log-sum-exp) in its slot, then count its
@@ -1153,30 +1180,18 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
           const int64_t wa = unit_first * nworkers / W;
           const bool is_tail = (seg_p0 == up0);
           const int64_t slot = 2 * wid + (is_tail ? 1 : 0);
-          if (tg == 0) {
+          for_owned([&](int j, int ch, const float* f, float mj, float l, bool lse_lane) {
+            // (a group row's row that attended nothing in this segment: a
+            // zero share of weight 0)
+            const float inv = (CK != kGroup || l > 0.f) ? vscale / l : 0.f;
+            float4* dst = reinterpret_cast<float4*>(a.sh_o + (slot * G + j) * D + ch * EPV);
 #pragma unroll
-            for (int j = 0; j < G; ++j) {
-              // (a group row's row that attended nothing in this segment: a
-              // zero share of weight 0)
-              const float inv = (CK != kGroup || lall[j] > 0.f) ? vscale / lall[j] : 0.f;
-              float4* dst = reinterpret_cast<float4*>(a.sh_o + (slot * G + j) * D + c * EPV);
-#pragma unroll
-              for (int e4 = 0; e4 < EPV / 4; ++e4)
-                dst[e4] = make_float4(o[j][4 * e4] * inv, o[j][4 * e4 + 1] * inv, o[j][4 * e4 + 2] * inv,
-                                      o[j][4 * e4 + 3] * inv);
-            }
-          }
-          if (lane < G) {
-            float mj = m[0], lj = lall[0];
-#pragma unroll
-            for (int j = 1; j < G; ++j)
-              if (lane == j) {
-                mj = m[j];
-                lj = lall[j];
-              }
-            a.sh_lse[slot * G + lane] =
-                (CK == kGroup && !(lj > 0.f)) ? -INFINITY : (mj + log2f(lj)) * 0.69314718055994530942f;
-          }
+            for (int e4 = 0; e4 < EPV / 4; ++e4)
+              dst[e4] = make_float4(f[4 * e4] * inv, f[4 * e4 + 1] * inv, f[4 * e4 + 2] * inv, f[4 * e4 + 3] * inv);
+            if (lse_lane)
+              a.sh_lse[slot * G + j] =
+                  (CK == kGroup && !(l > 0.f)) ? -INFINITY : (mj + log2f(l)) * 0.69314718055994530942f;
+          });
           const bool last = share_done(a.ws_cnt + wa, cc.p - seg_p0 + 1, unp);
           if (is_tail)
             tail_in = true;

@@ -258,7 +258,7 @@ def test_fixed_workspace_layout():
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     n = pa.pa_decode_workspace_bytes(8, 32, 8, 128, 8192, 512)
     P = 8192 * 16 // 512
-    workers = sms * 12  # G = 4: 12 warps per SM
+    workers = sms * 16  # G = 4: 12 warps per SM over a bf16 cache, 16 over FP8 (the larger)
     shares = 2 * workers * 4 * 128 * 4 + (2 * workers * 4 * 4 + 255) // 256 * 256
     assert n == pa.PA_DECODE_WS_HEADER_BYTES + 8 * 32 * P * 128 * 4 + 8 * 32 * P * 4 + shares
 
