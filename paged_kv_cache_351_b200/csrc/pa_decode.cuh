@@ -130,7 +130,10 @@ struct DecodeCfg {
   // parts (high and low, 2 x 16 words for each of the 4 G lanes that hold a
   // real head) live in shared memory after the probabilities
   static constexpr bool MMA = sizeof(Tkv) == 1 && G >= kFp8MmaMinG;
-  static constexpr int QLO = MMA ? 4 * G * 128 : 0;
+  // G <= 4: the high and low parts share one 8-column B fragment (below):
+  // 16 words per lane
+  static constexpr bool PACKQ = MMA && G <= 4;
+  static constexpr int QLO = !MMA ? 0 : PACKQ ? 32 * 64 : 4 * G * 128;
   static constexpr int PBUF = G * kBS * 4 + QLO;   // probabilities of one page (+ low query parts)
   static constexpr int LOG2_NT = NT == 16 ? 4 : NT == 8 ? 3 : NT == 4 ? 2 : NT == 2 ? 1 : 0;
   static_assert(LPT >= 8 && LPT <= 32 && (LPT & (LPT - 1)) == 0, "row of 128, 256 or 512 bytes");
@@ -692,6 +695,10 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
     // lanes' query is zero): vector v (4 words) of lane l at qhl[v * 4 G + l],
     // qf in v = 0..3, ql in v = 4..7
     uint4* const qhl = reinterpret_cast<uint4*>(pbuf + G * kBS);
+    // G <= 4: the B fragment's 8 columns are the G heads' high parts
+    // (columns 0..3) and their low parts (columns 4..7), so one MMA per
+    // k-step covers both; lane (gr, tig) keeps the part of head gr & 3 that
+    // column gr holds at qhl[v * 32 + lane], v = 0..3
     float oacc[8][4];    // O^T fragments
     float mh[2], lh[2];  // running max and denominator of heads 2 tig, 2 tig + 1
     float sfac[2];       // power-of-two factor undoing the query's range normalisation
@@ -729,9 +736,10 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
         if constexpr (CK == kGroup) nreal = cg.n * a.g_real;
         if constexpr (kMma) {
           float qv[32];
-          if (gr < nreal) {
+          const int hq = C::PACKQ ? (gr & 3) : gr;  // the head whose query this lane holds
+          if (hq < nreal && hq < G) {
 #pragma unroll
-            for (int v = 0; v < 4; ++v) Elem<Tq>::unpack(qs[gr * (C::QROWB / 16) + tig * 4 + v], qv + 8 * v);
+            for (int v = 0; v < 4; ++v) Elem<Tq>::unpack(qs[hq * (C::QROWB / 16) + tig * 4 + v], qv + 8 * v);
           } else {
 #pragma unroll
             for (int e = 0; e < 32; ++e) qv[e] = 0.f;
@@ -758,11 +766,18 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
             f16x2_to_f32(qf[j2], h0, h1);
             ql[j2] = pack_f16x2(a0 - h0, a1 - h1);
           }
+          if constexpr (C::PACKQ) {
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            if (gr < G) {
-              qhl[v * 4 * G + lane] = make_uint4(qf[4 * v], qf[4 * v + 1], qf[4 * v + 2], qf[4 * v + 3]);
-              qhl[(v + 4) * 4 * G + lane] = make_uint4(ql[4 * v], ql[4 * v + 1], ql[4 * v + 2], ql[4 * v + 3]);
+            for (int v = 0; v < 4; ++v)
+              qhl[v * 32 + lane] = gr < 4 ? make_uint4(qf[4 * v], qf[4 * v + 1], qf[4 * v + 2], qf[4 * v + 3])
+                                          : make_uint4(ql[4 * v], ql[4 * v + 1], ql[4 * v + 2], ql[4 * v + 3]);
+          } else {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              if (gr < G) {
+                qhl[v * 4 * G + lane] = make_uint4(qf[4 * v], qf[4 * v + 1], qf[4 * v + 2], qf[4 * v + 3]);
+                qhl[(v + 4) * 4 * G + lane] = make_uint4(ql[4 * v], ql[4 * v + 1], ql[4 * v + 2], ql[4 * v + 3]);
+              }
             }
           }
           const float up = ldexpf(1.f, ex);
@@ -839,15 +854,41 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
             // dims + {2, 3} -> k 2 tig + 8, 2 tig + 9
             const uint32_t af[4] = {e4m3x2_lo_to_f16x2(r0[kk]), e4m3x2_lo_to_f16x2(r1[kk]),
                                     e4m3x2_hi_to_f16x2(r0[kk]), e4m3x2_hi_to_f16x2(r1[kk])};
-            const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
-            const uint4 hw = gr < G ? qhl[(kk >> 1) * 4 * G + lane] : z4;
-            const uint4 lw = gr < G ? qhl[(4 + (kk >> 1)) * 4 * G + lane] : z4;
-            mma_16816_f16((kk & 1) ? sb : sa, af, (kk & 1) ? hw.z : hw.x, (kk & 1) ? hw.w : hw.y);
-            mma_16816_f16((kk & 1) ? lb : la, af, (kk & 1) ? lw.z : lw.x, (kk & 1) ? lw.w : lw.y);
+            if constexpr (C::PACKQ) {
+              const uint4 qw = qhl[(kk >> 1) * 32 + lane];
+              mma_16816_f16((kk & 1) ? sb : sa, af, (kk & 1) ? qw.z : qw.x, (kk & 1) ? qw.w : qw.y);
+            } else {
+              const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+              const uint4 hw = gr < G ? qhl[(kk >> 1) * 4 * G + lane] : z4;
+              const uint4 lw = gr < G ? qhl[(4 + (kk >> 1)) * 4 * G + lane] : z4;
+              mma_16816_f16((kk & 1) ? sb : sa, af, (kk & 1) ? hw.z : hw.x, (kk & 1) ? hw.w : hw.y);
+              mma_16816_f16((kk & 1) ? lb : la, af, (kk & 1) ? lw.z : lw.x, (kk & 1) ? lw.w : lw.y);
+            }
           }
+          if constexpr (C::PACKQ) {
+            // columns 2 tig, 2 tig + 1 (high parts, tig < 2) plus columns
+            // 2 tig + 4, 2 tig + 5 (low parts), held by lane tig ^ 2
 #pragma unroll
-          for (int k = 0; k < 4; ++k) sa[k] = (sa[k] + sb[k]) + (la[k] + lb[k]);
+            for (int k = 0; k < 4; ++k) {
+              sa[k] += sb[k];
+              sa[k] += __shfl_xor_sync(0xffffffffu, sa[k], 2);
+            }
+          } else {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) sa[k] = (sa[k] + sb[k]) + (la[k] + lb[k]);
+          }
         }
+        // this lane's V rows, loaded before the softmax so that their latency
+        // overlaps it; tokens past the context may hold any codes (NaN would
+        // survive p = 0)
+        const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+        const uint4 va = 2 * tig < valid ? *reinterpret_cast<const uint4*>(Vb + (2 * tig) * 128 + gr * 16) : zero;
+        const uint4 vb =
+            2 * tig + 1 < valid ? *reinterpret_cast<const uint4*>(Vb + (2 * tig + 1) * 128 + gr * 16) : zero;
+        const uint4 vc =
+            2 * tig + 8 < valid ? *reinterpret_cast<const uint4*>(Vb + (2 * tig + 8) * 128 + gr * 16) : zero;
+        const uint4 vd =
+            2 * tig + 9 < valid ? *reinterpret_cast<const uint4*>(Vb + (2 * tig + 9) * 128 + gr * 16) : zero;
         // sa = {S[gr][2tig], S[gr][2tig+1], S[gr+8][2tig], S[gr+8][2tig+1]} (log2 units)
         float sc4[4] = {sa[0] * sfac[0], sa[1] * sfac[1], sa[2] * sfac[0], sa[3] * sfac[1]};
         if (gr >= valid) sc4[0] = sc4[1] = -INFINITY;
@@ -905,15 +946,6 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
         }
         // ---- O^T += V^T P: rows = dims 16 gr + 2 mm (+1), k = tokens ----
         {
-          const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
-          // tokens past the context may hold any codes (NaN would survive p = 0)
-          const uint4 va = 2 * tig < valid ? *reinterpret_cast<const uint4*>(Vb + (2 * tig) * 128 + gr * 16) : zero;
-          const uint4 vb =
-              2 * tig + 1 < valid ? *reinterpret_cast<const uint4*>(Vb + (2 * tig + 1) * 128 + gr * 16) : zero;
-          const uint4 vc =
-              2 * tig + 8 < valid ? *reinterpret_cast<const uint4*>(Vb + (2 * tig + 8) * 128 + gr * 16) : zero;
-          const uint4 vd =
-              2 * tig + 9 < valid ? *reinterpret_cast<const uint4*>(Vb + (2 * tig + 9) * 128 + gr * 16) : zero;
           const uint32_t wa[4] = {va.x, va.y, va.z, va.w}, wb[4] = {vb.x, vb.y, vb.z, vb.w};
           const uint32_t wc[4] = {vc.x, vc.y, vc.z, vc.w}, wd[4] = {vd.x, vd.y, vd.z, vd.w};
 #pragma unroll
