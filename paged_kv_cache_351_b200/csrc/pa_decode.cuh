@@ -360,15 +360,21 @@ __device__ __forceinline__ bool worker_empty(int64_t k, int64_t W, int64_t N) {
 __device__ __forceinline__ int64_t share_slot(int64_t k, int64_t wa) { return 2 * k + (k == wa ? 1 : 0); }
 
 // Counts `mine` pages of a row into its counter (one lane; every lane of the
-// warp has published its part of the share and fenced before).  True for
+// warp has published its part of the share before a warp barrier).  True for
 // the worker whose pages complete the row: it resets the counter, so every
 // counter is zero again when the launch ends, and it alone merges the row.
 // Nobody waits for anybody.  A counter that overshoots the row (a workspace
 // whose counters did not start at zero) sets PA_DEV_BAD_WORKSPACE.
 __device__ __forceinline__ bool count_in(unsigned int* cnt, unsigned int mine, unsigned int total) {
-  const unsigned int now = atomicAdd(cnt, mine) + mine;
+  // acquire-release: the caller's share (made visible to this lane by the
+  // warp barrier before) is released with the count, and the last arriver
+  // acquires every other worker's share with it
+  unsigned int old;
+  asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], %2;" : "=r"(old) : "l"(cnt), "r"(mine) : "memory");
+  const unsigned int now = old + mine;
   if (now < total) return false;
-  atomicExch(cnt, 0u);
+  // nobody else touches the counter again in this launch
+  asm volatile("st.relaxed.gpu.u32 [%0], %1;" ::"l"(cnt), "r"(0u) : "memory");
   if (now > total) {
     flag(PA_DEV_BAD_WORKSPACE);
     return false;
@@ -377,14 +383,15 @@ __device__ __forceinline__ bool count_in(unsigned int* cnt, unsigned int mine, u
 }
 
 // Warp-collective: publish-then-count for this warp's share of a cut row.
-// Returns (in every lane) whether this worker completes the row.
+// Returns (in every lane) whether this worker completes the row.  The warp
+// barriers order every lane's share stores before lane 0's release, and
+// lane 0's acquire before every lane's reads of the other shares.
 __device__ __forceinline__ bool share_done(unsigned int* cnt, int mine, int total) {
-  __threadfence();  // each lane's share stores, before the count
   __syncwarp();
   int last = 0;
   if ((threadIdx.x & 31) == 0) last = count_in(cnt, unsigned(mine), unsigned(total));
   last = __shfl_sync(0xffffffffu, last, 0);
-  if (last) __threadfence();  // the count, before reading the other shares
+  __syncwarp();
   return last != 0;
 }
 
@@ -403,10 +410,18 @@ __device__ __forceinline__ void merge_shares(const float* ws_o, const float* ws_
   constexpr int PER = D / 32;
   constexpr float kLog2e = 1.4426950408889634f;
   const int lane = threadIdx.x & 31;
-  float mx[G], wsum[G];
+  // the lse values of the first 32 shares stay in registers (lane t: share
+  // wa + t); most rows have only a few shares
+  float l0[G], mx[G], wsum[G];
+  {
+    const int64_t kl = wa + lane;
+    const bool mine = kl <= wb && !worker_empty(kl, W, N);
 #pragma unroll
-  for (int j = 0; j < G; ++j) mx[j] = -INFINITY;
-  for (int64_t k = wa + lane; k <= wb; k += 32) {
+    for (int j = 0; j < G; ++j) l0[j] = mine ? __ldcg(ws_lse + share_slot(kl, wa) * G + j) : -INFINITY;
+  }
+#pragma unroll
+  for (int j = 0; j < G; ++j) mx[j] = l0[j];
+  for (int64_t k = wa + 32 + lane; k <= wb; k += 32) {
     if (worker_empty(k, W, N)) continue;
     const int64_t slot = share_slot(k, wa);
 #pragma unroll
@@ -421,23 +436,33 @@ __device__ __forceinline__ void merge_shares(const float* ws_o, const float* ws_
     for (int e = 0; e < PER; ++e) acc[j][e] = 0.f;
   }
   for (int64_t k0 = wa; k0 <= wb; k0 += 32) {
-    // this lane's share of the chunk: its weights (0 for none)
+    // this lane's share of the chunk: its weights (0 for none, and for a row
+    // with no weight anywhere: a row of a group that attended nothing)
     const int64_t kl = k0 + lane;
-    const bool mine = kl <= wb && !worker_empty(kl, W, N);
     float wl[G];
+    if (k0 == wa) {
 #pragma unroll
-    for (int j = 0; j < G; ++j)  // (a row with no weight anywhere: a row of a group that attended nothing)
-      wl[j] = (mine && mx[j] != -INFINITY) ? ex2((__ldcg(ws_lse + share_slot(kl, wa) * G + j) - mx[j]) * kLog2e)
-                                            : 0.f;
+      for (int j = 0; j < G; ++j) wl[j] = (l0[j] != -INFINITY && mx[j] != -INFINITY) ? ex2((l0[j] - mx[j]) * kLog2e) : 0.f;
+    } else {
+      const bool mine = kl <= wb && !worker_empty(kl, W, N);
+#pragma unroll
+      for (int j = 0; j < G; ++j)
+        wl[j] = (mine && mx[j] != -INFINITY) ? ex2((__ldcg(ws_lse + share_slot(kl, wa) * G + j) - mx[j]) * kLog2e)
+                                              : 0.f;
+    }
     const int n = int(wb - k0 + 1 < 32 ? wb - k0 + 1 : 32);
 #pragma unroll 4
     for (int t = 0; t < n; ++t) {
       float w[G];
+      bool any = false;
 #pragma unroll
-      for (int j = 0; j < G; ++j) w[j] = __shfl_sync(0xffffffffu, wl[j], t);
-      // an empty worker's slot was never written: skip it (its weight is 0)
+      for (int j = 0; j < G; ++j) {
+        w[j] = __shfl_sync(0xffffffffu, wl[j], t);
+        any |= w[j] != 0.f;
+      }
+      // a share of no weight (an empty worker's slot, never written) is skipped
+      if (!any) continue;
       const int64_t slot = share_slot(k0 + t, wa);
-      if (w[0] == 0.f && worker_empty(k0 + t, W, N)) continue;
 #pragma unroll
       for (int j = 0; j < G; ++j) {
         wsum[j] += w[j];
@@ -557,30 +582,6 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
   const unsigned char* vcb = reinterpret_cast<const unsigned char*>(a.vc);
 
   if (lo < hi) {
-    // The cut units this worker holds pages of (at most two: one that began
-    // in an earlier worker, one that continues in a later one), so that a
-    // worker giving up early still counts its pages in and leaves every
-    // counter at zero.
-    int64_t head_wa = -1, tail_wa = -1;
-    int head_pages = 0, head_np = 0, tail_pages = 0, tail_np = 0;
-    if (a.mode != kNoSplit) {
-      int64_t f0, f1;
-      int n0, n1;
-      unit_of(locate(S, U, Hkv, lo), S, a.mode, a.part_pages, &f0, &n0);
-      if (lo != f0) {
-        head_wa = f0 * nworkers / W;
-        head_np = n0;
-        head_pages = int((hi < f0 + n0 ? hi : f0 + n0) - lo);
-      }
-      unit_of(locate(S, U, Hkv, hi - 1), S, a.mode, a.part_pages, &f1, &n1);
-      if (hi != f1 + n1 && f1 >= lo) {
-        tail_wa = wid;
-        tail_np = n1;
-        tail_pages = int(hi - f1);
-      }
-    }
-    bool head_in = false, tail_in = false;  // counted in already
-
     // ---- producer cursor (warp-uniform) ----
     RowPos pc = locate(S, U, Hkv, lo);
     int64_t px = lo;
@@ -718,11 +719,20 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
           const int s2 = int((s + (y - cx)) % a.stages);
           mbar_wait_bounded(smem_u32(&bars[s2]), (phase >> s2) & 1u, a.timeout_ns);
         }
-        // count the unfinished shares in (their rows are left unwritten; the
-        // status word reports the timeout) so the counters end at zero
-        if (lane == 0) {
-          if (head_wa >= 0 && !head_in) count_in(a.ws_cnt + head_wa, unsigned(head_pages), unsigned(head_np));
-          if (tail_wa >= 0 && !tail_in) count_in(a.ws_cnt + tail_wa, unsigned(tail_pages), unsigned(tail_np));
+        // Count the unfinished shares in (their rows are left unwritten; the
+        // status word reports the timeout) so the counters end at zero.  A
+        // worker holds pages of at most two cut units: one that began in an
+        // earlier worker (counted in once the consumer has passed its end)
+        // and one that continues in a later one (at the end of the range,
+        // not yet counted in while the consumer is inside the range).
+        if (lane == 0 && a.mode != kNoSplit) {
+          int64_t f0, f1;
+          int n0, n1;
+          unit_of(locate(S, U, Hkv, lo), S, a.mode, a.part_pages, &f0, &n0);
+          const int64_t e0 = hi < f0 + n0 ? hi : f0 + n0;
+          if (lo != f0 && cx < e0) count_in(a.ws_cnt + f0 * nworkers / W, unsigned(e0 - lo), unsigned(n0));
+          unit_of(locate(S, U, Hkv, hi - 1), S, a.mode, a.part_pages, &f1, &n1);
+          if (hi != f1 + n1 && f1 >= lo) count_in(a.ws_cnt + wid, unsigned(hi - f1), unsigned(n1));
         }
         return;
       }
@@ -1225,10 +1235,6 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
                   (CK == kGroup && !(l > 0.f)) ? -INFINITY : (mj + log2f(l)) * 0.69314718055994530942f;
           });
           const bool last = share_done(a.ws_cnt + wa, cc.p - seg_p0 + 1, unp);
-          if (is_tail)
-            tail_in = true;
-          else
-            head_in = true;
           if (last) {
             constexpr int PER = D / 32;
             const int64_t wb = (unit_first + unp - 1) * nworkers / W;
