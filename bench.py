@@ -24,6 +24,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import math
 import os
@@ -176,11 +177,19 @@ def measured_tensor_peak():
         return 1590.0, "fallback"
 
 
+_CODE_TOKENS = re.compile(r'"(?:\\.|[^"\\\n])*"|//[^\n]*|/\*.*?\*/', re.S)
+
+
 def kernel_source_hash(files=("pa_decode.cuh", "pa_common.cuh")):
+    """Hash of a kernel's source files with comments removed and blank
+    space collapsed: it changes when the code does, not when a comment is
+    reworded (string literals, such as inline PTX, are kept)."""
     h = hashlib.sha256()
     for f in files:
-        with open(os.path.join(ROOT, "paged_kv_cache_351_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "paged_kv_cache_351_b200", "csrc", f)) as fh:
+            text = fh.read()
+        code = _CODE_TOKENS.sub(lambda m: m.group(0) if m.group(0).startswith('"') else " ", text)
+        h.update(" ".join(code.split()).encode())
     return h.hexdigest()[:16]
 
 

@@ -740,7 +740,7 @@ static pa_status launch_kind(const DecodeCall& dc, int G, const pa::DecodeArgs& 
     if (dt == PA_FP8_E4M3 && D == 128)
       return dispatch_group<__nv_fp8_e4m3, __nv_bfloat16, 128, CK>(G, a, plan, s, dev);
   } else {
-    // shared-prefix passes: bf16 head size 128 and fp32 head size 64
+    // shared-prefix decode: bf16 head size 128 and fp32 head size 64
     if (dt == PA_BF16 && D == 128) return dispatch_group<__nv_bfloat16, __nv_bfloat16, 128, CK>(G, a, plan, s, dev);
     if (dt == PA_F32 && D == 64) return dispatch_group<float, float, 64, CK>(G, a, plan, s, dev);
   }

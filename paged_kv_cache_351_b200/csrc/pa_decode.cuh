@@ -705,7 +705,7 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
     float sfac[2];       // power-of-two factor undoing the query's range normalisation
     float vscale = 1.f;
     int ctx_i = 0;
-    int nreal = G;       // query rows that belong to a sequence (prefix pass: members x g_real)
+    int nreal = G;       // query rows that belong to a sequence (a group row: members x g_real)
     uint32_t phase = 0;  // bit s = parity of the next wait on stage s
     int s = 0;
 

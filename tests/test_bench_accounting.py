@@ -216,3 +216,22 @@ def test_reference_arm_bounds_each_step(name):
     assert time.time() - t0 < 120
     d = json.loads([l for l in res.stdout.splitlines() if l.startswith("{")][0])
     assert d["steps"] == 2000 and d["value"] > 0
+
+
+def test_kernel_source_hash_ignores_comments_not_code(tmp_path, monkeypatch):
+    """The profiles' kernel_source_sha: rewording a comment or re-spacing keeps
+    the hash, any code change (including inside an inline-PTX string) does
+    not, and a '//' inside a string literal is code."""
+    csrc = tmp_path / "paged_kv_cache_351_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+
+    def h(text):
+        (csrc / "k.cuh").write_text(text)
+        return bench.kernel_source_hash(("k.cuh",))
+
+    base = h('int f(int x) {  // add one\n  /* block\n comment */ return x + 1;\n}\nconst char* s = "a//b";\n')
+    assert h('int f(int x) {  // add ONE, reworded\n  return   x + 1;\n}\nconst char* s = "a//b";\n') == base
+    assert h('int f(int x) {\n  return x + 2;\n}\nconst char* s = "a//b";\n') != base
+    assert h('int f(int x) {\n  return x + 1;\n}\nconst char* s = "a//c";\n') != base
+    assert h('int f(int x) {\n  return x + 1;\n}\nconst char* s = "a";\n') != base
