@@ -696,10 +696,12 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
     // lanes' query is zero): vector v (4 words) of lane l at qhl[v * 4 G + l],
     // qf in v = 0..3, ql in v = 4..7
     uint4* const qhl = reinterpret_cast<uint4*>(pbuf + G * kBS);
-    // G <= 4: the B fragment's 8 columns are the G heads' high parts
-    // (columns 0..3) and their low parts (columns 4..7), so one MMA per
-    // k-step covers both; lane (gr, tig) keeps the part of head gr & 3 that
-    // column gr holds at qhl[v * 32 + lane], v = 0..3
+    // G <= 4: the B fragment's 8 columns are each head's high part (column
+    // 2 h) and low part (column 2 h + 1), so one MMA per k-step covers both
+    // and lane (gr, tig) ends with both parts of head tig's scores; lane
+    // (gr, tig) keeps the part that column gr holds (head gr >> 1) at
+    // qhl[v * 32 + lane], v = 0..3.  Its softmax state (mh[0], lh[0]) is then
+    // that of head tig.
     float oacc[8][4];    // O^T fragments
     float mh[2], lh[2];  // running max and denominator of heads 2 tig, 2 tig + 1
     float sfac[2];       // power-of-two factor undoing the query's range normalisation
@@ -746,7 +748,7 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
         if constexpr (CK == kGroup) nreal = cg.n * a.g_real;
         if constexpr (kMma) {
           float qv[32];
-          const int hq = C::PACKQ ? (gr & 3) : gr;  // the head whose query this lane holds
+          const int hq = C::PACKQ ? (gr >> 1) : gr;  // the head whose query this lane holds
           if (hq < nreal && hq < G) {
 #pragma unroll
             for (int v = 0; v < 4; ++v) Elem<Tq>::unpack(qs[hq * (C::QROWB / 16) + tig * 4 + v], qv + 8 * v);
@@ -779,8 +781,8 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
           if constexpr (C::PACKQ) {
 #pragma unroll
             for (int v = 0; v < 4; ++v)
-              qhl[v * 32 + lane] = gr < 4 ? make_uint4(qf[4 * v], qf[4 * v + 1], qf[4 * v + 2], qf[4 * v + 3])
-                                          : make_uint4(ql[4 * v], ql[4 * v + 1], ql[4 * v + 2], ql[4 * v + 3]);
+              qhl[v * 32 + lane] = (gr & 1) == 0 ? make_uint4(qf[4 * v], qf[4 * v + 1], qf[4 * v + 2], qf[4 * v + 3])
+                                                 : make_uint4(ql[4 * v], ql[4 * v + 1], ql[4 * v + 2], ql[4 * v + 3]);
           } else {
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
@@ -876,13 +878,9 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
             }
           }
           if constexpr (C::PACKQ) {
-            // columns 2 tig, 2 tig + 1 (high parts, tig < 2) plus columns
-            // 2 tig + 4, 2 tig + 5 (low parts), held by lane tig ^ 2
+            // columns 2 tig (high part) and 2 tig + 1 (low part) of head tig
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              sa[k] += sb[k];
-              sa[k] += __shfl_xor_sync(0xffffffffu, sa[k], 2);
-            }
+            for (int k = 0; k < 4; ++k) sa[k] += sb[k];
           } else {
 #pragma unroll
             for (int k = 0; k < 4; ++k) sa[k] = (sa[k] + sb[k]) + (la[k] + lb[k]);
@@ -899,52 +897,93 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
             2 * tig + 8 < valid ? *reinterpret_cast<const uint4*>(Vb + (2 * tig + 8) * 128 + gr * 16) : zero;
         const uint4 vd =
             2 * tig + 9 < valid ? *reinterpret_cast<const uint4*>(Vb + (2 * tig + 9) * 128 + gr * 16) : zero;
-        // sa = {S[gr][2tig], S[gr][2tig+1], S[gr+8][2tig], S[gr+8][2tig+1]} (log2 units)
-        float sc4[4] = {sa[0] * sfac[0], sa[1] * sfac[1], sa[2] * sfac[0], sa[3] * sfac[1]};
-        if (gr >= valid) sc4[0] = sc4[1] = -INFINITY;
-        if (gr + 8 >= valid) sc4[2] = sc4[3] = -INFINITY;
-        if constexpr (CK == kGroup) {  // rows (heads) that do not attend this page
-          if (2 * tig < alo || 2 * tig >= ahi) sc4[0] = sc4[2] = -INFINITY;
-          if (2 * tig + 1 < alo || 2 * tig + 1 >= ahi) sc4[1] = sc4[3] = -INFINITY;
-        }
-        float pm0 = fmaxf(sc4[0], sc4[2]), pm1 = fmaxf(sc4[1], sc4[3]);
-#pragma unroll
-        for (int msk = 4; msk < 32; msk <<= 1) {
-          pm0 = fmaxf(pm0, __shfl_xor_sync(0xffffffffu, pm0, msk));
-          pm1 = fmaxf(pm1, __shfl_xor_sync(0xffffffffu, pm1, msk));
-        }
-        // token 0 of every page is valid, so the maxima are finite; in a
-        // group row a row that has attended nothing yet keeps -inf (no
-        // rescale, zero probabilities)
-        const float mn0 = fmaxf(mh[0], pm0), mn1 = fmaxf(mh[1], pm1);
-        float al0 = ex2(mh[0] - mn0), al1 = ex2(mh[1] - mn1);
-        const bool grew = __any_sync(0xffffffffu, mn0 != mh[0] || mn1 != mh[1]);
-        mh[0] = mn0;
-        mh[1] = mn1;
-        float p0 = ex2(sc4[0] - mn0), p1 = ex2(sc4[1] - mn1), p2 = ex2(sc4[2] - mn0), p3 = ex2(sc4[3] - mn1);
-        if constexpr (CK == kGroup) {
-          if (mn0 == -INFINITY) al0 = 1.f, p0 = p2 = 0.f;
-          if (mn1 == -INFINITY) al1 = 1.f, p1 = p3 = 0.f;
-        }
-        lh[0] = lh[0] * al0 + (p0 + p2);
-        lh[1] = lh[1] * al1 + (p1 + p3);
-        if (grew) {
-#pragma unroll
-          for (int mm = 0; mm < 8; ++mm) {
-            oacc[mm][0] *= al0;
-            oacc[mm][1] *= al1;
-            oacc[mm][2] *= al0;
-            oacc[mm][3] *= al1;
+        if constexpr (C::PACKQ) {
+          // head tig at tokens gr and gr + 8 (log2 units)
+          float t0 = (sa[0] + sa[1]) * sfac[0], t1 = (sa[2] + sa[3]) * sfac[0];
+          if (gr >= valid) t0 = -INFINITY;
+          if (gr + 8 >= valid) t1 = -INFINITY;
+          if constexpr (CK == kGroup) {  // a row (head) that does not attend this page
+            if (tig < alo || tig >= ahi) t0 = t1 = -INFINITY;
           }
-        }
-        // probabilities [head][token] through shared memory into the B layout of P V
-        if (2 * tig < G) {
-          pbuf[(2 * tig) * kBS + gr] = p0;
-          pbuf[(2 * tig) * kBS + gr + 8] = p2;
-        }
-        if (2 * tig + 1 < G) {
-          pbuf[(2 * tig + 1) * kBS + gr] = p1;
-          pbuf[(2 * tig + 1) * kBS + gr + 8] = p3;
+          float pm = fmaxf(t0, t1);
+#pragma unroll
+          for (int msk = 4; msk < 32; msk <<= 1) pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, msk));
+          const float mn = fmaxf(mh[0], pm);
+          float al = ex2(mh[0] - mn);
+          const bool grew = __any_sync(0xffffffffu, mn != mh[0]);
+          mh[0] = mn;
+          float p0 = ex2(t0 - mn), p1 = ex2(t1 - mn);
+          if constexpr (CK == kGroup) {
+            if (mn == -INFINITY) al = 1.f, p0 = p1 = 0.f;
+          }
+          lh[0] = lh[0] * al + (p0 + p1);
+          if (grew) {
+            // the O^T columns of this lane are heads 2 tig and 2 tig + 1: their
+            // factors from lanes tig' = 2 tig, 2 tig + 1 (columns past the heads
+            // hold zeros)
+            const float alA = __shfl_sync(0xffffffffu, al, (2 * tig) & 3);
+            const float alB = __shfl_sync(0xffffffffu, al, (2 * tig + 1) & 3);
+#pragma unroll
+            for (int mm = 0; mm < 8; ++mm) {
+              oacc[mm][0] *= alA;
+              oacc[mm][1] *= alB;
+              oacc[mm][2] *= alA;
+              oacc[mm][3] *= alB;
+            }
+          }
+          // probabilities [head][token] through shared memory into the B layout of P V
+          if (tig < G) {
+            pbuf[tig * kBS + gr] = p0;
+            pbuf[tig * kBS + gr + 8] = p1;
+          }
+        } else {
+          // sa = {S[gr][2tig], S[gr][2tig+1], S[gr+8][2tig], S[gr+8][2tig+1]} (log2 units)
+          float sc4[4] = {sa[0] * sfac[0], sa[1] * sfac[1], sa[2] * sfac[0], sa[3] * sfac[1]};
+          if (gr >= valid) sc4[0] = sc4[1] = -INFINITY;
+          if (gr + 8 >= valid) sc4[2] = sc4[3] = -INFINITY;
+          if constexpr (CK == kGroup) {  // rows (heads) that do not attend this page
+            if (2 * tig < alo || 2 * tig >= ahi) sc4[0] = sc4[2] = -INFINITY;
+            if (2 * tig + 1 < alo || 2 * tig + 1 >= ahi) sc4[1] = sc4[3] = -INFINITY;
+          }
+          float pm0 = fmaxf(sc4[0], sc4[2]), pm1 = fmaxf(sc4[1], sc4[3]);
+#pragma unroll
+          for (int msk = 4; msk < 32; msk <<= 1) {
+            pm0 = fmaxf(pm0, __shfl_xor_sync(0xffffffffu, pm0, msk));
+            pm1 = fmaxf(pm1, __shfl_xor_sync(0xffffffffu, pm1, msk));
+          }
+          // token 0 of every page is valid, so the maxima are finite; in a
+          // group row a row that has attended nothing yet keeps -inf (no
+          // rescale, zero probabilities)
+          const float mn0 = fmaxf(mh[0], pm0), mn1 = fmaxf(mh[1], pm1);
+          float al0 = ex2(mh[0] - mn0), al1 = ex2(mh[1] - mn1);
+          const bool grew = __any_sync(0xffffffffu, mn0 != mh[0] || mn1 != mh[1]);
+          mh[0] = mn0;
+          mh[1] = mn1;
+          float p0 = ex2(sc4[0] - mn0), p1 = ex2(sc4[1] - mn1), p2 = ex2(sc4[2] - mn0), p3 = ex2(sc4[3] - mn1);
+          if constexpr (CK == kGroup) {
+            if (mn0 == -INFINITY) al0 = 1.f, p0 = p2 = 0.f;
+            if (mn1 == -INFINITY) al1 = 1.f, p1 = p3 = 0.f;
+          }
+          lh[0] = lh[0] * al0 + (p0 + p2);
+          lh[1] = lh[1] * al1 + (p1 + p3);
+          if (grew) {
+#pragma unroll
+            for (int mm = 0; mm < 8; ++mm) {
+              oacc[mm][0] *= al0;
+              oacc[mm][1] *= al1;
+              oacc[mm][2] *= al0;
+              oacc[mm][3] *= al1;
+            }
+          }
+          // probabilities [head][token] through shared memory into the B layout of P V
+          if (2 * tig < G) {
+            pbuf[(2 * tig) * kBS + gr] = p0;
+            pbuf[(2 * tig) * kBS + gr + 8] = p2;
+          }
+          if (2 * tig + 1 < G) {
+            pbuf[(2 * tig + 1) * kBS + gr] = p1;
+            pbuf[(2 * tig + 1) * kBS + gr + 8] = p3;
+          }
         }
         __syncwarp();
         uint32_t pb0 = 0u, pb1 = 0u;
@@ -1127,6 +1166,7 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
         // there (no gather into a per-lane copy of every row).
         float lall[G];
         float lrow[2];
+        float mrow[2];
         if constexpr (kMma) {
           lrow[0] = lh[0];
           lrow[1] = lh[1];
@@ -1134,6 +1174,17 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
           for (int msk = 4; msk < 32; msk <<= 1) {
             lrow[0] += __shfl_xor_sync(0xffffffffu, lrow[0], msk);
             lrow[1] += __shfl_xor_sync(0xffffffffu, lrow[1], msk);
+          }
+          mrow[0] = mh[0];
+          mrow[1] = mh[1];
+          if constexpr (C::PACKQ) {
+            // this lane's state is head tig's; its output columns are heads
+            // 2 tig and 2 tig + 1
+            const float l0 = lrow[0], m0 = mh[0];
+            lrow[0] = __shfl_sync(0xffffffffu, l0, (2 * tig) & 3);
+            lrow[1] = __shfl_sync(0xffffffffu, l0, (2 * tig + 1) & 3);
+            mrow[0] = __shfl_sync(0xffffffffu, m0, (2 * tig) & 3);
+            mrow[1] = __shfl_sync(0xffffffffu, m0, (2 * tig + 1) & 3);
           }
         } else {
 #pragma unroll
@@ -1166,7 +1217,7 @@ __global__ void __launch_bounds__(max_warps_for(G, 16 / int(sizeof(Tkv))) * 32, 
                 float f[EPV];
 #pragma unroll
                 for (int e = 0; e < EPV; ++e) f[e] = oacc[e >> 1][hh + 2 * (e & 1)];
-                put(j, gr, f, mh[hh], lrow[hh], gr == 0);
+                put(j, gr, f, mrow[hh], lrow[hh], gr == 0);
               }
             }
           } else {
