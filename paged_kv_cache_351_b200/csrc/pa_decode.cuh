@@ -52,13 +52,12 @@ constexpr int kMaxWarps = 16;  // workers per CTA (the most any shape allows)
 // Warps per CTA the register budget allows without spills: a lane of the
 // scalar path keeps the query and output of G heads x EPV dims in registers
 // (2 G EPV floats); at 128 or more (bf16 G = 8) only 8 warps fit.  The FP8
-// path (EPV = 16) runs 16 warps up to G = 4: its G = 1 scalar path fits 126
-// registers, and its tensor-core path (G >= 2) keeps the query's f16 parts
-// in shared memory and writes its results straight from the MMA fragments
-// (measured on the GQA batch-256 FP8 decode: 0.186 ms with 12 warps and the
-// query in registers, 0.169 ms with 12 warps and 0.161 ms with 16 after the
-// change).  Registers are split per SM sub-partition: 13 to 16 warps leave
-// 128 registers per thread, 9 to 12 warps 168, 8 warps 255.
+// path (EPV = 16) runs 16 warps up to G = 4: its G = 1 scalar path fits in
+// 128 registers, and so does its tensor-core path (G >= 2), which keeps the
+// query's f16 parts in shared memory and writes its results straight from
+// the MMA fragments (measured on the GQA batch-256 FP8 decode: 0.169 ms with
+// 12 warps, 0.161 ms with 16).  Registers are split per SM sub-partition: 13
+// to 16 warps leave 128 registers per thread, 9 to 12 warps 168, 8 warps 255.
 __host__ __device__ constexpr int max_warps_for(int G, int EPV) {
   return EPV == 16 ? (G >= 8 ? 8 : 16) : (2 * G * EPV >= 128 ? 8 : 12);
 }
@@ -127,14 +126,14 @@ struct DecodeCfg {
   static constexpr int STAGE = 2 * PAGE + QBYTES;  // K page, V page, query rows
   static constexpr int GH = G >= 2 ? G / 2 : 1;    // heads a lane holds after the butterfly
   // FP8 cache, G >= kFp8MmaMinG: tensor-core page math, whose f16 query
-  // parts (high and low, 2 x 16 words for each of the 4 G lanes that hold a
-  // real head) live in shared memory after the probabilities
+  // parts live in shared memory after the probabilities: for G <= 4 (PACKQ)
+  // a head's high and low parts are two columns of one 8-column B fragment,
+  // 16 words per lane; for G = 8 both parts, 2 x 16 words for each of the
+  // 4 G lanes that hold a head
   static constexpr bool MMA = sizeof(Tkv) == 1 && G >= kFp8MmaMinG;
-  // G <= 4: the high and low parts share one 8-column B fragment (below):
-  // 16 words per lane
   static constexpr bool PACKQ = MMA && G <= 4;
   static constexpr int QLO = !MMA ? 0 : PACKQ ? 32 * 64 : 4 * G * 128;
-  static constexpr int PBUF = G * kBS * 4 + QLO;   // probabilities of one page (+ low query parts)
+  static constexpr int PBUF = G * kBS * 4 + QLO;   // probabilities of one page (+ the query parts)
   static constexpr int LOG2_NT = NT == 16 ? 4 : NT == 8 ? 3 : NT == 4 ? 2 : NT == 2 ? 1 : 0;
   static_assert(LPT >= 8 && LPT <= 32 && (LPT & (LPT - 1)) == 0, "row of 128, 256 or 512 bytes");
   static_assert(2 * NT == LPT, "lane layout");
