@@ -1,6 +1,7 @@
 /* A plain C99 client of libpa.so: include/pa.h must compile as strict C
- * (no C++ constructs) and the host allocator must be usable through it
- * alone.  Built and run by tests/test_c_client.py; needs no GPU. */
+ * (no C++ constructs) and the host allocator (fork, copy-on-write, prefix
+ * groups for the shared-prefix decode) must be usable through it alone.
+ * Built and run by tests/test_c_client.py; needs no GPU. */
 #include <stdio.h>
 
 #include "pa.h"
@@ -23,6 +24,13 @@ int main(void) {
   if (pa_seq_block_table(a, 8, table, 4, &n) != PA_OK || n != 2) return 16;
   printf("%lld %lld %d %d %d %d\n", (long long)pair[0], (long long)pair[1], table[0], table[1],
          pa_block_refcount(a, 0), pa_alloc_num_free(a));
+  {
+    /* parent and fork share their one full block: one group of two */
+    const int64_t ids[2] = {7, 8};
+    int32_t gs[3] = {-1, -1, -1}, gb[2] = {-1, -1}, ng = -1;
+    if (pa_alloc_prefix_groups(a, ids, 2, 4, gs, gb, &ng) != PA_OK) return 19;
+    printf("%d %d %d %d\n", ng, gs[0], gs[1], gb[0]);
+  }
   if (pa_seq_free(a, 7) != PA_OK || pa_seq_free(a, 8) != PA_OK) return 17;
   if (pa_seq_free(a, 8) != PA_ERR_INVALID_ARG) return 18; /* double free */
   printf("%d %s\n", pa_alloc_num_free(a), pa_status_string(PA_ERR_OUT_OF_BLOCKS));

@@ -1,6 +1,6 @@
 """The C ABI from C: tests/c_abi_client.c includes include/pa.h as strict
 C99 (-pedantic -Werror), links libpa.so and drives the host allocator
-through a fork and its copy-on-write (CPU only)."""
+through a fork, its copy-on-write and the prefix grouping (CPU only)."""
 
 import os
 import shutil
@@ -31,4 +31,6 @@ def test_plain_c_client():
     # held by both; 8 - 3 blocks in use; all free again; the status text
     lines = run.stdout.splitlines()
     assert lines[0].split() == ["1", "2", "0", "2", "2", "5"]
-    assert lines[1] == "8 out of free blocks"
+    # prefix groups: one group of both sequences sharing block 0
+    assert lines[1].split() == ["1", "0", "2", "1"]
+    assert lines[2] == "8 out of free blocks"
