@@ -1,9 +1,9 @@
 """Host-side argument checking of every device entry point, fuzzed on CPU:
-descriptors of valid calls (decode, FP8 decode, the no-scratch decode,
-prefill, cache writes, copy-on-write and swap copies) with zero to two
-fields changed at random — the pointer (null, misaligned), the dtype, the
-rank, a size or a stride (negative, zero, at and past 2^31, huge) — plus odd
-scales, head counts and options.  Every call must return one of the
+descriptors of valid calls (decode, FP8 decode, the no-scratch decode, the
+shared-prefix decode, prefill, cache writes, copy-on-write and swap copies)
+with zero to two fields changed at random — the pointer (null, misaligned),
+the dtype, the rank, a size or a stride (negative, zero, at and past 2^31,
+huge) — plus odd scales, head counts, group sizes and options.  Every call must return one of the
 documented status codes without crashing the process.
 
 The calls run in a child process that sees no CUDA device
@@ -71,7 +71,7 @@ def call(r):
     max_nb, T = r.choice([0, 1, 5, 128]), r.choice([0, 1, 7, 300])
     dt = r.choice([0, 1, 4])
     qdt = 1 if dt == 4 else dt
-    which = r.randrange(7)
+    which = r.randrange(8)
     cache = lambda d=dt: [tensor((NB, Hkv, 16, D), d), tensor((NB, Hkv, 16, D), d)]  # noqa: E731
     if which == 0:
         ts = [tensor((T, Hkv, D), dt), tensor((T, Hkv, D), dt), *cache(), tensor((T,), 3)]
@@ -88,8 +88,12 @@ def call(r):
     elif which == 5:
         ts = [tensor((T, H, D), 1), tensor((T, H, D), 1), *cache(1), tensor((B, max_nb), 2), tensor((B,), 2),
               tensor((B + 1,), 2)]
-    else:
+    elif which == 6:
         ts = [*cache(), *cache(), tensor((T, 2), 3)]
+    else:
+        ng = r.choice([0, 1, B, B + 1])
+        ts = [tensor((B, H, D), qdt), tensor((B, H, D), qdt), *cache(), tensor((B, max_nb), 2), tensor((B,), 2),
+              tensor((ng + 1,), 2), tensor((ng,), 2)]
     for _ in range(r.randrange(3)):
         mutate(r, ts)
     p = [ctypes.byref(t) if r.random() > 0.03 else None for t in ts]
@@ -108,7 +112,9 @@ def call(r):
         return lib.pa_decode_fp8(*p[:6], r.choice([1.0, float("nan")]), heads, p[6], p[7], o)
     if which == 5:
         return lib.pa_prefill(*p, r.choice([-1, 0, 1, T, T + 1]), r.choice([1.0, 0.0, -1.0]), heads, o)
-    return lib.pa_swap_blocks(*p, o)
+    if which == 6:
+        return lib.pa_swap_blocks(*p, o)
+    return lib.pa_decode_cascade(*p[:8], r.choice([-1, 0, 1, 2, 4, 9]), r.choice([1.0, float("nan")]), heads, o)
 
 
 r = random.Random(int(sys.argv[1]))
