@@ -305,6 +305,12 @@ pa_status pa_decode_cascade_workspace_bytes(int32_t num_seqs, int32_t num_heads,
  *   nearest even and saturation to +-448 (NaN stays NaN).
  * pa_decode_fp8: as pa_decode over an FP8 cache with bf16 query and output;
  *   K[t] = e4m3_value(code) * k_scale[g], V likewise; fp32 accumulation.
+ *   For G = H / H_kv >= 2 the page dot products run on the tensor cores
+ *   (mma.sync, f16 operands): the e4m3 codes are exact in f16 and the
+ *   query, scaled per head by a power of two, is carried as an f16 high
+ *   part plus the f16 rounding of the rest (about 22 bits), so the logits
+ *   keep close to fp32 accuracy at any query magnitude; the probabilities
+ *   enter the PV product as f16.
  * k_scale, v_scale: [H_kv] fp32 on the device, contiguous, positive.
  * pa_reshape_and_cache and pa_decode reject FP8 caches (they have no scales).
  * ------------------------------------------------------------------------- */
